@@ -1,0 +1,438 @@
+/*
+ * lowbit_oracle.c -- the CPU oracle for the packed low-bit products.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, obviously-correct
+ * statement of what the GPU library computes.  Only the test-suite, the smoke
+ * check and the benchmark's CPU-baseline leg may load it.  It shares no code,
+ * header, table or constant with the CUDA library, and the CUDA library never
+ * calls it.
+ *
+ * Style rules kept on purpose:
+ *   - single-threaded, no SIMD intrinsics, no blocking, no reordering;
+ *   - floating point products are formed and summed in IEEE double, with the
+ *     reduction index ascending, exactly as the defining sums are written;
+ *   - integer products are summed in int64 and only then reduced mod 2^16.
+ *
+ * Sources (web pages; section named after the page title):
+ *   [Z80]    "Show HN: Z80-uLM, a conversational AI that fits in 40KB"
+ *            -- feature list (2-bit weights {-2,-1,0,+1}, 4 per byte; 16-bit
+ *            integer inference), architecture list (128 query + 128 context
+ *            trigram buckets, hidden layers, ReLU between hidden layers, one
+ *            output neuron per character), the "unpack 2-bit weight" listing,
+ *            the MULADD listing, and the per-layer arithmetic shift listing.
+ *   [BONSAI] "Bonsai-27B-gguf technical white paper digest", section
+ *            "technical architecture highlights" (one sign bit per weight,
+ *            -1 or +1; one FP16 scale shared by every 128 weights; 1.125 bits
+ *            per weight; 14.2x smaller than FP16).
+ *   [ACORN]  "acorn-llm 0.11.4" project page, section "int4 quantisation
+ *            quality: group quantisation" (one scale per group of values along
+ *            the input dimension; symmetric round-to-nearest int4; the scale
+ *            changes every 64 values).
+ *
+ * Readings taken where the pages are silent (each is listed in the design doc):
+ *   - Q1 bit polarity: bit 1 -> +1, bit 0 -> -1.
+ *   - Q1 bit order: weight k of a row is bit (k % 8) of byte (k / 8), LSB first
+ *     (the same LSB-first order the Z80 listing uses for its 2-bit fields).
+ *   - Q1 scale group: 128 consecutive weights along K of one row.
+ *   - INT4: two's-complement nibble, even k in the low nibble, no zero point,
+ *     group of 64 consecutive weights along K with one FP16 scale.
+ *   - Q2 weight matrix is row-major [out][in], codes packed along `in`.
+ *   - Shift after the output layer too; argmax ties go to the lowest index.
+ *   - Trigram hash: FNV-1a 32-bit of the three bytes, bucket = hash mod 128,
+ *     +32 per trigram, words padded with one space on each side.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* Scalar decoders, written from the IEEE 754 / bfloat16 bit layouts.        */
+/* ------------------------------------------------------------------------ */
+
+/* binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits. */
+double orc_f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int expo = (h >> 10) & 0x1F;
+    int frac = h & 0x3FF;
+    double v;
+    if (expo == 0)
+        v = ldexp((double)frac, -24);                 /* subnormal: frac * 2^-24 */
+    else if (expo == 31)
+        v = frac ? NAN : INFINITY;
+    else
+        v = ldexp((double)(frac + 1024), expo - 25);  /* (1.frac) * 2^(expo-15) */
+    return sign ? -v : v;
+}
+
+/* bfloat16: 1 sign, 8 exponent (bias 127), 7 fraction bits. */
+double orc_bf16_to_f64(uint16_t b)
+{
+    int sign = (b >> 15) & 1;
+    int expo = (b >> 7) & 0xFF;
+    int frac = b & 0x7F;
+    double v;
+    if (expo == 0)
+        v = ldexp((double)frac, -133);                /* subnormal: frac * 2^-133 */
+    else if (expo == 255)
+        v = frac ? NAN : INFINITY;
+    else
+        v = ldexp((double)(frac + 128), expo - 134);  /* (1.frac) * 2^(expo-127) */
+    return sign ? -v : v;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Q1_0_g128 [BONSAI]: one sign bit per weight, FP16 scale per 128 weights.  */
+/* ------------------------------------------------------------------------ */
+
+/* codes[r][c] in {0,1} -> packed[r][c/8], bit (c%8).  Returns 0, or -1 when
+   cols is not a multiple of 8 or a code is out of range. */
+int orc_q1_pack(const int8_t *codes, int64_t rows, int64_t cols, uint8_t *packed)
+{
+    if (cols % 8 != 0) return -1;
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t j = 0; j < cols / 8; j++) {
+            unsigned byte = 0;
+            for (int i = 0; i < 8; i++) {
+                int8_t c = codes[r * cols + 8 * j + i];
+                if (c != 0 && c != 1) return -1;
+                byte |= (unsigned)c << i;
+            }
+            packed[r * (cols / 8) + j] = (uint8_t)byte;
+        }
+    }
+    return 0;
+}
+
+int orc_q1_unpack(const uint8_t *packed, int64_t rows, int64_t cols, int8_t *codes)
+{
+    if (cols % 8 != 0) return -1;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c++)
+            codes[r * cols + c] = (int8_t)((packed[r * (cols / 8) + c / 8] >> (c % 8)) & 1);
+    return 0;
+}
+
+/* The dequantised weight w[n][k] = (bit ? +1 : -1) * d[n][k/128]. */
+double orc_q1_weight(const uint8_t *bits, const uint16_t *scales, int64_t K, int64_t n, int64_t k)
+{
+    int bit = (bits[n * (K / 8) + k / 8] >> (k % 8)) & 1;
+    double d = orc_f16_to_f64(scales[n * (K / 128) + k / 128]);
+    return bit ? d : -d;
+}
+
+/* y[m][n] = sum_k w[n][k] * x[m][k], in double, k ascending.
+   absdot[m][n] = sum_k |w[n][k] * x[m][k]| (may be NULL). */
+int orc_q1_gemv(const uint8_t *bits, const uint16_t *scales, const uint16_t *x,
+                int64_t M, int64_t N, int64_t K, double *y, double *absdot)
+{
+    if (K % 128 != 0) return -1;
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                double p = orc_q1_weight(bits, scales, K, n, k) * orc_bf16_to_f64(x[m * K + k]);
+                acc += p;
+                aacc += fabs(p);
+            }
+            y[m * N + n] = acc;
+            if (absdot) absdot[m * N + n] = aacc;
+        }
+    }
+    return 0;
+}
+
+/* The same definition evaluated only at the listed (m, n) output elements. */
+int orc_q1_gemv_at(const uint8_t *bits, const uint16_t *scales, const uint16_t *x,
+                   int64_t K, const int64_t *ms, const int64_t *ns, int64_t count,
+                   double *y, double *absdot)
+{
+    if (K % 128 != 0) return -1;
+    for (int64_t i = 0; i < count; i++) {
+        double acc = 0.0, aacc = 0.0;
+        for (int64_t k = 0; k < K; k++) {
+            double p = orc_q1_weight(bits, scales, K, ns[i], k) * orc_bf16_to_f64(x[ms[i] * K + k]);
+            acc += p;
+            aacc += fabs(p);
+        }
+        y[i] = acc;
+        if (absdot) absdot[i] = aacc;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* INT4, symmetric, FP16 scale per 64 weights along K [ACORN].               */
+/* ------------------------------------------------------------------------ */
+
+/* codes[r][c] in [-8,7] -> packed[r][c/2]; even c in the low nibble. */
+int orc_int4_pack(const int8_t *codes, int64_t rows, int64_t cols, uint8_t *packed)
+{
+    if (cols % 2 != 0) return -1;
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t j = 0; j < cols / 2; j++) {
+            int8_t lo = codes[r * cols + 2 * j];
+            int8_t hi = codes[r * cols + 2 * j + 1];
+            if (lo < -8 || lo > 7 || hi < -8 || hi > 7) return -1;
+            unsigned lo4 = (unsigned)(lo < 0 ? lo + 16 : lo);   /* two's complement in 4 bits */
+            unsigned hi4 = (unsigned)(hi < 0 ? hi + 16 : hi);
+            packed[r * (cols / 2) + j] = (uint8_t)(lo4 | (hi4 << 4));
+        }
+    }
+    return 0;
+}
+
+static int nibble_value(unsigned nib)
+{
+    return nib >= 8 ? (int)nib - 16 : (int)nib;
+}
+
+int orc_int4_unpack(const uint8_t *packed, int64_t rows, int64_t cols, int8_t *codes)
+{
+    if (cols % 2 != 0) return -1;
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t c = 0; c < cols; c++) {
+            uint8_t byte = packed[r * (cols / 2) + c / 2];
+            unsigned nib = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+            codes[r * cols + c] = (int8_t)nibble_value(nib);
+        }
+    }
+    return 0;
+}
+
+/* w[n][k] = q[n][k] * d[n][k/64]. */
+double orc_int4_weight(const uint8_t *q, const uint16_t *scales, int64_t K, int64_t n, int64_t k)
+{
+    uint8_t byte = q[n * (K / 2) + k / 2];
+    unsigned nib = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+    return (double)nibble_value(nib) * orc_f16_to_f64(scales[n * (K / 64) + k / 64]);
+}
+
+int orc_int4_gemv(const uint8_t *q, const uint16_t *scales, const uint16_t *x,
+                  int64_t M, int64_t N, int64_t K, double *y, double *absdot)
+{
+    if (K % 64 != 0) return -1;
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                double p = orc_int4_weight(q, scales, K, n, k) * orc_bf16_to_f64(x[m * K + k]);
+                acc += p;
+                aacc += fabs(p);
+            }
+            y[m * N + n] = acc;
+            if (absdot) absdot[m * N + n] = aacc;
+        }
+    }
+    return 0;
+}
+
+int orc_int4_gemv_at(const uint8_t *q, const uint16_t *scales, const uint16_t *x,
+                     int64_t K, const int64_t *ms, const int64_t *ns, int64_t count,
+                     double *y, double *absdot)
+{
+    if (K % 64 != 0) return -1;
+    for (int64_t i = 0; i < count; i++) {
+        double acc = 0.0, aacc = 0.0;
+        for (int64_t k = 0; k < K; k++) {
+            double p = orc_int4_weight(q, scales, K, ns[i], k) * orc_bf16_to_f64(x[ms[i] * K + k]);
+            acc += p;
+            aacc += fabs(p);
+        }
+        y[i] = acc;
+        if (absdot) absdot[i] = aacc;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Z80-style 2-bit integer MLP [Z80].                                        */
+/* ------------------------------------------------------------------------ */
+
+/* codes[r][c] in {0,1,2,3} -> packed[r][c/4], code of c at bits 2*(c%4). */
+int orc_q2_pack(const int8_t *codes, int64_t rows, int64_t cols, uint8_t *packed)
+{
+    if (cols % 4 != 0) return -1;
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t j = 0; j < cols / 4; j++) {
+            unsigned byte = 0;
+            for (int i = 0; i < 4; i++) {
+                int8_t c = codes[r * cols + 4 * j + i];
+                if (c < 0 || c > 3) return -1;
+                byte |= (unsigned)c << (2 * i);
+            }
+            packed[r * (cols / 4) + j] = (uint8_t)byte;
+        }
+    }
+    return 0;
+}
+
+int orc_q2_unpack(const uint8_t *packed, int64_t rows, int64_t cols, int8_t *codes)
+{
+    if (cols % 4 != 0) return -1;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c++)
+            codes[r * cols + c] = (int8_t)((packed[r * (cols / 4) + c / 4] >> (2 * (c % 4))) & 3);
+    return 0;
+}
+
+/* Code -> weight: the "sub 2" step of the unpack listing maps 0,1,2,3 to
+   -2,-1,0,+1. */
+int orc_q2_weight(const uint8_t *packed, int64_t in_dim, int64_t o, int64_t i)
+{
+    int code = (packed[o * (in_dim / 4) + i / 4] >> (2 * (i % 4))) & 3;
+    return code - 2;
+}
+
+/* Reduce an exact integer sum to the 16-bit two's-complement register it
+   would leave in a wrapping 16-bit accumulator. */
+static int16_t wrap16(int64_t v)
+{
+    uint16_t u = (uint16_t)((uint64_t)v & 0xFFFFu);
+    return (int16_t)(u >= 0x8000u ? (int32_t)u - 0x10000 : (int32_t)u);
+}
+
+/* Arithmetic right shift by 2 of a 16-bit register: the listing's
+   "sra h / rr l" pair done twice.  Written as floor division by 4, which is
+   what a sign-preserving shift of a two's-complement value computes. */
+static int16_t sra2(int16_t v)
+{
+    int32_t q = v / 4;
+    if ((v % 4) != 0 && v < 0) q -= 1;   /* C division truncates; floor it */
+    return (int16_t)q;
+}
+
+/* One layer, exact form: acc = sum_i w[o][i] * a[i] in int64, then wrapped
+   to 16 bits, then shifted.  Hidden layers apply ReLU; the output layer does
+   not.  out[] receives the post-shift (and post-ReLU for hidden) values. */
+void orc_q2_layer(const uint8_t *packed, int64_t in_dim, int64_t out_dim,
+                  const int16_t *a, int is_hidden, int16_t *out)
+{
+    for (int64_t o = 0; o < out_dim; o++) {
+        int64_t acc = 0;
+        for (int64_t i = 0; i < in_dim; i++)
+            acc += (int64_t)orc_q2_weight(packed, in_dim, o, i) * (int64_t)a[i];
+        int16_t z = sra2(wrap16(acc));
+        out[o] = (is_hidden && z < 0) ? 0 : z;
+    }
+}
+
+/* One layer, register-level form: the MULADD listing taken literally in its
+   arithmetic meaning -- weight 0 skips, +1 adds the activation once, -1
+   subtracts it once, -2 subtracts it twice -- with the 16-bit accumulator
+   wrapping after every single add or subtract. */
+void orc_q2_layer_muladd16(const uint8_t *packed, int64_t in_dim, int64_t out_dim,
+                           const int16_t *a, int is_hidden, int16_t *out)
+{
+    for (int64_t o = 0; o < out_dim; o++) {
+        int16_t hl = 0;
+        for (int64_t i = 0; i < in_dim; i++) {
+            int w = orc_q2_weight(packed, in_dim, o, i);
+            int16_t de = a[i];
+            if (w == 0) continue;
+            if (w == 1) { hl = wrap16((int64_t)hl + de); continue; }
+            hl = wrap16((int64_t)hl - de);
+            if (w == -2) hl = wrap16((int64_t)hl - de);
+        }
+        int16_t z = sra2(hl);
+        out[o] = (is_hidden && z < 0) ? 0 : z;
+    }
+}
+
+/* Smallest index of the maximum. */
+int32_t orc_argmax16(const int16_t *v, int64_t n)
+{
+    int32_t best = 0;
+    for (int64_t i = 1; i < n; i++)
+        if (v[i] > v[best]) best = (int32_t)i;
+    return best;
+}
+
+/* Whole network for a batch of input vectors.
+   packed_layers[l] is [dims[l+1]][dims[l]/4].  logits[b][dims[n_layers]];
+   argmax may be NULL.  use_muladd16 selects the register-level form.
+   dims[] must not exceed 4096. */
+int orc_q2_mlp_forward(const uint8_t *const *packed_layers, const int32_t *dims, int n_layers,
+                       const int16_t *x, int64_t batch, int16_t *logits, int32_t *argmax,
+                       int use_muladd16)
+{
+    static int16_t bufa[4096], bufb[4096];
+    if (n_layers < 1) return -1;
+    for (int l = 0; l <= n_layers; l++)
+        if (dims[l] < 1 || dims[l] > 4096 || (l < n_layers && dims[l] % 4 != 0)) return -1;
+    for (int64_t b = 0; b < batch; b++) {
+        memcpy(bufa, x + b * dims[0], sizeof(int16_t) * (size_t)dims[0]);
+        int16_t *cur = bufa, *nxt = bufb;
+        for (int l = 0; l < n_layers; l++) {
+            int hidden = (l < n_layers - 1);
+            if (use_muladd16)
+                orc_q2_layer_muladd16(packed_layers[l], dims[l], dims[l + 1], cur, hidden, nxt);
+            else
+                orc_q2_layer(packed_layers[l], dims[l], dims[l + 1], cur, hidden, nxt);
+            int16_t *t = cur; cur = nxt; nxt = t;
+        }
+        int64_t nout = dims[n_layers];
+        memcpy(logits + b * nout, cur, sizeof(int16_t) * (size_t)nout);
+        if (argmax) argmax[b] = orc_argmax16(cur, nout);
+    }
+    return 0;
+}
+
+/* Trigram-bucket encoder [Z80 "trigram hash encoding"]: the text is lower-
+   cased and split on spaces; each word, padded with one space on each side,
+   contributes +32 to bucket (FNV-1a-32 of each 3-byte window) mod 128.  Word
+   order does not change the result, because every trigram lies inside one
+   word. */
+static uint32_t fnv1a3(const unsigned char *p)
+{
+    uint32_t h = 2166136261u;
+    for (int i = 0; i < 3; i++) {
+        h ^= p[i];
+        h *= 16777619u;
+    }
+    return h;
+}
+
+void orc_trigram_encode(const char *text, int16_t *buckets /* [128] */)
+{
+    unsigned char word[258];
+    memset(buckets, 0, 128 * sizeof(int16_t));
+    size_t n = strlen(text), i = 0;
+    while (i < n) {
+        while (i < n && text[i] == ' ') i++;
+        size_t len = 0;
+        word[len++] = ' ';
+        while (i < n && text[i] != ' ' && len < 256) {
+            unsigned char c = (unsigned char)text[i++];
+            if (c >= 'A' && c <= 'Z') c = (unsigned char)(c - 'A' + 'a');
+            word[len++] = c;
+        }
+        while (i < n && text[i] != ' ') i++;   /* overlong word: rest ignored */
+        if (len == 1) break;                     /* no more words */
+        word[len++] = ' ';
+        for (size_t t = 0; t + 3 <= len; t++)
+            buckets[fnv1a3(word + t) % 128] += 32;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Glue between the projections of a layer stack: RMS normalisation.         */
+/* r[m][d] = v[m][d] / sqrt(mean_d v[m][d]^2 + eps), v = a (+ b when b is     */
+/* given), in double.  The caller rounds r to bfloat16.                       */
+/* ------------------------------------------------------------------------ */
+void orc_rmsnorm(const float *a, const float *b, int64_t M, int64_t D, double eps, double *r)
+{
+    for (int64_t m = 0; m < M; m++) {
+        double ss = 0.0;
+        for (int64_t d = 0; d < D; d++) {
+            double v = (double)a[m * D + d] + (b ? (double)b[m * D + d] : 0.0);
+            ss += v * v;
+        }
+        double inv = 1.0 / sqrt(ss / (double)D + eps);
+        for (int64_t d = 0; d < D; d++) {
+            double v = (double)a[m * D + d] + (b ? (double)b[m * D + d] : 0.0);
+            r[m * D + d] = v * inv;
+        }
+    }
+}

@@ -1,0 +1,368 @@
+"""Pins for the CPU oracle: every check here compares the oracle with
+something other than itself -- the pages' fixed facts (tests/golden), an
+emulation of the Z80 listing's instructions, library routines (numpy's
+unpackbits / float16, torch's bfloat16, numpy matmul), closed forms and
+brute-force enumeration.  No GPU is used."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from conftest import read_golden
+
+
+# ---------------------------------------------------------------------------
+# scalar decoders
+# ---------------------------------------------------------------------------
+
+def test_f16_decode_all_patterns_match_numpy():
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = pats.view(np.float16).astype(np.float64)
+    got = np.array([oracle.f16_to_f64(int(p)) for p in pats])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_bf16_decode_all_patterns_match_torch():
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(pats.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    got = np.array([oracle.bf16_to_f64(int(p)) for p in pats])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+# ---------------------------------------------------------------------------
+# Q1_0_g128
+# ---------------------------------------------------------------------------
+
+def test_q1_format_facts_from_page():
+    g = {r[0]: float(r[1]) for r in read_golden("q1_format.txt")}
+    K, N = 4096, 8
+    codes = synth.q1_codes(1, N, K)
+    packed = oracle.pack("q1", codes)
+    scales = synth.q1_scales(1, N, K)
+    bits = 8 * (packed.nbytes + scales.nbytes)
+    assert bits / (N * K) == g["bits_per_weight"]
+    assert g["sign_bits_per_weight"] + g["scale_bits"] / g["group_size"] == g["bits_per_weight"]
+    assert round(16 / (bits / (N * K)), 1) == g["ratio_vs_fp16"]
+    assert scales.shape == (N, K // int(g["group_size"]))
+
+
+def test_q1_unpack_all_bytes_matches_numpy_unpackbits():
+    allb = np.arange(256, dtype=np.uint8).reshape(256, 1)
+    got = oracle.unpack("q1", allb, 8)
+    ref = np.unpackbits(allb, axis=1, bitorder="little").astype(np.int8)
+    assert np.array_equal(got, ref)
+    assert np.array_equal(oracle.pack("q1", got), allb)
+
+
+def test_q1_pack_roundtrip_random():
+    codes = synth.q1_codes(2, 33, 1024)
+    p = oracle.pack("q1", codes)
+    assert np.array_equal(oracle.unpack("q1", p, 1024), codes)
+    with pytest.raises(ValueError):
+        oracle.pack("q1", np.full((1, 8), 2, np.int8))
+
+
+def _np_q1_dense(bits, scales, K):
+    signs = np.where(np.unpackbits(bits, axis=1, bitorder="little")[:, :K] == 1, 1.0, -1.0)
+    d = np.repeat(scales.view(np.float16).astype(np.float64), 128, axis=1)
+    return signs * d
+
+
+def test_q1_gemv_matches_numpy_matmul():
+    M, N, K = 3, 37, 384
+    bits = oracle.pack("q1", synth.q1_codes(3, N, K))
+    scales = synth.q1_scales(3, N, K)
+    x = synth.bf16_normal(3, (M, K))
+    y, ab = oracle.q1_gemv(bits, scales, x, want_abs=True)
+    W = _np_q1_dense(bits, scales, K)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    np.testing.assert_allclose(y, xf @ W.T, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ab, np.abs(xf) @ np.abs(W).T, rtol=1e-12)
+
+
+def test_q1_onehot_probe_reads_back_every_weight():
+    N, K = 5, 256
+    bits = oracle.pack("q1", synth.q1_codes(4, N, K))
+    scales = synth.q1_scales(4, N, K)
+    one = 0x3F80  # bf16 1.0
+    for k in (0, 1, 7, 8, 127, 128, 200, 255):
+        x = np.zeros((1, K), np.uint16)
+        x[0, k] = one
+        y = oracle.q1_gemv(bits, scales, x)[0]
+        for n in range(N):
+            bit = (int(bits[n, k // 8]) >> (k % 8)) & 1
+            d = float(scales[n, k // 128:k // 128 + 1].view(np.float16)[0])
+            assert y[n] == (d if bit else -d)
+
+
+def test_q1_all_ones_closed_form():
+    N, K = 9, 512
+    bits = oracle.pack("q1", synth.q1_codes(5, N, K))
+    scales = synth.q1_scales(5, N, K)
+    x = np.full((1, K), 0x3F80, np.uint16)
+    y = oracle.q1_gemv(bits, scales, x)[0]
+    for n in range(N):
+        exp = 0.0
+        for g in range(K // 128):
+            pop = sum(bin(int(b)).count("1") for b in bits[n, 16 * g:16 * g + 16])
+            exp += float(scales[n, g:g + 1].view(np.float16)[0]) * (2 * pop - 128)
+        assert y[n] == exp
+
+
+def test_q1_unit_scales_integer_x_exact_int64():
+    N, K = 16, 256
+    codes = synth.q1_codes(6, N, K)
+    bits = oracle.pack("q1", codes)
+    scales = np.full((N, K // 128), 0x3C00, np.uint16)  # fp16 1.0
+    xi = synth.rng(6, 99).integers(-100, 101, size=(2, K))
+    x = synth.to_bf16_bits(xi.astype(np.float64))
+    y = oracle.q1_gemv(bits, scales, x)
+    ref = xi.astype(np.int64) @ (2 * codes.astype(np.int64) - 1).T
+    assert np.array_equal(y, ref.astype(np.float64))
+
+
+def test_q1_bruteforce_all_sign_patterns_of_one_byte():
+    # x_k = 2^k on k = 0..7 and 0 elsewhere; sum_k (2 b_k - 1) 2^k = 2 v - 255.
+    K = 128
+    x = np.zeros((1, K), np.uint16)
+    x[0, :8] = synth.to_bf16_bits(2.0 ** np.arange(8))
+    scales = np.full((1, 1), 0x3C00, np.uint16)
+    for v in range(256):
+        bits = np.zeros((1, K // 8), np.uint8)
+        bits[0, 0] = v
+        assert oracle.q1_gemv(bits, scales, x)[0, 0] == 2 * v - 255
+
+
+def test_q1_gemv_at_equals_full():
+    M, N, K = 2, 11, 256
+    bits = oracle.pack("q1", synth.q1_codes(7, N, K))
+    scales = synth.q1_scales(7, N, K)
+    x = synth.bf16_normal(7, (M, K))
+    y = oracle.q1_gemv(bits, scales, x)
+    ms = np.array([0, 1, 1, 0])
+    ns = np.array([0, 10, 3, 5])
+    ys, _ = oracle.q1_gemv_at(bits, scales, x, ms, ns)
+    assert np.array_equal(ys, y[ms, ns])
+
+
+# ---------------------------------------------------------------------------
+# INT4-g64
+# ---------------------------------------------------------------------------
+
+def test_int4_group_fact_and_layout():
+    g = {r[0]: int(r[1]) for r in read_golden("int4_group.txt")}
+    assert g["group_size"] == 64 and g["values_per_byte"] == 2
+    codes = synth.int4_codes(1, 4, 128)
+    assert codes.min() >= g["code_min"] and codes.max() <= g["code_max"]
+    scales = synth.int4_scales(1, 4, 128)
+    assert scales.shape == (4, 128 // g["group_size"])
+
+
+def test_int4_unpack_all_bytes_sign_extension():
+    allb = np.arange(256, dtype=np.uint8).reshape(256, 1)
+    got = oracle.unpack("int4", allb, 2)
+    lo = (allb[:, 0].astype(np.int8) << 4) >> 4           # arithmetic shift sign-extends
+    hi = allb[:, 0].astype(np.int8) >> 4
+    assert np.array_equal(got[:, 0], lo)
+    assert np.array_equal(got[:, 1], hi)
+    assert np.array_equal(oracle.pack("int4", got), allb)
+
+
+def test_int4_all_nibble_pairs_roundtrip():
+    pairs = np.array([[a, b] for a in range(-8, 8) for b in range(-8, 8)], np.int8)
+    p = oracle.pack("int4", pairs)
+    assert np.array_equal(oracle.unpack("int4", p, 2), pairs)
+    with pytest.raises(ValueError):
+        oracle.pack("int4", np.array([[8, 0]], np.int8))
+
+
+def test_int4_gemv_matches_numpy_matmul():
+    M, N, K = 4, 29, 320
+    codes = synth.int4_codes(8, N, K)
+    q = oracle.pack("int4", codes)
+    scales = synth.int4_scales(8, N, K)
+    x = synth.bf16_normal(8, (M, K))
+    y, ab = oracle.int4_gemv(q, scales, x, want_abs=True)
+    W = codes.astype(np.float64) * np.repeat(scales.view(np.float16).astype(np.float64), 64, axis=1)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    np.testing.assert_allclose(y, xf @ W.T, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ab, np.abs(xf) @ np.abs(W).T, rtol=1e-12)
+
+
+def test_int4_group_isolation_probe():
+    # Only group g has a non-zero scale: y must equal d * sum over that group.
+    N, K = 3, 256
+    codes = synth.int4_codes(9, N, K)
+    q = oracle.pack("int4", codes)
+    x = np.full((1, K), 0x3F80, np.uint16)
+    for g in range(K // 64):
+        scales = np.zeros((N, K // 64), np.uint16)
+        scales[:, g] = 0x3C00
+        y = oracle.int4_gemv(q, scales, x)[0]
+        assert np.array_equal(y, codes[:, 64 * g:64 * g + 64].sum(axis=1).astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# Z80-style 2-bit integer MLP
+# ---------------------------------------------------------------------------
+
+def _z80_unpack_byte(byte):
+    """Emulate the page's listing on an 8-bit A register: `and 03h; sub 2`
+    gives one weight, `rrca` twice rotates the next field into place."""
+    a = byte
+    out = []
+    for _ in range(4):
+        w = ((a & 0x03) - 2) & 0xFF
+        out.append(w - 256 if w >= 128 else w)
+        for _ in range(2):                      # rrca: bit 0 -> bit 7 and carry
+            a = ((a >> 1) | ((a & 1) << 7)) & 0xFF
+    return out
+
+
+def test_q2_code_map_from_page():
+    cmap = {int(c): int(w) for c, w in read_golden("q2_code_map.txt")}
+    assert cmap == {0: -2, 1: -1, 2: 0, 3: 1}
+    for code, w in cmap.items():
+        packed = np.array([[code]], np.uint8)   # code in the first field
+        assert oracle.unpack("q2", packed, 4)[0, 0] == code
+        assert _z80_unpack_byte(code)[0] == w
+
+
+def test_q2_unpack_matches_z80_listing_for_every_byte():
+    cmap = {int(c): int(w) for c, w in read_golden("q2_code_map.txt")}
+    allb = np.arange(256, dtype=np.uint8).reshape(256, 1)
+    codes = oracle.unpack("q2", allb, 4)
+    for v in range(256):
+        assert [cmap[int(c)] for c in codes[v]] == _z80_unpack_byte(v)
+    assert np.array_equal(oracle.pack("q2", codes), allb)
+
+
+def _z80_sra2(v16):
+    """`sra h; rr l` twice on the 16-bit pair HL, bit by bit."""
+    h, l = (v16 >> 8) & 0xFF, v16 & 0xFF
+    for _ in range(2):
+        carry = h & 1
+        h = ((h >> 1) | (h & 0x80)) & 0xFF      # sra h keeps the sign bit
+        l = ((l >> 1) | (carry << 7)) & 0xFF    # rr l takes the carry
+    v = (h << 8) | l
+    return v - 65536 if v >= 32768 else v
+
+
+def test_q2_shift_matches_z80_sra_rr_pair_exhaustive():
+    # out layer with one +1 weight on input 0: acc = a0, out = shift(a0).
+    packed = np.array([[0b10101011]], np.uint8)  # codes 3,2,2,2 -> +1,0,0,0
+    vals = np.arange(-32768, 32768, 37, dtype=np.int64)
+    for v in vals:
+        a = np.array([v, 5, -5, 1], np.int16)
+        got = int(oracle.q2_layer(packed, 4, 1, a, hidden=False)[0])
+        assert got == _z80_sra2(int(v) & 0xFFFF)
+        assert got == int(v) // 4
+
+
+def test_q2_bruteforce_one_byte_all_codes():
+    a = np.array([1, 10, 100, 1000], np.int16)
+    for v in range(256):
+        packed = np.array([[v]], np.uint8)
+        ws = _z80_unpack_byte(v)
+        acc = sum(w * int(x) for w, x in zip(ws, a))
+        got = int(oracle.q2_layer(packed, 4, 1, a, hidden=False)[0])
+        assert got == acc // 4
+
+
+def _np_q2_layer(codes, a, hidden):
+    acc = (codes.astype(np.int64) - 2) @ a.astype(np.int64)
+    v = ((acc + 32768) % 65536) - 32768
+    z = v // 4
+    return np.maximum(z, 0) if hidden else z
+
+
+def test_q2_layer_matches_numpy_and_muladd16_with_overflow():
+    g = synth.rng(11, 0)
+    for trial in range(20):
+        cin, cout = 64, 24
+        codes = g.integers(0, 4, size=(cout, cin), dtype=np.int8)
+        # large activations force 16-bit wrap-around
+        a = g.integers(-32768, 32768, size=cin).astype(np.int16)
+        packed = oracle.pack("q2", codes)
+        for hidden in (True, False):
+            ref = _np_q2_layer(codes, a, hidden)
+            assert np.array_equal(oracle.q2_layer(packed, cin, cout, a, hidden), ref)
+            assert np.array_equal(oracle.q2_layer(packed, cin, cout, a, hidden, muladd16=True), ref)
+
+
+def test_q2_forward_matches_numpy_stack_and_relu_placement():
+    rows = {r[0]: r[1:] for r in read_golden("q2_topology.txt")}
+    dims = tuple(int(d) for d in rows["layers"])
+    assert dims == synth.Q2_DIMS
+    layers = synth.q2_codes(12, dims)
+    packed = [oracle.pack("q2", c) for c in layers]
+    x = synth.q2_inputs(12, 64)
+    logits, am = oracle.q2_mlp_forward(packed, dims, x)
+    logits16, am16 = oracle.q2_mlp_forward(packed, dims, x, muladd16=True)
+    assert np.array_equal(logits, logits16) and np.array_equal(am, am16)
+    for b in range(x.shape[0]):
+        a = x[b].astype(np.int64)
+        for l, c in enumerate(layers):
+            a = _np_q2_layer(c, a, hidden=(l < len(layers) - 1))
+        assert np.array_equal(logits[b], a)
+        assert am[b] == int(np.argmax(a))        # numpy argmax: first maximum
+    assert (logits < 0).any()                    # no ReLU on the output layer
+
+
+def test_q2_mac_count_order_from_page():
+    rows = {r[0]: r[1:] for r in read_golden("q2_topology.txt")}
+    dims = [int(v) for v in rows["layers"]]
+    macs = sum(dims[i] * dims[i + 1] for i in range(len(dims) - 1))
+    assert macs == 78848
+    order = int(rows["macs_per_char_order"][0])
+    assert order / 10 < macs < order * 10
+    assert int(rows["query_buckets"][0]) + int(rows["context_buckets"][0]) == dims[0]
+
+
+def test_argmax_ties_lowest_index():
+    assert oracle.argmax16(np.array([3, 7, 7, -1], np.int16)) == 1
+    assert oracle.argmax16(np.array([-5, -5], np.int16)) == 0
+
+
+def test_trigram_relations_from_page():
+    for rel, a, b in read_golden("trigram_examples.txt"):
+        va, vb = oracle.trigram_encode(a), oracle.trigram_encode(b)
+        assert va.shape == (128,) and (va % 32 == 0).all() and va.sum() > 0
+        if rel == "equal":
+            assert np.array_equal(va, vb)
+        else:
+            shared = np.minimum(va, vb).sum()
+            assert shared >= 0.4 * min(va.sum(), vb.sum())
+    # case-insensitive and whitespace-insensitive
+    assert np.array_equal(oracle.trigram_encode("Hello  There "), oracle.trigram_encode("hello there"))
+
+
+def test_q2_inputs_shape_the_trigram_distribution():
+    x = synth.q2_inputs(13, 32)
+    assert x.shape == (32, 256)
+    for half in (x[:, :128], x[:, 128:]):
+        assert ((half != 0).sum(axis=1) == 8).all()
+        assert set(np.unique(half[half != 0]).tolist()) <= {32, 64, 96}
+
+
+# ---------------------------------------------------------------------------
+# RMS normalisation glue
+# ---------------------------------------------------------------------------
+
+def test_rmsnorm_matches_numpy_and_closed_forms():
+    g = synth.rng(14, 0)
+    a = g.standard_normal((3, 640)).astype(np.float32)
+    b = g.standard_normal((3, 640)).astype(np.float32)
+    for bb in (None, b):
+        v = a.astype(np.float64) + (0.0 if bb is None else bb.astype(np.float64))
+        ref = v / np.sqrt(np.mean(v * v, axis=1, keepdims=True) + 1e-6)
+        np.testing.assert_allclose(oracle.rmsnorm(a, bb), ref, rtol=1e-13)
+    c = np.full((1, 64), 3.0, np.float32)
+    np.testing.assert_allclose(oracle.rmsnorm(c), 3.0 / np.sqrt(9.0 + 1e-6), rtol=1e-15)
+    r = oracle.rmsnorm(a * 1000.0)
+    np.testing.assert_allclose(r, oracle.rmsnorm(a), rtol=1e-5)
