@@ -1,0 +1,207 @@
+// lowbit_abi.cu -- the extern "C" entry points declared in include/lowbit.h.
+// Every argument is validated here, on the host, before anything is enqueued.
+#include "common.cuh"
+
+namespace lowbit {
+lowbit_status pack_launch(lowbit_format, const int8_t *, int64_t, int64_t, uint8_t *, cudaStream_t);
+lowbit_status unpack_launch(lowbit_format, const uint8_t *, int64_t, int64_t, int8_t *, cudaStream_t);
+lowbit_status q1_gemv_simt_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
+                                  int, cudaStream_t);
+lowbit_status int4_gemv_simt_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
+                                    int, cudaStream_t);
+lowbit_status q2_mlp_launch(const uint8_t *const *, const int32_t *, int, const int16_t *, int, int16_t *,
+                            int32_t *, cudaStream_t);
+int q2_weight_bytes_padded(const int32_t *, int);
+lowbit_status rmsnorm_launch(const float *, const float *, int, int, float, uint16_t *, cudaStream_t);
+
+constexpr int64_t kMaxElems = int64_t(1) << 40;
+constexpr int kQ1MaxM = 16;
+}  // namespace lowbit
+
+using namespace lowbit;
+
+#define LB_CHECK(cond, code) \
+    do {                     \
+        if (!(cond)) return (code); \
+    } while (0)
+
+static int per_byte(lowbit_format f)
+{
+    switch (f) {
+    case LOWBIT_FMT_Q1_G128: return 8;
+    case LOWBIT_FMT_Q2: return 4;
+    case LOWBIT_FMT_INT4_G64: return 2;
+    default: return 0;
+    }
+}
+
+extern "C" {
+
+const char *lowbit_status_string(lowbit_status s)
+{
+    switch (s) {
+    case LOWBIT_OK: return "ok";
+    case LOWBIT_ERR_INVALID_ARG: return "invalid argument";
+    case LOWBIT_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case LOWBIT_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case LOWBIT_ERR_CUDA: return "CUDA launch failed";
+    default: return "unknown status";
+    }
+}
+
+int lowbit_version(void) { return 100; }
+
+lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, int64_t cols,
+                          uint8_t *packed, void *stream)
+{
+    const int per = per_byte(fmt);
+    LB_CHECK(per != 0, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(rows >= 0 && cols >= 0 && rows * cols < kMaxElems, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(cols % per == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    if (rows == 0 || cols == 0) return LOWBIT_OK;
+    LB_CHECK(codes != nullptr && packed != nullptr, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(codes) && aligned16(packed), LOWBIT_ERR_MISALIGNED);
+    return pack_launch(fmt, codes, rows, cols, packed, as_stream(stream));
+}
+
+lowbit_status lowbit_unpack(lowbit_format fmt, const uint8_t *packed, int64_t rows, int64_t cols,
+                            int8_t *codes, void *stream)
+{
+    const int per = per_byte(fmt);
+    LB_CHECK(per != 0, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(rows >= 0 && cols >= 0 && rows * cols < kMaxElems, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(cols % per == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    if (rows == 0 || cols == 0) return LOWBIT_OK;
+    LB_CHECK(codes != nullptr && packed != nullptr, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(codes) && aligned16(packed), LOWBIT_ERR_MISALIGNED);
+    return unpack_launch(fmt, packed, rows, cols, codes, as_stream(stream));
+}
+
+// ---------------------------------------------------------------------------
+// Q1_0_g128
+// ---------------------------------------------------------------------------
+
+static lowbit_status q1_shape_ok(int M, int N, int K)
+{
+    LB_CHECK(M >= 1 && M <= kQ1MaxM && N >= 1 && K >= 1, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(K % 128 == 0 && (int64_t)N * K < kMaxElems, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    return LOWBIT_OK;
+}
+
+size_t lowbit_q1g128_workspace_bytes(int M, int K)
+{
+    (void)M;
+    (void)K;
+    return 0;
+}
+
+size_t lowbit_q1g128_act_bytes(int M, int K)
+{
+    if (M < 1 || K < 1) return 0;
+    return (size_t)M * (size_t)K * 2u;
+}
+
+lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales, const uint16_t *x,
+                                 float *y, int M, int N, int K, void *workspace, size_t workspace_bytes,
+                                 void *stream)
+{
+    lowbit_status s = q1_shape_ok(M, N, K);
+    if (s != LOWBIT_OK) return s;
+    LB_CHECK(w_bits && w_scales && x && y, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(w_bits) && aligned16(w_scales) && aligned16(x) && aligned16(y), LOWBIT_ERR_MISALIGNED);
+    const size_t need = lowbit_q1g128_workspace_bytes(M, K);
+    LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
+    return q1_gemv_simt_launch(w_bits, w_scales, x, y, M, N, K, as_stream(stream));
+}
+
+lowbit_status lowbit_q1g128_prepare_act(const uint16_t *x, int M, int K, void *act, size_t act_bytes,
+                                        void *stream)
+{
+    LB_CHECK(M >= 1 && M <= kQ1MaxM && K >= 1, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(K % 128 == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    LB_CHECK(x && act, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(x) && aligned16(act), LOWBIT_ERR_MISALIGNED);
+    const size_t need = lowbit_q1g128_act_bytes(M, K);
+    LB_CHECK(act_bytes >= need, LOWBIT_ERR_INVALID_ARG);
+    return cudaMemcpyAsync(act, x, need, cudaMemcpyDeviceToDevice, as_stream(stream)) == cudaSuccess
+               ? LOWBIT_OK
+               : LOWBIT_ERR_CUDA;
+}
+
+lowbit_status lowbit_q1g128_gemv_act(const uint8_t *w_bits, const uint16_t *w_scales, const void *act,
+                                     float *y, int M, int N, int K, void *stream)
+{
+    lowbit_status s = q1_shape_ok(M, N, K);
+    if (s != LOWBIT_OK) return s;
+    LB_CHECK(w_bits && w_scales && act && y, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(w_bits) && aligned16(w_scales) && aligned16(act) && aligned16(y),
+             LOWBIT_ERR_MISALIGNED);
+    return q1_gemv_simt_launch(w_bits, w_scales, static_cast<const uint16_t *>(act), y, M, N, K,
+                               as_stream(stream));
+}
+
+// ---------------------------------------------------------------------------
+// INT4_G64
+// ---------------------------------------------------------------------------
+
+size_t lowbit_int4g64_workspace_bytes(int M, int N, int K)
+{
+    (void)M;
+    (void)N;
+    (void)K;
+    return 0;
+}
+
+lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales, const uint16_t *x, float *y,
+                                  int M, int N, int K, void *workspace, size_t workspace_bytes, void *stream)
+{
+    LB_CHECK(M >= 1 && N >= 1 && K >= 1, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(K % 64 == 0 && (int64_t)N * K < kMaxElems && (int64_t)M * K < kMaxElems,
+             LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    LB_CHECK(w_q && w_scales && x && y, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(w_q) && aligned16(w_scales) && aligned16(x) && aligned16(y), LOWBIT_ERR_MISALIGNED);
+    const size_t need = lowbit_int4g64_workspace_bytes(M, N, K);
+    LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
+    return int4_gemv_simt_launch(w_q, w_scales, x, y, M, N, K, as_stream(stream));
+}
+
+// ---------------------------------------------------------------------------
+// Q2 MLP
+// ---------------------------------------------------------------------------
+
+lowbit_status lowbit_q2_mlp_forward(const uint8_t *const *w_packed, const int32_t *dims, int n_layers,
+                                    const int16_t *x, int batch, int16_t *logits, int32_t *argmax,
+                                    void *stream)
+{
+    LB_CHECK(w_packed && dims && n_layers >= 1 && n_layers <= 8 && batch >= 0, LOWBIT_ERR_INVALID_ARG);
+    for (int l = 0; l < n_layers; ++l) {
+        LB_CHECK(dims[l] >= 4 && dims[l] <= 1024, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+        LB_CHECK(dims[l] % 4 == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+        LB_CHECK(w_packed[l] != nullptr, LOWBIT_ERR_INVALID_ARG);
+        LB_CHECK(aligned16(w_packed[l]), LOWBIT_ERR_MISALIGNED);
+    }
+    LB_CHECK(dims[n_layers] >= 1 && dims[n_layers] <= 1024, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    LB_CHECK(q2_weight_bytes_padded(dims, n_layers) <= 96 * 1024, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    if (batch == 0) return LOWBIT_OK;
+    LB_CHECK(x && logits, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(x) && aligned16(logits) && (argmax == nullptr || aligned16(argmax)),
+             LOWBIT_ERR_MISALIGNED);
+    return q2_mlp_launch(w_packed, dims, n_layers, x, batch, logits, argmax, as_stream(stream));
+}
+
+// ---------------------------------------------------------------------------
+// glue
+// ---------------------------------------------------------------------------
+
+lowbit_status lowbit_rmsnorm_bf16(const float *a, const float *b, int M, int D, float eps, uint16_t *out,
+                                  void *stream)
+{
+    LB_CHECK(M >= 1 && D >= 1 && eps >= 0.f && a && out, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(D % 8 == 0 && (int64_t)M * D < kMaxElems, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    LB_CHECK(aligned16(a) && aligned16(out) && (b == nullptr || aligned16(b)), LOWBIT_ERR_MISALIGNED);
+    return rmsnorm_launch(a, b, M, D, eps, out, as_stream(stream));
+}
+
+}  // extern "C"

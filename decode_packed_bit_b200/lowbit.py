@@ -1,0 +1,172 @@
+"""Python binding of liblowbit.so (include/lowbit.h): argument marshalling only.
+
+Every function has the name of the C entry point it calls.  Tensors are
+torch CUDA tensors (torch supplies device memory and streams; every step of
+the computation runs in the library's own kernels).  fp16/bf16 operands may
+be given as float16/bfloat16 tensors or as int16/uint16 bit patterns.  A
+non-OK status raises LowbitError.  There is no fallback: if the shared
+library is missing, loading fails with an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "liblowbit.so")
+
+LOWBIT_OK = 0
+LOWBIT_ERR_INVALID_ARG = 1
+LOWBIT_ERR_MISALIGNED = 2
+LOWBIT_ERR_UNSUPPORTED_SHAPE = 3
+LOWBIT_ERR_CUDA = 4
+
+LOWBIT_FMT_Q1_G128 = 1
+LOWBIT_FMT_Q2 = 2
+LOWBIT_FMT_INT4_G64 = 3
+FORMATS = {"q1": LOWBIT_FMT_Q1_G128, "q2": LOWBIT_FMT_Q2, "int4": LOWBIT_FMT_INT4_G64}
+
+# (name, restype, argtypes) of every symbol include/lowbit.h declares.
+P, I32, I64, SZ, F32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+SYMBOLS = [
+    ("lowbit_status_string", ctypes.c_char_p, [I32]),
+    ("lowbit_version", I32, []),
+    ("lowbit_pack", I32, [I32, P, I64, I64, P, P]),
+    ("lowbit_unpack", I32, [I32, P, I64, I64, P, P]),
+    ("lowbit_q1g128_workspace_bytes", SZ, [I32, I32]),
+    ("lowbit_q1g128_gemv", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
+    ("lowbit_q1g128_act_bytes", SZ, [I32, I32]),
+    ("lowbit_q1g128_prepare_act", I32, [P, I32, I32, P, SZ, P]),
+    ("lowbit_q1g128_gemv_act", I32, [P, P, P, P, I32, I32, I32, P]),
+    ("lowbit_int4g64_workspace_bytes", SZ, [I32, I32, I32]),
+    ("lowbit_int4g64_gemm", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
+    ("lowbit_q2_mlp_forward", I32, [P, P, I32, P, I32, P, P, P]),
+    ("lowbit_rmsnorm_bf16", I32, [P, P, I32, I32, F32, P, P]),
+]
+
+_lib = None
+
+
+class LowbitError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().lowbit_status_string(status).decode()
+        super().__init__(f"{where}: {msg} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m decode_packed_bit_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SYMBOLS:
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != LOWBIT_OK:
+        raise LowbitError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _fmt(fmt):
+    return FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+# -- packing ----------------------------------------------------------------------
+
+def lowbit_pack(fmt, codes, packed, stream=None):
+    rows, cols = codes.shape
+    _check(lib().lowbit_pack(_fmt(fmt), _ptr(codes), rows, cols, _ptr(packed), _stream(stream)),
+           "lowbit_pack")
+
+
+def lowbit_unpack(fmt, packed, codes, stream=None):
+    rows, cols = codes.shape
+    _check(lib().lowbit_unpack(_fmt(fmt), _ptr(packed), rows, cols, _ptr(codes), _stream(stream)),
+           "lowbit_unpack")
+
+
+# -- Q1_0_g128 --------------------------------------------------------------------
+
+def lowbit_q1g128_workspace_bytes(M: int, K: int) -> int:
+    return int(lib().lowbit_q1g128_workspace_bytes(M, K))
+
+
+def lowbit_q1g128_act_bytes(M: int, K: int) -> int:
+    return int(lib().lowbit_q1g128_act_bytes(M, K))
+
+
+def lowbit_q1g128_gemv(w_bits, w_scales, x, y, workspace=None, stream=None):
+    M, K = x.shape
+    N = w_bits.shape[0]
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().lowbit_q1g128_gemv(_ptr(w_bits), _ptr(w_scales), _ptr(x), _ptr(y), M, N, K,
+                                    _ptr(workspace), wsb, _stream(stream)), "lowbit_q1g128_gemv")
+
+
+def lowbit_q1g128_prepare_act(x, act, stream=None):
+    M, K = x.shape
+    _check(lib().lowbit_q1g128_prepare_act(_ptr(x), M, K, _ptr(act), act.numel() * act.element_size(),
+                                           _stream(stream)), "lowbit_q1g128_prepare_act")
+
+
+def lowbit_q1g128_gemv_act(w_bits, w_scales, act, y, M: int, stream=None):
+    N = w_bits.shape[0]
+    K = w_bits.shape[1] * 8
+    _check(lib().lowbit_q1g128_gemv_act(_ptr(w_bits), _ptr(w_scales), _ptr(act), _ptr(y), M, N, K,
+                                        _stream(stream)), "lowbit_q1g128_gemv_act")
+
+
+# -- INT4_G64 ---------------------------------------------------------------------
+
+def lowbit_int4g64_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().lowbit_int4g64_workspace_bytes(M, N, K))
+
+
+def lowbit_int4g64_gemm(w_q, w_scales, x, y, workspace=None, stream=None):
+    M, K = x.shape
+    N = w_q.shape[0]
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().lowbit_int4g64_gemm(_ptr(w_q), _ptr(w_scales), _ptr(x), _ptr(y), M, N, K,
+                                     _ptr(workspace), wsb, _stream(stream)), "lowbit_int4g64_gemm")
+
+
+# -- Q2 MLP -----------------------------------------------------------------------
+
+def lowbit_q2_mlp_forward(w_packed, dims, x, logits, argmax=None, stream=None):
+    n_layers = len(w_packed)
+    ptrs = (ctypes.c_void_p * n_layers)(*[w.data_ptr() for w in w_packed])
+    dims_c = (ctypes.c_int32 * (n_layers + 1))(*[int(d) for d in dims])
+    _check(lib().lowbit_q2_mlp_forward(ctypes.cast(ptrs, ctypes.c_void_p), ctypes.cast(dims_c, ctypes.c_void_p),
+                                       n_layers, _ptr(x), x.shape[0], _ptr(logits), _ptr(argmax),
+                                       _stream(stream)), "lowbit_q2_mlp_forward")
+
+
+# -- glue -------------------------------------------------------------------------
+
+def lowbit_rmsnorm_bf16(a, b, out, eps=1e-6, stream=None):
+    M, D = a.shape
+    _check(lib().lowbit_rmsnorm_bf16(_ptr(a), _ptr(b), M, D, float(eps), _ptr(out), _stream(stream)),
+           "lowbit_rmsnorm_bf16")

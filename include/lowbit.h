@@ -1,0 +1,190 @@
+/*
+ * lowbit.h -- packed low-bit matrix-vector and small-batch matrix products
+ * for NVIDIA B200 (sm_100a).  C ABI of liblowbit.so.
+ *
+ * Three weight formats are supported.  Their definitions come from three web
+ * pages (named by title and section):
+ *
+ *   Q1_0_g128  "Bonsai-27B-gguf technical white paper digest", section
+ *              "technical architecture highlights": every weight is one sign
+ *              bit (-1 or +1) and every 128 weights share one FP16 scale
+ *              (1.125 bits per weight).
+ *   Q2         "Show HN: Z80-uLM, a conversational AI that fits in 40KB":
+ *              2-bit weights {-2,-1,0,+1}, four per byte (the "unpack 2-bit
+ *              weight" listing), a 16-bit two's-complement accumulator (the
+ *              MULADD listing), an arithmetic shift right by 2 after every
+ *              layer (the shift listing), ReLU between hidden layers (the
+ *              architecture list).
+ *   INT4_G64   "acorn-llm 0.11.4", section "int4 quantisation quality: group
+ *              quantisation": symmetric int4 with one scale per group of 64
+ *              values along the input dimension; here the scale is FP16.
+ *
+ * Conventions shared by every entry point
+ *   - N = output rows, K = reduction length, M = batch rows of x.
+ *   - Matrices are row-major.  x is [M][K] bfloat16, y is [M][N] float32.
+ *   - fp16 and bf16 values are passed as uint16_t bit patterns.
+ *   - Every pointer is a DEVICE pointer unless marked HOST.  All device
+ *     pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *     Calls are asynchronous and ordered on `stream`; none synchronises.
+ *   - Arguments are checked on the host before anything is enqueued.  On a
+ *     non-OK status nothing has been enqueued.  LOWBIT_ERR_CUDA reports a
+ *     failed launch (cudaGetLastError).  Faults inside a kernel are
+ *     asynchronous and surface at the caller's next synchronisation.
+ *   - The caller owns every buffer.  The library allocates no device memory
+ *     and keeps no global state; entry points are safe to call from several
+ *     host threads on different streams.  Kernels whose work needs scratch
+ *     memory take a caller-provided workspace, sized by the matching
+ *     *_workspace_bytes() query.
+ *
+ * Packed layouts (one row of a matrix is packed along K):
+ *   Q1_0_g128  bits   [N][K/8]:   weight k is bit (k%8) of byte k/8; bit 1
+ *                                 means +1, bit 0 means -1.
+ *              scales [N][K/128]: fp16; scale g covers k in [128g, 128g+128).
+ *   Q2         bytes  [out][in/4]: the code of input i is bits 2*(i%4)..+1
+ *                                 of byte i/4 (lowest field first); code c
+ *                                 stands for the weight c-2.
+ *   INT4_G64   bytes  [N][K/2]:   weight k is the low nibble (k even) or the
+ *                                 high nibble (k odd) of byte k/2, a 4-bit
+ *                                 two's-complement value in [-8, 7].
+ *              scales [N][K/64]:  fp16; scale g covers k in [64g, 64g+64).
+ */
+#ifndef LOWBIT_H
+#define LOWBIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LOWBIT_OK = 0,
+    LOWBIT_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, size < 0, ... */
+    LOWBIT_ERR_MISALIGNED = 2,        /* a device pointer is not 16-byte aligned */
+    LOWBIT_ERR_UNSUPPORTED_SHAPE = 3, /* K or a dimension breaks a format rule */
+    LOWBIT_ERR_CUDA = 4               /* a CUDA launch failed */
+} lowbit_status;
+
+typedef enum {
+    LOWBIT_FMT_Q1_G128 = 1,
+    LOWBIT_FMT_Q2 = 2,
+    LOWBIT_FMT_INT4_G64 = 3
+} lowbit_format;
+
+/* Static string for a status code (never NULL). */
+const char *lowbit_status_string(lowbit_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int lowbit_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Packing (all three formats).
+ *
+ * lowbit_pack: codes int8 [rows][cols] -> packed uint8 [rows][cols/per_byte]
+ * with per_byte = 8 (Q1_0_g128; codes 0 or 1), 4 (Q2; codes 0..3) or 2
+ * (INT4_G64; codes -8..7).  Codes outside the format's range are masked to
+ * the field width (the packer does not read the data on the host to check).
+ * lowbit_unpack is the exact inverse, for every packed byte value.
+ * cols must be a multiple of per_byte, else LOWBIT_ERR_UNSUPPORTED_SHAPE.
+ * rows == 0 is a no-op that returns LOWBIT_OK.
+ * ------------------------------------------------------------------------- */
+lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, int64_t cols,
+                          uint8_t *packed, void *stream);
+lowbit_status lowbit_unpack(lowbit_format fmt, const uint8_t *packed, int64_t rows, int64_t cols,
+                            int8_t *codes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Q1_0_g128 product (Bonsai white-paper digest, "technical architecture
+ * highlights"):
+ *     y[m][n] = sum_g d[n][g] * sum_{k in group g} s(b[n][k]) * x[m][k]
+ * with s(1) = +1, s(0) = -1, groups of 128 consecutive k, fp32 accumulate.
+ *
+ *   w_bits   [N][K/8]   packed sign bits
+ *   w_scales [N][K/128] fp16 scales
+ *   x        [M][K]     bf16
+ *   y        [M][N]     fp32 (written, not accumulated into)
+ * Shapes: 1 <= M <= 16, N >= 1, K >= 128, K % 128 == 0, N*K < 2^40.
+ * workspace: device scratch of at least lowbit_q1g128_workspace_bytes(M, K)
+ * bytes (may be NULL when that size is 0); its contents are overwritten.
+ * Calls that share one workspace must be ordered on one stream.
+ * ------------------------------------------------------------------------- */
+size_t lowbit_q1g128_workspace_bytes(int M, int K);
+lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales,
+                                 const uint16_t *x, float *y, int M, int N, int K,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/* Split form of the same product for an activation that feeds several
+ * weight matrices (for example the projections that read one normalised
+ * hidden state).  lowbit_q1g128_prepare_act converts x once into the operand
+ * form the product kernels read (act, lowbit_q1g128_act_bytes(M, K) bytes);
+ * lowbit_q1g128_gemv_act then computes y from that buffer.  The result is
+ * bit-identical to lowbit_q1g128_gemv on the same x.  Same shape rules. */
+size_t lowbit_q1g128_act_bytes(int M, int K);
+lowbit_status lowbit_q1g128_prepare_act(const uint16_t *x, int M, int K, void *act,
+                                        size_t act_bytes, void *stream);
+lowbit_status lowbit_q1g128_gemv_act(const uint8_t *w_bits, const uint16_t *w_scales,
+                                     const void *act, float *y, int M, int N, int K,
+                                     void *stream);
+
+/* ---------------------------------------------------------------------------
+ * INT4_G64 product (acorn-llm 0.11.4, "int4 quantisation quality: group
+ * quantisation"):
+ *     y[m][n] = sum_g d[n][g] * sum_{k in group g} q[n][k] * x[m][k]
+ * with q in [-8, 7], groups of 64 consecutive k, fp32 accumulate.
+ *
+ *   w_q      [N][K/2]  packed nibbles
+ *   w_scales [N][K/64] fp16 scales
+ *   x        [M][K]    bf16
+ *   y        [M][N]    fp32
+ * Shapes: M >= 1, N >= 1, K >= 64, K % 64 == 0, M*K, N*K < 2^40.
+ * The kernel is chosen by M: a weight-streaming GEMV for small M and a
+ * tensor-core (tcgen05) GEMM for M >= 128.
+ * workspace: at least lowbit_int4g64_workspace_bytes(M, N, K) bytes (NULL
+ * allowed when that is 0).
+ * ------------------------------------------------------------------------- */
+size_t lowbit_int4g64_workspace_bytes(int M, int N, int K);
+lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales,
+                                  const uint16_t *x, float *y, int M, int N, int K,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Z80-style 2-bit integer MLP ("Show HN: Z80-uLM"), fused over all layers:
+ * for each input vector, a_0 = x; for each layer l with weights w = code-2,
+ *     acc   = sum_i w[o][i] * a_l[i]   reduced mod 2^16 (16-bit wrapping)
+ *     z     = acc >> 2                 arithmetic shift (floor division by 4)
+ *     a_l+1 = max(z, 0) on hidden layers; logits = z on the last layer;
+ * argmax = smallest index of the largest logit.
+ *
+ *   w_packed  HOST array of n_layers device pointers; layer l is
+ *             [dims[l+1]][dims[l]/4] packed Q2 codes
+ *   dims      HOST array of n_layers+1 widths
+ *   x         [batch][dims[0]] int16
+ *   logits    [batch][dims[n_layers]] int16
+ *   argmax    [batch] int32, or NULL
+ * Shapes: 1 <= n_layers <= 8; 4 <= dims[l] <= 1024 and dims[l] % 4 == 0 for
+ * l < n_layers; 1 <= dims[n_layers] <= 1024; the packed weights of all layers
+ * together at most 96 KiB; batch >= 0.
+ * Bit-exact: the result equals the integer definition above for any input.
+ * ------------------------------------------------------------------------- */
+lowbit_status lowbit_q2_mlp_forward(const uint8_t *const *w_packed, const int32_t *dims,
+                                    int n_layers, const int16_t *x, int batch,
+                                    int16_t *logits, int32_t *argmax, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Glue between the projections of a layer stack: RMS normalisation with unit
+ * gain, rounded to bf16.
+ *     v[m][d] = a[m][d] (+ b[m][d] when b is not NULL)
+ *     out[m][d] = bf16_rne( v[m][d] / sqrt(mean_d v[m][d]^2 + eps) )
+ * computed in fp32.  a, b [M][D] fp32; out [M][D] bf16.  M >= 1, 1 <= D,
+ * D % 8 == 0, eps >= 0.
+ * ------------------------------------------------------------------------- */
+lowbit_status lowbit_rmsnorm_bf16(const float *a, const float *b, int M, int D, float eps,
+                                  uint16_t *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOWBIT_H */

@@ -1,0 +1,106 @@
+"""The C-ABI library loads, exports every symbol include/lowbit.h declares,
+and rejects bad arguments on the host before any CUDA call.  CPU only: no
+call here reaches a kernel launch (every case fails validation or is an
+empty no-op)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+from decode_packed_bit_b200 import build as lb_build
+
+
+@pytest.fixture(scope="module")
+def L():
+    lb_build.build()
+    from decode_packed_bit_b200 import lowbit
+    return lowbit.lib()
+
+
+def _header_symbols():
+    with open(os.path.join(ROOT, "include", "lowbit.h")) as f:
+        txt = f.read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(lowbit_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    from decode_packed_bit_b200 import lowbit
+    declared = _header_symbols()
+    assert len(declared) >= 12
+    bound = {name for name, _, _ in lowbit.SYMBOLS}
+    for name in declared:
+        assert hasattr(L, name), f"{name} missing from liblowbit.so"
+        assert name in bound, f"{name} has no Python binding"
+
+
+def test_status_strings(L):
+    for s in range(5):
+        assert L.lowbit_status_string(s)
+    assert L.lowbit_status_string(99) == b"unknown status"
+    assert L.lowbit_version() >= 100
+
+
+FAKE = ctypes.c_void_p(0x10000)      # aligned, never dereferenced: validation fails first
+MIS = ctypes.c_void_p(0x10008)
+
+
+def test_pack_validation(L):
+    assert L.lowbit_pack(7, FAKE, 4, 8, FAKE, None) == 1               # bad format
+    assert L.lowbit_pack(1, FAKE, 4, 12, FAKE, None) == 3              # cols % 8
+    assert L.lowbit_pack(2, FAKE, 4, 6, FAKE, None) == 3               # cols % 4
+    assert L.lowbit_pack(3, FAKE, 4, 3, FAKE, None) == 3               # cols % 2
+    assert L.lowbit_pack(1, None, 4, 8, FAKE, None) == 1               # null
+    assert L.lowbit_pack(1, MIS, 4, 8, FAKE, None) == 2                # misaligned
+    assert L.lowbit_pack(1, None, 0, 8, None, None) == 0               # empty: no-op
+    assert L.lowbit_unpack(1, FAKE, -1, 8, FAKE, None) == 1
+    assert L.lowbit_unpack(3, FAKE, 4, 8, MIS, None) == 2
+
+
+def test_q1_validation(L):
+    g = L.lowbit_q1g128_gemv
+    assert g(FAKE, FAKE, FAKE, FAKE, 0, 16, 128, None, 0, None) == 1   # M < 1
+    assert g(FAKE, FAKE, FAKE, FAKE, 17, 16, 128, None, 0, None) == 1  # M > 16
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 16, 192, None, 0, None) == 3   # K % 128
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 0, 128, None, 0, None) == 1    # N < 1
+    assert g(None, FAKE, FAKE, FAKE, 1, 16, 128, None, 0, None) == 1   # null
+    assert g(FAKE, FAKE, MIS, FAKE, 1, 16, 128, None, 0, None) == 2    # misaligned x
+    need = L.lowbit_q1g128_workspace_bytes(1, 4096)
+    if need:
+        assert g(FAKE, FAKE, FAKE, FAKE, 1, 16, 4096, FAKE, need - 1, None) == 1
+    assert L.lowbit_q1g128_act_bytes(1, 4096) > 0
+    assert L.lowbit_q1g128_prepare_act(FAKE, 1, 100, FAKE, 1 << 20, None) == 3
+    assert L.lowbit_q1g128_prepare_act(FAKE, 1, 128, FAKE, 0, None) == 1
+    assert L.lowbit_q1g128_gemv_act(FAKE, FAKE, None, FAKE, 1, 16, 128, None) == 1
+
+
+def test_int4_validation(L):
+    g = L.lowbit_int4g64_gemm
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 16, 96, None, 0, None) == 3    # K % 64
+    assert g(FAKE, FAKE, FAKE, FAKE, 0, 16, 64, None, 0, None) == 1
+    assert g(FAKE, None, FAKE, FAKE, 1, 16, 64, None, 0, None) == 1
+    assert g(FAKE, FAKE, FAKE, MIS, 1, 16, 64, None, 0, None) == 2
+
+
+def test_q2_and_glue_validation(L):
+    layers = (ctypes.c_void_p * 3)(0x10000, 0x10000, 0x10000)
+    dims = (ctypes.c_int32 * 4)(256, 192, 128, 40)
+    lp = ctypes.cast(layers, ctypes.c_void_p)
+    dp = ctypes.cast(dims, ctypes.c_void_p)
+    f = L.lowbit_q2_mlp_forward
+    assert f(lp, dp, 3, FAKE, 0, FAKE, None, None) == 0                 # empty batch
+    assert f(lp, dp, 0, FAKE, 4, FAKE, None, None) == 1                 # no layers
+    assert f(lp, dp, 3, FAKE, 4, None, None, None) == 1                 # null logits
+    bad = (ctypes.c_int32 * 4)(250, 192, 128, 40)
+    assert f(lp, ctypes.cast(bad, ctypes.c_void_p), 3, FAKE, 4, FAKE, None, None) == 3
+    big = (ctypes.c_int32 * 4)(1024, 1024, 1024, 40)                    # 512 KiB of weights
+    assert f(lp, ctypes.cast(big, ctypes.c_void_p), 3, FAKE, 4, FAKE, None, None) == 3
+    mis = (ctypes.c_void_p * 3)(0x10000, 0x10004, 0x10000)
+    assert f(ctypes.cast(mis, ctypes.c_void_p), dp, 3, FAKE, 4, FAKE, None, None) == 2
+    n = L.lowbit_rmsnorm_bf16
+    assert n(FAKE, None, 1, 12, 1e-6, FAKE, None) == 3
+    assert n(FAKE, None, 1, 16, -1.0, FAKE, None) == 1
+    assert n(FAKE, MIS, 1, 16, 1e-6, FAKE, None) == 2

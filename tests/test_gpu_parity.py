@@ -1,0 +1,269 @@
+"""GPU parity: every product of the library against the CPU oracle, through
+the C ABI, on seeded inputs.  Integer work (packing, the 2-bit MLP) must be
+bit-exact; float formats must meet relative L2 <= 1e-5 and per element
+|diff| <= 2e-3 * sum|w x| against the FP64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity_util import check_float, dev, host, sample_pairs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lb(cuda_device):
+    from decode_packed_bit_b200 import build
+    build.build()
+    from decode_packed_bit_b200 import lowbit
+    return lowbit
+
+
+def _sync():
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# packing: bit-exact, all formats
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt,per", [("q1", 8), ("q2", 4), ("int4", 2)])
+@pytest.mark.parametrize("rows,cols", [(1, 16), (37, 1024), (300, 136 * 8), (5, 4096)])
+def test_pack_unpack_bitexact(lb, fmt, per, rows, cols):
+    seed = 100 + rows
+    if fmt == "q1":
+        codes = synth.q1_codes(seed, rows, cols)
+    elif fmt == "q2":
+        codes = synth.rng(seed, 0).integers(0, 4, size=(rows, cols), dtype=np.int8)
+    else:
+        codes = synth.int4_codes(seed, rows, cols)
+    ref = oracle.pack(fmt, codes)
+    packed = torch.zeros((rows, cols // per), dtype=torch.uint8, device="cuda")
+    lb.lowbit_pack(fmt, dev(codes), packed)
+    back = torch.zeros((rows, cols), dtype=torch.int8, device="cuda")
+    lb.lowbit_unpack(fmt, packed, back)
+    _sync()
+    assert np.array_equal(host(packed), ref)
+    assert np.array_equal(host(back), codes)
+
+
+@pytest.mark.parametrize("fmt,per", [("q1", 8), ("q2", 4), ("int4", 2)])
+def test_unpack_every_byte_value(lb, fmt, per):
+    allb = np.tile(np.arange(256, dtype=np.uint8), 16).reshape(16, 256)   # 16-byte aligned rows
+    cols = 256 * per
+    ref = oracle.unpack(fmt, allb, cols)
+    out = torch.zeros((16, cols), dtype=torch.int8, device="cuda")
+    lb.lowbit_unpack(fmt, dev(allb), out)
+    repacked = torch.zeros((16, 256), dtype=torch.uint8, device="cuda")
+    lb.lowbit_pack(fmt, out, repacked)
+    _sync()
+    assert np.array_equal(host(out), ref)
+    assert np.array_equal(host(repacked), allb)
+
+
+# ---------------------------------------------------------------------------
+# Q1_0_g128
+# ---------------------------------------------------------------------------
+
+def _q1_problem(seed, M, N, K):
+    codes = synth.q1_codes(seed, N, K)
+    bits = oracle.pack("q1", codes)
+    scales = synth.q1_scales(seed, N, K)
+    x = synth.bf16_normal(seed, (M, K))
+    return bits, scales, x
+
+
+def _run_q1(lb, bits, scales, x, N, use_act=False):
+    M, K = x.shape
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    bits_d, scales_d, x_d = dev(bits), dev(scales), dev(x)
+    if use_act:
+        act = torch.zeros(lb.lowbit_q1g128_act_bytes(M, K), dtype=torch.uint8, device="cuda")
+        lb.lowbit_q1g128_prepare_act(x_d, act)
+        lb.lowbit_q1g128_gemv_act(bits_d, scales_d, act, y, M)
+    else:
+        nws = lb.lowbit_q1g128_workspace_bytes(M, K)
+        ws = torch.zeros(max(nws, 16), dtype=torch.uint8, device="cuda") if nws else None
+        lb.lowbit_q1g128_gemv(bits_d, scales_d, x_d, y, workspace=ws)
+    _sync()
+    return host(y)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 16])
+@pytest.mark.parametrize("N,K", [(1, 128), (333, 384), (1000, 1024), (77, 2176)])
+def test_q1_small_full_compare(lb, M, N, K):
+    bits, scales, x = _q1_problem(1000 + M * 7 + N, M, N, K)
+    y = _run_q1(lb, bits, scales, x, N)
+    y64, ab = oracle.q1_gemv(bits, scales, x, want_abs=True)
+    check_float(y, y64, ab, f"q1 M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_q1_prepared_activation_matches_direct(lb, M):
+    N, K = 515, 1280
+    bits, scales, x = _q1_problem(2000 + M, M, N, K)
+    y1 = _run_q1(lb, bits, scales, x, N)
+    y2 = _run_q1(lb, bits, scales, x, N, use_act=True)
+    assert np.array_equal(y1, y2)
+
+
+def test_q1_special_inputs(lb):
+    N, K = 64, 512
+    bits, scales, _ = _q1_problem(3000, 1, N, K)
+    zero = np.zeros((1, K), np.uint16)
+    assert np.array_equal(_run_q1(lb, bits, scales, zero, N), np.zeros((1, N), np.float32))
+    for k in (0, 5, 127, 128, 511):
+        onehot = np.zeros((1, K), np.uint16)
+        onehot[0, k] = 0x3F80
+        y = _run_q1(lb, bits, scales, onehot, N)[0]
+        ref = np.array([oracle.q1_weight(bits, scales, K, n, k) for n in range(N)])
+        assert np.array_equal(y.astype(np.float64), ref)
+    # extreme magnitudes: large and tiny activations in the same group
+    x = synth.bf16_normal(3001, (1, K)).copy()
+    x[0, ::3] = synth.to_bf16_bits(np.full(len(x[0, ::3]), 3.0e4))
+    x[0, 1::7] = synth.to_bf16_bits(np.full(len(x[0, 1::7]), 1.0e-20))
+    y = _run_q1(lb, bits, scales, x, N)
+    y64, ab = oracle.q1_gemv(bits, scales, x, want_abs=True)
+    check_float(y, y64, ab, "q1 extreme magnitudes")
+
+
+def test_q1_4096_square_full(lb):
+    """The 4096x4096 M=1 GEMV, every output compared."""
+    seed = synth.SEED_BASE + synth.W_Q1_4096
+    bits, scales, x = _q1_problem(seed, 1, 4096, 4096)
+    y = _run_q1(lb, bits, scales, x, 4096)
+    y64, ab = oracle.q1_gemv(bits, scales, x, want_abs=True)
+    check_float(y, y64, ab, "q1 4096^2")
+
+
+@pytest.mark.parametrize("shape", synth.Q1_SWEEP_SHAPES)
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_q1_layer_shapes_sampled(lb, shape, M):
+    N, K = shape
+    seed = synth.SEED_BASE + synth.W_Q1_SWEEP
+    bits = synth.q1_packed_random(seed, N, K, tag=N + K)
+    scales = synth.q1_scales(seed, N, K, tag=N + K)
+    x = synth.bf16_normal(seed, (M, K), tag=M)
+    y = _run_q1(lb, bits, scales, x, N)
+    ms, ns = sample_pairs(M, N, 160, seed + M)
+    y64, ab = oracle.q1_gemv_at(bits, scales, x, ms, ns)
+    check_float(y[ms, ns], y64, ab, f"q1 {shape} M={M}")
+
+
+# ---------------------------------------------------------------------------
+# INT4_G64
+# ---------------------------------------------------------------------------
+
+def _run_int4(lb, q, scales, x, N):
+    M, K = x.shape
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    nws = lb.lowbit_int4g64_workspace_bytes(M, N, K)
+    ws = torch.zeros(nws, dtype=torch.uint8, device="cuda") if nws else None
+    lb.lowbit_int4g64_gemm(dev(q), dev(scales), dev(x), y, workspace=ws)
+    _sync()
+    return host(y)
+
+
+@pytest.mark.parametrize("M", [1, 2, 7, 32, 33, 128, 130])
+@pytest.mark.parametrize("N,K", [(1, 64), (333, 448), (1000, 1024)])
+def test_int4_small_full_compare(lb, M, N, K):
+    seed = 4000 + M * 13 + N
+    codes = synth.int4_codes(seed, N, K)
+    q = oracle.pack("int4", codes)
+    scales = synth.int4_scales(seed, N, K)
+    x = synth.bf16_normal(seed, (M, K))
+    y = _run_int4(lb, q, scales, x, N)
+    y64, ab = oracle.int4_gemv(q, scales, x, want_abs=True)
+    check_float(y, y64, ab, f"int4 M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("M", [1, 32, 256])
+def test_int4_11008x4096_sampled(lb, M):
+    seed = synth.SEED_BASE + synth.W_INT4
+    N, K = synth.INT4_N, synth.INT4_K
+    codes = synth.int4_codes(seed, N, K)
+    q = oracle.pack("int4", codes)
+    scales = synth.int4_scales(seed, N, K)
+    x = synth.bf16_normal(seed, (M, K), tag=M)
+    y = _run_int4(lb, q, scales, x, N)
+    ms, ns = sample_pairs(M, N, 200, seed + M)
+    y64, ab = oracle.int4_gemv_at(q, scales, x, ms, ns)
+    check_float(y[ms, ns], y64, ab, f"int4 11008x4096 M={M}")
+
+
+# ---------------------------------------------------------------------------
+# Z80-style 2-bit MLP: bit-exact
+# ---------------------------------------------------------------------------
+
+def _run_q2(lb, packed, dims, x, with_argmax=True):
+    batch = x.shape[0]
+    logits = torch.full((batch, dims[-1]), -1, dtype=torch.int16, device="cuda")
+    am = torch.full((batch,), -1, dtype=torch.int32, device="cuda") if with_argmax else None
+    w_d = [dev(p) for p in packed]
+    lb.lowbit_q2_mlp_forward(w_d, dims, dev(x), logits, am)
+    _sync()
+    return host(logits), (host(am) if with_argmax else None)
+
+
+def test_q2_mlp_1024_vectors_bitexact(lb):
+    seed = synth.SEED_BASE + synth.W_Q2_MLP
+    dims = synth.Q2_DIMS
+    packed = [oracle.pack("q2", c) for c in synth.q2_codes(seed, dims)]
+    x = synth.q2_inputs(seed, 1024)
+    logits, am = _run_q2(lb, packed, dims, x)
+    ref_l, ref_a = oracle.q2_mlp_forward(packed, dims, x)
+    assert np.array_equal(logits, ref_l)
+    assert np.array_equal(am, ref_a)
+
+
+@pytest.mark.parametrize("batch", [1, 7, 9, 100])
+def test_q2_mlp_ragged_batches_and_overflow(lb, batch):
+    dims = (256, 192, 128, 40)
+    packed = [oracle.pack("q2", c) for c in synth.q2_codes(77, dims)]
+    g = synth.rng(77, 5)
+    x = g.integers(-32768, 32768, size=(batch, 256)).astype(np.int16)   # forces 16-bit wrap
+    logits, am = _run_q2(lb, packed, dims, x)
+    ref_l, ref_a = oracle.q2_mlp_forward(packed, dims, x)
+    assert np.array_equal(logits, ref_l)
+    assert np.array_equal(am, ref_a)
+    lg2, none = _run_q2(lb, packed, dims, x, with_argmax=False)
+    assert np.array_equal(lg2, ref_l) and none is None
+
+
+@pytest.mark.parametrize("dims", [(4, 4), (8, 12, 4), (64, 1024, 32, 1), (1024, 16, 1024)])
+def test_q2_mlp_other_topologies(lb, dims):
+    codes = [synth.rng(88, l).integers(0, 4, size=(dims[l + 1], dims[l]), dtype=np.int8)
+             for l in range(len(dims) - 1)]
+    packed = [oracle.pack("q2", c) for c in codes]
+    x = synth.rng(88, 9).integers(-3000, 3000, size=(19, dims[0])).astype(np.int16)
+    logits, am = _run_q2(lb, packed, dims, x)
+    ref_l, ref_a = oracle.q2_mlp_forward(packed, dims, x)
+    assert np.array_equal(logits, ref_l)
+    assert np.array_equal(am, ref_a)
+
+
+# ---------------------------------------------------------------------------
+# RMS-norm glue
+# ---------------------------------------------------------------------------
+
+def _bf16_ulp(v):
+    e = np.floor(np.log2(np.maximum(np.abs(v), 1e-38)))
+    return 2.0 ** (e - 7)
+
+
+@pytest.mark.parametrize("M,D,two", [(1, 5120, False), (8, 17408, True), (3, 64, True)])
+def test_rmsnorm_bf16_within_half_ulp(lb, M, D, two):
+    g = synth.rng(99, D)
+    a = (g.standard_normal((M, D)) * 0.7).astype(np.float32)
+    b = g.standard_normal((M, D)).astype(np.float32) if two else None
+    out = torch.zeros((M, D), dtype=torch.int16, device="cuda")
+    lb.lowbit_rmsnorm_bf16(dev(a), dev(b) if two else None, out, eps=1e-6)
+    _sync()
+    got = synth.bf16_bits_to_f32(host(out).view(np.uint16)).astype(np.float64)
+    r64 = oracle.rmsnorm(a, b, eps=1e-6)
+    # round-to-nearest to bf16 of an fp32 result: at most half a bf16 ulp
+    # plus the fp32 error of the normalisation itself
+    tol = 0.5 * _bf16_ulp(r64) + 1e-6 * np.abs(r64) + 1e-30
+    assert (np.abs(got - r64) <= tol).all()
