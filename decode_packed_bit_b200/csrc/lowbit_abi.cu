@@ -13,6 +13,14 @@ lowbit_status q2_mlp_launch(const uint8_t *const *, const int32_t *, int, const 
                             int32_t *, cudaStream_t);
 int q2_weight_bytes_padded(const int32_t *, int);
 lowbit_status rmsnorm_launch(const float *, const float *, int, int, float, uint16_t *, cudaStream_t);
+size_t q1m1_act_bytes(int K);
+size_t q1m1_ws_bytes(int R, int N, int K);
+bool q1m1_shape_supported(int R, int N, int K);
+int q1m1_max_group();
+size_t q1m1_xcopy_off(int K);
+lowbit_status q1m1_prepare_launch(const uint16_t *, int, void *, unsigned *, cudaStream_t);
+lowbit_status q1m1_gemv_launch(const uint8_t *const *, const uint16_t *const *, const void *, float *const *,
+                               int, int, int, void *, cudaStream_t);
 
 constexpr int64_t kMaxElems = int64_t(1) << 40;
 constexpr int kQ1MaxM = 16;
@@ -88,17 +96,37 @@ static lowbit_status q1_shape_ok(int M, int N, int K)
     return LOWBIT_OK;
 }
 
-size_t lowbit_q1g128_workspace_bytes(int M, int K)
-{
-    (void)M;
-    (void)K;
-    return 0;
-}
+static size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
 
 size_t lowbit_q1g128_act_bytes(int M, int K)
 {
-    if (M < 1 || K < 1) return 0;
-    return (size_t)M * (size_t)K * 2u;
+    if (M < 1 || M > kQ1MaxM || K < 128 || K % 128 != 0) return 0;
+    if (M == 1) return q1m1_act_bytes(K);
+    return al256((size_t)M * (size_t)K * 2u);
+}
+
+// M = 1 runs on the tensor-core kernel when the shape allows (K/128 even and
+// the activation slices fit in shared memory); otherwise, and for M >= 2, the
+// SIMT kernel reads a bf16 copy of x (kept in the prepared buffer at M = 1).
+static bool q1_tc_path(int R, int M, int N, int K) { return M == 1 && q1m1_shape_supported(R, N, K); }
+
+static const uint16_t *q1_simt_x(const void *act, int M, int K)
+{
+    const uint8_t *a = static_cast<const uint8_t *>(act);
+    return reinterpret_cast<const uint16_t *>(M == 1 ? a + q1m1_xcopy_off(K) : a);
+}
+
+size_t lowbit_q1g128_act_workspace_bytes(int R, int M, int N, int K)
+{
+    if (R < 1 || M < 1 || M > kQ1MaxM || N < 1 || K < 128 || K % 128 != 0) return 0;
+    return q1_tc_path(R, M, N, K) ? q1m1_ws_bytes(R, N, K) : 0;
+}
+
+size_t lowbit_q1g128_workspace_bytes(int M, int N, int K)
+{
+    if (M < 1 || M > kQ1MaxM || N < 1 || K < 128 || K % 128 != 0) return 0;
+    if (!q1_tc_path(1, M, N, K)) return 0;
+    return al256(q1m1_act_bytes(K)) + q1m1_ws_bytes(1, N, K);
 }
 
 lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales, const uint16_t *x,
@@ -109,10 +137,19 @@ lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales
     if (s != LOWBIT_OK) return s;
     LB_CHECK(w_bits && w_scales && x && y, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(aligned16(w_bits) && aligned16(w_scales) && aligned16(x) && aligned16(y), LOWBIT_ERR_MISALIGNED);
-    const size_t need = lowbit_q1g128_workspace_bytes(M, K);
+    const size_t need = lowbit_q1g128_workspace_bytes(M, N, K);
     LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
-    return q1_gemv_simt_launch(w_bits, w_scales, x, y, M, N, K, as_stream(stream));
+    cudaStream_t st = as_stream(stream);
+    if (q1_tc_path(1, M, N, K)) {
+        uint8_t *act = static_cast<uint8_t *>(workspace);
+        uint8_t *ws = act + al256(q1m1_act_bytes(K));
+        unsigned *cnt = q1m1_ws_bytes(1, N, K) ? reinterpret_cast<unsigned *>(ws) : nullptr;
+        s = q1m1_prepare_launch(x, K, act, cnt, st);
+        if (s != LOWBIT_OK) return s;
+        return q1m1_gemv_launch(&w_bits, &w_scales, act, &y, 1, N, K, ws, st);
+    }
+    return q1_gemv_simt_launch(w_bits, w_scales, x, y, M, N, K, st);
 }
 
 lowbit_status lowbit_q1g128_prepare_act(const uint16_t *x, int M, int K, void *act, size_t act_bytes,
@@ -124,21 +161,44 @@ lowbit_status lowbit_q1g128_prepare_act(const uint16_t *x, int M, int K, void *a
     LB_CHECK(aligned16(x) && aligned16(act), LOWBIT_ERR_MISALIGNED);
     const size_t need = lowbit_q1g128_act_bytes(M, K);
     LB_CHECK(act_bytes >= need, LOWBIT_ERR_INVALID_ARG);
-    return cudaMemcpyAsync(act, x, need, cudaMemcpyDeviceToDevice, as_stream(stream)) == cudaSuccess
+    cudaStream_t st = as_stream(stream);
+    if (M == 1) return q1m1_prepare_launch(x, K, act, nullptr, st);
+    return cudaMemcpyAsync(act, x, (size_t)M * K * 2u, cudaMemcpyDeviceToDevice, st) == cudaSuccess
                ? LOWBIT_OK
                : LOWBIT_ERR_CUDA;
 }
 
-lowbit_status lowbit_q1g128_gemv_act(const uint8_t *w_bits, const uint16_t *w_scales, const void *act,
-                                     float *y, int M, int N, int K, void *stream)
+lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits, const uint16_t *const *w_scales,
+                                           const void *act, float *const *y, int R, int M, int N, int K,
+                                           void *workspace, size_t workspace_bytes, void *stream)
 {
+    LB_CHECK(R >= 1 && R <= q1m1_max_group() && w_bits && w_scales && y, LOWBIT_ERR_INVALID_ARG);
     lowbit_status s = q1_shape_ok(M, N, K);
     if (s != LOWBIT_OK) return s;
-    LB_CHECK(w_bits && w_scales && act && y, LOWBIT_ERR_INVALID_ARG);
-    LB_CHECK(aligned16(w_bits) && aligned16(w_scales) && aligned16(act) && aligned16(y),
-             LOWBIT_ERR_MISALIGNED);
-    return q1_gemv_simt_launch(w_bits, w_scales, static_cast<const uint16_t *>(act), y, M, N, K,
-                               as_stream(stream));
+    LB_CHECK(act != nullptr, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(act), LOWBIT_ERR_MISALIGNED);
+    for (int r = 0; r < R; ++r) {
+        LB_CHECK(w_bits[r] && w_scales[r] && y[r], LOWBIT_ERR_INVALID_ARG);
+        LB_CHECK(aligned16(w_bits[r]) && aligned16(w_scales[r]) && aligned16(y[r]), LOWBIT_ERR_MISALIGNED);
+    }
+    const size_t need = lowbit_q1g128_act_workspace_bytes(R, M, N, K);
+    LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
+    cudaStream_t st = as_stream(stream);
+    if (q1_tc_path(R, M, N, K)) return q1m1_gemv_launch(w_bits, w_scales, act, y, R, N, K, workspace, st);
+    for (int r = 0; r < R; ++r) {
+        s = q1_gemv_simt_launch(w_bits[r], w_scales[r], q1_simt_x(act, M, K), y[r], M, N, K, st);
+        if (s != LOWBIT_OK) return s;
+    }
+    return LOWBIT_OK;
+}
+
+lowbit_status lowbit_q1g128_gemv_act(const uint8_t *w_bits, const uint16_t *w_scales, const void *act,
+                                     float *y, int M, int N, int K, void *workspace, size_t workspace_bytes,
+                                     void *stream)
+{
+    return lowbit_q1g128_gemv_act_group(&w_bits, &w_scales, act, &y, 1, M, N, K, workspace, workspace_bytes,
+                                        stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -33,11 +33,13 @@ SYMBOLS = [
     ("lowbit_version", I32, []),
     ("lowbit_pack", I32, [I32, P, I64, I64, P, P]),
     ("lowbit_unpack", I32, [I32, P, I64, I64, P, P]),
-    ("lowbit_q1g128_workspace_bytes", SZ, [I32, I32]),
+    ("lowbit_q1g128_workspace_bytes", SZ, [I32, I32, I32]),
     ("lowbit_q1g128_gemv", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
     ("lowbit_q1g128_act_bytes", SZ, [I32, I32]),
+    ("lowbit_q1g128_act_workspace_bytes", SZ, [I32, I32, I32, I32]),
     ("lowbit_q1g128_prepare_act", I32, [P, I32, I32, P, SZ, P]),
-    ("lowbit_q1g128_gemv_act", I32, [P, P, P, P, I32, I32, I32, P]),
+    ("lowbit_q1g128_gemv_act", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
+    ("lowbit_q1g128_gemv_act_group", I32, [P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
     ("lowbit_int4g64_workspace_bytes", SZ, [I32, I32, I32]),
     ("lowbit_int4g64_gemm", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
     ("lowbit_q2_mlp_forward", I32, [P, P, I32, P, I32, P, P, P]),
@@ -110,12 +112,20 @@ def lowbit_unpack(fmt, packed, codes, stream=None):
 
 # -- Q1_0_g128 --------------------------------------------------------------------
 
-def lowbit_q1g128_workspace_bytes(M: int, K: int) -> int:
-    return int(lib().lowbit_q1g128_workspace_bytes(M, K))
+def lowbit_q1g128_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().lowbit_q1g128_workspace_bytes(M, N, K))
 
 
 def lowbit_q1g128_act_bytes(M: int, K: int) -> int:
     return int(lib().lowbit_q1g128_act_bytes(M, K))
+
+
+def lowbit_q1g128_act_workspace_bytes(R: int, M: int, N: int, K: int) -> int:
+    return int(lib().lowbit_q1g128_act_workspace_bytes(R, M, N, K))
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
 
 
 def lowbit_q1g128_gemv(w_bits, w_scales, x, y, workspace=None, stream=None):
@@ -132,11 +142,31 @@ def lowbit_q1g128_prepare_act(x, act, stream=None):
                                            _stream(stream)), "lowbit_q1g128_prepare_act")
 
 
-def lowbit_q1g128_gemv_act(w_bits, w_scales, act, y, M: int, stream=None):
+def lowbit_q1g128_gemv_act(w_bits, w_scales, act, y, M: int, workspace=None, stream=None):
+    """workspace: zero-filled before its first use (calls leave it zeroed)."""
     N = w_bits.shape[0]
     K = w_bits.shape[1] * 8
     _check(lib().lowbit_q1g128_gemv_act(_ptr(w_bits), _ptr(w_scales), _ptr(act), _ptr(y), M, N, K,
-                                        _stream(stream)), "lowbit_q1g128_gemv_act")
+                                        _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "lowbit_q1g128_gemv_act")
+
+
+def _ptr_array(ts):
+    arr = (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def lowbit_q1g128_gemv_act_group(w_bits, w_scales, act, ys, M: int, workspace=None, stream=None):
+    """w_bits, w_scales, ys: equal-length lists of tensors (one per matrix)."""
+    R = len(w_bits)
+    N = w_bits[0].shape[0]
+    K = w_bits[0].shape[1] * 8
+    pb, kb = _ptr_array(w_bits)
+    ps, ks = _ptr_array(w_scales)
+    py, ky = _ptr_array(ys)
+    _check(lib().lowbit_q1g128_gemv_act_group(pb, ps, _ptr(act), py, R, M, N, K, _ptr(workspace),
+                                              _nbytes(workspace), _stream(stream)),
+           "lowbit_q1g128_gemv_act_group")
 
 
 # -- INT4_G64 ---------------------------------------------------------------------

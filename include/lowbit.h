@@ -106,11 +106,18 @@ lowbit_status lowbit_unpack(lowbit_format fmt, const uint8_t *packed, int64_t ro
  *   x        [M][K]     bf16
  *   y        [M][N]     fp32 (written, not accumulated into)
  * Shapes: 1 <= M <= 16, N >= 1, K >= 128, K % 128 == 0, N*K < 2^40.
- * workspace: device scratch of at least lowbit_q1g128_workspace_bytes(M, K)
- * bytes (may be NULL when that size is 0); its contents are overwritten.
+ * Activations must be finite; values below 2^-96 in magnitude count as 0 at
+ * M = 1 (the tensor-core path works in per-group 24-bit fixed point).
+ * workspace: device scratch of at least lowbit_q1g128_workspace_bytes(M, N,
+ * K) bytes (may be NULL when that size is 0); it holds the prepared
+ * activation and the split-K partial sums, and needs no initialisation.
  * Calls that share one workspace must be ordered on one stream.
+ * The weights are read before the kernel waits for the previous kernel on
+ * the stream (programmatic dependent launch): a kernel that writes w_bits or
+ * w_scales must not trigger its dependents early.  The library's packers
+ * never do.
  * ------------------------------------------------------------------------- */
-size_t lowbit_q1g128_workspace_bytes(int M, int K);
+size_t lowbit_q1g128_workspace_bytes(int M, int N, int K);
 lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales,
                                  const uint16_t *x, float *y, int M, int N, int K,
                                  void *workspace, size_t workspace_bytes, void *stream);
@@ -118,15 +125,31 @@ lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales
 /* Split form of the same product for an activation that feeds several
  * weight matrices (for example the projections that read one normalised
  * hidden state).  lowbit_q1g128_prepare_act converts x once into the operand
- * form the product kernels read (act, lowbit_q1g128_act_bytes(M, K) bytes);
- * lowbit_q1g128_gemv_act then computes y from that buffer.  The result is
- * bit-identical to lowbit_q1g128_gemv on the same x.  Same shape rules. */
+ * form the product kernels read (act, lowbit_q1g128_act_bytes(M, K) bytes).
+ * lowbit_q1g128_gemv_act_group then computes y_r = W_r x for R matrices of
+ * the same shape [N][K] in one launch:
+ *   w_bits, w_scales, y: HOST arrays of R device pointers (1 <= R <= 256);
+ *   each y_r equals a separate lowbit_q1g128_gemv call up to fp32 summation
+ *   order (the K-split depends on the amount of work in the launch).
+ * lowbit_q1g128_gemv_act is the R = 1 case.  Same shape rules as above.
+ * Workspace: lowbit_q1g128_act_workspace_bytes(R, M, N, K) bytes (NULL
+ * allowed when 0); it holds split-K partial sums and arrival counters.  It
+ * must be zero-filled before its first use, and every completed call leaves
+ * it valid for the next call of any shape.  Calls that share an act buffer
+ * or a workspace must be ordered on one stream.
+ * At M = 1 the tensor-core kernel takes every shape with K/128 even; other
+ * shapes run a CUDA-core kernel (same results within the float bar). */
 size_t lowbit_q1g128_act_bytes(int M, int K);
+size_t lowbit_q1g128_act_workspace_bytes(int R, int M, int N, int K);
 lowbit_status lowbit_q1g128_prepare_act(const uint16_t *x, int M, int K, void *act,
                                         size_t act_bytes, void *stream);
 lowbit_status lowbit_q1g128_gemv_act(const uint8_t *w_bits, const uint16_t *w_scales,
                                      const void *act, float *y, int M, int N, int K,
-                                     void *stream);
+                                     void *workspace, size_t workspace_bytes, void *stream);
+lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits,
+                                           const uint16_t *const *w_scales, const void *act,
+                                           float *const *y, int R, int M, int N, int K,
+                                           void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------
  * INT4_G64 product (acorn-llm 0.11.4, "int4 quantisation quality: group

@@ -68,13 +68,19 @@ def test_q1_validation(L):
     assert g(FAKE, FAKE, FAKE, FAKE, 1, 0, 128, None, 0, None) == 1    # N < 1
     assert g(None, FAKE, FAKE, FAKE, 1, 16, 128, None, 0, None) == 1   # null
     assert g(FAKE, FAKE, MIS, FAKE, 1, 16, 128, None, 0, None) == 2    # misaligned x
-    need = L.lowbit_q1g128_workspace_bytes(1, 4096)
-    if need:
-        assert g(FAKE, FAKE, FAKE, FAKE, 1, 16, 4096, FAKE, need - 1, None) == 1
+    need = L.lowbit_q1g128_workspace_bytes(1, 4096, 4096)
+    assert need > 0
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 4096, 4096, FAKE, need - 1, None) == 1
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 4096, 4096, None, need, None) == 1
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 4096, 4096, MIS, need, None) == 2
+    assert L.lowbit_q1g128_workspace_bytes(1, 16, 100) == 0            # invalid shape -> 0
     assert L.lowbit_q1g128_act_bytes(1, 4096) > 0
     assert L.lowbit_q1g128_prepare_act(FAKE, 1, 100, FAKE, 1 << 20, None) == 3
     assert L.lowbit_q1g128_prepare_act(FAKE, 1, 128, FAKE, 0, None) == 1
-    assert L.lowbit_q1g128_gemv_act(FAKE, FAKE, None, FAKE, 1, 16, 128, None) == 1
+    wsa = L.lowbit_q1g128_act_workspace_bytes(1, 1, 4096, 4096)
+    assert wsa > 0
+    assert L.lowbit_q1g128_gemv_act(FAKE, FAKE, None, FAKE, 1, 16, 128, None, 0, None) == 1
+    assert L.lowbit_q1g128_gemv_act(FAKE, FAKE, FAKE, FAKE, 1, 4096, 4096, FAKE, wsa - 1, None) == 1
 
 
 def test_int4_validation(L):

@@ -81,11 +81,14 @@ def _run_q1(lb, bits, scales, x, N, use_act=False):
     bits_d, scales_d, x_d = dev(bits), dev(scales), dev(x)
     if use_act:
         act = torch.zeros(lb.lowbit_q1g128_act_bytes(M, K), dtype=torch.uint8, device="cuda")
+        nws = lb.lowbit_q1g128_act_workspace_bytes(1, M, N, K)
+        ws = torch.zeros(nws, dtype=torch.uint8, device="cuda") if nws else None
         lb.lowbit_q1g128_prepare_act(x_d, act)
-        lb.lowbit_q1g128_gemv_act(bits_d, scales_d, act, y, M)
+        lb.lowbit_q1g128_gemv_act(bits_d, scales_d, act, y, M, workspace=ws)
     else:
-        nws = lb.lowbit_q1g128_workspace_bytes(M, K)
-        ws = torch.zeros(max(nws, 16), dtype=torch.uint8, device="cuda") if nws else None
+        nws = lb.lowbit_q1g128_workspace_bytes(M, N, K)
+        # garbage-filled on purpose: the one-shot call needs no initialised workspace
+        ws = torch.full((nws,), 0xA5, dtype=torch.uint8, device="cuda") if nws else None
         lb.lowbit_q1g128_gemv(bits_d, scales_d, x_d, y, workspace=ws)
     _sync()
     return host(y)
@@ -107,6 +110,54 @@ def test_q1_prepared_activation_matches_direct(lb, M):
     y1 = _run_q1(lb, bits, scales, x, N)
     y2 = _run_q1(lb, bits, scales, x, N, use_act=True)
     assert np.array_equal(y1, y2)
+
+
+def test_q1_act_workspace_reused_across_calls(lb):
+    """One prepared activation and one split-K workspace shared by several
+    products in a row: the arrival counters must come back to zero."""
+    K = 4096
+    x = synth.bf16_normal(2500, (1, K))
+    act = torch.zeros(lb.lowbit_q1g128_act_bytes(1, K), dtype=torch.uint8, device="cuda")
+    lb.lowbit_q1g128_prepare_act(dev(x), act)
+    ws = torch.zeros(max(lb.lowbit_q1g128_act_workspace_bytes(1, 1, N, K) for N in (4096, 1000, 5120)),
+                     dtype=torch.uint8, device="cuda")
+    for rep, N in enumerate((4096, 1000, 5120, 4096)):
+        bits = synth.q1_packed_random(2500 + rep, N, K)
+        scales = synth.q1_scales(2500 + rep, N, K)
+        y = torch.full((1, N), float("nan"), dtype=torch.float32, device="cuda")
+        lb.lowbit_q1g128_gemv_act(dev(bits), dev(scales), act, y, 1, workspace=ws)
+        _sync()
+        ms, ns = sample_pairs(1, N, 200, rep)
+        y64, ab = oracle.q1_gemv_at(bits, scales, x, ms, ns)
+        check_float(host(y)[ms, ns], y64, ab, f"q1 reuse {rep}")
+    cnt_region = host(ws)
+    assert not np.isnan(host(y)).any()
+    del cnt_region
+
+
+@pytest.mark.parametrize("R,N,K", [(3, 515, 1280), (20, 4096, 4096), (2, 17408, 512), (5, 33, 17408)])
+def test_q1_group_matches_oracle_and_single_calls(lb, R, N, K):
+    """R matrices that read one prepared activation, in one launch."""
+    x = synth.bf16_normal(2600 + R, (1, K))
+    x_d = dev(x)
+    act = torch.zeros(lb.lowbit_q1g128_act_bytes(1, K), dtype=torch.uint8, device="cuda")
+    lb.lowbit_q1g128_prepare_act(x_d, act)
+    mats = [(synth.q1_packed_random(2600 + r, N, K), synth.q1_scales(2600 + r, N, K)) for r in range(R)]
+    bits_d = [dev(b) for b, _ in mats]
+    scales_d = [dev(s) for _, s in mats]
+    ys = [torch.full((1, N), float("nan"), dtype=torch.float32, device="cuda") for _ in range(R)]
+    ws = torch.zeros(max(16, lb.lowbit_q1g128_act_workspace_bytes(R, 1, N, K)), dtype=torch.uint8,
+                     device="cuda")
+    lb.lowbit_q1g128_gemv_act_group(bits_d, scales_d, act, ys, 1, workspace=ws)
+    _sync()
+    for r in (0, R // 2, R - 1):
+        b, s = mats[r]
+        ms, ns = sample_pairs(1, N, 120, r)
+        y64, ab = oracle.q1_gemv_at(b, s, x, ms, ns)
+        check_float(host(ys[r])[ms, ns], y64, ab, f"q1 group R={R} r={r}")
+        # a lone call may split K differently (another fp32 summation order)
+        single = _run_q1(lb, b, s, x, N)
+        np.testing.assert_allclose(single, host(ys[r]), rtol=0, atol=1e-5 * float(np.abs(host(ys[r])).max()))
 
 
 def test_q1_special_inputs(lb):
