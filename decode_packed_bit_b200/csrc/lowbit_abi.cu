@@ -14,13 +14,12 @@ lowbit_status q2_mlp_launch(const uint8_t *const *, const int32_t *, int, const 
 int q2_weight_bytes_padded(const int32_t *, int);
 lowbit_status rmsnorm_launch(const float *, const float *, int, int, float, uint16_t *, cudaStream_t);
 size_t q1m1_act_bytes(int K);
-size_t q1m1_ws_bytes(int R, int N, int K);
 bool q1m1_shape_supported(int R, int N, int K);
 int q1m1_max_group();
 size_t q1m1_xcopy_off(int K);
-lowbit_status q1m1_prepare_launch(const uint16_t *, int, void *, unsigned *, cudaStream_t);
+lowbit_status q1m1_prepare_launch(const uint16_t *, int, void *, cudaStream_t);
 lowbit_status q1m1_gemv_launch(const uint8_t *const *, const uint16_t *const *, const void *, float *const *,
-                               int, int, int, void *, cudaStream_t);
+                               int, int, int, cudaStream_t);
 
 constexpr int64_t kMaxElems = int64_t(1) << 40;
 constexpr int kQ1MaxM = 16;
@@ -118,15 +117,15 @@ static const uint16_t *q1_simt_x(const void *act, int M, int K)
 
 size_t lowbit_q1g128_act_workspace_bytes(int R, int M, int N, int K)
 {
-    if (R < 1 || M < 1 || M > kQ1MaxM || N < 1 || K < 128 || K % 128 != 0) return 0;
-    return q1_tc_path(R, M, N, K) ? q1m1_ws_bytes(R, N, K) : 0;
+    (void)R; (void)M; (void)N; (void)K;
+    return 0;  // the split-K partial sums stay in thread-block-cluster shared memory
 }
 
 size_t lowbit_q1g128_workspace_bytes(int M, int N, int K)
 {
     if (M < 1 || M > kQ1MaxM || N < 1 || K < 128 || K % 128 != 0) return 0;
     if (!q1_tc_path(1, M, N, K)) return 0;
-    return al256(q1m1_act_bytes(K)) + q1m1_ws_bytes(1, N, K);
+    return al256(q1m1_act_bytes(K));  // the prepared activation
 }
 
 lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales, const uint16_t *x,
@@ -143,11 +142,9 @@ lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales
     cudaStream_t st = as_stream(stream);
     if (q1_tc_path(1, M, N, K)) {
         uint8_t *act = static_cast<uint8_t *>(workspace);
-        uint8_t *ws = act + al256(q1m1_act_bytes(K));
-        unsigned *cnt = q1m1_ws_bytes(1, N, K) ? reinterpret_cast<unsigned *>(ws) : nullptr;
-        s = q1m1_prepare_launch(x, K, act, cnt, st);
+        s = q1m1_prepare_launch(x, K, act, st);
         if (s != LOWBIT_OK) return s;
-        return q1m1_gemv_launch(&w_bits, &w_scales, act, &y, 1, N, K, ws, st);
+        return q1m1_gemv_launch(&w_bits, &w_scales, act, &y, 1, N, K, st);
     }
     return q1_gemv_simt_launch(w_bits, w_scales, x, y, M, N, K, st);
 }
@@ -162,7 +159,7 @@ lowbit_status lowbit_q1g128_prepare_act(const uint16_t *x, int M, int K, void *a
     const size_t need = lowbit_q1g128_act_bytes(M, K);
     LB_CHECK(act_bytes >= need, LOWBIT_ERR_INVALID_ARG);
     cudaStream_t st = as_stream(stream);
-    if (M == 1) return q1m1_prepare_launch(x, K, act, nullptr, st);
+    if (M == 1) return q1m1_prepare_launch(x, K, act, st);
     return cudaMemcpyAsync(act, x, (size_t)M * K * 2u, cudaMemcpyDeviceToDevice, st) == cudaSuccess
                ? LOWBIT_OK
                : LOWBIT_ERR_CUDA;
@@ -185,7 +182,7 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits, const u
     LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
     cudaStream_t st = as_stream(stream);
-    if (q1_tc_path(R, M, N, K)) return q1m1_gemv_launch(w_bits, w_scales, act, y, R, N, K, workspace, st);
+    if (q1_tc_path(R, M, N, K)) return q1m1_gemv_launch(w_bits, w_scales, act, y, R, N, K, st);
     for (int r = 0; r < R; ++r) {
         s = q1_gemv_simt_launch(w_bits[r], w_scales[r], q1_simt_x(act, M, K), y[r], M, N, K, st);
         if (s != LOWBIT_OK) return s;

@@ -110,8 +110,8 @@ lowbit_status lowbit_unpack(lowbit_format fmt, const uint8_t *packed, int64_t ro
  * M = 1 (the tensor-core path works in per-group 24-bit fixed point).
  * workspace: device scratch of at least lowbit_q1g128_workspace_bytes(M, N,
  * K) bytes (may be NULL when that size is 0); it holds the prepared
- * activation and the split-K partial sums, and needs no initialisation.
- * Calls that share one workspace must be ordered on one stream.
+ * activation and needs no initialisation.  Calls that share one workspace
+ * must be ordered on one stream.
  * The weights are read before the kernel waits for the previous kernel on
  * the stream (programmatic dependent launch): a kernel that writes w_bits or
  * w_scales must not trigger its dependents early.  The library's packers
@@ -133,10 +133,9 @@ lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales
  *   order (the K-split depends on the amount of work in the launch).
  * lowbit_q1g128_gemv_act is the R = 1 case.  Same shape rules as above.
  * Workspace: lowbit_q1g128_act_workspace_bytes(R, M, N, K) bytes (NULL
- * allowed when 0); it holds split-K partial sums and arrival counters.  It
- * must be zero-filled before its first use, and every completed call leaves
- * it valid for the next call of any shape.  Calls that share an act buffer
- * or a workspace must be ordered on one stream.
+ * allowed when 0; the current kernels need none: split-K partial sums are
+ * reduced in thread-block-cluster shared memory).  Calls that share an act
+ * buffer must be ordered on one stream.
  * At M = 1 the tensor-core kernel takes every shape with K/128 even; other
  * shapes run a CUDA-core kernel (same results within the float bar). */
 size_t lowbit_q1g128_act_bytes(int M, int K);

@@ -77,10 +77,16 @@ def test_q1_validation(L):
     assert L.lowbit_q1g128_act_bytes(1, 4096) > 0
     assert L.lowbit_q1g128_prepare_act(FAKE, 1, 100, FAKE, 1 << 20, None) == 3
     assert L.lowbit_q1g128_prepare_act(FAKE, 1, 128, FAKE, 0, None) == 1
-    wsa = L.lowbit_q1g128_act_workspace_bytes(1, 1, 4096, 4096)
-    assert wsa > 0
+    assert L.lowbit_q1g128_act_workspace_bytes(1, 1, 4096, 4096) == 0
     assert L.lowbit_q1g128_gemv_act(FAKE, FAKE, None, FAKE, 1, 16, 128, None, 0, None) == 1
-    assert L.lowbit_q1g128_gemv_act(FAKE, FAKE, FAKE, FAKE, 1, 4096, 4096, FAKE, wsa - 1, None) == 1
+    assert L.lowbit_q1g128_gemv_act(FAKE, FAKE, MIS, FAKE, 1, 16, 128, None, 0, None) == 2
+    ptrs = (ctypes.c_void_p * 2)(0x10000, 0x10000)
+    pp = ctypes.cast(ptrs, ctypes.c_void_p)
+    grp = L.lowbit_q1g128_gemv_act_group
+    assert grp(pp, pp, FAKE, pp, 0, 1, 16, 256, None, 0, None) == 1      # R < 1
+    assert grp(pp, pp, FAKE, pp, 257, 1, 16, 256, None, 0, None) == 1    # R > 256
+    bad = (ctypes.c_void_p * 2)(0x10000, 0)
+    assert grp(pp, ctypes.cast(bad, ctypes.c_void_p), FAKE, pp, 2, 1, 16, 256, None, 0, None) == 1
 
 
 def test_int4_validation(L):
