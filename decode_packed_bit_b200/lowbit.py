@@ -40,6 +40,7 @@ SYMBOLS = [
     ("lowbit_q1g128_prepare_act", I32, [P, I32, I32, P, SZ, P]),
     ("lowbit_q1g128_gemv_act", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
     ("lowbit_q1g128_gemv_act_group", I32, [P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
+    ("lowbit_q1g128_gemv_noalloc", I32, [P, P, P, P, I32, I32, I32, P]),
     ("lowbit_int4g64_workspace_bytes", SZ, [I32, I32, I32]),
     ("lowbit_int4g64_gemm", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
     ("lowbit_q2_mlp_forward", I32, [P, P, I32, P, I32, P, P, P]),
@@ -167,6 +168,15 @@ def lowbit_q1g128_gemv_act_group(w_bits, w_scales, act, ys, M: int, workspace=No
     _check(lib().lowbit_q1g128_gemv_act_group(pb, ps, _ptr(act), py, R, M, N, K, _ptr(workspace),
                                               _nbytes(workspace), _stream(stream)),
            "lowbit_q1g128_gemv_act_group")
+
+
+def lowbit_q1g128_gemv_noalloc(w_bits, w_scales, x, y, stream=None):
+    """The product without a workspace (scratch in the library's own fixed
+    device array; K <= 32768 at M = 1; calls must not overlap on the GPU)."""
+    M, K = x.shape
+    N = w_bits.shape[0]
+    _check(lib().lowbit_q1g128_gemv_noalloc(_ptr(w_bits), _ptr(w_scales), _ptr(x), _ptr(y), M, N, K,
+                                            _stream(stream)), "lowbit_q1g128_gemv_noalloc")
 
 
 # -- INT4_G64 ---------------------------------------------------------------------

@@ -150,6 +150,27 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits,
                                            float *const *y, int R, int M, int N, int K,
                                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* Allocation-free form of lowbit_q1g128_gemv.  The pages have no
+ * counterpart: it exists for callers that cannot allocate device memory --
+ * a plugin whose host framework owns every device allocation, a real-time or
+ * embedded deployment that reserves all device memory up front, or code that
+ * must not call cudaMalloc at the point where the product runs.
+ *   Same arguments and result as lowbit_q1g128_gemv, without a workspace.
+ *   The scratch the M = 1 path needs lives in a fixed 512 KiB array in the
+ *   library's own device memory, present on every device that loads the
+ *   library until the process exits; it limits K to 32768 at M = 1 (larger K
+ *   returns LOWBIT_ERR_UNSUPPORTED_SHAPE).  The call allocates nothing.
+ *   The first call on a device looks up that array's device address (with
+ *   the device current) and caches it; make that first call before any
+ *   stream capture.
+ *   All calls share the one array, so calls that overlap on the GPU (for
+ *   example on two streams without ordering between them) race; order them
+ *   on one stream.  Each call overwrites the part it reads, so the contents a
+ *   previous call left behind do no harm. */
+lowbit_status lowbit_q1g128_gemv_noalloc(const uint8_t *w_bits, const uint16_t *w_scales,
+                                         const uint16_t *x, float *y, int M, int N, int K,
+                                         void *stream);
+
 /* ---------------------------------------------------------------------------
  * INT4_G64 product (acorn-llm 0.11.4, "int4 quantisation quality: group
  * quantisation"):
