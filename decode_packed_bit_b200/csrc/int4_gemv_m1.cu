@@ -1,0 +1,431 @@
+// int4_gemv_m1.cu -- INT4_G64 matrix-vector product at M = 1 on the integer
+// tensor cores (mma.sync m16n8k32, u8 x s8 -> s32).
+//
+// What is computed ("acorn-llm 0.11.4", section "int4 quantisation quality:
+// group quantisation": one scale per group of values along the input
+// dimension, here 64 values and an FP16 scale):
+//     y[n] = sum_g d[n][g] * sum_{k in g} q[n][k] * x[k],  q in [-8, 7].
+//
+// As the acorn page observes, a grouped kernel must keep the scale switch and
+// the group bookkeeping out of the inner loop.  Here the inner loop is pure
+// integer tensor-core work and the scale is applied once per (row, group):
+//
+//   A operand: one lop3 per 32-bit word and nibble half, (w & 0x0F0F0F0F) ^
+//     0x08080808 gives the four low nibbles as u8 q+8, (w & 0xF0F0F0F0) ^
+//     0x80808080 the four high nibbles as u8 16*(q+8).
+//   B operand: per 64-group, x as 24-bit fixed point X_k = round(x_k *
+//     2^(23-E_g)); even k (low nibbles) take 16*X_k, odd k take X_k, so every
+//     product is 16*(q+8)*X; split into four signed 8-bit limbs, one per B
+//     column.  Columns 0-3 carry the first group of a 128-k pair, 4-7 the
+//     second.
+//   Epilogue: sum_k q X = D/16 - 8*sum_k X, with D = sum_l D_l 2^(8l); so
+//     y += d * (2^(E-27) * D - 2^(E-20) * sum_k X_k).
+//
+// Work split and weight streaming follow the Q1 kernels: a step is 32 rows
+// (two mma tiles) x one 128-k pair of groups, staged per warp by cp.async; a
+// thread-block cluster splits K and reduces through distributed shared memory
+// when the rows alone cannot fill the GPU.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace lowbit {
+
+constexpr int kI4PairK = 128;               // k per step (two 64-groups)
+constexpr int kI4FragBytesPerPair = 1024;   // 4 mma x 32 lanes x 8 bytes
+constexpr int kI4InfoBytesPerPair = 16;     // two groups x (G, S)
+constexpr int kI4Warps = 8;
+constexpr int kI4SplitWarps = 4;
+constexpr int kI4StepRows = 32;
+constexpr int kI4Stages = 6;                // a warp's whole K-slice in flight
+constexpr int kI4RowStride = 64;            // 16-byte reads of a row quad are conflict free
+constexpr int kI4StageW = kI4StepRows * kI4RowStride;
+constexpr int kI4StageBytes = kI4StageW + kI4StepRows * 4;
+constexpr int kI4WarpRing = kI4Stages * kI4StageBytes;
+constexpr int kI4MinExp = -96;
+constexpr int kI4MaxSmem = 226 * 1024;
+constexpr int kI4MaxCluster = 8;
+constexpr int kI4SplitRows = kI4SplitWarps * kI4StepRows;
+
+static inline size_t i4_align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------------------
+// activation prepare
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float i4_warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ int i4_warp_sum(int v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// One CTA of 128 threads per 128-k pair.  Thread kk turns x[k] into limbs;
+// then thread t writes B fragment words of lane t%32 for mma t/32.
+__global__ void __launch_bounds__(128) k_i4_prep_m1(const uint16_t *__restrict__ x, int K, uint8_t *__restrict__ act,
+                                                   size_t info_off)
+{
+    __shared__ float smax[4];
+    __shared__ int ssum[4];
+    __shared__ int8_t limb[4][128];
+    pdl_launch_dependents();
+    const int pr = blockIdx.x;
+    const int kk = threadIdx.x;
+    const int k = pr * kI4PairK + kk;
+    const int warp = kk >> 5, lane = kk & 31;
+    const int h = kk >> 6;  // group within the pair
+    pdl_wait_primary();
+
+    const float xv = k < K ? bf16_bits_to_float(x[k]) : 0.f;
+    const float wm = i4_warp_max(fabsf(xv));
+    if (lane == 0) smax[warp] = wm;
+    __syncthreads();
+    const float m = fmaxf(smax[2 * h], smax[2 * h + 1]);
+    const int e8 = (int)((__float_as_uint(m) >> 23) & 0xFFu);
+    const int E = max(e8 == 0 ? kI4MinExp : e8 - 126, kI4MinExp);
+    const int X = __float2int_rn(ldexpf(xv, 23 - E));       // |X| < 2^23
+    const int B = (k & 1) ? X : X * 16;                      // low nibbles carry q+8, high 16(q+8)
+    int l0 = (int)(int8_t)(B & 0xFF);
+    int r = (B - l0) >> 8;
+    int l1 = (int)(int8_t)(r & 0xFF);
+    r = (r - l1) >> 8;
+    int l2 = (int)(int8_t)(r & 0xFF);
+    const int l3 = (r - l2) >> 8;                            // |B| < 2^27: l3 in [-8, 8]
+    limb[0][kk] = (int8_t)l0;
+    limb[1][kk] = (int8_t)l1;
+    limb[2][kk] = (int8_t)l2;
+    limb[3][kk] = (int8_t)l3;
+    const int ws = i4_warp_sum(X);
+    if (lane == 0) ssum[warp] = ws;
+    __syncthreads();
+    if ((kk & 63) == 0) {
+        const int T = ssum[2 * h] + ssum[2 * h + 1];
+        const int grp = 2 * pr + h;
+        float2 info = make_float2(0.f, 0.f);
+        if (grp * 64 < K) info = make_float2(ldexpf(1.0f, E - 27), ldexpf((float)T, E - 20));
+        reinterpret_cast<float2 *>(act + info_off)[grp] = info;
+    }
+
+    // B fragments: mma u (4 per pair), lane (n, t).  Register j, byte c holds
+    // the k-slot of A register a(2j) byte c of thread t: nibble j of packed
+    // byte 4*wi + c of group t/2, wi = 4(t&1) + u, i.e. k = 64(t/2) + 32(t&1)
+    // + 8u + 2c + j.  Column n = 4*group + limb; the other group's lanes get 0.
+    for (int e = kk; e < 4 * 32; e += 128) {
+        const int u = e >> 5, ln = e & 31;
+        const int n = ln >> 2, t = ln & 3;
+        uint32_t w[2] = {0u, 0u};
+        if ((n >> 2) == (t >> 1)) {
+            const int8_t *lb = limb[n & 3];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    w[j] |= (uint32_t)(uint8_t)lb[64 * (t >> 1) + 32 * (t & 1) + 8 * u + 2 * c + j] << (8 * c);
+        }
+        reinterpret_cast<uint2 *>(act + (size_t)pr * kI4FragBytesPerPair)[e] = make_uint2(w[0], w[1]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// product
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void i4_mma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                       uint32_t b1, bool zero)
+{
+    if (zero)
+        asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                     "{%10,%10,%10,%10};"
+                     : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+    else
+        asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                     "{%0,%1,%2,%3};"
+                     : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void i4_cp16(unsigned dst, const void *src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void i4_cp4(unsigned dst, const void *src, bool valid)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
+__device__ __forceinline__ void i4_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void i4_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+struct I4Params {
+    const uint8_t *q;
+    const uint16_t *scales;
+    float *y;
+    const uint8_t *act;
+    size_t info_off;
+    int N, K, npairs;
+    int L;          // pairs per K-slice
+    int act_smem;
+};
+
+// Issue one step: rows blk*32..+32, pair pidx (must be < pend).  Lane L
+// copies 16-byte column L%4 of rows L/4 + {0,8,16,24}, and the two scales
+// (4 bytes) of row L.
+__device__ __forceinline__ void i4_issue(unsigned stage, const I4Params &p, int blk, int pidx, int pend, int lane)
+{
+    const int rowbytes = p.K >> 1, G = p.K >> 6;
+    const int col = lane & 3;
+    const int row0 = blk * kI4StepRows + (lane >> 2);
+    const bool pok = pidx < pend;
+    const uint8_t *src = p.q + (size_t)row0 * rowbytes + pidx * 64 + col * 16;
+    const unsigned dst = stage + (lane >> 2) * kI4RowStride + col * 16;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const bool ok = pok && row0 + 8 * u < p.N;
+        i4_cp16(dst + 8 * u * kI4RowStride, ok ? src + (size_t)(8 * u) * rowbytes : p.q, ok);
+    }
+    const int srow = blk * kI4StepRows + lane;
+    const bool sok = pok && srow < p.N;
+    i4_cp4(stage + kI4StageW + lane * 4, sok ? p.scales + (size_t)srow * G + 2 * pidx : p.scales, sok);
+}
+
+// Consume one staged step.  bf: this lane's fragments of the pair; gi: the
+// (G, S) of this lane's group.
+__device__ __forceinline__ void i4_consume(const uint8_t *st, const uint8_t *bf, float2 gi, int lane,
+                                           float (&yacc)[2][2])
+{
+    const int g = lane >> 2, tq = lane & 3, h = tq >> 1;
+    uint4 w[2][2];  // [tile][row g / g+8]: words 4(tq&1)..+3 of group h
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+            w[t][r] = *reinterpret_cast<const uint4 *>(st + (16 * t + g + 8 * r) * kI4RowStride + h * 32 +
+                                                       (tq & 1) * 16);
+    int d[2][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const uint2 b = *reinterpret_cast<const uint2 *>(bf + u * 256);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const uint32_t w0 = u == 0 ? w[t][0].x : u == 1 ? w[t][0].y : u == 2 ? w[t][0].z : w[t][0].w;
+            const uint32_t w1 = u == 0 ? w[t][1].x : u == 1 ? w[t][1].y : u == 2 ? w[t][1].z : w[t][1].w;
+            const uint32_t lo0 = (w0 & 0x0F0F0F0Fu) ^ 0x08080808u, hi0 = (w0 & 0xF0F0F0F0u) ^ 0x80808080u;
+            const uint32_t lo1 = (w1 & 0x0F0F0F0Fu) ^ 0x08080808u, hi1 = (w1 & 0xF0F0F0F0u) ^ 0x80808080u;
+            i4_mma(d[t], lo0, lo1, hi0, hi1, b.x, b.y, u == 0);
+        }
+    }
+    const float coef = gi.x * ((tq & 1) ? 65536.f : 1.f);
+    const float sub = (tq & 1) ? 0.f : gi.y;
+    const float magic = 12582912.f;
+    const float subc = fmaf(coef, magic, sub);
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint16_t sc = *reinterpret_cast<const uint16_t *>(st + kI4StageW + (16 * t + g + 8 * r) * 4 + h * 2);
+            const float hi = __int_as_float(d[t][2 * r + 1] + 0x4B400000) - magic;
+            const float vm = fmaf(256.f, hi, __int_as_float(d[t][2 * r] + 0x4B400000));
+            yacc[t][r] = fmaf(f16_bits_to_float(sc), fmaf(coef, vm, -subc), yacc[t][r]);
+        }
+}
+
+__device__ __forceinline__ void i4_stage_act(uint8_t *smem, const I4Params &p, int p_lo, int n)
+{
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.act + (size_t)p_lo * kI4FragBytesPerPair);
+    uint4 *dst = reinterpret_cast<uint4 *>(smem);
+    for (int i = threadIdx.x; i < n * (kI4FragBytesPerPair / 16); i += blockDim.x) dst[i] = __ldg(src + i);
+    const uint4 *isrc = reinterpret_cast<const uint4 *>(p.act + p.info_off + (size_t)p_lo * kI4InfoBytesPerPair);
+    uint4 *idst = reinterpret_cast<uint4 *>(smem + (size_t)n * kI4FragBytesPerPair);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) idst[i] = __ldg(isrc + i);
+}
+
+template <typename Out>
+__device__ __forceinline__ void i4_finish(float (&yacc)[2][2], int lane, Out out)
+{
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            yacc[t][r] += __shfl_xor_sync(0xffffffffu, yacc[t][r], 1);
+            yacc[t][r] += __shfl_xor_sync(0xffffffffu, yacc[t][r], 2);
+        }
+    const int tq = lane & 3, g = lane >> 2;
+    const int t = tq >> 1, r = tq & 1;
+    const float v = t ? (r ? yacc[1][1] : yacc[1][0]) : (r ? yacc[0][1] : yacc[0][0]);
+    out(16 * t + g + 8 * r, v);
+    yacc[0][0] = yacc[0][1] = yacc[1][0] = yacc[1][1] = 0.f;
+}
+
+__device__ __forceinline__ void i4_cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Read a float of rank `rank`'s shared memory.  volatile keeps the load after
+// the cluster barrier; the callers issue all ranks' loads before using any,
+// so they overlap.
+__device__ __forceinline__ float i4_ld_cluster(const float *local, unsigned rank)
+{
+    const unsigned a = (unsigned)__cvta_generic_to_shared(local);
+    unsigned ra;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra));
+    return v;
+}
+
+// grid: x = K-slice (cluster rank), y = 128-row block.  With one slice the
+// cluster is a single CTA and its partial sums are the result.
+__global__ void __launch_bounds__(kI4SplitWarps * 32) k_i4_m1_split(const I4Params p)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ float part[kI4SplitRows];
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int slice = blockIdx.x, nsl = gridDim.x, rb = blockIdx.y;
+    const int blk = rb * kI4SplitWarps + warp;
+    const int p_lo = slice * p.L, p_hi = min(p.npairs, p_lo + p.L);
+    const int nsteps = blk * kI4StepRows < p.N && p_hi > p_lo ? p_hi - p_lo : 0;
+    uint8_t *ring = smem + p.act_smem + warp * kI4WarpRing;
+    const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
+
+    int ist = 0;
+    auto issue_next = [&]() {
+        if (ist < nsteps) i4_issue(ring_s + (ist % kI4Stages) * kI4StageBytes, p, blk, p_lo + ist, p_hi, lane);
+        ++ist;
+        i4_commit();
+    };
+#pragma unroll
+    for (int t = 0; t < kI4Stages - 1; ++t) issue_next();
+
+    pdl_wait_primary();
+    if (p_hi > p_lo) i4_stage_act(smem, p, p_lo, p_hi - p_lo);
+    __syncthreads();
+
+    const uint8_t *bfrag = smem + lane * 8;
+    const float2 *sinfo = reinterpret_cast<const float2 *>(smem + (size_t)(p_hi - p_lo) * kI4FragBytesPerPair) +
+                          ((lane & 3) >> 1);
+    float yacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    for (int s = 0; s < nsteps; ++s) {
+        issue_next();
+        i4_wait<kI4Stages - 1>();
+        __syncwarp();
+        i4_consume(ring + (s % kI4Stages) * kI4StageBytes, bfrag + s * kI4FragBytesPerPair, sinfo[2 * s], lane,
+                   yacc);
+        __syncwarp();
+    }
+    i4_wait<0>();
+    i4_finish(yacc, lane, [&](int row, float v) { part[warp * kI4StepRows + row] = v; });
+
+    if (nsl == 1) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < kI4SplitRows; i += blockDim.x)
+            if (rb * kI4SplitRows + i < p.N) p.y[rb * kI4SplitRows + i] = part[i];
+        return;
+    }
+    i4_cluster_sync();  // every slice's partial sums are in its CTA's shared memory
+    // rank q adds up rows [q*per, (q+1)*per) over all ranks, in rank order
+    const int per = (kI4SplitRows + nsl - 1) / nsl;
+    for (int i = slice * per + threadIdx.x; i < min(kI4SplitRows, (slice + 1) * per); i += blockDim.x) {
+        float v[kI4MaxCluster];
+#pragma unroll
+        for (int q = 0; q < kI4MaxCluster; ++q) v[q] = q < nsl ? i4_ld_cluster(part + i, (unsigned)q) : 0.f;
+        float sum = 0.f;
+#pragma unroll
+        for (int q = 0; q < kI4MaxCluster; ++q) sum += v[q];
+        if (rb * kI4SplitRows + i < p.N) p.y[rb * kI4SplitRows + i] = sum;
+    }
+    i4_cluster_sync();  // peers keep their shared memory until every rank has read it
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+struct I4Plan {
+    int npairs, L, nslices, blocks;
+    size_t info_off, act_bytes, act_smem, smem;
+    bool ok;
+};
+
+static I4Plan i4_plan(int N, int K, int sms)
+{
+    I4Plan P = {};
+    P.npairs = (K + kI4PairK - 1) / kI4PairK;
+    P.info_off = i4_align256((size_t)P.npairs * kI4FragBytesPerPair);
+    P.act_bytes = i4_align256(P.info_off + (size_t)P.npairs * kI4InfoBytesPerPair);
+    P.blocks = (N + kI4SplitRows - 1) / kI4SplitRows;
+    const size_t per_pair = kI4FragBytesPerPair + kI4InfoBytesPerPair;
+    const size_t ring = (size_t)kI4SplitWarps * kI4WarpRing;
+    // enough CTAs for several per SM, and each CTA's activation slice in smem
+    int S = (int)std::min<long long>(kI4MaxCluster, std::max<long long>(1, (4LL * sms + P.blocks - 1) / P.blocks));
+    S = std::max(S, (P.npairs + kI4Stages - 1) / kI4Stages);  // whole slice in flight when possible
+    S = std::min(std::min(S, kI4MaxCluster), P.npairs);
+    while (true) {
+        P.L = (P.npairs + S - 1) / S;
+        P.nslices = (P.npairs + P.L - 1) / P.L;
+        P.act_smem = ((size_t)P.L * per_pair + 15) & ~size_t(15);
+        P.smem = P.act_smem + ring;
+        if (P.smem <= (size_t)kI4MaxSmem || S >= kI4MaxCluster) break;
+        S = std::min(kI4MaxCluster, S * 2);
+    }
+    P.ok = P.smem <= (size_t)kI4MaxSmem && P.blocks < 65536 && (K / 64) % 2 == 0;
+    return P;
+}
+
+static int i4_num_sms()
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+bool i4m1_supported(int N, int K) { return i4_plan(N, K, i4_num_sms()).ok; }
+size_t i4m1_act_bytes(int K) { return i4_plan(1, K, 148).act_bytes; }
+
+lowbit_status i4m1_launch(const uint8_t *q, const uint16_t *scales, const uint16_t *x, float *y, int N, int K,
+                          void *act, cudaStream_t st)
+{
+    const I4Plan P = i4_plan(N, K, i4_num_sms());
+    cudaError_t e = launch_pdl(k_i4_prep_m1, dim3(P.npairs), dim3(128), 0, st, x, K, static_cast<uint8_t *>(act),
+                               P.info_off);
+    if (e != cudaSuccess) return LOWBIT_ERR_CUDA;
+    I4Params p = {};
+    p.q = q;
+    p.scales = scales;
+    p.y = y;
+    p.act = static_cast<const uint8_t *>(act);
+    p.info_off = P.info_off;
+    p.N = N;
+    p.K = K;
+    p.npairs = P.npairs;
+    p.L = P.L;
+    p.act_smem = (int)P.act_smem;
+    if (cudaFuncSetAttribute(k_i4_m1_split, cudaFuncAttributeMaxDynamicSharedMemorySize, kI4MaxSmem) != cudaSuccess)
+        return LOWBIT_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(P.nslices, P.blocks);
+    cfg.blockDim = dim3(kI4SplitWarps * 32);
+    cfg.dynamicSmemBytes = P.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = P.nslices;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, k_i4_m1_split, p);
+    return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
+}  // namespace lowbit

@@ -17,6 +17,10 @@ size_t q1m1_act_bytes(int K);
 bool q1m1_shape_supported(int R, int N, int K);
 int q1m1_max_group();
 size_t q1m1_xcopy_off(int K);
+bool i4m1_supported(int N, int K);
+size_t i4m1_act_bytes(int K);
+lowbit_status i4m1_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, void *,
+                          cudaStream_t);
 lowbit_status q1m1_prepare_launch(const uint16_t *, int, void *, cudaStream_t);
 lowbit_status q1m1_gemv_launch(const uint8_t *const *, const uint16_t *const *, const void *, float *const *,
                                int, int, int, cudaStream_t);
@@ -204,9 +208,8 @@ lowbit_status lowbit_q1g128_gemv_act(const uint8_t *w_bits, const uint16_t *w_sc
 
 size_t lowbit_int4g64_workspace_bytes(int M, int N, int K)
 {
-    (void)M;
-    (void)N;
-    (void)K;
+    if (M < 1 || N < 1 || K < 64 || K % 64 != 0) return 0;
+    if (M == 1 && i4m1_supported(N, K)) return al256(i4m1_act_bytes(K));  // the prepared activation
     return 0;
 }
 
@@ -221,7 +224,9 @@ lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales, 
     const size_t need = lowbit_int4g64_workspace_bytes(M, N, K);
     LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
-    return int4_gemv_simt_launch(w_q, w_scales, x, y, M, N, K, as_stream(stream));
+    cudaStream_t st = as_stream(stream);
+    if (M == 1 && i4m1_supported(N, K)) return i4m1_launch(w_q, w_scales, x, y, N, K, workspace, st);
+    return int4_gemv_simt_launch(w_q, w_scales, x, y, M, N, K, st);
 }
 
 // ---------------------------------------------------------------------------

@@ -504,15 +504,21 @@ __device__ __forceinline__ void cluster_sync()
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Read a float of rank `rank`'s shared memory.  volatile keeps the load after
+// the cluster barrier; the callers issue all ranks' loads before using any,
+// so they overlap.
 __device__ __forceinline__ float ld_cluster_f32(const float *local, unsigned rank)
 {
     const unsigned a = (unsigned)__cvta_generic_to_shared(local);
     unsigned ra;
     float v;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra));
     return v;
 }
+
+constexpr int kQ1SplitStages = 6;  // a split warp's whole K-slice in flight
+constexpr int kQ1SplitRing = kQ1SplitStages * kQ1StageBytes;
 
 constexpr int kQ1SplitRows = kQ1SplitWarps * kQ1StepRows;  // rows of one CTA
 
@@ -531,19 +537,19 @@ __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid
     const int ch_lo = slice * p.L, ch_hi = min(p.nchunks, ch_lo + p.L);
     const int nsteps = blk * kQ1StepRows < p.N && ch_hi > ch_lo
                            ? (ch_hi - ch_lo + kQ1StepChunks - 1) / kQ1StepChunks : 0;
-    uint8_t *ring = smem + p.act_smem + warp * kQ1WarpRing;
+    uint8_t *ring = smem + p.act_smem + warp * kQ1SplitRing;
     const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
 
     int ist = 0;
     auto issue_next = [&]() {
         if (ist < nsteps)
-            issue_any(ring_s + (ist % kQ1Stages) * kQ1StageBytes, grp, p, r, blk, ch_lo + ist * kQ1StepChunks,
-                      ch_hi, lane);
+            issue_any(ring_s + (ist % kQ1SplitStages) * kQ1StageBytes, grp, p, r, blk,
+                      ch_lo + ist * kQ1StepChunks, ch_hi, lane);
         ++ist;
         cp_async_commit();
     };
 #pragma unroll
-    for (int t = 0; t < kQ1Stages - 1; ++t) issue_next();
+    for (int t = 0; t < kQ1SplitStages - 1; ++t) issue_next();
 
     pdl_wait_primary();
     if (ch_hi > ch_lo) stage_act(smem, p, ch_lo, ch_hi - ch_lo);
@@ -555,26 +561,35 @@ __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid
     float yacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
     for (int s = 0; s < nsteps; ++s) {
         issue_next();
-        cp_async_wait<kQ1Stages - 1>();
+        cp_async_wait<kQ1SplitStages - 1>();
         __syncwarp();
         const int lch = s * kQ1StepChunks;
-        consume_step(ring + (s % kQ1Stages) * kQ1StageBytes, bfrag + lch * kQ1FragBytesPerChunk, sinfo + 2 * lch,
-                     min(kQ1StepChunks, ch_hi - ch_lo - lch), lc, yacc);
+        consume_step(ring + (s % kQ1SplitStages) * kQ1StageBytes, bfrag + lch * kQ1FragBytesPerChunk,
+                     sinfo + 2 * lch, min(kQ1StepChunks, ch_hi - ch_lo - lch), lc, yacc);
         __syncwarp();
     }
     cp_async_wait<0>();
     finish_cell(yacc, lane, [&](int row, float v) { part[warp * kQ1StepRows + row] = v; });
 
-    cluster_sync();  // every slice's partial sums are in its CTA's shared memory
-    if (slice == 0) {
-        for (int i = threadIdx.x; i < kQ1SplitRows; i += blockDim.x) {
-            const int row = rb * kQ1SplitRows + i;
-            float sum = 0.f;
-            for (int q = 0; q < nsl; ++q) sum += ld_cluster_f32(part + i, (unsigned)q);
-            if (row < p.N) grp.y[r][row] = sum;
-        }
+    if (nsl == 1) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < kQ1SplitRows; i += blockDim.x)
+            if (rb * kQ1SplitRows + i < p.N) grp.y[r][rb * kQ1SplitRows + i] = part[i];
+        return;
     }
-    cluster_sync();  // peers keep their shared memory until rank 0 has read it
+    cluster_sync();  // every slice's partial sums are in its CTA's shared memory
+    // rank q adds up rows [q*per, (q+1)*per) over all ranks, in rank order
+    const int per = (kQ1SplitRows + nsl - 1) / nsl;
+    for (int i = slice * per + threadIdx.x; i < min(kQ1SplitRows, (slice + 1) * per); i += blockDim.x) {
+        float v[kQ1MaxCluster];
+#pragma unroll
+        for (int q = 0; q < kQ1MaxCluster; ++q) v[q] = q < nsl ? ld_cluster_f32(part + i, (unsigned)q) : 0.f;
+        float sum = 0.f;
+#pragma unroll
+        for (int q = 0; q < kQ1MaxCluster; ++q) sum += v[q];
+        if (rb * kQ1SplitRows + i < p.N) grp.y[r][rb * kQ1SplitRows + i] = sum;
+    }
+    cluster_sync();  // peers keep their shared memory until every rank has read it
 }
 
 // ---------------------------------------------------------------------------
@@ -624,10 +639,11 @@ static Q1Plan q1_plan(int R, int N, int K, int sms)
     }
     // split kernel: S slices so that the CTAs fill the SMs several times over
     P.stream = false;
-    const size_t ring_split = (size_t)kQ1SplitWarps * kQ1WarpRing;
+    const size_t ring_split = (size_t)kQ1SplitWarps * kQ1SplitRing;
     const long long blocks = (long long)R * ((N + kQ1SplitRows - 1) / kQ1SplitRows);
     int S = (int)std::min<long long>(kQ1MaxCluster, std::max<long long>(1, (4LL * sms + blocks - 1) / blocks));
-    S = std::min(S, P.nchunks);
+    S = std::max(S, (P.nchunks + kQ1StepChunks * kQ1SplitStages - 1) / (kQ1StepChunks * kQ1SplitStages));
+    S = std::min(std::min(S, kQ1MaxCluster), P.nchunks);
     while (true) {
         P.L = (P.nchunks + S - 1) / S;
         P.nslices = (P.nchunks + P.L - 1) / P.L;
