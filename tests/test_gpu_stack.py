@@ -1,0 +1,108 @@
+"""The 64-layer Q1_0_g128 projection stack (hidden 5120, ffn 17408), one
+decode step at M = 1 and M = 8, checked teacher-forced: every recorded
+projection against the FP64 oracle on sampled output rows, given the bf16
+input it actually received; every normalisation against the oracle's RMS
+norm fed the same fp32 input."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity_util import check_float, host
+
+pytestmark = pytest.mark.gpu
+
+H, F, L = synth.STACK_HIDDEN, synth.STACK_FFN, synth.STACK_LAYERS
+
+
+@pytest.fixture(scope="module")
+def stack_weights(cuda_device):
+    from decode_packed_bit_b200 import build
+    build.build()
+    from decode_packed_bit_b200.stack import Q1Layer
+    seed = synth.SEED_BASE + synth.W_Q1_STACK
+    layers = []
+    for li in range(L):
+        w = {}
+        for pi, (name, n, k) in enumerate(synth.STACK_PROJ):
+            w[name] = synth.torch_q1_layer(seed, n, k, li * 16 + pi, cuda_device)
+        layers.append(Q1Layer(w))
+    return layers
+
+
+def _bf16_ulp(v):
+    e = np.floor(np.log2(np.maximum(np.abs(v), 1e-38)))
+    return 2.0 ** (e - 7)
+
+
+def _next_input_key(li, name):
+    nxt = {"q": (li, "k"), "k": (li, "v"), "v": (li, "o"), "o": (li, "gate"), "gate+up": (li, "down"),
+           "down": (li + 1, "q")}
+    return nxt[name]
+
+
+def _run(stack_weights, M, which):
+    from decode_packed_bit_b200.stack import Q1Stack, StackRecord
+    st = Q1Stack(stack_weights, H, F, M, "cuda")
+    x0 = synth.bf16_normal(synth.SEED_BASE + synth.W_Q1_STACK, (M, H), tag=M)
+    st.x.copy_(torch.from_numpy(x0.view(np.int16)).view(torch.bfloat16).cuda())
+    rec = StackRecord(which=which)
+    st.step(record=rec)
+    torch.cuda.synchronize()
+    return st, rec
+
+
+def _check_projections(stack_weights, rec, M, rows_per_proj, seed):
+    g = np.random.default_rng(seed)
+    for (li, name), xin in rec.inputs.items():
+        if (li, name) not in rec.outputs:
+            continue
+        bits, scales = stack_weights[li].w[name]
+        N = bits.shape[0]
+        rows = np.unique(np.concatenate([[0, N - 1], g.integers(0, N, size=rows_per_proj)]))
+        b = host(bits[torch.as_tensor(rows, device=bits.device)])
+        s = host(scales[torch.as_tensor(rows, device=bits.device)].view(torch.int16)).view(np.uint16)
+        x = host(xin.view(torch.int16)).view(np.uint16)
+        ms = np.repeat(np.arange(M), len(rows))
+        ns = np.tile(np.arange(len(rows)), M)
+        y64, ab = oracle.q1_gemv_at(b, s, x, ms, ns)
+        yg = host(rec.outputs[(li, name)])[:, rows].reshape(-1)
+        check_float(yg, y64, ab, f"stack M={M} layer {li} {name}")
+
+
+def _check_glue(rec, M):
+    checked = 0
+    for (li, name), v in rec.norm_in.items():
+        key = _next_input_key(li, name)
+        if key not in rec.inputs:
+            continue
+        if name == "gate+up":
+            a, b = host(v[0]), host(v[1])
+            r64 = oracle.rmsnorm(a, b, eps=1e-6)
+        else:
+            r64 = oracle.rmsnorm(host(v), None, eps=1e-6)
+        got = synth.bf16_bits_to_f32(host(rec.inputs[key].view(torch.int16)).view(np.uint16)).astype(np.float64)
+        tol = 0.5 * _bf16_ulp(r64) + 1e-6 * np.abs(r64) + 1e-30
+        assert (np.abs(got - r64) <= tol).all(), f"normalisation after layer {li} {name}"
+        checked += 1
+    assert checked > 0
+
+
+def test_stack_m1_all_layers_teacher_forced(stack_weights):
+    st, rec = _run(stack_weights, 1, which=None)
+    assert st.bytes_per_step == 3350200320
+    assert len(rec.outputs) == 7 * L
+    _check_projections(stack_weights, rec, 1, rows_per_proj=12, seed=11)
+    _check_glue(rec, 1)
+    assert torch.isfinite(st.x.float()).all()
+
+
+def test_stack_m8_sampled_layers_teacher_forced(stack_weights):
+    layers = [0, 1, 9, 23, 40, 55, 62, 63]
+    which = {(li, name) for li in layers for name, _, _ in synth.STACK_PROJ}
+    which |= {(li + 1, "q") for li in layers if li + 1 < L}
+    st, rec = _run(stack_weights, 8, which=which)
+    _check_projections(stack_weights, rec, 8, rows_per_proj=6, seed=12)
+    _check_glue(rec, 8)
+    assert torch.isfinite(st.x.float()).all()
