@@ -18,6 +18,9 @@ bool q1m1_shape_supported(int R, int N, int K);
 int q1m1_max_group();
 size_t q1m1_xcopy_off(int K);
 bool i4m1_supported(int N, int K);
+bool i4tc_supported(int M, int N, int K);
+lowbit_status i4tc_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
+int i4tc_fault_flag();
 size_t i4m1_act_bytes(int K);
 lowbit_status i4m1_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, void *,
                           cudaStream_t);
@@ -61,6 +64,12 @@ const char *lowbit_status_string(lowbit_status s)
 }
 
 int lowbit_version(void) { return 100; }
+
+int lowbit_fault_flags(void)
+{
+    const int f = i4tc_fault_flag();
+    return f < 0 ? -1 : f;
+}
 
 lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, int64_t cols,
                           uint8_t *packed, void *stream)
@@ -226,6 +235,7 @@ lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales, 
     LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
     cudaStream_t st = as_stream(stream);
     if (M == 1 && i4m1_supported(N, K)) return i4m1_launch(w_q, w_scales, x, y, N, K, workspace, st);
+    if (i4tc_supported(M, N, K)) return i4tc_launch(w_q, w_scales, x, y, M, N, K, st);
     return int4_gemv_simt_launch(w_q, w_scales, x, y, M, N, K, st);
 }
 

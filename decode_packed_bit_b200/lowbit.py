@@ -31,6 +31,7 @@ P, I32, I64, SZ, F32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_s
 SYMBOLS = [
     ("lowbit_status_string", ctypes.c_char_p, [I32]),
     ("lowbit_version", I32, []),
+    ("lowbit_fault_flags", I32, []),
     ("lowbit_pack", I32, [I32, P, I64, I64, P, P]),
     ("lowbit_unpack", I32, [I32, P, I64, I64, P, P]),
     ("lowbit_q1g128_workspace_bytes", SZ, [I32, I32, I32]),
@@ -95,6 +96,10 @@ def _stream(stream):
 
 def _fmt(fmt):
     return FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def lowbit_fault_flags() -> int:
+    return int(lib().lowbit_fault_flags())
 
 
 # -- packing ----------------------------------------------------------------------

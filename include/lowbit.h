@@ -79,6 +79,12 @@ const char *lowbit_status_string(lowbit_status s);
 /* Library version, major*10000 + minor*100 + patch. */
 int lowbit_version(void);
 
+/* Faults the kernels of the current device recorded since the last call,
+ * and clears them: 0 = none; bit 0 = a bounded wait inside the tensor-core
+ * GEMM ran out (its results are then not valid); -1 = the flag could not be
+ * read.  Synchronises with the device. */
+int lowbit_fault_flags(void);
+
 /* ---------------------------------------------------------------------------
  * Packing (all three formats).
  *
@@ -182,8 +188,10 @@ lowbit_status lowbit_q1g128_gemv_noalloc(const uint8_t *w_bits, const uint16_t *
  *   x        [M][K]    bf16
  *   y        [M][N]    fp32
  * Shapes: M >= 1, N >= 1, K >= 64, K % 64 == 0, M*K, N*K < 2^40.
- * The kernel is chosen by M: a weight-streaming GEMV for small M and a
- * tensor-core (tcgen05) GEMM for M >= 128.
+ * The kernel is chosen by M: at M = 1 a weight-streaming tensor-core GEMV
+ * (mma.sync on the packed nibbles); for M >= 16 a tcgen05 GEMM that
+ * dequantises each weight tile into shared memory as two exact bf16 halves
+ * (hi + lo = q*d) and accumulates in TMEM; otherwise a CUDA-core kernel.
  * workspace: at least lowbit_int4g64_workspace_bytes(M, N, K) bytes (NULL
  * allowed when that is 0).
  * ------------------------------------------------------------------------- */

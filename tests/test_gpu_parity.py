@@ -217,7 +217,7 @@ def _run_int4(lb, q, scales, x, N):
     return host(y)
 
 
-@pytest.mark.parametrize("M", [1, 2, 7, 32, 33, 128, 130])
+@pytest.mark.parametrize("M", [1, 2, 7, 16, 32, 33, 64, 128, 130, 256, 300])
 @pytest.mark.parametrize("N,K", [(1, 64), (333, 448), (1000, 1024)])
 def test_int4_small_full_compare(lb, M, N, K):
     seed = 4000 + M * 13 + N
@@ -242,6 +242,7 @@ def test_int4_11008x4096_sampled(lb, M):
     ms, ns = sample_pairs(M, N, 200, seed + M)
     y64, ab = oracle.int4_gemv_at(q, scales, x, ms, ns)
     check_float(y[ms, ns], y64, ab, f"int4 11008x4096 M={M}")
+    assert lb.lowbit_fault_flags() == 0
 
 
 # ---------------------------------------------------------------------------
