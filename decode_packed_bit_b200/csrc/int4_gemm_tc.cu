@@ -37,6 +37,7 @@ namespace lowbit {
 constexpr int kTcBN = 128;             // weight rows per CTA
 constexpr int kTcBK = 64;              // k per stage (one scale group)
 constexpr int kTcStages = 3;
+constexpr int kTcPrefetch = 4;          // groups of packed weights loaded ahead
 constexpr int kTcProdWarps = 8;
 constexpr int kTcTmaWarp = kTcProdWarps;
 constexpr int kTcMmaWarp = kTcProdWarps + 1;
@@ -211,32 +212,50 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
         const bool valid = n < N;
         const uint8_t *qrow = q + (size_t)(valid ? n : 0) * (K / 2) + hf * 16;
         const uint16_t *srow = scales + (size_t)(valid ? n : 0) * (K / 64);
-        for (int it = 0; it < ngroups && ok; ++it) {
-            const int s = it % kTcStages, j = it / kTcStages;
-            uint4 pk = make_uint4(0u, 0u, 0u, 0u);
-            float d = 0.f;
-            if (valid) {
-                pk = __ldg(reinterpret_cast<const uint4 *>(qrow + it * 32));
-                d = f16_bits_to_float(__ldg(srow + it));
-            }
-            if (it >= kTcStages && !mbar_wait(empty + s, (j - 1) & 1)) {
-                ok = false;
-                break;
-            }
-            uint8_t *ahi = smem + s * kTcStageBytes, *alo = ahi + kTcATile;
-            const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+        // packed weights and scales are loaded kTcPrefetch groups ahead
+        uint4 pkb[kTcPrefetch];
+        float db[kTcPrefetch];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint4 hi, lo;
-                dequant8(words[c], d, hi, lo);
-                const int chunk = hf * 4 + c;                       // 16-byte chunk = 8 k
-                const int off = r * 128 + ((chunk ^ (r & 7)) << 4); // 128-byte swizzle
-                *reinterpret_cast<uint4 *>(ahi + off) = hi;
-                *reinterpret_cast<uint4 *>(alo + off) = lo;
+        for (int u = 0; u < kTcPrefetch; ++u) {
+            pkb[u] = make_uint4(0u, 0u, 0u, 0u);
+            db[u] = 0.f;
+            if (valid && u < ngroups) {
+                pkb[u] = __ldg(reinterpret_cast<const uint4 *>(qrow + u * 32));
+                db[u] = f16_bits_to_float(__ldg(srow + u));
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(full_a + s);
+        }
+        for (int it0 = 0; it0 < ngroups && ok; it0 += kTcPrefetch) {
+#pragma unroll
+            for (int u = 0; u < kTcPrefetch; ++u) {
+                const int it = it0 + u;
+                if (it >= ngroups || !ok) break;
+                const int s = it % kTcStages, j = it / kTcStages;
+                const uint4 pk = pkb[u];
+                const float d = db[u];
+                const int nx = it + kTcPrefetch;
+                if (valid && nx < ngroups) {
+                    pkb[u] = __ldg(reinterpret_cast<const uint4 *>(qrow + nx * 32));
+                    db[u] = f16_bits_to_float(__ldg(srow + nx));
+                }
+                if (it >= kTcStages && !mbar_wait(empty + s, (j - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *ahi = smem + s * kTcStageBytes, *alo = ahi + kTcATile;
+                const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint4 hi, lo;
+                    dequant8(words[c], d, hi, lo);
+                    const int chunk = hf * 4 + c;                       // 16-byte chunk = 8 k
+                    const int off = r * 128 + ((chunk ^ (r & 7)) << 4); // 128-byte swizzle
+                    *reinterpret_cast<uint4 *>(ahi + off) = hi;
+                    *reinterpret_cast<uint4 *>(alo + off) = lo;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full_a + s);
+            }
         }
     } else if (warp == kTcTmaWarp) {
         if (lane == 0) {
