@@ -351,6 +351,198 @@ def run_q1_4096(args, world, rank, local):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# the other workloads (one JSON line each, with their own metric)
+# ---------------------------------------------------------------------------
+
+def _graph_time(step, stream, steps, warmup):
+    """Capture step() in a CUDA graph on `stream`; return ms per replay."""
+    import torch
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    for _ in range(warmup):
+        graph.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del graph
+    return ms
+
+
+def _emit(rank, line):
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_q1_stack(args, world, rank, local):
+    """64-layer Q1_0_g128 projection stack, one decode step per replay."""
+    import torch
+    import synth
+    from decode_packed_bit_b200 import build as lb_build
+    lb_build.build()
+    from decode_packed_bit_b200.stack import Q1Layer, Q1Stack
+    dev = torch.device("cuda", local)
+    seed = synth.SEED_BASE + synth.W_Q1_STACK + 1000 * rank
+    layers = [Q1Layer({name: synth.torch_q1_layer(seed, n, k, li * 16 + pi, dev)
+                       for pi, (name, n, k) in enumerate(synth.STACK_PROJ)})
+              for li in range(synth.STACK_LAYERS)]
+    M = args.m
+    st = Q1Stack(layers, synth.STACK_HIDDEN, synth.STACK_FFN, M, dev)
+    st.x.copy_(torch.from_numpy(synth.bf16_normal(seed, (M, synth.STACK_HIDDEN)).view(np.int16))
+               .view(torch.bfloat16).to(dev))
+    stream = torch.cuda.Stream(device=dev)
+    with ClockSampler(local) as clk:
+        ms = _graph_time(lambda: st.step(stream=stream), stream, args.steps, args.warmup)
+    ms = max_over_ranks(ms, world)
+    gbs = st.bytes_per_step / (ms * 1e-3) / 1e9
+    _emit(rank, {"metric": f"decode tokens/s through the 64-layer Q1 stack (M={M})",
+                 "value": round(M * world * 1e3 / ms, 2), "unit": "tokens/s", "n_gpus": world,
+                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+                 "higher_is_better": True, "scaling": "weak", "dtype": KERNEL_DTYPE if M == 1 else "bf16xsign->f32",
+                 "data": "synthetic",
+                 "config": {"workload": "Q1_0_g128 64-layer stack, hidden 5120, ffn 17408", "M": M,
+                            "bytes_per_step": st.bytes_per_step, "l2": "inputs larger than L2 (3.35 GB)"},
+                 "weight_gbs": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / measured_peaks()[0], 2),
+                 "gpu_launches": st.launches_per_step() * args.steps, "clocks": clk.summary()})
+    return 0
+
+
+def _rotation(per_bytes, l2):
+    return max(4, -(-3 * l2 // per_bytes))
+
+
+def run_q1_sweep(args, world, rank, local):
+    """Q1_0_g128 at the three layer shapes and M in {1, 4, 16}."""
+    import torch
+    import synth
+    from decode_packed_bit_b200 import build as lb_build
+    lb_build.build()
+    from decode_packed_bit_b200 import lowbit as lb
+    dev = torch.device("cuda", local)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    seed = synth.SEED_BASE + synth.W_Q1_SWEEP + 1000 * rank
+    results = []
+    for (N, K) in synth.Q1_SWEEP_SHAPES:
+        per = q1_bytes(N, K)
+        R = min(256, _rotation(per, l2))
+        mats = [synth.torch_q1_layer(seed, N, K, r, dev) for r in range(R)]
+        for M in (1, 4, 16):
+            x = torch.from_numpy(synth.bf16_normal(seed, (M, K), tag=M).view(np.int16)).to(dev)
+            ys = [torch.empty((M, N), dtype=torch.float32, device=dev) for _ in range(R)]
+            stream = torch.cuda.Stream(device=dev)
+            if M == 1:
+                act = torch.empty(lb.lowbit_q1g128_act_bytes(1, K), dtype=torch.uint8, device=dev)
+
+                def step():
+                    lb.lowbit_q1g128_prepare_act(x, act, stream=stream)
+                    lb.lowbit_q1g128_gemv_act_group([b for b, _ in mats], [s for _, s in mats], act, ys, 1,
+                                                    stream=stream)
+            else:
+                def step():
+                    for r in range(R):
+                        lb.lowbit_q1g128_gemv(mats[r][0], mats[r][1], x, ys[r], stream=stream)
+            ms = max_over_ranks(_graph_time(step, stream, max(3, args.steps // 5), args.warmup), world)
+            results.append({"N": N, "K": K, "M": M, "weight_sets": R,
+                            "gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
+                            "us_per_gemv": round(ms * 1e3 / R, 3)})
+        del mats
+    _emit(rank, {"metric": "packed-weight GB/s, Q1_0_g128 layer-shape sweep", "unit": "GB/s",
+                 "value": results[0]["gbs"], "n_gpus": world, "higher_is_better": True, "data": "synthetic",
+                 "config": {"workload": "Q1_0_g128 (5120,5120),(17408,5120),(5120,17408) x M in {1,4,16}",
+                            "l2": "inputs larger than L2 (rotating weight sets)"},
+                 "results": results})
+    return 0
+
+
+def run_int4(args, world, rank, local):
+    """INT4_G64 11008 x 4096 at M in {1, 32, 256}."""
+    import torch
+    import synth
+    from decode_packed_bit_b200 import build as lb_build
+    lb_build.build()
+    from decode_packed_bit_b200 import lowbit as lb
+    dev = torch.device("cuda", local)
+    N, K = synth.INT4_N, synth.INT4_K
+    per = N * K // 2 + 2 * N * (K // 64)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = _rotation(per, l2)
+    g = torch.Generator(device=dev)
+    g.manual_seed(synth.SEED_BASE + synth.W_INT4 + 1000 * rank)
+    qs = [torch.randint(0, 256, (N, K // 2), generator=g, device=dev, dtype=torch.uint8) for _ in range(R)]
+    ss = [(torch.randn((N, K // 64), generator=g, device=dev) * 0.01).abs().half() for _ in range(R)]
+    results = []
+    for M in (1, 32, 256):
+        x = torch.randn((M, K), generator=g, device=dev).bfloat16()
+        y = torch.empty((R, M, N), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(16, lb.lowbit_int4g64_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
+        stream = torch.cuda.Stream(device=dev)
+
+        def step():
+            for r in range(R):
+                lb.lowbit_int4g64_gemm(qs[r], ss[r], x, y[r], workspace=ws, stream=stream)
+        ms = max_over_ranks(_graph_time(step, stream, max(3, args.steps // 5), args.warmup), world)
+        results.append({"M": M, "us_per_call": round(ms * 1e3 / R, 3),
+                        "weight_gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
+                        "tflops": round(2.0 * M * N * K * R / (ms * 1e-3) / 1e12, 2)})
+    assert lb.lowbit_fault_flags() == 0
+    _emit(rank, {"metric": "INT4_G64 11008x4096: packed-weight GB/s (M=1) and TFLOP/s (M=32, 256)",
+                 "unit": "GB/s", "value": results[0]["weight_gbs"], "n_gpus": world, "higher_is_better": True,
+                 "data": "synthetic",
+                 "config": {"workload": "INT4_G64 N=11008 K=4096 M in {1,32,256}", "weight_sets": R,
+                            "l2": "inputs larger than L2 (rotating weight sets)"},
+                 "results": results})
+    return 0
+
+
+def run_q2_mlp(args, world, rank, local):
+    """The 2-bit integer MLP (256->192->128->40) over 1024 and 1M vectors."""
+    import torch
+    import synth
+    from decode_packed_bit_b200 import build as lb_build
+    lb_build.build()
+    from decode_packed_bit_b200 import lowbit as lb
+    dev = torch.device("cuda", local)
+    seed = synth.SEED_BASE + synth.W_Q2_MLP + 1000 * rank
+    dims = synth.Q2_DIMS
+    w = []
+    for c in synth.q2_codes(seed, dims):
+        codes = torch.from_numpy(c).to(dev)
+        packed = torch.empty((c.shape[0], c.shape[1] // 4), dtype=torch.uint8, device=dev)
+        lb.lowbit_pack("q2", codes, packed)
+        w.append(packed)
+    macs = sum(dims[i] * dims[i + 1] for i in range(len(dims) - 1))
+    results = []
+    for batch in (1024, 1 << 20):
+        xb = synth.q2_inputs(seed, 1024)
+        x = torch.from_numpy(np.tile(xb, (batch // 1024, 1))).to(dev)
+        logits = torch.empty((batch, dims[-1]), dtype=torch.int16, device=dev)
+        am = torch.empty((batch,), dtype=torch.int32, device=dev)
+        stream = torch.cuda.Stream(device=dev)
+        ms = max_over_ranks(_graph_time(lambda: lb.lowbit_q2_mlp_forward(w, dims, x, logits, am, stream=stream),
+                                        stream, args.steps, args.warmup), world)
+        results.append({"batch": batch, "us": round(ms * 1e3, 3), "vectors_per_s": round(batch / (ms * 1e-3), 1),
+                        "gmac_per_s": round(batch * macs / (ms * 1e-3) / 1e9, 2)})
+    _emit(rank, {"metric": "2-bit integer MLP vectors/s (256->192->128->40)", "unit": "vectors/s",
+                 "value": results[0]["vectors_per_s"], "n_gpus": world, "higher_is_better": True,
+                 "dtype": "int16 wrap / int32", "data": "synthetic",
+                 "config": {"workload": "Z80-style 2-bit MLP, 1024 and 1048576 vectors", "macs_per_vector": macs},
+                 "results": results})
+    return 0
+
+
+OTHER_WORKLOADS = {"q1_stack": run_q1_stack, "q1_sweep": run_q1_sweep, "int4": run_int4, "q2_mlp": run_q2_mlp}
+
+
 KERNEL_DTYPE = "u8xs8->s32 (tensor core), f32 epilogue"
 
 
@@ -381,6 +573,7 @@ def main():
     ap.add_argument("--workload", default="q1_4096",
                     choices=["q1_4096", "q1_sweep", "q1_stack", "int4", "q2_mlp"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--m", type=int, default=1, help="batch rows for --workload q1_stack")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -394,8 +587,7 @@ def main():
     try:
         if args.workload == "q1_4096":
             return run_q1_4096(args, world, rank, local)
-        import bench_workloads
-        return bench_workloads.run(args, world, rank, local)
+        return OTHER_WORKLOADS[args.workload](args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist
