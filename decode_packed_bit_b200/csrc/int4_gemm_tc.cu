@@ -25,12 +25,10 @@
 //              stage's "empty" barrier.
 // Every mbarrier wait is bounded in time; a wait that runs out records a
 // fault flag and the CTA leaves its loops, releases TMEM and exits.
-#include <cuda.h>
-
 #include <algorithm>
 #include <mutex>
 
-#include "common.cuh"
+#include "tc_common.cuh"
 
 namespace lowbit {
 
@@ -46,67 +44,8 @@ constexpr int kTcATile = kTcBN * kTcBK * 2;        // 16 KiB of bf16
 constexpr int kTcBTile = 256 * kTcBK * 2;          // 32 KiB of bf16 (BM <= 256)
 constexpr int kTcStageBytes = 2 * kTcATile + kTcBTile;
 constexpr int kTcSmemBytes = kTcStages * kTcStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-constexpr unsigned long long kTcWaitNs = 2000000000ull;  // 2 s
 
 __device__ unsigned g_tc_fault;  // set when a bounded wait ran out
-
-__device__ __forceinline__ unsigned long long globaltimer_ns()
-{
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"((unsigned)__cvta_generic_to_shared(bar)), "r"(count)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"((unsigned)__cvta_generic_to_shared(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, unsigned bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
-                     (unsigned)__cvta_generic_to_shared(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-
-// Wait until phase `parity` of the barrier has completed; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity)
-{
-    const unsigned a = (unsigned)__cvta_generic_to_shared(bar);
-    const unsigned long long t0 = globaltimer_ns();
-    while (true) {
-        unsigned ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(a), "r"(parity)
-            : "memory");
-        if (ok) return true;
-        if (globaltimer_ns() - t0 > kTcWaitNs) {
-            atomicExch(&g_tc_fault, 1u);
-            return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            (unsigned)__cvta_generic_to_shared(dst)),
-        "l"(map), "r"(c0), "r"(c1), "r"((unsigned)__cvta_generic_to_shared(bar))
-        : "memory");
-}
 
 // UMMA shared-memory descriptor: K-major operand with 128-byte swizzle, rows
 // 128 bytes apart, 8-row groups 1024 bytes apart (tile base 1024-aligned).
@@ -117,21 +56,16 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(const void *smem_tile)
            (1ull << 46) /*version*/ | (2ull << 61) /*SWIZZLE_128B*/;
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          bool accumulate)
+// D (+)= A x B, both from shared memory.  ACC (accumulate into D) is an
+// immediate: a predicate computed from a register slows every MMA issue.
+template <bool ACC>
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc)
 {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"((unsigned)accumulate));
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t *bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     (unsigned)__cvta_generic_to_shared(bar))
-                 : "memory");
+        "l"(adesc), "l"(bdesc), "r"(idesc), "n"(ACC ? 1 : 0));
 }
 
 // bf16 pair, round to nearest even, lo in the low half
@@ -192,16 +126,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
             mbar_init(empty + s, 1);
         }
         mbar_init(done, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_fence_init();
     }
     if (warp == kTcMmaWarp) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         (unsigned)__cvta_generic_to_shared(tmem_slot)),
-                     "r"(256));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        tmem_alloc(tmem_slot, 256);
     }
     __syncthreads();
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    tc_fence_after();
     const uint32_t tmem_d = *tmem_slot;
     bool ok = true;
 
@@ -237,7 +168,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
                     pkb[u] = __ldg(reinterpret_cast<const uint4 *>(qrow + nx * 32));
                     db[u] = f16_bits_to_float(__ldg(srow + nx));
                 }
-                if (it >= kTcStages && !mbar_wait(empty + s, (j - 1) & 1)) {
+                if (it >= kTcStages && !mbar_wait(empty + s, (j - 1) & 1, &g_tc_fault)) {
                     ok = false;
                     break;
                 }
@@ -262,44 +193,54 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
             pdl_wait_primary();  // x follows stream order
             for (int it = 0; it < ngroups; ++it) {
                 const int s = it % kTcStages, j = it / kTcStages;
-                if (it >= kTcStages && !mbar_wait(empty + s, (j - 1) & 1)) break;
+                if (it >= kTcStages && !mbar_wait(empty + s, (j - 1) & 1, &g_tc_fault)) break;
                 mbar_arrive_expect_tx(full_b + s, (unsigned)(BM * kTcBK * 2));
                 tma_load_2d(smem + s * kTcStageBytes + 2 * kTcATile, &tmap_x, it * kTcBK, m0, full_b + s);
             }
         }
     } else {
-        if (lane == 0) {
-            // instruction descriptor: f32 accumulate, bf16 A and B, both K-major,
-            // N = BM, M = 128
-            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BM >> 3) << 17) |
-                                   ((uint32_t)(kTcBN >> 4) << 24);
-            for (int it = 0; it < ngroups; ++it) {
-                const int s = it % kTcStages, j = it / kTcStages;
-                if (!mbar_wait(full_a + s, j & 1) || !mbar_wait(full_b + s, j & 1)) {
-                    ok = false;
-                    break;
-                }
-                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                uint8_t *st = smem + s * kTcStageBytes;
-                const uint64_t ahi = umma_desc_sw128(st), alo = umma_desc_sw128(st + kTcATile),
-                               bd = umma_desc_sw128(st + 2 * kTcATile);
+        // MMA issue: the whole warp runs the loop (uniform operands), one
+        // elected lane issues.  instruction descriptor: f32 accumulate, bf16
+        // A and B, both K-major, N = BM, M = 128
+        const uint32_t idesc =
+            (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BM >> 3) << 17) | ((uint32_t)(kTcBN >> 4) << 24);
+        for (int it = 0; it < ngroups; ++it) {
+            const int s = it % kTcStages, j = it / kTcStages;
+            if (!mbar_wait_warp(full_a + s, j & 1, &g_tc_fault) || !mbar_wait_warp(full_b + s, j & 1, &g_tc_fault)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint8_t *st = smem + s * kTcStageBytes;
+            const uint64_t ahi = umma_desc_sw128(st), alo = umma_desc_sw128(st + kTcATile),
+                           bd = umma_desc_sw128(st + 2 * kTcATile);
+            if (elect_one()) {
+                // advancing 16 k (32 bytes) inside the swizzle atom: +2 in 16-byte units
+                if (it == 0)
+                    umma_bf16<false>(tmem_d, ahi, bd, idesc);
+                else
+                    umma_bf16<true>(tmem_d, ahi, bd, idesc);
+                umma_bf16<true>(tmem_d, alo, bd, idesc);
 #pragma unroll
-                for (int kk = 0; kk < kTcBK / 16; ++kk) {
-                    // advancing 16 k (32 bytes) inside the swizzle atom: +2 in 16-byte units
-                    umma_bf16(tmem_d, ahi + 2 * kk, bd + 2 * kk, idesc, it > 0 || kk > 0);
-                    umma_bf16(tmem_d, alo + 2 * kk, bd + 2 * kk, idesc, true);
+                for (int kk = 1; kk < kTcBK / 16; ++kk) {
+                    umma_bf16<true>(tmem_d, ahi + 2 * kk, bd + 2 * kk, idesc);
+                    umma_bf16<true>(tmem_d, alo + 2 * kk, bd + 2 * kk, idesc);
                 }
                 umma_commit(empty + s);
             }
-            if (ok) umma_commit(done);
+            __syncwarp();
         }
+        // also after a failed wait: `done` then tells that every MMA issued
+        // has completed, before tensor memory is released
+        if (elect_one()) umma_commit(done);
         __syncwarp();
+        mbar_wait_warp(done, 0, &g_tc_fault);
     }
 
     // ---- epilogue: TMEM -> y (warps 0-7: lane quarter warp%4, column half warp/4) ----
     if (warp < kTcProdWarps) {
-        const bool got = ok && mbar_wait(done, 0);
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const bool got = mbar_wait_warp(done, 0, &g_tc_fault) && ok;
+        tc_fence_after();
         pdl_wait_primary();  // y may still be read by an earlier kernel
         const int quarter = warp & 3, half = warp >> 2;
         const int n = n0 + quarter * 32 + lane;
@@ -326,12 +267,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
                 }
             }
         }
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        tc_fence_before();
     }
     __syncthreads();
     if (warp == kTcMmaWarp) {
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(256));
+        tc_fence_after();
+        tmem_dealloc(tmem_d, 256);
     }
 }
 

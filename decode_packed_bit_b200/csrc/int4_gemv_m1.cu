@@ -53,18 +53,6 @@ static inline size_t i4_align256(size_t v) { return (v + 255) & ~size_t(255); }
 // activation prepare
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ float i4_warp_max(float v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-__device__ __forceinline__ int i4_warp_sum(int v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
 
 // One CTA of 128 threads per 128-k pair.  Thread kk turns x[k] into limbs;
 // then thread t writes B fragment words of lane t%32 for mma t/32.
@@ -83,7 +71,7 @@ __global__ void __launch_bounds__(128) k_i4_prep_m1(const uint16_t *__restrict__
     pdl_wait_primary();
 
     const float xv = k < K ? bf16_bits_to_float(x[k]) : 0.f;
-    const float wm = i4_warp_max(fabsf(xv));
+    const float wm = warp_max(fabsf(xv));
     if (lane == 0) smax[warp] = wm;
     __syncthreads();
     const float m = fmaxf(smax[2 * h], smax[2 * h + 1]);
@@ -101,7 +89,7 @@ __global__ void __launch_bounds__(128) k_i4_prep_m1(const uint16_t *__restrict__
     limb[1][kk] = (int8_t)l1;
     limb[2][kk] = (int8_t)l2;
     limb[3][kk] = (int8_t)l3;
-    const int ws = i4_warp_sum(X);
+    const int ws = warp_sum_int(X);
     if (lane == 0) ssum[warp] = ws;
     __syncthreads();
     if ((kk & 63) == 0) {

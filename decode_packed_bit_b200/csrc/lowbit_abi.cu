@@ -21,6 +21,7 @@ bool i4m1_supported(int N, int K);
 bool i4tc_supported(int M, int N, int K);
 lowbit_status i4tc_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 int i4tc_fault_flag();
+int q1tc_fault_flag();
 size_t i4m1_act_bytes(int K);
 lowbit_status i4m1_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, void *,
                           cudaStream_t);
@@ -67,8 +68,9 @@ int lowbit_version(void) { return 100; }
 
 int lowbit_fault_flags(void)
 {
-    const int f = i4tc_fault_flag();
-    return f < 0 ? -1 : f;
+    const int f4 = i4tc_fault_flag(), f1 = q1tc_fault_flag();
+    if (f4 < 0 || f1 < 0) return -1;
+    return (f4 ? 1 : 0) | (f1 ? 2 : 0);
 }
 
 lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, int64_t cols,

@@ -45,7 +45,7 @@
 //     distributed shared memory (deterministic, no global scratch).
 #include <algorithm>
 
-#include "common.cuh"
+#include "q1_common.cuh"
 
 namespace lowbit {
 
@@ -67,36 +67,15 @@ constexpr int kQ1InfoBytesPerChunk = 16;    // two groups x (G, S) floats
 #endif
 constexpr int kQ1Warps = LOWBIT_Q1_WARPS;
 constexpr int kQ1MinExp = -96;              // activations below 2^-96 round to 0
-constexpr int kQ1MaxGroup = 256;
 constexpr int kQ1MaxSmem = 226 * 1024;     // dynamic part; leaves room for static smem
 constexpr int kQ1MaxCluster = 8;
 
 
-struct Q1Group {
-    const uint8_t *bits[kQ1MaxGroup];
-    const uint16_t *scales[kQ1MaxGroup];
-    float *y[kQ1MaxGroup];
-};
 
-static inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // ---------------------------------------------------------------------------
 // activation prepare: x (bf16) -> limb fragments + per-group (G, S) + copy
 // ---------------------------------------------------------------------------
-
-__device__ __forceinline__ float warp_max(float v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
-__device__ __forceinline__ int warp_sum_int(int v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
 
 // One CTA of 256 threads per 256-k chunk.  Thread kk first turns x[k] into
 // four limbs; then thread t writes the 8-byte B fragment of lane t%32 for
@@ -658,12 +637,23 @@ static Q1Plan q1_plan(int R, int N, int K, int sms)
     return P;
 }
 
-size_t q1m1_act_bytes(int K) { return q1_plan(1, 1, K, 148).act_bytes; }
-size_t q1m1_xcopy_off(int K) { return q1_plan(1, 1, K, 148).xcopy_off; }
+// With LOWBIT_Q1_TC=1 at build time, K a multiple of 1024 goes to the
+// tcgen05 kernel (q1_gemv_tc.cu) instead.  It is off by default: measured on
+// B200 it streams 1.4 TB/s against 3.5 TB/s for the mma.sync kernels above,
+// because every 128-row tile needs a four-warp hand-off to the MMA warp per
+// 256 k, where the mma.sync warps run independently.
+#ifndef LOWBIT_Q1_TC
+#define LOWBIT_Q1_TC 0
+#endif
+static bool use_tc(int K) { return LOWBIT_Q1_TC && q1tc_supported(1, 1, K); }
+
+size_t q1m1_act_bytes(int K) { return use_tc(K) ? q1tc_act_bytes(K) : q1_plan(1, 1, K, 148).act_bytes; }
+size_t q1m1_xcopy_off(int K) { return use_tc(K) ? q1tc_xcopy_off(K) : q1_plan(1, 1, K, 148).xcopy_off; }
 int q1m1_max_group() { return kQ1MaxGroup; }
 
 bool q1m1_shape_supported(int R, int N, int K)
 {
+    if (use_tc(K)) return q1tc_supported(R, N, K);
     if ((K / 128) % 2 != 0) return false;  // scale pairs must be 4-byte aligned
     if (R < 1 || R > kQ1MaxGroup) return false;
     return q1_plan(R, N, K, num_sms()).ok;
@@ -671,6 +661,7 @@ bool q1m1_shape_supported(int R, int N, int K)
 
 lowbit_status q1m1_prepare_launch(const uint16_t *x, int K, void *act, cudaStream_t st)
 {
+    if (use_tc(K)) return q1tc_prepare_launch(x, K, act, st);
     const Q1Plan P = q1_plan(1, 1, K, 148);
     cudaError_t e = launch_pdl(k_q1_prep_m1, dim3(P.nchunks), dim3(256), 0, st, x, K, static_cast<uint8_t *>(act),
                                P.info_off, P.xcopy_off);
@@ -680,6 +671,7 @@ lowbit_status q1m1_prepare_launch(const uint16_t *x, int K, void *act, cudaStrea
 lowbit_status q1m1_gemv_launch(const uint8_t *const *bits, const uint16_t *const *scales, const void *act,
                                float *const *y, int R, int N, int K, cudaStream_t st)
 {
+    if (use_tc(K)) return q1tc_gemv_launch(bits, scales, act, y, R, N, K, st);
     const Q1Plan P = q1_plan(R, N, K, num_sms());
     Q1Group grp;
     for (int r = 0; r < R; ++r) {

@@ -80,9 +80,10 @@ const char *lowbit_status_string(lowbit_status s);
 int lowbit_version(void);
 
 /* Faults the kernels of the current device recorded since the last call,
- * and clears them: 0 = none; bit 0 = a bounded wait inside the tensor-core
- * GEMM ran out (its results are then not valid); -1 = the flag could not be
- * read.  Synchronises with the device. */
+ * and clears them: 0 = none; bit 0 = a bounded wait inside the INT4_G64
+ * tcgen05 GEMM ran out, bit 1 = one inside the Q1_0_g128 tcgen05 product
+ * (the results of that call are then not valid); -1 = the flags could not
+ * be read.  Synchronises with the device. */
 int lowbit_fault_flags(void);
 
 /* ---------------------------------------------------------------------------

@@ -135,7 +135,8 @@ def test_q1_act_workspace_reused_across_calls(lb):
     del cnt_region
 
 
-@pytest.mark.parametrize("R,N,K", [(3, 515, 1280), (20, 4096, 4096), (2, 17408, 512), (5, 33, 17408)])
+@pytest.mark.parametrize("R,N,K", [(3, 515, 1280), (20, 4096, 4096), (2, 17408, 512), (5, 33, 17408),
+                                   (40, 300, 3072), (200, 200, 2048)])
 def test_q1_group_matches_oracle_and_single_calls(lb, R, N, K):
     """R matrices that read one prepared activation, in one launch."""
     x = synth.bf16_normal(2600 + R, (1, K))
