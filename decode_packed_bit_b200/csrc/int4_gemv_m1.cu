@@ -37,7 +37,17 @@ constexpr int kI4InfoBytesPerPair = 16;     // two groups x (G, S)
 constexpr int kI4Warps = 8;
 constexpr int kI4SplitWarps = 4;
 constexpr int kI4StepRows = 32;
-constexpr int kI4Stages = 6;                // a warp's whole K-slice in flight
+// Tuning knobs (compile-time; the defaults are the measured best).
+#ifndef LOWBIT_I4_STAGES
+#define LOWBIT_I4_STAGES 6
+#endif
+#ifndef LOWBIT_I4_CTAS_PER_SM
+#define LOWBIT_I4_CTAS_PER_SM 2
+#endif
+#ifndef LOWBIT_I4_FILL
+#define LOWBIT_I4_FILL 0
+#endif
+constexpr int kI4Stages = LOWBIT_I4_STAGES;  // steps of a warp in flight
 constexpr int kI4RowStride = 64;            // 16-byte reads of a row quad are conflict free
 constexpr int kI4StageW = kI4StepRows * kI4RowStride;
 constexpr int kI4StageBytes = kI4StageW + kI4StepRows * 4;
@@ -47,78 +57,6 @@ constexpr int kI4MaxSmem = 226 * 1024;
 constexpr int kI4MaxCluster = 8;
 constexpr int kI4SplitRows = kI4SplitWarps * kI4StepRows;
 
-static inline size_t i4_align256(size_t v) { return (v + 255) & ~size_t(255); }
-
-// ---------------------------------------------------------------------------
-// activation prepare
-// ---------------------------------------------------------------------------
-
-
-// One CTA of 128 threads per 128-k pair.  Thread kk turns x[k] into limbs;
-// then thread t writes B fragment words of lane t%32 for mma t/32.
-__global__ void __launch_bounds__(128) k_i4_prep_m1(const uint16_t *__restrict__ x, int K, uint8_t *__restrict__ act,
-                                                   size_t info_off)
-{
-    __shared__ float smax[4];
-    __shared__ int ssum[4];
-    __shared__ int8_t limb[4][128];
-    pdl_launch_dependents();
-    const int pr = blockIdx.x;
-    const int kk = threadIdx.x;
-    const int k = pr * kI4PairK + kk;
-    const int warp = kk >> 5, lane = kk & 31;
-    const int h = kk >> 6;  // group within the pair
-    pdl_wait_primary();
-
-    const float xv = k < K ? bf16_bits_to_float(x[k]) : 0.f;
-    const float wm = warp_max(fabsf(xv));
-    if (lane == 0) smax[warp] = wm;
-    __syncthreads();
-    const float m = fmaxf(smax[2 * h], smax[2 * h + 1]);
-    const int e8 = (int)((__float_as_uint(m) >> 23) & 0xFFu);
-    const int E = max(e8 == 0 ? kI4MinExp : e8 - 126, kI4MinExp);
-    const int X = __float2int_rn(ldexpf(xv, 23 - E));       // |X| < 2^23
-    const int B = (k & 1) ? X : X * 16;                      // low nibbles carry q+8, high 16(q+8)
-    int l0 = (int)(int8_t)(B & 0xFF);
-    int r = (B - l0) >> 8;
-    int l1 = (int)(int8_t)(r & 0xFF);
-    r = (r - l1) >> 8;
-    int l2 = (int)(int8_t)(r & 0xFF);
-    const int l3 = (r - l2) >> 8;                            // |B| < 2^27: l3 in [-8, 8]
-    limb[0][kk] = (int8_t)l0;
-    limb[1][kk] = (int8_t)l1;
-    limb[2][kk] = (int8_t)l2;
-    limb[3][kk] = (int8_t)l3;
-    const int ws = warp_sum_int(X);
-    if (lane == 0) ssum[warp] = ws;
-    __syncthreads();
-    if ((kk & 63) == 0) {
-        const int T = ssum[2 * h] + ssum[2 * h + 1];
-        const int grp = 2 * pr + h;
-        float2 info = make_float2(0.f, 0.f);
-        if (grp * 64 < K) info = make_float2(ldexpf(1.0f, E - 27), ldexpf((float)T, E - 20));
-        reinterpret_cast<float2 *>(act + info_off)[grp] = info;
-    }
-
-    // B fragments: mma u (4 per pair), lane (n, t).  Register j, byte c holds
-    // the k-slot of A register a(2j) byte c of thread t: nibble j of packed
-    // byte 4*wi + c of group t/2, wi = 4(t&1) + u, i.e. k = 64(t/2) + 32(t&1)
-    // + 8u + 2c + j.  Column n = 4*group + limb; the other group's lanes get 0.
-    for (int e = kk; e < 4 * 32; e += 128) {
-        const int u = e >> 5, ln = e & 31;
-        const int n = ln >> 2, t = ln & 3;
-        uint32_t w[2] = {0u, 0u};
-        if ((n >> 2) == (t >> 1)) {
-            const int8_t *lb = limb[n & 3];
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    w[j] |= (uint32_t)(uint8_t)lb[64 * (t >> 1) + 32 * (t & 1) + 8 * u + 2 * c + j] << (8 * c);
-        }
-        reinterpret_cast<uint2 *>(act + (size_t)pr * kI4FragBytesPerPair)[e] = make_uint2(w[0], w[1]);
-    }
-}
 
 // ---------------------------------------------------------------------------
 // product
@@ -152,11 +90,10 @@ template <int N>
 __device__ __forceinline__ void i4_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 struct I4Params {
+    const uint16_t *x;  // bf16 activation; each CTA builds its slice's fragments from it
     const uint8_t *q;
     const uint16_t *scales;
     float *y;
-    const uint8_t *act;
-    size_t info_off;
     int N, K, npairs;
     int L;          // pairs per K-slice
     int act_smem;
@@ -224,14 +161,70 @@ __device__ __forceinline__ void i4_consume(const uint8_t *st, const uint8_t *bf,
         }
 }
 
-__device__ __forceinline__ void i4_stage_act(uint8_t *smem, const I4Params &p, int p_lo, int n)
+constexpr int kI4BuildScratch = kI4SplitWarps * 4 * 128;  // limb scratch of the build
+
+// Build the B fragments and group constants of one 128-k pair from x, in one
+// warp: lane l takes k = 128 pr + 32 j + l (j = 0..3; j < 2 is the pair's
+// first group), so every per-group reduction is a warp shuffle; the limbs
+// go through lw (this warp's 4 x 128-byte scratch) to the fragment layout.
+__device__ __forceinline__ void i4_build_pair_warp(const uint16_t *__restrict__ x, int K, int pr, uint8_t *frag,
+                                                   float2 *info, int8_t (*lw)[128], int lane)
 {
-    const uint4 *src = reinterpret_cast<const uint4 *>(p.act + (size_t)p_lo * kI4FragBytesPerPair);
-    uint4 *dst = reinterpret_cast<uint4 *>(smem);
-    for (int i = threadIdx.x; i < n * (kI4FragBytesPerPair / 16); i += blockDim.x) dst[i] = __ldg(src + i);
-    const uint4 *isrc = reinterpret_cast<const uint4 *>(p.act + p.info_off + (size_t)p_lo * kI4InfoBytesPerPair);
-    uint4 *idst = reinterpret_cast<uint4 *>(smem + (size_t)n * kI4FragBytesPerPair);
-    for (int i = threadIdx.x; i < n; i += blockDim.x) idst[i] = __ldg(isrc + i);
+    float xv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int k = pr * kI4PairK + 32 * j + lane;
+        xv[j] = k < K ? bf16_bits_to_float(x[k]) : 0.f;
+    }
+    int E[2], T[2] = {0, 0};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float mh = warp_max(fmaxf(fabsf(xv[2 * h]), fabsf(xv[2 * h + 1])));
+        const int e8 = (int)((__float_as_uint(mh) >> 23) & 0xFFu);
+        E[h] = max(e8 == 0 ? kI4MinExp : e8 - 126, kI4MinExp);  // smallest E with max|x| < 2^E
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int X = __float2int_rn(ldexpf(xv[j], 23 - E[j >> 1]));  // |X| <= 2^23
+        T[j >> 1] += X;
+        const int B = (lane & 1) ? X : X * 16;  // k & 1 == lane & 1: low nibbles carry q+8, high 16(q+8)
+        const int l0 = (int)(int8_t)(B & 0xFF);
+        int r = (B - l0) >> 8;
+        const int l1 = (int)(int8_t)(r & 0xFF);
+        r = (r - l1) >> 8;
+        const int l2 = (int)(int8_t)(r & 0xFF);
+        lw[0][32 * j + lane] = (int8_t)l0;
+        lw[1][32 * j + lane] = (int8_t)l1;
+        lw[2][32 * j + lane] = (int8_t)l2;
+        lw[3][32 * j + lane] = (int8_t)((r - l2) >> 8);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int Th = warp_sum_int(T[h]);
+        if (lane == 0)
+            info[h] = (2 * pr + h) * 64 < K ? make_float2(ldexpf(1.0f, E[h] - 27), ldexpf((float)Th, E[h] - 20))
+                                            : make_float2(0.f, 0.f);
+    }
+    __syncwarp();
+    // B fragments: mma u (4 per pair), lane (n, t).  Register j, byte c holds
+    // the k-slot of A register a(2j) byte c of thread t: nibble j of packed
+    // byte 4*wi + c of group t/2, wi = 4(t&1) + u, i.e. k = 64(t/2) + 32(t&1)
+    // + 8u + 2c + j.  Column n = 4*group + limb; the other group's lanes get 0.
+    const int n = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        uint32_t w[2] = {0u, 0u};
+        if ((n >> 2) == (t >> 1)) {
+            const int8_t *lb = lw[n & 3];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    w[j] |= (uint32_t)(uint8_t)lb[64 * (t >> 1) + 32 * (t & 1) + 8 * u + 2 * c + j] << (8 * c);
+        }
+        reinterpret_cast<uint2 *>(frag)[32 * u + lane] = make_uint2(w[0], w[1]);
+    }
+    __syncwarp();  // the scratch is reused for the warp's next pair
 }
 
 template <typename Out>
@@ -294,7 +287,14 @@ __global__ void __launch_bounds__(kI4SplitWarps * 32) k_i4_m1_split(const I4Para
     for (int t = 0; t < kI4Stages - 1; ++t) issue_next();
 
     pdl_wait_primary();
-    if (p_hi > p_lo) i4_stage_act(smem, p, p_lo, p_hi - p_lo);
+    if (p_hi > p_lo) {
+        const int n = p_hi - p_lo;
+        int8_t(*lw)[128] = reinterpret_cast<int8_t(*)[128]>(smem + p.act_smem + kI4SplitWarps * kI4WarpRing +
+                                                             warp * 4 * 128);
+        float2 *info = reinterpret_cast<float2 *>(smem + (size_t)n * kI4FragBytesPerPair);
+        for (int c = warp; c < n; c += kI4SplitWarps)
+            i4_build_pair_warp(p.x, p.K, p_lo + c, smem + (size_t)c * kI4FragBytesPerPair, info + 2 * c, lw, lane);
+    }
     __syncthreads();
 
     const uint8_t *bfrag = smem + lane * 8;
@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(kI4SplitWarps * 32) k_i4_m1_split(const I4Para
 
 struct I4Plan {
     int npairs, L, nslices, blocks;
-    size_t info_off, act_bytes, act_smem, smem;
+    size_t act_smem, smem;
     bool ok;
 };
 
@@ -347,20 +347,19 @@ static I4Plan i4_plan(int N, int K, int sms)
 {
     I4Plan P = {};
     P.npairs = (K + kI4PairK - 1) / kI4PairK;
-    P.info_off = i4_align256((size_t)P.npairs * kI4FragBytesPerPair);
-    P.act_bytes = i4_align256(P.info_off + (size_t)P.npairs * kI4InfoBytesPerPair);
     P.blocks = (N + kI4SplitRows - 1) / kI4SplitRows;
     const size_t per_pair = kI4FragBytesPerPair + kI4InfoBytesPerPair;
     const size_t ring = (size_t)kI4SplitWarps * kI4WarpRing;
     // enough CTAs for several per SM, and each CTA's activation slice in smem
-    int S = (int)std::min<long long>(kI4MaxCluster, std::max<long long>(1, (4LL * sms + P.blocks - 1) / P.blocks));
-    S = std::max(S, (P.npairs + kI4Stages - 1) / kI4Stages);  // whole slice in flight when possible
+    int S = (int)std::min<long long>(
+        kI4MaxCluster, std::max<long long>(1, ((long long)LOWBIT_I4_CTAS_PER_SM * sms + P.blocks - 1) / P.blocks));
+    if (LOWBIT_I4_FILL) S = std::max(S, (P.npairs + kI4Stages - 1) / kI4Stages);  // whole slice in flight
     S = std::min(std::min(S, kI4MaxCluster), P.npairs);
     while (true) {
         P.L = (P.npairs + S - 1) / S;
         P.nslices = (P.npairs + P.L - 1) / P.L;
         P.act_smem = ((size_t)P.L * per_pair + 15) & ~size_t(15);
-        P.smem = P.act_smem + ring;
+        P.smem = P.act_smem + ring + kI4BuildScratch;
         if (P.smem <= (size_t)kI4MaxSmem || S >= kI4MaxCluster) break;
         S = std::min(kI4MaxCluster, S * 2);
     }
@@ -376,21 +375,18 @@ static int i4_num_sms()
 }
 
 bool i4m1_supported(int N, int K) { return i4_plan(N, K, i4_num_sms()).ok; }
-size_t i4m1_act_bytes(int K) { return i4_plan(1, K, 148).act_bytes; }
 
 lowbit_status i4m1_launch(const uint8_t *q, const uint16_t *scales, const uint16_t *x, float *y, int N, int K,
-                          void *act, cudaStream_t st)
+                          cudaStream_t st)
 {
+    // one launch: every CTA turns its K-slice of x into fragments itself
     const I4Plan P = i4_plan(N, K, i4_num_sms());
-    cudaError_t e = launch_pdl(k_i4_prep_m1, dim3(P.npairs), dim3(128), 0, st, x, K, static_cast<uint8_t *>(act),
-                               P.info_off);
-    if (e != cudaSuccess) return LOWBIT_ERR_CUDA;
+    cudaError_t e;
     I4Params p = {};
+    p.x = x;
     p.q = q;
     p.scales = scales;
     p.y = y;
-    p.act = static_cast<const uint8_t *>(act);
-    p.info_off = P.info_off;
     p.N = N;
     p.K = K;
     p.npairs = P.npairs;

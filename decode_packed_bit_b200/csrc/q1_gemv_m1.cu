@@ -203,6 +203,7 @@ constexpr int kQ1SplitWarps = 4;
 
 struct Q1Params {
     const uint8_t *act;
+    const uint16_t *x;  // split kernel: build the activation from x itself (act unused)
     size_t info_off;
     int R, N, K, nchunks;
     int L;              // chunks per K-slice (split kernel) or nchunks (stream kernel)
@@ -379,6 +380,72 @@ __device__ __forceinline__ void stage_act(uint8_t *smem, const Q1Params &p, int 
     for (int i = threadIdx.x; i < n; i += blockDim.x) idst[i] = __ldg(isrc + i);
 }
 
+constexpr int kQ1BuildScratch = kQ1SplitWarps * 4 * 256;  // limb scratch of the fused split kernel
+
+// The work of k_q1_prep_m1 for one 256-k chunk, done by one warp: lane l
+// takes k = 256 ch + 32 j + l (j = 0..7; j < 4 is the chunk's first group),
+// so every per-group reduction is a warp shuffle.  lw: this warp's limb
+// scratch (4 x 256 bytes).
+__device__ __forceinline__ void q1_build_chunk_warp(const uint16_t *__restrict__ x, int K, int ch, uint8_t *frag,
+                                                    float2 *info, int8_t (*lw)[256], int lane)
+{
+    float xv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int k = ch * kQ1ChunkK + 32 * j + lane;
+        xv[j] = k < K ? bf16_bits_to_float(x[k]) : 0.f;
+    }
+    float m[2] = {0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m[j >> 2] = fmaxf(m[j >> 2], fabsf(xv[j]));
+    int E[2], T[2] = {0, 0};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float mh = warp_max(m[h]);
+        const int e8 = (int)((__float_as_uint(mh) >> 23) & 0xFFu);
+        E[h] = max(e8 == 0 ? kQ1MinExp : e8 - 126, kQ1MinExp);  // smallest E with max|x| < 2^E
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int X = __float2int_rn(ldexpf(xv[j], 23 - E[j >> 2]));  // |X| <= 2^23
+        T[j >> 2] += X;
+        const int B = X * (1 << (7 - (lane & 7)));                    // k & 7 == lane & 7
+        const int l0 = (int)(int8_t)(B & 0xFF);
+        int r = (B - l0) >> 8;
+        const int l1 = (int)(int8_t)(r & 0xFF);
+        r = (r - l1) >> 8;
+        const int l2 = (int)(int8_t)(r & 0xFF);
+        lw[0][32 * j + lane] = (int8_t)l0;
+        lw[1][32 * j + lane] = (int8_t)l1;
+        lw[2][32 * j + lane] = (int8_t)l2;
+        lw[3][32 * j + lane] = (int8_t)((r - l2) >> 8);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int Th = warp_sum_int(T[h]);  // |T| <= 2^30
+        if (lane == 0)
+            info[h] = (2 * ch + h) * 128 < K ? make_float2(ldexpf(1.0f, E[h] - 29), ldexpf((float)Th, E[h] - 23))
+                                             : make_float2(0.f, 0.f);
+    }
+    __syncwarp();
+    // fragment words: the same layout as k_q1_prep_m1 writes
+    const int n = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t w[2] = {0u, 0u};
+        if ((n >> 2) == (t >> 1)) {
+            const int8_t *lb = lw[n & 3];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    w[j] |= (uint32_t)(uint8_t)lb[64 * t + 32 * j + 8 * c + i] << (8 * c);
+        }
+        reinterpret_cast<uint2 *>(frag)[32 * i + lane] = make_uint2(w[0], w[1]);
+    }
+    __syncwarp();  // the scratch is reused for the warp's next chunk
+}
+
 // Final per-cell reduction: lanes tq = 0..3 of a row group hold the two
 // groups' low/high limb partials; lane tq writes row g + 8*(tq&1) of tile
 // tq>>1 into out(tile, row).
@@ -496,7 +563,16 @@ __device__ __forceinline__ float ld_cluster_f32(const float *local, unsigned ran
     return v;
 }
 
-constexpr int kQ1SplitStages = 6;  // a split warp's whole K-slice in flight
+#ifndef LOWBIT_Q1_SPLIT_STAGES
+#define LOWBIT_Q1_SPLIT_STAGES 3
+#endif
+#ifndef LOWBIT_Q1_SPLIT_CTAS_PER_SM
+#define LOWBIT_Q1_SPLIT_CTAS_PER_SM 2
+#endif
+#ifndef LOWBIT_Q1_SPLIT_FILL
+#define LOWBIT_Q1_SPLIT_FILL 0
+#endif
+constexpr int kQ1SplitStages = LOWBIT_Q1_SPLIT_STAGES;  // steps of a split warp in flight
 constexpr int kQ1SplitRing = kQ1SplitStages * kQ1StageBytes;
 
 constexpr int kQ1SplitRows = kQ1SplitWarps * kQ1StepRows;  // rows of one CTA
@@ -531,7 +607,20 @@ __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid
     for (int t = 0; t < kQ1SplitStages - 1; ++t) issue_next();
 
     pdl_wait_primary();
-    if (ch_hi > ch_lo) stage_act(smem, p, ch_lo, ch_hi - ch_lo);
+    if (ch_hi > ch_lo) {
+        const int n = ch_hi - ch_lo;
+        if (p.x != nullptr) {
+            // fused: each warp turns its share of the slice's chunks of x into fragments
+            int8_t(*lw)[256] = reinterpret_cast<int8_t(*)[256]>(smem + p.act_smem + kQ1SplitWarps * kQ1SplitRing +
+                                                                 warp * 4 * 256);
+            float2 *info = reinterpret_cast<float2 *>(smem + (size_t)n * kQ1FragBytesPerChunk);
+            for (int c = warp; c < n; c += kQ1SplitWarps)
+                q1_build_chunk_warp(p.x, p.K, ch_lo + c, smem + (size_t)c * kQ1FragBytesPerChunk, info + 2 * c, lw,
+                                    lane);
+        } else {
+            stage_act(smem, p, ch_lo, n);
+        }
+    }
     __syncthreads();
 
     const LaneConst lc = lane_const(lane);
@@ -620,14 +709,16 @@ static Q1Plan q1_plan(int R, int N, int K, int sms)
     P.stream = false;
     const size_t ring_split = (size_t)kQ1SplitWarps * kQ1SplitRing;
     const long long blocks = (long long)R * ((N + kQ1SplitRows - 1) / kQ1SplitRows);
-    int S = (int)std::min<long long>(kQ1MaxCluster, std::max<long long>(1, (4LL * sms + blocks - 1) / blocks));
-    S = std::max(S, (P.nchunks + kQ1StepChunks * kQ1SplitStages - 1) / (kQ1StepChunks * kQ1SplitStages));
+    int S = (int)std::min<long long>(
+        kQ1MaxCluster, std::max<long long>(1, ((long long)LOWBIT_Q1_SPLIT_CTAS_PER_SM * sms + blocks - 1) / blocks));
+    if (LOWBIT_Q1_SPLIT_FILL)  // whole slice in flight
+        S = std::max(S, (P.nchunks + kQ1StepChunks * kQ1SplitStages - 1) / (kQ1StepChunks * kQ1SplitStages));
     S = std::min(std::min(S, kQ1MaxCluster), P.nchunks);
     while (true) {
         P.L = (P.nchunks + S - 1) / S;
         P.nslices = (P.nchunks + P.L - 1) / P.L;
         P.act_smem = ((size_t)P.L * per_chunk + 15) & ~size_t(15);
-        P.smem = P.act_smem + ring_split;
+        P.smem = P.act_smem + ring_split + kQ1BuildScratch;
         if (P.smem <= (size_t)kQ1MaxSmem || S >= kQ1MaxCluster) break;
         S = std::min(kQ1MaxCluster, S * 2);
     }
@@ -668,11 +759,10 @@ lowbit_status q1m1_prepare_launch(const uint16_t *x, int K, void *act, cudaStrea
     return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
 
-lowbit_status q1m1_gemv_launch(const uint8_t *const *bits, const uint16_t *const *scales, const void *act,
-                               float *const *y, int R, int N, int K, cudaStream_t st)
+static lowbit_status q1m1_launch(const Q1Plan &P, const uint8_t *const *bits, const uint16_t *const *scales,
+                                 const void *act, const uint16_t *x, float *const *y, int R, int N, int K,
+                                 cudaStream_t st)
 {
-    if (use_tc(K)) return q1tc_gemv_launch(bits, scales, act, y, R, N, K, st);
-    const Q1Plan P = q1_plan(R, N, K, num_sms());
     Q1Group grp;
     for (int r = 0; r < R; ++r) {
         grp.bits[r] = bits[r];
@@ -681,6 +771,7 @@ lowbit_status q1m1_gemv_launch(const uint8_t *const *bits, const uint16_t *const
     }
     Q1Params p = {};
     p.act = static_cast<const uint8_t *>(act);
+    p.x = x;
     p.info_off = P.info_off;
     p.R = R;
     p.N = N;
@@ -714,6 +805,25 @@ lowbit_status q1m1_gemv_launch(const uint8_t *const *bits, const uint16_t *const
     cfg.numAttrs = na;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, grp, p);
     return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
+lowbit_status q1m1_gemv_launch(const uint8_t *const *bits, const uint16_t *const *scales, const void *act,
+                               float *const *y, int R, int N, int K, cudaStream_t st)
+{
+    if (use_tc(K)) return q1tc_gemv_launch(bits, scales, act, y, R, N, K, st);
+    return q1m1_launch(q1_plan(R, N, K, num_sms()), bits, scales, act, nullptr, y, R, N, K, st);
+}
+
+// One matrix straight from x, in one launch (the split kernel builds its
+// slice of the activation itself).  LOWBIT_ERR_UNSUPPORTED_SHAPE when the
+// shape takes the stream kernel, which needs a prepared activation.
+lowbit_status q1m1_gemv_fused_launch(const uint8_t *bits, const uint16_t *scales, const uint16_t *x, float *y, int N,
+                                     int K, cudaStream_t st)
+{
+    if (use_tc(K) || !q1m1_shape_supported(1, N, K)) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    const Q1Plan P = q1_plan(1, N, K, num_sms());
+    if (P.stream) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    return q1m1_launch(P, &bits, &scales, nullptr, x, &y, 1, N, K, st);
 }
 
 }  // namespace lowbit

@@ -194,7 +194,9 @@ lowbit_status lowbit_q1g128_gemv_noalloc(const uint8_t *w_bits, const uint16_t *
  * dequantises each weight tile into shared memory as two exact bf16 halves
  * (hi + lo = q*d) and accumulates in TMEM; otherwise a CUDA-core kernel.
  * workspace: at least lowbit_int4g64_workspace_bytes(M, N, K) bytes (NULL
- * allowed when that is 0).
+ * allowed when that is 0, which it is for every shape today: each kernel
+ * builds its operands in shared memory; the argument is kept so that a
+ * kernel needing scratch can be added without changing the call).
  * ------------------------------------------------------------------------- */
 size_t lowbit_int4g64_workspace_bytes(int M, int N, int K);
 lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales,
