@@ -24,6 +24,8 @@ int i4tc_fault_flag();
 int q1tc_fault_flag();
 lowbit_status i4m1_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, cudaStream_t);
 lowbit_status q1m1_prepare_launch(const uint16_t *, int, void *, cudaStream_t);
+bool q1sm_supported(int M, int N, int K);
+lowbit_status q1sm_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 lowbit_status q1m1_gemv_fused_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
                                      cudaStream_t);
 lowbit_status q1m1_gemv_launch(const uint8_t *const *, const uint16_t *const *, const void *, float *const *,
@@ -163,6 +165,7 @@ lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales
         if (s != LOWBIT_OK) return s;
         return q1m1_gemv_launch(&w_bits, &w_scales, act, &y, 1, N, K, st);
     }
+    if (M >= 2 && q1sm_supported(M, N, K)) return q1sm_launch(w_bits, w_scales, x, y, M, N, K, st);
     return q1_gemv_simt_launch(w_bits, w_scales, x, y, M, N, K, st);
 }
 
@@ -200,8 +203,11 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits, const u
     LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
     cudaStream_t st = as_stream(stream);
     if (q1_tc_path(R, M, N, K)) return q1m1_gemv_launch(w_bits, w_scales, act, y, R, N, K, st);
+    const bool sm = M >= 2 && q1sm_supported(M, N, K);
     for (int r = 0; r < R; ++r) {
-        s = q1_gemv_simt_launch(w_bits[r], w_scales[r], q1_simt_x(act, M, K), y[r], M, N, K, st);
+        const uint16_t *xr = q1_simt_x(act, M, K);
+        s = sm ? q1sm_launch(w_bits[r], w_scales[r], xr, y[r], M, N, K, st)
+               : q1_gemv_simt_launch(w_bits[r], w_scales[r], xr, y[r], M, N, K, st);
         if (s != LOWBIT_OK) return s;
     }
     return LOWBIT_OK;

@@ -21,6 +21,8 @@ lowbit_status q1m1_gemv_launch(const uint8_t *const *, const uint16_t *const *, 
                                int, int, int, cudaStream_t);
 lowbit_status q1_gemv_simt_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int,
                                   cudaStream_t);
+bool q1sm_supported(int M, int N, int K);
+lowbit_status q1sm_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 }  // namespace lowbit
 
 using namespace lowbit;
@@ -62,6 +64,7 @@ extern "C" lowbit_status lowbit_q1g128_gemv_noalloc(const uint8_t *w_bits, const
     if (!aligned16(w_bits) || !aligned16(w_scales) || !aligned16(x) || !aligned16(y)) return LOWBIT_ERR_MISALIGNED;
     cudaStream_t st = as_stream(stream);
     // Only the M = 1 tensor-core path needs scratch; the others read x directly.
+    if (M >= 2 && q1sm_supported(M, N, K)) return q1sm_launch(w_bits, w_scales, x, y, M, N, K, st);
     if (M != 1 || !q1m1_shape_supported(1, N, K)) return q1_gemv_simt_launch(w_bits, w_scales, x, y, M, N, K, st);
     if (K > kNoAllocMaxK || q1m1_act_bytes(K) > kNoAllocScratchBytes) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
     void *scratch = nullptr;

@@ -103,6 +103,23 @@ def test_q1_small_full_compare(lb, M, N, K):
     check_float(y, y64, ab, f"q1 M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("M", [2, 7, 8, 9, 16])
+@pytest.mark.parametrize("N,K", [(129, 256), (1000, 2048), (300, 5120), (77, 17408)])
+def test_q1_small_batch_tensor_core(lb, M, N, K):
+    """2 <= M <= 16 with K % 256 == 0 takes the bf16 tensor-core kernel: one
+    or two batch tiles, ragged row blocks, one or several K slices."""
+    bits, scales, x = _q1_problem(1700 + M, M, N, K)
+    y = _run_q1(lb, bits, scales, x, N)
+    if N * K <= 1000 * 2048:
+        y64, ab = oracle.q1_gemv(bits, scales, x, want_abs=True)
+        check_float(y, y64, ab, f"q1 small-M M={M} N={N} K={K}")
+    else:
+        ms, ns = sample_pairs(M, N, 160, M)
+        y64, ab = oracle.q1_gemv_at(bits, scales, x, ms, ns)
+        check_float(y[ms, ns], y64, ab, f"q1 small-M M={M} N={N} K={K}")
+    assert np.isfinite(y).all()
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_q1_prepared_activation_matches_direct(lb, M):
     N, K = 515, 1280
