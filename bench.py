@@ -142,11 +142,13 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """The largest of every rank's v (a device time): one all-reduce of a
+    scalar, on the GPU under NCCL, on the host under gloo."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
