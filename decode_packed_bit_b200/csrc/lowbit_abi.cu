@@ -25,6 +25,10 @@ int q1tc_fault_flag();
 lowbit_status i4m1_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, cudaStream_t);
 lowbit_status q1m1_prepare_launch(const uint16_t *, int, void *, cudaStream_t);
 bool q1sm_supported(int M, int N, int K);
+lowbit_status q1stack_launch(const uint8_t *const *, const uint16_t *const *, int, int, int, uint16_t *, float, void *,
+                             uint16_t *, float *, cudaStream_t);
+size_t q1stack_workspace_bytes(int F);
+int q1stack_fault_flag();
 lowbit_status q1sm_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 lowbit_status q1m1_gemv_fused_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
                                      cudaStream_t);
@@ -70,9 +74,9 @@ int lowbit_version(void) { return 100; }
 
 int lowbit_fault_flags(void)
 {
-    const int f4 = i4tc_fault_flag(), f1 = q1tc_fault_flag();
-    if (f4 < 0 || f1 < 0) return -1;
-    return (f4 ? 1 : 0) | (f1 ? 2 : 0);
+    const int f4 = i4tc_fault_flag(), f1 = q1tc_fault_flag(), fs = q1stack_fault_flag();
+    if (f4 < 0 || f1 < 0 || fs < 0) return -1;
+    return (f4 ? 1 : 0) | (f1 ? 2 : 0) | (fs ? 4 : 0);
 }
 
 lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, int64_t cols,
@@ -219,6 +223,32 @@ lowbit_status lowbit_q1g128_gemv_act(const uint8_t *w_bits, const uint16_t *w_sc
 {
     return lowbit_q1g128_gemv_act_group(&w_bits, &w_scales, act, &y, 1, M, N, K, workspace, workspace_bytes,
                                         stream);
+}
+
+size_t lowbit_q1g128_stack_workspace_bytes(int n_layers, int hidden, int ffn)
+{
+    if (n_layers < 1 || hidden < 1 || ffn < 1) return 0;
+    return al256(q1stack_workspace_bytes(ffn));
+}
+
+lowbit_status lowbit_q1g128_stack_step(const uint8_t *const *w_bits, const uint16_t *const *w_scales, int n_layers,
+                                       int hidden, int ffn, uint16_t *x, float eps, void *workspace,
+                                       size_t workspace_bytes, uint16_t *record_inputs, float *record_outputs,
+                                       void *stream)
+{
+    LB_CHECK(w_bits && w_scales && x && workspace, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(n_layers >= 1 && n_layers <= 73 && hidden >= 1 && ffn >= hidden && eps >= 0.f, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(hidden % 1024 == 0 && ffn % 1024 == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    LB_CHECK(workspace_bytes >= lowbit_q1g128_stack_workspace_bytes(n_layers, hidden, ffn), LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(x) && aligned16(workspace), LOWBIT_ERR_MISALIGNED);
+    LB_CHECK(record_inputs == nullptr || aligned16(record_inputs), LOWBIT_ERR_MISALIGNED);
+    LB_CHECK(record_outputs == nullptr || aligned16(record_outputs), LOWBIT_ERR_MISALIGNED);
+    for (int i = 0; i < 7 * n_layers; ++i) {
+        LB_CHECK(w_bits[i] && w_scales[i], LOWBIT_ERR_INVALID_ARG);
+        LB_CHECK(aligned16(w_bits[i]) && aligned16(w_scales[i]), LOWBIT_ERR_MISALIGNED);
+    }
+    return q1stack_launch(w_bits, w_scales, n_layers, hidden, ffn, x, eps, workspace, record_inputs, record_outputs,
+                          as_stream(stream));
 }
 
 // ---------------------------------------------------------------------------

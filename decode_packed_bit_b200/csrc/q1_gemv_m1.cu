@@ -44,6 +44,7 @@
 //     cluster, and their partial sums are added in fixed rank order through
 //     distributed shared memory (deterministic, no global scratch).
 #include <algorithm>
+#include <mutex>
 
 #include "q1_common.cuh"
 
@@ -446,6 +447,13 @@ __device__ __forceinline__ void q1_build_chunk_warp(const uint16_t *__restrict__
     __syncwarp();  // the scratch is reused for the warp's next chunk
 }
 
+__device__ __forceinline__ unsigned long long globaltimer_ns_q1()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Final per-cell reduction: lanes tq = 0..3 of a row group hold the two
 // groups' low/high limb partials; lane tq writes row g + 8*(tq&1) of tile
 // tq>>1 into out(tile, row).
@@ -824,6 +832,398 @@ lowbit_status q1m1_gemv_fused_launch(const uint8_t *bits, const uint16_t *scales
     const Q1Plan P = q1_plan(1, N, K, num_sms());
     if (P.stream) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
     return q1m1_launch(P, &bits, &scales, nullptr, x, &y, 1, N, K, st);
+}
+
+
+// ---------------------------------------------------------------------------
+// one decode step through a stack of Q1_0_g128 projections, in one launch
+// ---------------------------------------------------------------------------
+//
+// Per layer: q, k, v, o (hidden -> hidden), gate and up (hidden -> ffn, the
+// same input, outputs summed before the next normalisation), down (ffn ->
+// hidden); each projection's input is bf16(RMSNorm(previous fp32 output)),
+// unit gain; the layer's output, normalised, is the next layer's input.
+// The step runs as 6 phases per layer in one cooperative launch (every CTA
+// resident), separated by a grid barrier: a global counter every CTA adds to
+// once per phase, waited on with a bounded spin.  In a phase every CTA
+//   1. normalises the previous phase's output (it reads all of it) and turns
+//      its own 1024-k slice into B fragments (four warps, one 256-k chunk
+//      each);
+//   2. its warps run (32-row block, slice) units through the same mma.sync
+//      inner loop as the split kernel and add each unit's partial sums into
+//      the phase's output with fp32 atomics (outputs rotate through three
+//      buffers: the one two phases ahead is zeroed meanwhile);
+// while the warps' cp.async rings keep fetching the next units' weights
+// across the phase boundaries (weights never depend on activations).
+
+constexpr int kStWarps = 16;
+constexpr int kStThreads = kStWarps * 32;
+constexpr int kStSliceK = 1024;                 // k per slice: four 256-k chunks
+constexpr int kStSliceChunks = kStSliceK / kQ1ChunkK;
+constexpr int kStStages = 3;
+constexpr int kStMaxProj = 512;
+constexpr int kStPhasesPerLayer = 6;
+constexpr unsigned long long kStWaitNs = 2000000000ull;
+
+__device__ unsigned g_q1stack_fault;  // set when a grid-barrier wait ran out
+
+struct StackW {
+    const uint8_t *bits[kStMaxProj];     // projection 7 l + {q, k, v, o, gate, up, down}
+    const uint16_t *scales[kStMaxProj];
+};
+
+struct StackP {
+    uint16_t *x;         // [H] bf16: the step input, then its output
+    float *buf;          // 3 x [2F] fp32 phase outputs
+    unsigned *bar;       // grid barrier counter (zero at launch)
+    uint16_t *rec_in;    // optional [7L][F] bf16: every projection's input
+    float *rec_out;      // optional [7L][F] fp32: every projection's output
+    int L, H, F;
+    float eps;
+};
+
+struct StPhase {
+    int ph, layer, K, N, nblocks, nmat;  // nmat: 1, or 2 for gate+up (rows of up follow those of gate)
+};
+
+__device__ __forceinline__ StPhase st_phase(const StackP &p, int ph_idx)
+{
+    StPhase q;
+    q.layer = ph_idx / kStPhasesPerLayer;
+    q.ph = ph_idx % kStPhasesPerLayer;
+    q.K = q.ph == 5 ? p.F : p.H;
+    q.N = q.ph == 4 ? p.F : (q.ph == 5 ? p.H : p.H);
+    q.nmat = q.ph == 4 ? 2 : 1;
+    q.nblocks = q.nmat * q.N / 32;
+    return q;
+}
+
+__device__ __forceinline__ int st_proj(const StPhase &q, int mat) { return 7 * q.layer + (q.ph < 4 ? q.ph : (q.ph == 4 ? 4 + mat : 6)); }
+
+// A warp's position in its sequence of steps (phase, j-th unit of the warp
+// in that phase, step t of the unit).
+struct StIt {
+    int p, j, t;
+};
+
+// Block of unit j of warp `warp` of CTA `c` in phase q, or -1.
+__device__ __forceinline__ int st_block(const StPhase &q, int G, int c, int warp, int j)
+{
+    const int S = q.K / kStSliceK;
+    const int s = c % S, rk = c / S;
+    const int cps = (G - 1 - s) / S + 1;  // CTAs that work on slice s
+    const int b = rk + cps * (warp + j * kStWarps);
+    return b < q.nblocks ? b : -1;
+}
+
+// Move to the next step that exists (or past the last phase).
+__device__ __forceinline__ void st_next(StIt &it, const StackP &p, int G, int c, int warp, int nph)
+{
+    if (++it.t < kStSliceChunks / kQ1StepChunks) return;
+    it.t = 0;
+    ++it.j;
+    while (it.p < nph && st_block(st_phase(p, it.p), G, c, warp, it.j) < 0) {
+        ++it.p;
+        it.j = 0;
+    }
+}
+
+__device__ __forceinline__ void st_first(StIt &it, const StackP &p, int G, int c, int warp, int nph)
+{
+    it.p = 0;
+    it.j = 0;
+    it.t = 0;
+    while (it.p < nph && st_block(st_phase(p, it.p), G, c, warp, 0) < 0) ++it.p;
+}
+
+// Copy one step: 32 rows x 2 chunks of one matrix (all rows and chunks exist).
+__device__ __forceinline__ void st_issue(unsigned stage, const StackW &W, const StackP &p, const StIt &it, int G,
+                                         int c, int warp, int lane)
+{
+    const StPhase q = st_phase(p, it.p);
+    const int b = st_block(q, G, c, warp, it.j);
+    const int mat = b / (q.N / 32), row0 = (b % (q.N / 32)) * 32;
+    const int pi = st_proj(q, mat);
+    const int ch0 = (c % (q.K / kStSliceK)) * kStSliceChunks + it.t * kQ1StepChunks;
+    const int rowbytes = q.K >> 3, G16 = q.K >> 7;
+    const int col = lane & 3;
+    const uint8_t *bsrc = W.bits[pi] + (size_t)(row0 + (lane >> 2)) * rowbytes + ch0 * 32 + col * 16;
+    const unsigned bdst = stage + (lane >> 2) * kQ1RowStride + col * 16;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) cp_async16(bdst + 8 * u * kQ1RowStride, bsrc + (size_t)(8 * u) * rowbytes, true);
+    const int sc = lane & 1;
+    const uint16_t *ssrc = W.scales[pi] + (size_t)(row0 + (lane >> 1)) * G16 + 2 * (ch0 + sc);
+    const unsigned sdst = stage + kQ1StageW + (lane >> 1) * 8 + sc * 4;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) cp_async4(sdst + 16 * u * 8, ssrc + (size_t)(16 * u) * G16, true);
+}
+
+// Bring phase ph's weights into L2 ahead of time: CTA c takes blocks c,
+// c + G, ...; a block's 32 rows of signs (and of scales) are contiguous.
+constexpr int kStPrefetchAhead = 2;  // phases
+
+__device__ __forceinline__ void st_prefetch_l2(const StackW &W, const StackP &p, int ph, int G, int c)
+{
+    if (ph >= p.L * kStPhasesPerLayer) return;
+    const StPhase q = st_phase(p, ph);
+    const unsigned bbytes = 32u * (unsigned)(q.K / 8), sbytes = 32u * (unsigned)(q.K / 128) * 2u;
+    for (int b = c + G * (int)threadIdx.x; b < q.nblocks; b += G * kStThreads) {
+        const int mat = b / (q.N / 32), row0 = (b % (q.N / 32)) * 32;
+        const int pi = st_proj(q, mat);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(W.bits[pi] + (size_t)row0 * (q.K / 8)),
+                     "r"(bbytes)
+                     : "memory");
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(W.scales[pi] + (size_t)row0 * (q.K / 128)),
+                     "r"(sbytes)
+                     : "memory");
+    }
+}
+
+__device__ __forceinline__ float st_block_sum(float v, float *red)
+{
+    v = warp_sum(v);
+    __syncthreads();  // red is free
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kStWarps; ++w) t += red[w];
+    return t;
+}
+
+// Grid barrier: every CTA adds 1 per phase; wait until all G have.
+__device__ __forceinline__ void st_grid_sync(const StackP &p, unsigned target)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(p.bar, 1u);
+        unsigned v = 0;
+        const unsigned long long t0 = globaltimer_ns_q1();
+        while (true) {
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.bar) : "memory");
+            if (v >= target) break;
+            // after one wait has run out the results are void: do not wait again
+            if (*reinterpret_cast<volatile unsigned *>(&g_q1stack_fault) != 0u) break;
+            if (globaltimer_ns_q1() - t0 > kStWaitNs) {
+                atomicExch(&g_q1stack_fault, 1u);
+                break;
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_constant__ StackW W, const StackP p)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ float red[kStWarps];
+    uint8_t *frag = smem;                                                  // 4 chunks of fragments
+    float2 *info = reinterpret_cast<float2 *>(smem + kStSliceChunks * kQ1FragBytesPerChunk);
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem + kStSliceChunks * kQ1FragBytesPerChunk + 256);
+    int8_t(*lwall)[256] = reinterpret_cast<int8_t(*)[256]>(reinterpret_cast<uint8_t *>(xs) + kStSliceK * 2);
+    float *xsf = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(lwall) + 4 * 4 * 256);  // raw slice values
+    uint8_t *rings = reinterpret_cast<uint8_t *>(xsf) + kStSliceK * 4;
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int nph = p.L * kStPhasesPerLayer;
+    const size_t bufn = 2 * (size_t)p.F;
+    uint8_t *ring = rings + warp * kStStages * kQ1StageBytes;
+    const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
+
+    for (int ph = 0; ph < kStPrefetchAhead; ++ph) st_prefetch_l2(W, p, ph, G, c);
+    StIt is;  // issue position (runs up to kStStages - 1 steps ahead)
+    st_first(is, p, G, c, warp, nph);
+    int nis = 0;
+    auto issue_next = [&]() {
+        if (is.p < nph) {
+            st_issue(ring_s + (nis % kStStages) * kQ1StageBytes, W, p, is, G, c, warp, lane);
+            st_next(is, p, G, c, warp, nph);
+        }
+        ++nis;
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int t = 0; t < kStStages - 1; ++t) issue_next();
+
+    pdl_wait_primary();  // x is produced by earlier kernels
+    const LaneConst lc = lane_const(lane);
+    StIt cs;  // consume position
+    st_first(cs, p, G, c, warp, nph);
+    int ncs = 0;
+
+    for (int ph_idx = 0; ph_idx <= nph; ++ph_idx) {
+        st_prefetch_l2(W, p, ph_idx + kStPrefetchAhead, G, c);
+        // ---- input of this phase: normalise the previous output (or take x) ----
+        const bool last = ph_idx == nph;
+        const StPhase q = st_phase(p, last ? nph - 1 : ph_idx);
+        const int Kin = last ? p.H : q.K;
+        const float *prev = ph_idx > 0 ? p.buf + (size_t)((ph_idx - 1) % 3) * bufn : nullptr;
+        // down reads gate + up: kept apart only when they are recorded, else
+        // the gate+up phase adds both into one vector
+        const bool two = !last && q.ph == 5 && p.rec_out != nullptr;
+        float inv = 1.f;
+        const int S = q.K / kStSliceK, s = c % S;
+        if (prev != nullptr) {
+            // sum of squares of the whole input, 16 loads in flight per thread;
+            // this CTA's slice is kept on the way (raw, scaled once inv is known)
+            const int sl0 = last ? -1 : s * (kStSliceK / 4), sl1 = sl0 + kStSliceK / 4;
+            float ss = 0.f;
+            const int n4 = Kin / 4;
+            const float4 *a4 = reinterpret_cast<const float4 *>(prev);
+            const float4 *b4 = reinterpret_cast<const float4 *>(prev + p.F);
+            for (int base = threadIdx.x; base < n4; base += 16 * kStThreads) {
+                float4 v[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int i = base + u * kStThreads;
+                    v[u] = i < n4 ? a4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                if (two) {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int i = base + u * kStThreads;
+                        if (i < n4) {
+                            const float4 w = b4[i];
+                            v[u].x += w.x; v[u].y += w.y; v[u].z += w.z; v[u].w += w.w;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int i = base + u * kStThreads;
+                    if (i >= sl0 && i < sl1) reinterpret_cast<float4 *>(xsf)[i - sl0] = v[u];
+                    ss = fmaf(v[u].x, v[u].x, ss);
+                    ss = fmaf(v[u].y, v[u].y, ss);
+                    ss = fmaf(v[u].z, v[u].z, ss);
+                    ss = fmaf(v[u].w, v[u].w, ss);
+                }
+            }
+            ss = st_block_sum(ss, red);
+            inv = 1.0f / sqrtf(ss / (float)Kin + p.eps);
+        }
+        // the previous phase's outputs, recorded (its buffer is stable until the next phase)
+        if (p.rec_out != nullptr && ph_idx > 0) {
+            const StPhase pq = st_phase(p, ph_idx - 1);
+            for (int m = 0; m < pq.nmat; ++m) {
+                const int pi = st_proj(pq, m);
+                for (int i = c * kStThreads + threadIdx.x; i < pq.N; i += G * kStThreads)
+                    p.rec_out[(size_t)pi * p.F + i] = prev[(size_t)m * p.F + i];
+            }
+        }
+        if (last) {
+            // the step's output: x = bf16(norm(down output)), written by slices of CTAs
+            for (int i = c * kStThreads + threadIdx.x; i < p.H; i += G * kStThreads)
+                p.x[i] = __bfloat16_as_ushort(__float2bfloat16_rn(prev[i] * inv));
+            break;
+        }
+        for (int i = threadIdx.x; i < kStSliceK; i += kStThreads) {
+            const int k = s * kStSliceK + i;
+            uint16_t xb;
+            if (prev == nullptr)
+                xb = p.x[k];
+            else
+                xb = __bfloat16_as_ushort(__float2bfloat16_rn(xsf[i] * inv));  // stored before the block sum
+            xs[i] = xb;
+            if (p.rec_in != nullptr && c < S)  // the first CTA of each slice records it
+                for (int m = 0; m < q.nmat; ++m) p.rec_in[(size_t)st_proj(q, m) * p.F + k] = xb;
+        }
+        // zero the buffer two phases ahead (read last by the previous phase's prologue)
+        {
+            float *z = p.buf + (size_t)((ph_idx + 1) % 3) * bufn;
+            for (size_t i = (size_t)c * kStThreads + threadIdx.x; i < bufn; i += (size_t)G * kStThreads) z[i] = 0.f;
+        }
+        __syncthreads();
+        if (warp < kStSliceChunks)
+            q1_build_chunk_warp(xs - s * kStSliceK, q.K, s * kStSliceChunks + warp,
+                                frag + warp * kQ1FragBytesPerChunk, info + 2 * warp, lwall + 4 * warp, lane);
+        __syncthreads();
+
+        // ---- this warp's units of the phase ----
+        float *out = p.buf + (size_t)(ph_idx % 3) * bufn;
+        const int fold = (q.ph == 4 && p.rec_out == nullptr) ? q.N : 0;  // up's rows land on gate's
+        const float2 *sinfo = info + lc.h;
+        while (cs.p == ph_idx) {
+            float yacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            const int b = st_block(q, G, c, warp, cs.j);
+            for (int t = 0; t < kStSliceChunks / kQ1StepChunks; ++t) {
+                issue_next();
+                cp_async_wait<kStStages - 1>();
+                __syncwarp();
+                const int lch = t * kQ1StepChunks;
+                consume_step(ring + (ncs % kStStages) * kQ1StageBytes, frag + lane * 8 + lch * kQ1FragBytesPerChunk,
+                             sinfo + 2 * lch, kQ1StepChunks, lc, yacc);
+                __syncwarp();
+                ++ncs;
+                st_next(cs, p, G, c, warp, nph);
+            }
+            finish_cell(yacc, lane, [&](int row, float v) {
+                size_t o = (size_t)b * 32 + row;
+                if (fold != 0 && o >= (size_t)fold) o -= fold;
+                atomicAdd(out + o, v);
+            });
+        }
+        st_grid_sync(p, (unsigned)G * (unsigned)(ph_idx + 1));
+    }
+    cp_async_wait<0>();
+}
+
+lowbit_status q1stack_launch(const uint8_t *const *bits, const uint16_t *const *scales, int L, int H, int F,
+                             uint16_t *x, float eps, void *ws, uint16_t *rec_in, float *rec_out, cudaStream_t st)
+{
+    if (L < 1 || 7 * L > kStMaxProj || H % kStSliceK != 0 || F % kStSliceK != 0) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    static StackW W;  // large: kept off the stack
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < 7 * L; ++i) {
+        W.bits[i] = bits[i];
+        W.scales[i] = scales[i];
+    }
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    StackP p = {};
+    p.x = x;
+    p.bar = reinterpret_cast<unsigned *>(w8);
+    p.buf = reinterpret_cast<float *>(w8 + 256);
+    p.rec_in = rec_in;
+    p.rec_out = rec_out;
+    p.L = L;
+    p.H = H;
+    p.F = F;
+    p.eps = eps;
+    const size_t smem = kStSliceChunks * kQ1FragBytesPerChunk + 256 + kStSliceK * 2 + 4 * 4 * 256 + kStSliceK * 4 +
+                        (size_t)kStWarps * kStStages * kQ1StageBytes;
+    if (cudaFuncSetAttribute(k_q1_stack_m1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return LOWBIT_ERR_CUDA;
+    int per_sm = 0, sms = num_sms();
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_q1_stack_m1, kStThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+        return LOWBIT_ERR_CUDA;
+    // the barrier counter and phase 0's output start at zero
+    if (cudaMemsetAsync(w8, 0, 256 + 2 * (size_t)F * 4, st) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms * per_sm);
+    cfg.blockDim = dim3(kStThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barrier cannot deadlock
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_q1_stack_m1, W, p);
+    return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
+size_t q1stack_workspace_bytes(int F) { return 256 + 3 * 2 * (size_t)F * 4; }
+
+int q1stack_fault_flag()
+{
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_q1stack_fault, sizeof(v)) != cudaSuccess) return -1;
+    cudaMemcpyToSymbol(g_q1stack_fault, &zero, sizeof(zero));
+    return (int)v;
 }
 
 }  // namespace lowbit

@@ -46,6 +46,8 @@ SYMBOLS = [
     ("lowbit_int4g64_gemm", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
     ("lowbit_q2_mlp_forward", I32, [P, P, I32, P, I32, P, P, P]),
     ("lowbit_rmsnorm_bf16", I32, [P, P, I32, I32, F32, P, P]),
+    ("lowbit_q1g128_stack_workspace_bytes", SZ, [I32, I32, I32]),
+    ("lowbit_q1g128_stack_step", I32, [P, P, I32, I32, I32, P, F32, P, SZ, P, P, P]),
 ]
 
 _lib = None
@@ -215,3 +217,21 @@ def lowbit_rmsnorm_bf16(a, b, out, eps=1e-6, stream=None):
     M, D = a.shape
     _check(lib().lowbit_rmsnorm_bf16(_ptr(a), _ptr(b), M, D, float(eps), _ptr(out), _stream(stream)),
            "lowbit_rmsnorm_bf16")
+
+
+# -- the fused decode step of a Q1 stack ------------------------------------------
+
+def lowbit_q1g128_stack_workspace_bytes(n_layers: int, hidden: int, ffn: int) -> int:
+    return int(lib().lowbit_q1g128_stack_workspace_bytes(n_layers, hidden, ffn))
+
+
+def lowbit_q1g128_stack_step(w_bits, w_scales, x, hidden, ffn, workspace, eps=1e-6, record_inputs=None,
+                             record_outputs=None, stream=None):
+    """w_bits / w_scales: lists of 7 * n_layers device tensors (q, k, v, o, gate, up, down per layer)."""
+    n = len(w_bits)
+    bits, bits_keep = _ptr_array(w_bits)
+    scales, scales_keep = _ptr_array(w_scales)
+    wsb = workspace.numel() * workspace.element_size()
+    _check(lib().lowbit_q1g128_stack_step(bits, scales, n // 7, hidden, ffn, _ptr(x), float(eps), _ptr(workspace), wsb,
+                                          _ptr(record_inputs), _ptr(record_outputs), _stream(stream)),
+           "lowbit_q1g128_stack_step")

@@ -72,6 +72,45 @@ class Q1Stack:
         per = 5 * 2 + 2 + 6 if self.M == 1 else 7 + 6
         return per * len(self.layers)
 
+    def fused_supported(self) -> bool:
+        return self.M == 1 and self.hidden % 1024 == 0 and self.ffn % 1024 == 0
+
+    def step_fused(self, stream=None, record: StackRecord | None = None):
+        """The same step as step() at M = 1, as one launch of
+        lowbit_q1g128_stack_step (every projection and normalisation inside)."""
+        if not hasattr(self, "_fused_ws"):
+            dev = self.x.device
+            self._fused_ws = torch.empty(
+                lb.lowbit_q1g128_stack_workspace_bytes(len(self.layers), self.hidden, self.ffn), dtype=torch.uint8,
+                device=dev)
+            self._fused_bits = [layer.w[name][0] for layer in self.layers for name in PROJ]
+            self._fused_scales = [layer.w[name][1] for layer in self.layers for name in PROJ]
+        rin = rout = None
+        if record is not None:
+            n = 7 * len(self.layers)
+            rin = torch.zeros((n, self.ffn), dtype=torch.bfloat16, device=self.x.device)
+            rout = torch.zeros((n, self.ffn), dtype=torch.float32, device=self.x.device)
+        lb.lowbit_q1g128_stack_step(self._fused_bits, self._fused_scales, self.x, self.hidden, self.ffn,
+                                    self._fused_ws, eps=self.eps, record_inputs=rin, record_outputs=rout,
+                                    stream=stream)
+        if record is not None:
+            H, F = self.hidden, self.ffn
+            for li in range(len(self.layers)):
+                for pi, name in enumerate(PROJ):
+                    i = 7 * li + pi
+                    K = F if name == "down" else H
+                    N = F if name in ("gate", "up") else H
+                    if not record.want(li, name):
+                        continue
+                    record.inputs[(li, name)] = rin[i, :K].reshape(1, K).clone()
+                    record.outputs[(li, name)] = rout[i, :N].reshape(1, N).clone()
+                    if name in ("q", "k", "v", "o", "down"):
+                        record.norm_in[(li, name)] = rout[i, :N].reshape(1, N).clone()
+                if record.want(li, "gate") or record.want(li, "up"):
+                    record.norm_in[(li, "gate+up")] = (rout[7 * li + 4, :F].reshape(1, F).clone(),
+                                                       rout[7 * li + 5, :F].reshape(1, F).clone())
+        return self.x
+
     def step(self, stream=None, record: StackRecord | None = None):
         """One decode step: self.x (bf16 [M][hidden]) -> self.x."""
         M = self.M

@@ -81,9 +81,10 @@ int lowbit_version(void);
 
 /* Faults the kernels of the current device recorded since the last call,
  * and clears them: 0 = none; bit 0 = a bounded wait inside the INT4_G64
- * tcgen05 GEMM ran out, bit 1 = one inside the Q1_0_g128 tcgen05 product
- * (the results of that call are then not valid); -1 = the flags could not
- * be read.  Synchronises with the device. */
+ * tcgen05 GEMM ran out, bit 1 = one inside the Q1_0_g128 tcgen05 product,
+ * bit 2 = a grid barrier of lowbit_q1g128_stack_step (the results of that
+ * call are then not valid); -1 = the flags could not be read.  Synchronises
+ * with the device. */
 int lowbit_fault_flags(void);
 
 /* ---------------------------------------------------------------------------
@@ -177,6 +178,38 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits,
 lowbit_status lowbit_q1g128_gemv_noalloc(const uint8_t *w_bits, const uint16_t *w_scales,
                                          const uint16_t *x, float *y, int M, int N, int K,
                                          void *stream);
+
+/* ---------------------------------------------------------------------------
+ * One decode step (M = 1) through a stack of Q1_0_g128 linear projections,
+ * in one launch.  The pages fix only the weight format ("Bonsai-27B-gguf
+ * technical white paper digest", "technical architecture highlights") and
+ * that decode streams every layer's weights once per token; the chaining is
+ * this library's reading of the workload: per layer q, k, v, o (hidden ->
+ * hidden), gate and up (hidden -> ffn, same input, outputs summed), down
+ * (ffn -> hidden); every projection's input is bf16_rne(v / sqrt(mean(v^2)
+ * + eps)) of the previous fp32 output (v = gate + up before down), and the
+ * step output is that normalisation of the last down output.  Layer 0's q
+ * reads x as given.
+ *   w_bits, w_scales: HOST arrays of 7 * n_layers device pointers, in the
+ *     order q, k, v, o, gate, up, down for each layer; shapes as for
+ *     lowbit_q1g128_gemv ([N][K/8] and [N][K/128]).
+ *   x: [hidden] bf16, the step input, overwritten with the step output.
+ *   workspace: lowbit_q1g128_stack_workspace_bytes(...) bytes; the call
+ *     initialises what it needs (it enqueues a memset first).
+ *   record_inputs / record_outputs: NULL, or [7 * n_layers][ffn] bf16 /
+ *     fp32 that receive every projection's input and fp32 output (row i
+ *     uses the first K or N entries).
+ * Needs hidden and ffn multiples of 1024, ffn >= hidden, 1 <= n_layers <=
+ * 73.  The kernel is a cooperative launch (every CTA resident) whose phases
+ * are separated by a grid barrier; a barrier wait bounded at 2 s that runs
+ * out sets bit 2 of lowbit_fault_flags().  The projections' partial sums
+ * are added with fp32 atomics, so results can differ in the last bits from
+ * run to run. */
+size_t lowbit_q1g128_stack_workspace_bytes(int n_layers, int hidden, int ffn);
+lowbit_status lowbit_q1g128_stack_step(const uint8_t *const *w_bits, const uint16_t *const *w_scales,
+                                       int n_layers, int hidden, int ffn, uint16_t *x, float eps,
+                                       void *workspace, size_t workspace_bytes,
+                                       uint16_t *record_inputs, float *record_outputs, void *stream);
 
 /* ---------------------------------------------------------------------------
  * INT4_G64 product (acorn-llm 0.11.4, "int4 quantisation quality: group

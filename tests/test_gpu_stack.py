@@ -42,13 +42,16 @@ def _next_input_key(li, name):
     return nxt[name]
 
 
-def _run(stack_weights, M, which):
+def _run(stack_weights, M, which, fused=False):
     from decode_packed_bit_b200.stack import Q1Stack, StackRecord
     st = Q1Stack(stack_weights, H, F, M, "cuda")
     x0 = synth.bf16_normal(synth.SEED_BASE + synth.W_Q1_STACK, (M, H), tag=M)
     st.x.copy_(torch.from_numpy(x0.view(np.int16)).view(torch.bfloat16).cuda())
     rec = StackRecord(which=which)
-    st.step(record=rec)
+    if fused:
+        st.step_fused(record=rec)
+    else:
+        st.step(record=rec)
     torch.cuda.synchronize()
     return st, rec
 
@@ -106,3 +109,23 @@ def test_stack_m8_sampled_layers_teacher_forced(stack_weights):
     _check_projections(stack_weights, rec, 8, rows_per_proj=6, seed=12)
     _check_glue(rec, 8)
     assert torch.isfinite(st.x.float()).all()
+
+
+def test_stack_m1_one_launch_teacher_forced(stack_weights):
+    """lowbit_q1g128_stack_step: all 448 projections and their
+    normalisations in one cooperative launch, checked like the per-call
+    step, plus the step output against the oracle's last normalisation."""
+    from decode_packed_bit_b200 import lowbit as lb
+    st, rec = _run(stack_weights, 1, which=None, fused=True)
+    assert lb.lowbit_fault_flags() == 0
+    assert len(rec.outputs) == 7 * L
+    # layer 0's q input is the step input itself
+    x0 = synth.bf16_normal(synth.SEED_BASE + synth.W_Q1_STACK, (1, H), tag=1)
+    assert np.array_equal(host(rec.inputs[(0, "q")].view(torch.int16)).view(np.uint16), x0)
+    _check_projections(stack_weights, rec, 1, rows_per_proj=12, seed=13)
+    _check_glue(rec, 1)
+    # the step output: the last down output, normalised
+    r64 = oracle.rmsnorm(host(rec.norm_in[(L - 1, "down")]), None, eps=1e-6)
+    got = synth.bf16_bits_to_f32(host(st.x.view(torch.int16)).view(np.uint16)).astype(np.float64)
+    tol = 0.5 * _bf16_ulp(r64) + 1e-6 * np.abs(r64) + 1e-30
+    assert (np.abs(got - r64) <= tol).all()
