@@ -1,5 +1,8 @@
-// q1_gemm_smallm.cu -- Q1_0_g128 products at small batch (2 <= M <= 16) on
-// the bf16 tensor cores (mma.sync m16n8k16, fp32 accumulate).
+// gemm_smallm.cu -- products at small batch on the bf16 tensor cores
+// (mma.sync m16n8k16, fp32 accumulate): Q1_0_g128 for 2 <= M <= 16 and
+// INT4_G64 for 2 <= M <= 32.  Both formats share the work split, the
+// staging of x and the split-K reduction; they differ in how a thread turns
+// its packed weights into exact bf16 A operands.
 //
 // What is computed ("Bonsai-27B-gguf technical white paper digest",
 // "technical architecture highlights": one sign bit per weight, one FP16
@@ -34,8 +37,8 @@ constexpr int kSmStepK = 256;              // k per pipeline step (two groups)
 constexpr int kSmRowStride = 48;           // 32 bytes of signs per row, padded: conflict-free 16-byte reads
 constexpr int kSmStageW = 32 * kSmRowStride;
 constexpr int kSmStageBytes = kSmStageW + 32 * 4;  // + two fp16 scales per row
-constexpr int kSmStages = 4;
-constexpr int kSmRing = kSmStages * kSmStageBytes;
+constexpr int kSmStages = 3;  // weight and x rings (three CTAs fit on an SM)
+static_assert(kSmStages == 3, "the per-step wait depth below assumes a lookahead of two steps");
 constexpr int kSmMaxM = 16;
 constexpr int kSmMaxCluster = 8;
 constexpr int kSmMaxSmem = 220 * 1024;
@@ -48,8 +51,7 @@ struct SmParams {
     int M, N, K;
     int nsteps;  // K / 256
     int L;       // steps per K-slice
-    int NT;      // n8 tiles of the batch: 1 (M <= 8) or 2
-    int xfrag;   // bytes of staged x fragments
+    int NT;      // n8 tiles of the batch (8 vectors each)
 };
 
 __device__ __forceinline__ void sm_cp16(unsigned dst, const void *src, bool valid)
@@ -171,10 +173,131 @@ __device__ __forceinline__ void sm_consume(const uint8_t *stage, const uint2 *xf
     }
 }
 
-// grid: x = K-slice (cluster rank), y = 128-row block
-template <int NT>
-__global__ void __launch_bounds__(kSmWarps * 32) k_q1_smallm(const SmParams p)
+// ---------------------------------------------------------------------------
+// INT4_G64 ("acorn-llm 0.11.4", "int4 quantisation quality: group
+// quantisation"): y[m][n] = sum_g d[n][g] sum_{k in g} q[n][k] x[m][k].
+// A is q as an exact bf16: a thread's four k slots of a 16-k step are the two
+// packed bytes 2t, 2t+1 of the row's 8 bytes (k 4t..4t+3, low nibble first),
+// so B is again x[m][k..k+3].  A byte b becomes the bf16 pair {q_lo, q_hi}:
+// prmt isolates b, b * 0x1001 puts its nibbles at bits 0 and 16, and with the
+// sign bit of each nibble flipped (n ^ 8 = q + 8) and 0x4300 (128.0) or-ed in,
+// each half reads 136 + q exactly; a bf16 subtraction of 136 leaves q.
+// ---------------------------------------------------------------------------
+
+constexpr int kI4sStepK = 128;                // k per pipeline step (two groups of 64)
+constexpr int kI4sRowStride = 80;             // 64 bytes per row, padded: conflict-free 8-byte reads
+constexpr int kI4sStageW = 32 * kI4sRowStride;
+constexpr int kI4sStageBytes = kI4sStageW + 32 * 4;  // + two fp16 scales per row
+constexpr int kI4sMaxM = 32;
+
+// Copy step `st` (128 k) of rows blk*32..+32: lane L copies 16-byte column L%4
+// of rows L/4 + {0, 8, 16, 24}, and the scale pair of row L.
+__device__ __forceinline__ void i4s_issue(unsigned stage, const SmParams &p, int blk, int st, int lane)
 {
+    const int rowbytes = p.K >> 1, G = p.K >> 6;
+    const int col = lane & 3, r0 = blk * 32 + (lane >> 2);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int row = r0 + 8 * u;
+        const bool ok = row < p.N;
+        sm_cp16(stage + ((lane >> 2) + 8 * u) * kI4sRowStride + col * 16,
+                ok ? p.bits + (size_t)row * rowbytes + st * 64 + col * 16 : p.bits, ok);
+    }
+    const int srow = blk * 32 + lane;
+    const bool sok = srow < p.N;
+    sm_cp4(stage + kI4sStageW + lane * 4, sok ? p.scales + (size_t)srow * G + 2 * st : p.scales, sok);
+}
+
+// bf16 pair {q(low nibble), q(high nibble)} of byte `sel` (0..3) of w, exact
+__device__ __forceinline__ uint32_t i4_pair_bf16(uint32_t w, uint32_t sel)
+{
+    const uint32_t b = __byte_perm(w, 0u, sel | 0x4440u);       // the byte alone
+    const uint32_t v = ((b * 0x1001u) & 0x000F000Fu) ^ 0x43084308u;  // 136 + q in each half
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(0x43084308u));  // - 136
+    return r;
+}
+
+template <int NT>
+__device__ __forceinline__ void i4s_consume(const uint8_t *stage, const uint2 *xf, int lane, float (&yacc)[2][NT][4])
+{
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp) {
+        float acc[2][NT][4];
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) acc[tt][nt][0] = acc[tt][nt][1] = acc[tt][nt][2] = acc[tt][nt][3] = 0.f;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const int ks = 4 * grp + s;  // k16 step within the 128-k stage: bytes 8 ks .. 8 ks + 7 of a row
+            uint2 b[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) b[nt] = xf[(ks * NT + nt) * 32 + lane];
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                uint32_t a[2][2];  // [row g / g+8][k 4t..4t+1 / 4t+2..4t+3]
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    // this lane's two bytes: 2t, 2t+1 of the step's 8
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(
+                        stage + (16 * tt + 8 * r + g) * kI4sRowStride + 8 * ks + 4 * (t >> 1));
+                    const uint32_t s0 = 2u * (t & 1);
+                    a[r][0] = i4_pair_bf16(w, s0);
+                    a[r][1] = i4_pair_bf16(w, s0 + 1u);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    hmma(acc[tt][nt], a[0][0], a[1][0], a[0][1], a[1][1], b[nt].x, b[nt].y);
+            }
+        }
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+            const float d0 = f16_bits_to_float(
+                *reinterpret_cast<const uint16_t *>(stage + kI4sStageW + (16 * tt + g) * 4 + 2 * grp));
+            const float d1 = f16_bits_to_float(
+                *reinterpret_cast<const uint16_t *>(stage + kI4sStageW + (16 * tt + 8 + g) * 4 + 2 * grp));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                yacc[tt][nt][0] = fmaf(d0, acc[tt][nt][0], yacc[tt][nt][0]);
+                yacc[tt][nt][1] = fmaf(d0, acc[tt][nt][1], yacc[tt][nt][1]);
+                yacc[tt][nt][2] = fmaf(d1, acc[tt][nt][2], yacc[tt][nt][2]);
+                yacc[tt][nt][3] = fmaf(d1, acc[tt][nt][3], yacc[tt][nt][3]);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// the kernel (both formats)
+// ---------------------------------------------------------------------------
+//
+// grid: x = K-slice (cluster rank), y = 128-row block.  Per pipeline step the
+// CTA's four warps each copy their 32 rows' packed weights into their own
+// ring slot, and all 128 threads copy a share of the step's x fragments
+// (k16 step ks, batch tile nt, lane (g, t) -> x[8 nt + g][k .. k+3], k = 16 ks
+// + 4 t; zeros past the batch) into a CTA-wide ring.  A step is consumed
+// after every thread's copies of it have landed (its own wait, then a CTA
+// barrier), and that barrier also frees the slot of the previous step.
+
+template <int FMT>
+struct SmFmt;
+template <>
+struct SmFmt<1> {
+    static constexpr int kStepK = kSmStepK, kStageBytes = kSmStageBytes;
+};
+template <>
+struct SmFmt<3> {
+    static constexpr int kStepK = kI4sStepK, kStageBytes = kI4sStageBytes;
+};
+
+template <int FMT, int NT>
+__global__ void __launch_bounds__(kSmWarps * 32) k_smallm(const SmParams p)
+{
+    constexpr int kK16 = SmFmt<FMT>::kStepK / 16;
+    constexpr int kSB = SmFmt<FMT>::kStageBytes;
+    constexpr int kXFrags = kK16 * NT * 32;  // uint2 per step
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ uint2 lut[16];
     pdl_launch_dependents();
@@ -182,53 +305,74 @@ __global__ void __launch_bounds__(kSmWarps * 32) k_q1_smallm(const SmParams p)
     const int slice = blockIdx.x, nsl = gridDim.x, rb = blockIdx.y;
     const int blk = rb * kSmWarps + warp;
     const int s_lo = slice * p.L, s_hi = min(p.nsteps, s_lo + p.L);
-    const int nst = blk * 32 < p.N && s_hi > s_lo ? s_hi - s_lo : 0;
-    uint8_t *ring = smem + p.xfrag + warp * kSmRing;
-    const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
-    float *part = reinterpret_cast<float *>(smem + p.xfrag + kSmWarps * kSmRing);  // [M][128]
+    const int ns = max(0, s_hi - s_lo);      // steps of this CTA (the same for all its warps)
+    const bool rows = blk * 32 < p.N;        // this warp has rows
+    uint2 *xr = reinterpret_cast<uint2 *>(smem);                          // x ring: kSmStages x kXFrags
+    uint8_t *wring = smem + (size_t)kSmStages * kXFrags * 8 + warp * kSmStages * kSB;
+    float *part = reinterpret_cast<float *>(smem + (size_t)kSmStages * kXFrags * 8 + kSmWarps * kSmStages * kSB);
+    const unsigned xr_s = (unsigned)__cvta_generic_to_shared(xr);
+    const unsigned wr_s = (unsigned)__cvta_generic_to_shared(wring);
 
-    int ist = 0;
-    auto issue_next = [&]() {
-        if (ist < nst) sm_issue(ring_s + (ist % kSmStages) * kSmStageBytes, p, blk, s_lo + ist, lane);
-        ++ist;
-        sm_commit();
+    auto issue_w = [&](int s) {
+        if (s < ns && rows) {
+            if (FMT == 1)
+                sm_issue(wr_s + (s % kSmStages) * kSB, p, blk, s_lo + s, lane);
+            else
+                i4s_issue(wr_s + (s % kSmStages) * kSB, p, blk, s_lo + s, lane);
+        }
     };
+    auto issue_x = [&](int s) {
+        if (s >= ns) return;
+        const unsigned dst = xr_s + (unsigned)((s % kSmStages) * kXFrags) * 8u;
+        for (int i = threadIdx.x; i < kXFrags; i += kSmWarps * 32) {
+            const int ln = i & 31, nt = (i >> 5) % NT, ks = (i >> 5) / NT;
+            const int m = 8 * nt + (ln >> 2);
+            const int k = (s_lo + s) * SmFmt<FMT>::kStepK + 16 * ks + 4 * (ln & 3);
+            sm_cp8(dst + 8u * i, m < p.M ? p.x + (size_t)m * p.K + k : p.x, m < p.M);
+        }
+    };
+    // weights of the first steps go out before the previous kernel ends; x after it
 #pragma unroll
-    for (int t = 0; t < kSmStages - 1; ++t) issue_next();
-
-    // nibble -> two bf16x2: bit j of the nibble is the sign of k slot 4t + j
-    if (threadIdx.x < 16) {
+    for (int t = 0; t < kSmStages - 1; ++t) {
+        issue_w(t);
+        sm_commit();
+    }
+    if (FMT == 1 && threadIdx.x < 16) {
+        // nibble -> two bf16x2: bit j of the nibble is the sign of k slot 4t + j
         const uint32_t v = threadIdx.x;
-        auto s = [&](int j) -> uint32_t { return ((v >> j) & 1u) ? 0x3F80u : 0xBF80u; };
-        lut[threadIdx.x] = make_uint2(s(0) | (s(1) << 16), s(2) | (s(3) << 16));
+        auto sg = [&](int j) -> uint32_t { return ((v >> j) & 1u) ? 0x3F80u : 0xBF80u; };
+        lut[threadIdx.x] = make_uint2(sg(0) | (sg(1) << 16), sg(2) | (sg(3) << 16));
     }
     pdl_wait_primary();  // x is produced by earlier kernels
-    // x fragments of this slice: step ks, tile nt, lane (g, t) -> x[8 nt + g][k .. k+3], k = 16 ks + 4 t,
-    // copied asynchronously (all in flight at once; zeros past the batch)
-    uint2 *xf = reinterpret_cast<uint2 *>(smem);
-    const unsigned xf_s = (unsigned)__cvta_generic_to_shared(xf);
-    const int nfr = (s_hi - s_lo) * 16 * NT * 32;
-    for (int i = threadIdx.x; i < nfr; i += blockDim.x) {
-        const int ln = i & 31, nt = (i >> 5) % NT, ks = (i >> 5) / NT;
-        const int m = 8 * nt + (ln >> 2);
-        const int k = s_lo * kSmStepK + 16 * ks + 4 * (ln & 3);
-        sm_cp8(xf_s + 8u * i, m < p.M ? p.x + (size_t)m * p.K + k : p.x, m < p.M);
-    }
+#pragma unroll
+    for (int t = 0; t < kSmStages - 1; ++t) issue_x(t);
     sm_commit();
-    sm_wait<0>();  // (also the weight stages issued so far)
-    __syncthreads();
 
     float yacc[2][NT][4];
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) yacc[tt][nt][0] = yacc[tt][nt][1] = yacc[tt][nt][2] = yacc[tt][nt][3] = 0.f;
-    for (int s = 0; s < nst; ++s) {
-        issue_next();
-        sm_wait<kSmStages - 1>();
-        __syncwarp();
-        sm_consume<NT>(ring + (s % kSmStages) * kSmStageBytes, xf + s * 16 * NT * 32, lut, lane, yacc);
-        __syncwarp();
+    for (int s = 0; s < ns; ++s) {
+        // this thread's copies of step s are done once at most the one group
+        // committed after them is pending (at s = 0 the prologue's x group,
+        // which holds step 0's x, is the newest)
+        if (s == 0)
+            sm_wait<0>();
+        else
+            sm_wait<kSmStages - 2>();
+        __syncthreads();  // every thread's copies of step s landed; step s-1's slots are free
+        issue_w(s + kSmStages - 1);
+        issue_x(s + kSmStages - 1);
+        sm_commit();
+        if (rows) {
+            const uint8_t *st = wring + (s % kSmStages) * kSB;
+            const uint2 *xf = xr + (s % kSmStages) * kXFrags;
+            if (FMT == 1)
+                sm_consume<NT>(st, xf, lut, lane, yacc);
+            else
+                i4s_consume<NT>(st, xf, lane, yacc);
+        }
     }
     sm_wait<0>();
 
@@ -274,30 +418,28 @@ __global__ void __launch_bounds__(kSmWarps * 32) k_q1_smallm(const SmParams p)
 
 struct SmPlan {
     int nsteps, L, S, blocks, NT;
-    size_t xfrag, smem;
+    size_t smem;
     bool ok;
 };
 
-static SmPlan sm_plan(int M, int N, int K, int sms)
+// fmt: 1 = Q1_0_g128 (256 k per step), 3 = INT4_G64 (128 k per step)
+static SmPlan sm_plan(int fmt, int M, int N, int K, int sms)
 {
     SmPlan P = {};
-    P.NT = M <= 8 ? 1 : 2;
-    P.nsteps = K / kSmStepK;
+    const int stepk = fmt == 1 ? kSmStepK : kI4sStepK, maxm = fmt == 1 ? kSmMaxM : kI4sMaxM;
+    const int k16 = stepk / 16;
+    P.NT = (M + 7) / 8;
+    P.nsteps = K / stepk;
     P.blocks = (N + kSmRows - 1) / kSmRows;
-    if (M < 2 || M > kSmMaxM || N < 1 || K % kSmStepK != 0 || P.nsteps < 1) return P;  // ok = false
-    const size_t ring = (size_t)kSmWarps * kSmRing, part = (size_t)M * kSmRows * 4;
-    int S = (int)std::min<long long>(kSmMaxCluster, std::max<long long>(1, (2LL * sms + P.blocks - 1) / P.blocks));
-    S = std::min(S, P.nsteps);
-    while (true) {
-        P.L = (P.nsteps + S - 1) / S;
-        P.S = (P.nsteps + P.L - 1) / P.L;
-        P.xfrag = (size_t)P.L * 16 * P.NT * 32 * 8;
-        P.smem = P.xfrag + ring + part;
-        if (P.smem <= (size_t)kSmMaxSmem || S >= std::min(kSmMaxCluster, P.nsteps)) break;
-        S = std::min(std::min(kSmMaxCluster, P.nsteps), S * 2);
-    }
-    P.ok = M >= 2 && M <= kSmMaxM && K % kSmStepK == 0 && P.nsteps >= 1 && P.smem <= (size_t)kSmMaxSmem &&
-           P.blocks < 65536;
+    if (M < 2 || M > maxm || N < 1 || K % stepk != 0 || P.nsteps < 1) return P;  // ok = false
+    const size_t ring = (size_t)kSmWarps * kSmStages * (fmt == 1 ? kSmStageBytes : kI4sStageBytes);
+    const size_t xring = (size_t)kSmStages * k16 * P.NT * 32 * 8, part = (size_t)M * kSmRows * 4;
+    // K slices: as many as keep every CTA resident in one wave (three per SM)
+    P.S = (int)std::min<long long>(std::min(kSmMaxCluster, P.nsteps), std::max<long long>(1, 3LL * sms / P.blocks));
+    P.L = (P.nsteps + P.S - 1) / P.S;
+    P.S = (P.nsteps + P.L - 1) / P.L;
+    P.smem = xring + ring + part;
+    P.ok = P.smem <= (size_t)kSmMaxSmem && P.blocks < 65536;
     return P;
 }
 
@@ -308,12 +450,13 @@ static int sm_num_sms()
     return sms;
 }
 
-bool q1sm_supported(int M, int N, int K) { return sm_plan(M, N, K, sm_num_sms()).ok; }
+bool q1sm_supported(int M, int N, int K) { return sm_plan(1, M, N, K, sm_num_sms()).ok; }
+bool i4sm_supported(int M, int N, int K) { return sm_plan(3, M, N, K, sm_num_sms()).ok; }
 
-lowbit_status q1sm_launch(const uint8_t *bits, const uint16_t *scales, const uint16_t *x, float *y, int M, int N,
-                          int K, cudaStream_t st)
+static lowbit_status sm_launch(int fmt, const uint8_t *bits, const uint16_t *scales, const uint16_t *x, float *y,
+                               int M, int N, int K, cudaStream_t st)
 {
-    const SmPlan P = sm_plan(M, N, K, sm_num_sms());
+    const SmPlan P = sm_plan(fmt, M, N, K, sm_num_sms());
     if (!P.ok) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
     SmParams p = {};
     p.bits = bits;
@@ -326,8 +469,11 @@ lowbit_status q1sm_launch(const uint8_t *bits, const uint16_t *scales, const uin
     p.nsteps = P.nsteps;
     p.L = P.L;
     p.NT = P.NT;
-    p.xfrag = (int)P.xfrag;
-    void (*kern)(const SmParams) = P.NT == 1 ? k_q1_smallm<1> : k_q1_smallm<2>;
+    void (*kern)(const SmParams);
+    if (fmt == 1)
+        kern = P.NT == 1 ? k_smallm<1, 1> : k_smallm<1, 2>;
+    else
+        kern = P.NT == 1 ? k_smallm<3, 1> : P.NT == 2 ? k_smallm<3, 2> : P.NT == 3 ? k_smallm<3, 3> : k_smallm<3, 4>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmMaxSmem) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
@@ -346,6 +492,18 @@ lowbit_status q1sm_launch(const uint8_t *bits, const uint16_t *scales, const uin
     cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
     return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
+lowbit_status q1sm_launch(const uint8_t *bits, const uint16_t *scales, const uint16_t *x, float *y, int M, int N,
+                          int K, cudaStream_t st)
+{
+    return sm_launch(1, bits, scales, x, y, M, N, K, st);
+}
+
+lowbit_status i4sm_launch(const uint8_t *q, const uint16_t *scales, const uint16_t *x, float *y, int M, int N, int K,
+                          cudaStream_t st)
+{
+    return sm_launch(3, q, scales, x, y, M, N, K, st);
 }
 
 }  // namespace lowbit

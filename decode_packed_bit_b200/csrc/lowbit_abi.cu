@@ -25,6 +25,8 @@ int q1tc_fault_flag();
 lowbit_status i4m1_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, cudaStream_t);
 lowbit_status q1m1_prepare_launch(const uint16_t *, int, void *, cudaStream_t);
 bool q1sm_supported(int M, int N, int K);
+bool i4sm_supported(int M, int N, int K);
+lowbit_status i4sm_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 lowbit_status q1stack_launch(const uint8_t *const *, const uint16_t *const *, int, int, int, uint16_t *, float, void *,
                              uint16_t *, float *, cudaStream_t);
 size_t q1stack_workspace_bytes(int F);
@@ -276,6 +278,7 @@ lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales, 
     LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
     cudaStream_t st = as_stream(stream);
     if (M == 1 && i4m1_supported(N, K)) return i4m1_launch(w_q, w_scales, x, y, N, K, st);
+    if (M >= 2 && i4sm_supported(M, N, K)) return i4sm_launch(w_q, w_scales, x, y, M, N, K, st);
     if (i4tc_supported(M, N, K)) return i4tc_launch(w_q, w_scales, x, y, M, N, K, st);
     return int4_gemv_simt_launch(w_q, w_scales, x, y, M, N, K, st);
 }

@@ -223,9 +223,11 @@ lowbit_status lowbit_q1g128_stack_step(const uint8_t *const *w_bits, const uint1
  *   y        [M][N]    fp32
  * Shapes: M >= 1, N >= 1, K >= 64, K % 64 == 0, M*K, N*K < 2^40.
  * The kernel is chosen by M: at M = 1 a weight-streaming tensor-core GEMV
- * (mma.sync on the packed nibbles); for M >= 16 a tcgen05 GEMM that
- * dequantises each weight tile into shared memory as two exact bf16 halves
- * (hi + lo = q*d) and accumulates in TMEM; otherwise a CUDA-core kernel.
+ * (mma.sync on the packed nibbles, integer limbs of x); for 2 <= M <= 32
+ * (K % 128 == 0) mma.sync on bf16 operands, q exact in bf16 and the group
+ * scale applied once per group; above that a tcgen05 GEMM that dequantises
+ * each weight tile into shared memory as two exact bf16 halves (hi + lo =
+ * q*d) and accumulates in TMEM; other shapes a CUDA-core kernel.
  * workspace: at least lowbit_int4g64_workspace_bytes(M, N, K) bytes (NULL
  * allowed when that is 0, which it is for every shape today: each kernel
  * builds its operands in shared memory; the argument is kept so that a

@@ -235,6 +235,21 @@ def _run_int4(lb, q, scales, x, N):
     return host(y)
 
 
+@pytest.mark.parametrize("M", [2, 9, 17, 32])
+@pytest.mark.parametrize("N,K", [(129, 128), (300, 4096), (77, 11008)])
+def test_int4_small_batch_tensor_core(lb, M, N, K):
+    """2 <= M <= 32 with K % 128 == 0 takes the bf16 tensor-core kernel: one
+    to four batch tiles, ragged row blocks, one or several K slices."""
+    seed = 4400 + M * 7 + N
+    codes = synth.int4_codes(seed, N, K)
+    q = oracle.pack("int4", codes)
+    scales = synth.int4_scales(seed, N, K)
+    x = synth.bf16_normal(seed, (M, K))
+    y = _run_int4(lb, q, scales, x, N)
+    y64, ab = oracle.int4_gemv(q, scales, x, want_abs=True)
+    check_float(y, y64, ab, f"int4 small-M M={M} N={N} K={K}")
+
+
 @pytest.mark.parametrize("M", [1, 2, 7, 16, 32, 33, 64, 128, 130, 256, 300])
 @pytest.mark.parametrize("N,K", [(1, 64), (333, 448), (1000, 1024)])
 def test_int4_small_full_compare(lb, M, N, K):
