@@ -18,6 +18,8 @@
 // weights of every layer are staged once into shared memory as bytes; the
 // activations of the CTA's vectors ping-pong between two shared buffers, so
 // no intermediate layer output ever leaves the SM.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace lowbit {
@@ -108,6 +110,183 @@ __global__ void __launch_bounds__(256) k_q2_mlp(Q2Net net, const int16_t *__rest
     }
 }
 
+// ---------------------------------------------------------------------------
+// the same network on the integer tensor cores (layer widths <= 256)
+// ---------------------------------------------------------------------------
+//
+// Persistent CTAs expand every layer's codes once into signed bytes (c - 2)
+// in shared memory, row-major, rows padded to 16 and inputs to 32 with zero
+// weights.  Vectors go 32 at a time (four 8-column MMA tiles).  An int16
+// activation a is held as two byte limbs, lo = a & 0xFF (unsigned) and hi =
+// a >> 8 (signed), so a = lo + 256 hi; a layer is two mma.sync m16n8k32 per
+// 32 inputs (s8 x u8 for lo, s8 x s8 for hi) and acc = D_lo + 256 D_hi is the
+// exact int32 sum (|acc| < 2^27).  The epilogue wraps it to int16, shifts
+// right by 2, applies ReLU between hidden layers and writes the next layer's
+// limbs; nothing leaves the SM until the logits.
+
+constexpr int kQ2tVecs = 32;        // vectors per tile (4 MMA columns tiles)
+constexpr int kQ2tMaxDim = 256;
+constexpr int kQ2tPad = 16;         // row padding (bytes): conflict-free fragment reads
+constexpr int kQ2tThreads = 256;
+
+struct Q2TNet {
+    const uint8_t *w[kQ2MaxLayers];
+    int dims[kQ2MaxLayers + 1];
+    int rows[kQ2MaxLayers];   // dims[l+1] rounded up to 16
+    int cols[kQ2MaxLayers];   // dims[l] rounded up to 32
+    int woff[kQ2MaxLayers];   // byte offset of layer l's expanded weights
+    int wbytes;
+    int n_layers;
+};
+
+__device__ __forceinline__ void imma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void imma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kQ2tThreads) k_q2_mlp_tc(const Q2TNet net, const int16_t *__restrict__ x,
+                                                           int batch, int16_t *__restrict__ logits,
+                                                           int32_t *__restrict__ argmax)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    int8_t *wsm = reinterpret_cast<int8_t *>(smem);
+    // activation limbs: [buffer 2][limb 2][vector 32][kQ2tMaxDim + pad]
+    constexpr int kAStride = kQ2tMaxDim + kQ2tPad;
+    uint8_t *abuf = smem + net.wbytes;
+    auto limb = [&](int buf, int l, int v) { return abuf + ((size_t)(buf * 2 + l) * kQ2tVecs + v) * kAStride; };
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+
+    pdl_launch_dependents();
+    pdl_wait_primary();
+    // expand the codes once: weight (c - 2) as a signed byte; padding is 0
+    for (int i = threadIdx.x; i < net.wbytes / 16; i += kQ2tThreads)
+        reinterpret_cast<uint4 *>(wsm)[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    for (int l = 0; l < net.n_layers; ++l) {
+        const int din = net.dims[l], dout = net.dims[l + 1], rowb = din / 4, cols = net.cols[l] + kQ2tPad;
+        int8_t *dst = wsm + net.woff[l];
+        if (rowb % 4 == 0) {
+            // one 32-bit word of codes (16 weights) per thread and step, four loads in flight
+            const int wpr = rowb / 4, nw = dout * wpr;
+            for (int i0 = threadIdx.x; i0 < nw; i0 += 4 * kQ2tThreads) {
+                uint32_t word[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = i0 + u * kQ2tThreads;
+                    const int o = i / wpr, j = i - o * wpr;
+                    word[u] = i < nw ? reinterpret_cast<const uint32_t *>(net.w[l] + (size_t)o * rowb)[j] : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = i0 + u * kQ2tThreads;
+                    if (i >= nw) break;
+                    const int o = i / wpr, j = i - o * wpr;
+                    uint32_t out[4];
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {  // packed byte b: weights 16 j + 4 b .. + 3
+                        const uint32_t byte = (word[u] >> (8 * b)) & 0xFFu;
+                        uint32_t v = 0;
+#pragma unroll
+                        for (int f = 0; f < 4; ++f) v |= (uint32_t)(uint8_t)(int8_t)q2_code_to_weight(byte, f) << (8 * f);
+                        out[b] = v;
+                    }
+                    *reinterpret_cast<uint4 *>(dst + (size_t)o * cols + 16 * j) = make_uint4(out[0], out[1], out[2], out[3]);
+                }
+            }
+        } else {
+            for (int i = threadIdx.x; i < dout * din; i += kQ2tThreads) {
+                const int o = i / din, k = i - o * din;
+                dst[(size_t)o * cols + k] = (int8_t)q2_code_to_weight(net.w[l][(size_t)o * rowb + k / 4], k & 3);
+            }
+        }
+    }
+    __syncthreads();
+
+    const int ntiles = (batch + kQ2tVecs - 1) / kQ2tVecs;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int v0 = tile * kQ2tVecs, nv = min(kQ2tVecs, batch - v0);
+        const int d0 = net.dims[0];
+        // input limbs (zeros past the batch and past the input width)
+        for (int i = threadIdx.x; i < kQ2tVecs * net.cols[0]; i += kQ2tThreads) {
+            const int v = i / net.cols[0], k = i - v * net.cols[0];
+            const int a = (v < nv && k < d0) ? (int)x[(int64_t)(v0 + v) * d0 + k] : 0;
+            limb(0, 0, v)[k] = (uint8_t)(a & 0xFF);
+            limb(0, 1, v)[k] = (uint8_t)(int8_t)(a >> 8);
+        }
+        __syncthreads();
+        int cur = 0;
+        for (int l = 0; l < net.n_layers; ++l) {
+            const bool hidden = l < net.n_layers - 1;
+            const int mts = net.rows[l] / 16, kcs = net.cols[l] / 32, wcols = net.cols[l] + kQ2tPad;
+            const int8_t *wl = wsm + net.woff[l];
+            // (16-row tile, 8-vector tile) pairs, round-robin over the warps
+            for (int pr = warp; pr < mts * (kQ2tVecs / 8); pr += kQ2tThreads / 32) {
+                const int mt = pr / (kQ2tVecs / 8), nt = pr - mt * (kQ2tVecs / 8);
+                int dlo[4] = {0, 0, 0, 0}, dhi[4] = {0, 0, 0, 0};
+                const int8_t *wa = wl + (size_t)(mt * 16 + g) * wcols + 4 * t;
+                const uint8_t *blo = limb(cur, 0, nt * 8 + g) + 4 * t, *bhi = limb(cur, 1, nt * 8 + g) + 4 * t;
+                for (int kc = 0; kc < kcs; ++kc) {
+                    const int k0 = 32 * kc;
+                    const uint32_t a0 = *reinterpret_cast<const uint32_t *>(wa + k0);
+                    const uint32_t a1 = *reinterpret_cast<const uint32_t *>(wa + 8 * wcols + k0);
+                    const uint32_t a2 = *reinterpret_cast<const uint32_t *>(wa + k0 + 16);
+                    const uint32_t a3 = *reinterpret_cast<const uint32_t *>(wa + 8 * wcols + k0 + 16);
+                    imma_s8u8(dlo, a0, a1, a2, a3, *reinterpret_cast<const uint32_t *>(blo + k0),
+                              *reinterpret_cast<const uint32_t *>(blo + k0 + 16));
+                    imma_s8s8(dhi, a0, a1, a2, a3, *reinterpret_cast<const uint32_t *>(bhi + k0),
+                              *reinterpret_cast<const uint32_t *>(bhi + k0 + 16));
+                }
+                // d[j]: row mt*16 + g + 8 (j >> 1), vector nt*8 + 2t + (j & 1)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int acc = dlo[j] + 256 * dhi[j];                         // exact: |acc| < 2^27
+                    const int16_t wrapped = (int16_t)(uint16_t)(uint32_t)acc;      // mod 2^16
+                    int16_t z = (int16_t)(wrapped >> 2);                           // arithmetic shift
+                    if (hidden && z < 0) z = 0;
+                    const int o = mt * 16 + g + 8 * (j >> 1), v = nt * 8 + 2 * t + (j & 1);
+                    if (hidden) {
+                        limb(cur ^ 1, 0, v)[o] = (uint8_t)(z & 0xFF);
+                        limb(cur ^ 1, 1, v)[o] = (uint8_t)(int8_t)(z >> 8);
+                    } else if (o < net.dims[l + 1]) {
+                        // logits as int16: vector v's row spans both limb regions of the buffer
+                        reinterpret_cast<int16_t *>(limb(cur ^ 1, 0, 0))[v * kAStride + o] = z;
+                    }
+                }
+            }
+            __syncthreads();
+            cur ^= 1;
+        }
+        // logits (int16, in the last buffer) and argmax
+        const int dl = net.dims[net.n_layers];
+        const int16_t *lg = reinterpret_cast<const int16_t *>(limb(cur, 0, 0));
+        for (int i = threadIdx.x; i < nv * dl; i += kQ2tThreads) {
+            const int v = i / dl, c = i - v * dl;
+            logits[(int64_t)(v0 + v) * dl + c] = lg[v * kAStride + c];
+        }
+        if (argmax != nullptr && threadIdx.x < nv) {
+            const int16_t *a = lg + threadIdx.x * kAStride;
+            int best = 0;
+            for (int c = 1; c < dl; ++c)
+                if (a[c] > a[best]) best = c;  // strict: the lowest index wins ties
+            argmax[v0 + threadIdx.x] = best;
+        }
+        __syncthreads();  // the buffers are reused by the next tile
+    }
+}
+
 lowbit_status q2_mlp_launch(const uint8_t *const *w_packed, const int32_t *dims, int n_layers,
                             const int16_t *x, int batch, int16_t *logits, int32_t *argmax,
                             cudaStream_t st)
@@ -123,6 +302,39 @@ lowbit_status q2_mlp_launch(const uint8_t *const *w_packed, const int32_t *dims,
     }
     net.wbytes = off;
     if (batch == 0) return LOWBIT_OK;
+    {
+        Q2TNet tn = {};
+        tn.n_layers = n_layers;
+        bool fits = true;
+        int toff = 0;
+        for (int l = 0; l <= n_layers; ++l) {
+            tn.dims[l] = dims[l];
+            fits = fits && dims[l] <= kQ2tMaxDim;
+        }
+        for (int l = 0; l < n_layers && fits; ++l) {
+            tn.w[l] = w_packed[l];
+            tn.rows[l] = (dims[l + 1] + 15) / 16 * 16;
+            tn.cols[l] = (dims[l] + 31) / 32 * 32;
+            tn.woff[l] = toff;
+            toff += tn.rows[l] * (tn.cols[l] + kQ2tPad);
+        }
+        tn.wbytes = (toff + 15) & ~15;
+        const size_t tsmem = (size_t)tn.wbytes + 4u * kQ2tVecs * (kQ2tMaxDim + kQ2tPad);
+        if (fits && tsmem <= 200u * 1024u) {
+            if (cudaFuncSetAttribute(k_q2_mlp_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+                cudaSuccess)
+                return LOWBIT_ERR_CUDA;
+            int dev = 0, sms = 148, per_sm = 1;
+            if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_q2_mlp_tc, kQ2tThreads, tsmem) != cudaSuccess ||
+                per_sm < 1)
+                per_sm = 1;
+            const int tiles = (batch + kQ2tVecs - 1) / kQ2tVecs;
+            dim3 tgrid(std::min(tiles, per_sm * sms)), tblock(kQ2tThreads);  // persistent: every CTA resident
+            cudaError_t e = launch_pdl(k_q2_mlp_tc, tgrid, tblock, tsmem, st, tn, x, batch, logits, argmax);
+            return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+        }
+    }
     const size_t smem = (size_t)off + 2u * kVecs * kQ2MaxDim * sizeof(int16_t);
     // per-device function attribute, always set to the same (largest) value so
     // concurrent callers never shrink it under each other

@@ -303,7 +303,7 @@ def test_q2_mlp_1024_vectors_bitexact(lb):
     assert np.array_equal(am, ref_a)
 
 
-@pytest.mark.parametrize("batch", [1, 7, 9, 100])
+@pytest.mark.parametrize("batch", [1, 7, 9, 100, 5000])
 def test_q2_mlp_ragged_batches_and_overflow(lb, batch):
     dims = (256, 192, 128, 40)
     packed = [oracle.pack("q2", c) for c in synth.q2_codes(77, dims)]
@@ -317,7 +317,8 @@ def test_q2_mlp_ragged_batches_and_overflow(lb, batch):
     assert np.array_equal(lg2, ref_l) and none is None
 
 
-@pytest.mark.parametrize("dims", [(4, 4), (8, 12, 4), (64, 1024, 32, 1), (1024, 16, 1024)])
+@pytest.mark.parametrize("dims", [(4, 4), (8, 12, 4), (64, 1024, 32, 1), (1024, 16, 1024), (200, 256, 152),
+                                  (256, 96, 255 // 4 * 4, 44)])
 def test_q2_mlp_other_topologies(lb, dims):
     codes = [synth.rng(88, l).integers(0, 4, size=(dims[l + 1], dims[l]), dtype=np.int8)
              for l in range(len(dims) - 1)]
