@@ -23,11 +23,17 @@
 //     per B column.  Each D column then holds sum_k b_k * limb_l(X_k 2^(7-i))
 //     exactly, in int32.
 //   Two groups share one accumulator: B columns 0-3 carry the four limbs of
-//     the first group of a 256-k chunk, columns 4-7 those of the second.
+//     the first group of a 256-k chunk, columns 4-7 those of the second.  A
+//     lane's B registers are zero whenever its column group differs from the
+//     group of its k slots, so only 16 of the 32 lanes' fragments are stored
+//     (1 KB per chunk); the other lanes read a zero block.
 //   Epilogue per (row, group): 2^7 sum_k b X = sum_l D_l 2^(8l); the signed
-//     sum is sum s x = 2 sum b x - sum x, so y += d * (2^(E-29) * sum_l D_l
-//     2^(8l) - S_g) with S_g = 2^(E-23) * sum_k X_k.  Integer-exact up to the
-//     24-bit rounding of x and the fp32 epilogue.
+//     sum is sum s x = 2 sum b x - sum x.  Lane quarter tq holds the limb
+//     pair 2(tq&1), 2(tq&1)+1 of group tq>>1; it forms v = D_lo + 256 D_hi in
+//     int32 (|v| < 2^29), converts it once, and adds d * (c_tq v + n_tq),
+//     with c_tq = 2^(E-29) (times 2^16 for the high pair) and n_tq = -2^(E-23)
+//     sum_k X_k for the low pair (0 for the high pair).  Integer-exact up to
+//     the 24-bit rounding of x and the fp32 epilogue.
 //
 // Weight streaming: each warp owns a ring of shared-memory stages filled by
 // cp.async; a stage is 32 rows x 2 chunks (64 bytes of each row) plus their
@@ -51,20 +57,15 @@
 namespace lowbit {
 
 constexpr int kQ1ChunkK = 256;
-constexpr int kQ1FragBytesPerChunk = 2048;  // 8 mma x 32 lanes x 8 bytes (zeros outside each lane's group)
-constexpr int kQ1InfoBytesPerChunk = 16;    // two groups x (G, S) floats
+constexpr int kQ1FragBytesPerChunk = 1024;  // 8 mma x 16 live lanes x 8 bytes
+constexpr int kQ1InfoBytesPerChunk = 32;    // four lane quarters x (c, n) floats
+constexpr int kQ1ZeroBytes = 4096;          // zero block read by the dead lanes (covers a 4-chunk step)
 // Tuning knobs (compile-time; the defaults are the measured best).
 #ifndef LOWBIT_Q1_WARPS
 #define LOWBIT_Q1_WARPS 8
 #endif
 #ifndef LOWBIT_Q1_STAGES
 #define LOWBIT_Q1_STAGES 3
-#endif
-#ifndef LOWBIT_Q1_SPLIT_CHAINS
-#define LOWBIT_Q1_SPLIT_CHAINS 0
-#endif
-#ifndef LOWBIT_Q1_I2F
-#define LOWBIT_Q1_I2F 0
 #endif
 constexpr int kQ1Warps = LOWBIT_Q1_WARPS;
 constexpr int kQ1MinExp = -96;              // activations below 2^-96 round to 0
@@ -75,13 +76,44 @@ constexpr int kQ1MaxCluster = 8;
 
 
 // ---------------------------------------------------------------------------
-// activation prepare: x (bf16) -> limb fragments + per-group (G, S) + copy
+// activation prepare: x (bf16) -> limb fragments + per-lane epilogue constants
 // ---------------------------------------------------------------------------
 
+// The two epilogue constant pairs of one group (lane quarters 2h, 2h+1).
+__device__ __forceinline__ void q1_write_info(float2 *dst, bool exists, int E, int T)
+{
+    float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);
+    if (exists) {
+        lo = make_float2(ldexpf(1.0f, E - 29), -ldexpf((float)T, E - 23));
+        hi = make_float2(ldexpf(1.0f, E - 13), 0.f);
+    }
+    dst[0] = lo;
+    dst[1] = hi;
+}
+
+// B fragment of live entry e (0..15) of mma i, from a chunk's limbs
+// lb[limb][k - 256 ch].  Entry e is the lane with k quarter t = e & 3 and
+// column 4 (t >> 1) + (e >> 2), i.e. limb e >> 2 of the group of its k slots.
+// Register j, byte c holds B[k-slot 16j + 4t + c]; k-slot 16j + 4t + c of mma
+// i carries bit i of packed byte 8t + 4j + c of the row's 32-byte chunk, i.e.
+// k = 64t + 32j + 8c + i.
+__device__ __forceinline__ uint2 q1_fragment(const int8_t (*lb)[256], int i, int e)
+{
+    const int t = e & 3;
+    const int8_t *l = lb[e >> 2];
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) w[j] |= (uint32_t)(uint8_t)l[64 * t + 32 * j + 8 * c + i] << (8 * c);
+    return make_uint2(w[0], w[1]);
+}
+
 // One CTA of 256 threads per 256-k chunk.  Thread kk first turns x[k] into
-// four limbs; then thread t writes the 8-byte B fragment of lane t%32 for
-// mma t/32.  A plain bf16 copy of x is kept after the fragments for shapes
-// the tensor kernels do not take (K/128 odd), which the SIMT kernel reads.
+// four limbs; then thread t < 128 writes the 8-byte B fragment of live entry
+// t%16 for mma t/16.  A plain bf16 copy of x is kept after the fragments for
+// shapes the tensor kernels do not take (K/128 odd), which the SIMT kernel
+// reads.
 __global__ void __launch_bounds__(256) k_q1_prep_m1(const uint16_t *__restrict__ x, int K,
                                                     uint8_t *__restrict__ act, size_t info_off,
                                                     size_t xcopy_off)
@@ -125,29 +157,12 @@ __global__ void __launch_bounds__(256) k_q1_prep_m1(const uint16_t *__restrict__
     __syncthreads();
     if ((kk & 127) == 0) {
         const int T = ssum[4 * h] + ssum[4 * h + 1] + ssum[4 * h + 2] + ssum[4 * h + 3];  // |T| < 2^30
-        const int grp = 2 * ch + h;
-        float2 info = make_float2(0.f, 0.f);
-        if (grp * 128 < K) info = make_float2(ldexpf(1.0f, E - 29), ldexpf((float)T, E - 23));
-        reinterpret_cast<float2 *>(act + info_off)[grp] = info;
+        q1_write_info(reinterpret_cast<float2 *>(act + info_off) + 4 * ch + 2 * h, (2 * ch + h) * 128 < K, E, T);
     }
-
-    // B fragment of lane ln for mma i.  Register j, byte c of lane (n, t)
-    // holds B[k-slot 16j + 4t + c][column n]; k-slot 16j + 4t + c of mma i
-    // carries bit i of packed byte 8t + 4j + c of the row's 32-byte chunk,
-    // i.e. k = 64t + 32j + 8c + i.  Column n = 4*group + limb; lanes of the
-    // other group get zeros.
-    const int i = kk >> 5, ln = kk & 31;
-    const int n = ln >> 2, t = ln & 3;
-    uint32_t w[2] = {0u, 0u};
-    if ((n >> 2) == (t >> 1)) {
-        const int8_t *lb = limb[n & 3];
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                w[j] |= (uint32_t)(uint8_t)lb[64 * t + 32 * j + 8 * c + i] << (8 * c);
+    if (kk < 128) {
+        const uint2 f = q1_fragment(limb, kk >> 4, kk & 15);
+        reinterpret_cast<uint2 *>(act + (size_t)ch * kQ1FragBytesPerChunk)[kk] = f;
     }
-    reinterpret_cast<uint2 *>(act + (size_t)ch * kQ1FragBytesPerChunk)[kk] = make_uint2(w[0], w[1]);
 }
 
 // ---------------------------------------------------------------------------
@@ -257,8 +272,9 @@ __device__ __forceinline__ void issue_any(unsigned stage, const Q1Group &grp, co
 
 struct LaneConst {
     int woff, soff;     // offsets inside a stage (row g of tile 0, chunk 0)
-    float limb_scale;
     int tq, h;
+    int e;              // fragment entry this lane reads (lane & 15)
+    bool live;          // its column group is the group of its k slots
 };
 
 __device__ __forceinline__ LaneConst lane_const(int lane)
@@ -269,18 +285,26 @@ __device__ __forceinline__ LaneConst lane_const(int lane)
     lc.h = lc.tq >> 1;
     lc.woff = g * kQ1RowStride + lc.tq * 8;
     lc.soff = kQ1StageW + g * 8 + lc.h * 2;
-    lc.limb_scale = (lc.tq & 1) ? 65536.f : 1.f;
+    lc.e = lane & 15;
+    lc.live = (lane >> 4) == lc.h;
     return lc;
 }
 
-// float(d) for |d| < 2^22, exactly, without an int->float conversion
-// instruction: the integer add lands d in the mantissa of 1.5*2^23.
-constexpr float kQ1Magic = 12582912.f;
-__device__ __forceinline__ float magic_biased(int d) { return __int_as_float(d + 0x4B400000); }
+// The B fragment base of a step: a live lane reads its entry of the step's
+// first chunk, a dead lane the zero block.
+__device__ __forceinline__ const uint8_t *bfrag_base(const uint8_t *frags, const uint8_t *zero, int chunk,
+                                                     const LaneConst &lc)
+{
+    return lc.live ? frags + (size_t)chunk * kQ1FragBytesPerChunk + lc.e * 8 : zero + lc.e * 8;
+}
+
+// D_lo + 256 D_hi of one limb pair, as a float (one rounding; |v| < 2^29).
+__device__ __forceinline__ float limb_pair(int lo, int hi) { return (float)(lo + (hi << 8)); }
 
 // Multiply-accumulate one staged step of nch (1 or 2) chunks.  bf: this
-// lane's B fragments of the step's first chunk; inf: the (G, S) pair of this
-// lane's group in that chunk.  yacc[t][r]: row g + 8r of tile t.
+// lane's B fragment base for the step (bfrag_base); inf: this lane's (c, n)
+// pair of the step's first chunk (stride 4 per chunk).  yacc[t][r]: row
+// g + 8r of tile t.
 __device__ __forceinline__ void consume_step(const uint8_t *st, const uint8_t *bf, const float2 *inf, int nch,
                                              const LaneConst &lc, float (&yacc)[2][2])
 {
@@ -294,45 +318,28 @@ __device__ __forceinline__ void consume_step(const uint8_t *st, const uint8_t *b
                 w[t][r][c] = *reinterpret_cast<const uint2 *>(st + lc.woff + (16 * t + 8 * r) * kQ1RowStride + c * 32);
     int d[2][kQ1StepChunks][4];
     if (nch == kQ1StepChunks) {
-#if LOWBIT_Q1_SPLIT_CHAINS
-        int e[2][kQ1StepChunks][4];  // odd bit positions: a second independent chain
-#endif
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const uint32_t m = 0x01010101u << i;
 #pragma unroll
             for (int c = 0; c < kQ1StepChunks; ++c) {
-                const uint2 b = *reinterpret_cast<const uint2 *>(bf + c * kQ1FragBytesPerChunk + i * 256);
+                const uint2 b = *reinterpret_cast<const uint2 *>(bf + c * kQ1FragBytesPerChunk + i * 128);
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
-#if LOWBIT_Q1_SPLIT_CHAINS
-                    int (&acc)[4] = (i & 1) ? e[t][c] : d[t][c];
-                    if (i < 2)
-#else
-                    int (&acc)[4] = d[t][c];
                     if (i == 0)
-#endif
-                        mma_u8s8_z(acc, w[t][0][c].x & m, w[t][1][c].x & m, w[t][0][c].y & m, w[t][1][c].y & m,
+                        mma_u8s8_z(d[t][c], w[t][0][c].x & m, w[t][1][c].x & m, w[t][0][c].y & m, w[t][1][c].y & m,
                                    b.x, b.y);
                     else
-                        mma_u8s8(acc, w[t][0][c].x & m, w[t][1][c].x & m, w[t][0][c].y & m, w[t][1][c].y & m,
+                        mma_u8s8(d[t][c], w[t][0][c].x & m, w[t][1][c].x & m, w[t][0][c].y & m, w[t][1][c].y & m,
                                  b.x, b.y);
                 }
             }
         }
-#if LOWBIT_Q1_SPLIT_CHAINS
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int c = 0; c < kQ1StepChunks; ++c)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) d[t][c][q] += e[t][c][q];
-#endif
     } else {  // one chunk left
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const uint32_t m = 0x01010101u << i;
-            const uint2 b = *reinterpret_cast<const uint2 *>(bf + i * 256);
+            const uint2 b = *reinterpret_cast<const uint2 *>(bf + i * 128);
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 if (i == 0)
@@ -348,29 +355,22 @@ __device__ __forceinline__ void consume_step(const uint8_t *st, const uint8_t *b
     }
 #pragma unroll
     for (int c = 0; c < kQ1StepChunks; ++c) {
-        // a chunk past the end holds zero weights and zero scales
-        const float2 gi = c < nch ? inf[2 * c] : make_float2(0.f, 0.f);
-        const float coef = gi.x * lc.limb_scale;
-        const float subc = fmaf(coef, kQ1Magic, (lc.tq & 1) ? 0.f : gi.y);
+        // a chunk past the end holds zero weights and contributes nothing
+        const float2 ci = c < nch ? inf[4 * c] : make_float2(0.f, 0.f);
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const uint16_t sc =
                     *reinterpret_cast<const uint16_t *>(st + lc.soff + (16 * t + 8 * r) * 8 + c * 4);
-#if LOWBIT_Q1_I2F
-                const float v = (float)(d[t][c][2 * r] + 256 * d[t][c][2 * r + 1]);
-                yacc[t][r] = fmaf(f16_bits_to_float(sc), fmaf(coef, v, -(subc - coef * kQ1Magic)), yacc[t][r]);
-#else
-                const float hi = magic_biased(d[t][c][2 * r + 1]) - kQ1Magic;      // exact limb-pair high part
-                const float vm = fmaf(256.f, hi, magic_biased(d[t][c][2 * r]));    // 256 d_hi + d_lo + magic
-                yacc[t][r] = fmaf(f16_bits_to_float(sc), fmaf(coef, vm, -subc), yacc[t][r]);
-#endif
+                const float v = limb_pair(d[t][c][2 * r], d[t][c][2 * r + 1]);
+                yacc[t][r] = fmaf(f16_bits_to_float(sc), fmaf(ci.x, v, ci.y), yacc[t][r]);
             }
     }
 }
 
-// Copy prepared chunks [ch_lo, ch_lo+n) (fragments, then info) to smem.
+// Copy prepared chunks [ch_lo, ch_lo+n) (fragments, then the per-lane
+// constants) to smem, and clear the zero block that follows them.
 __device__ __forceinline__ void stage_act(uint8_t *smem, const Q1Params &p, int ch_lo, int n)
 {
     const uint4 *src = reinterpret_cast<const uint4 *>(p.act + (size_t)ch_lo * kQ1FragBytesPerChunk);
@@ -378,7 +378,14 @@ __device__ __forceinline__ void stage_act(uint8_t *smem, const Q1Params &p, int 
     for (int i = threadIdx.x; i < n * (kQ1FragBytesPerChunk / 16); i += blockDim.x) dst[i] = __ldg(src + i);
     const uint4 *isrc = reinterpret_cast<const uint4 *>(p.act + p.info_off + (size_t)ch_lo * kQ1InfoBytesPerChunk);
     uint4 *idst = reinterpret_cast<uint4 *>(smem + (size_t)n * kQ1FragBytesPerChunk);
-    for (int i = threadIdx.x; i < n; i += blockDim.x) idst[i] = __ldg(isrc + i);
+    for (int i = threadIdx.x; i < n * (kQ1InfoBytesPerChunk / 16); i += blockDim.x) idst[i] = __ldg(isrc + i);
+}
+
+// Zero block of kQ1ZeroBytes at `z` (16-byte aligned).
+__device__ __forceinline__ void clear_zero_block(uint8_t *z)
+{
+    for (int i = threadIdx.x; i < kQ1ZeroBytes / 16; i += blockDim.x)
+        reinterpret_cast<uint4 *>(z)[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 constexpr int kQ1BuildScratch = kQ1SplitWarps * 4 * 256;  // limb scratch of the fused split kernel
@@ -386,7 +393,7 @@ constexpr int kQ1BuildScratch = kQ1SplitWarps * 4 * 256;  // limb scratch of the
 // The work of k_q1_prep_m1 for one 256-k chunk, done by one warp: lane l
 // takes k = 256 ch + 32 j + l (j = 0..7; j < 4 is the chunk's first group),
 // so every per-group reduction is a warp shuffle.  lw: this warp's limb
-// scratch (4 x 256 bytes).
+// scratch (4 x 256 bytes); info: the chunk's four (c, n) pairs.
 __device__ __forceinline__ void q1_build_chunk_warp(const uint16_t *__restrict__ x, int K, int ch, uint8_t *frag,
                                                     float2 *info, int8_t (*lw)[256], int lane)
 {
@@ -424,25 +431,15 @@ __device__ __forceinline__ void q1_build_chunk_warp(const uint16_t *__restrict__
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int Th = warp_sum_int(T[h]);  // |T| <= 2^30
-        if (lane == 0)
-            info[h] = (2 * ch + h) * 128 < K ? make_float2(ldexpf(1.0f, E[h] - 29), ldexpf((float)Th, E[h] - 23))
-                                             : make_float2(0.f, 0.f);
+        if (lane == 0) q1_write_info(info + 2 * h, (2 * ch + h) * 128 < K, E[h], Th);
     }
     __syncwarp();
-    // fragment words: the same layout as k_q1_prep_m1 writes
-    const int n = lane >> 2, t = lane & 3;
+    // fragment words: the same layout as k_q1_prep_m1 writes; lane l takes
+    // entry l & 15 of mmas 4 (l >> 4) .. 4 (l >> 4) + 3
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        uint32_t w[2] = {0u, 0u};
-        if ((n >> 2) == (t >> 1)) {
-            const int8_t *lb = lw[n & 3];
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    w[j] |= (uint32_t)(uint8_t)lb[64 * t + 32 * j + 8 * c + i] << (8 * c);
-        }
-        reinterpret_cast<uint2 *>(frag)[32 * i + lane] = make_uint2(w[0], w[1]);
+    for (int q = 0; q < 4; ++q) {
+        const int i = 4 * (lane >> 4) + q;
+        reinterpret_cast<uint2 *>(frag)[16 * i + (lane & 15)] = q1_fragment(lw, i, lane & 15);
     }
     __syncwarp();  // the scratch is reused for the warp's next chunk
 }
@@ -513,12 +510,13 @@ __global__ void __launch_bounds__(kQ1Warps * 32, (kQ1Warps <= 8 ? 2 : 1)) k_q1_m
     for (int t = 0; t < kQ1Stages - 1; ++t) issue_next();
 
     pdl_wait_primary();  // the activation and the outputs follow stream order from here
+    uint8_t *zero = smem + p.act_smem - kQ1ZeroBytes;
     if (c1 > c0) stage_act(smem, p, 0, p.nchunks);
+    clear_zero_block(zero);
     __syncthreads();
 
     const LaneConst lc = lane_const(lane);
-    const uint8_t *bfrag = smem + lane * 8;
-    const float2 *sinfo = reinterpret_cast<const float2 *>(smem + (size_t)p.nchunks * kQ1FragBytesPerChunk) + lc.h;
+    const float2 *sinfo = reinterpret_cast<const float2 *>(smem + (size_t)p.nchunks * kQ1FragBytesPerChunk) + lc.tq;
 
     int cell = c0 + warp, r = cell / p.blocksN, blk = cell - r * p.blocksN;
     int slot = 0;
@@ -529,7 +527,7 @@ __global__ void __launch_bounds__(kQ1Warps * 32, (kQ1Warps <= 8 ? 2 : 1)) k_q1_m
             cp_async_wait<kQ1Stages - 1>();
             __syncwarp();
             const int chs = s * kQ1StepChunks;
-            consume_step(ring + slot * kQ1StageBytes, bfrag + chs * kQ1FragBytesPerChunk, sinfo + 2 * chs,
+            consume_step(ring + slot * kQ1StageBytes, bfrag_base(smem, zero, chs, lc), sinfo + 4 * chs,
                          min(kQ1StepChunks, p.nchunks - chs), lc, yacc);
             __syncwarp();  // every lane is done with this stage before it is refilled
             slot = slot + 1 == kQ1Stages ? 0 : slot + 1;
@@ -541,6 +539,169 @@ __global__ void __launch_bounds__(kQ1Warps * 32, (kQ1Warps <= 8 ? 2 : 1)) k_q1_m
         });
         cell += kQ1Warps;
         blk += kQ1Warps;
+        while (blk >= p.blocksN) {
+            blk -= p.blocksN;
+            ++r;
+        }
+    }
+    cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
+// lean stream kernel: the stream kernel's cells with 1024 k per step, for
+// K % 1024 == 0, N % 32 == 0 and 16-byte aligned operands (no bounds tests)
+// ---------------------------------------------------------------------------
+//
+// A stage holds 32 rows x 128 bytes of signs and, after them, each row's
+// 16-byte run of eight fp16 scales.  Row q's 16-byte piece p sits at piece
+// p ^ 2(q & 3): the 8-byte fragment reads of a warp then cover all 32 banks
+// once per 128 bytes.  A lane copies piece (lane & 7) of rows (lane >> 3) +
+// 4u, u = 0..7 (four whole rows per instruction), and the scale run of row
+// `lane`.  One CTA per SM; every warp has its own ring of S stages.
+
+constexpr int kQ1LChunks = 4;                                  // chunks per step
+constexpr int kQ1LRowBytes = kQ1LChunks * 32;
+constexpr int kQ1LStageW = kQ1StepRows * kQ1LRowBytes;
+constexpr int kQ1LStageBytes = kQ1LStageW + kQ1StepRows * 16;
+#ifndef LOWBIT_Q1_LEAN_STAGES
+#define LOWBIT_Q1_LEAN_STAGES 2
+#endif
+#ifndef LOWBIT_Q1_LEAN_WARPS
+#define LOWBIT_Q1_LEAN_WARPS 16
+#endif
+constexpr int kQ1LStages = LOWBIT_Q1_LEAN_STAGES;
+constexpr int kQ1LMaxWarps = LOWBIT_Q1_LEAN_WARPS;
+constexpr int kQ1LMinWarps = 8;
+
+__device__ __forceinline__ void cp_async16_full(unsigned dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// One staged step.  woff[c]: this lane's byte offset of chunk c in row g of
+// a stage; soff: its scale offset (row g, group h of chunk 0); bf: its B
+// fragment base (bfrag_base); inf: its (c, n) pair of the step's first chunk.
+__device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *bf, const float2 *inf,
+                                             const int (&woff)[kQ1LChunks], int soff, float (&yacc)[2][2])
+{
+#pragma unroll
+    for (int c = 0; c < kQ1LChunks; ++c) {
+        uint2 w[2][2];  // [tile][row g / g+8]
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+                w[t][r] = *reinterpret_cast<const uint2 *>(st + woff[c] + (16 * t + 8 * r) * kQ1LRowBytes);
+        int d[2][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t m = 0x01010101u << i;
+            const uint2 b = *reinterpret_cast<const uint2 *>(bf + c * kQ1FragBytesPerChunk + i * 128);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (i == 0)
+                    mma_u8s8_z(d[t], w[t][0].x & m, w[t][1].x & m, w[t][0].y & m, w[t][1].y & m, b.x, b.y);
+                else
+                    mma_u8s8(d[t], w[t][0].x & m, w[t][1].x & m, w[t][0].y & m, w[t][1].y & m, b.x, b.y);
+            }
+        }
+        const float2 ci = inf[4 * c];
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint16_t sc = *reinterpret_cast<const uint16_t *>(st + soff + (16 * t + 8 * r) * 16 + c * 4);
+                yacc[t][r] =
+                    fmaf(f16_bits_to_float(sc), fmaf(ci.x, limb_pair(d[t][2 * r], d[t][2 * r + 1]), ci.y), yacc[t][r]);
+            }
+    }
+}
+
+__global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __grid_constant__ Q1Group grp,
+                                                                     const Q1Params p)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int c0 = (int)((long long)blockIdx.x * p.cells / gridDim.x);
+    const int c1 = (int)((long long)(blockIdx.x + 1) * p.cells / gridDim.x);
+    const int spc = p.nchunks / kQ1LChunks;  // steps per cell
+    const size_t rowbytes = (size_t)(p.K >> 3);
+    const int G = p.K >> 7;
+    uint8_t *ring = smem + p.act_smem + warp * (kQ1LStages * kQ1LStageBytes);
+    const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
+
+    // issue side: cell icell = (matrix ir, 32-row block iblk), step istep
+    const int rq = lane >> 3;
+    const unsigned wdst = (unsigned)(rq * kQ1LRowBytes + (((lane & 7) ^ (rq << 1)) << 4));
+    const unsigned sdst = (unsigned)(kQ1LStageW + lane * 16);
+    int icell = c0 + warp, ir = icell / p.blocksN, iblk = icell - ir * p.blocksN, istep = 0, islot = 0;
+    const uint8_t *wsrc = nullptr;
+    const uint16_t *ssrc = nullptr;
+    auto cell_src = [&]() {
+        wsrc = grp.bits[ir] + (size_t)(iblk * kQ1StepRows + rq) * rowbytes + (lane & 7) * 16;
+        ssrc = grp.scales[ir] + (size_t)(iblk * kQ1StepRows + lane) * G;
+    };
+    if (icell < c1) cell_src();
+    auto issue_next = [&]() {
+        if (icell < c1) {
+            const unsigned st = ring_s + islot * kQ1LStageBytes;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                cp_async16_full(st + wdst + u * 4 * kQ1LRowBytes, wsrc + (size_t)(4 * u) * rowbytes);
+            cp_async16_full(st + sdst, ssrc);
+            wsrc += kQ1LRowBytes;
+            ssrc += 2 * kQ1LChunks;
+            if (++istep == spc) {
+                istep = 0;
+                icell += nw;
+                iblk += nw;
+                while (iblk >= p.blocksN) {
+                    iblk -= p.blocksN;
+                    ++ir;
+                }
+                if (icell < c1) cell_src();
+            }
+        }
+        cp_async_commit();
+        islot = islot + 1 == kQ1LStages ? 0 : islot + 1;
+    };
+#pragma unroll
+    for (int t = 0; t < kQ1LStages - 1; ++t) issue_next();
+
+    pdl_wait_primary();  // the activation and the outputs follow stream order from here
+    uint8_t *zero = smem + p.act_smem - kQ1ZeroBytes;
+    if (c1 > c0) stage_act(smem, p, 0, p.nchunks);
+    clear_zero_block(zero);
+    __syncthreads();
+
+    const int g = lane >> 2, tq = lane & 3;
+    int woff[kQ1LChunks];
+#pragma unroll
+    for (int c = 0; c < kQ1LChunks; ++c)
+        woff[c] = g * kQ1LRowBytes + (((2 * c + (tq >> 1)) ^ ((g & 3) << 1)) << 4) + (tq & 1) * 8;
+    const int soff = kQ1LStageW + g * 16 + (tq >> 1) * 2;
+    const bool live = (lane >> 4) == (tq >> 1);
+    const uint8_t *bf_live = smem + (lane & 15) * 8, *bf_dead = zero + (lane & 15) * 8;
+    const float2 *inf0 = reinterpret_cast<const float2 *>(smem + (size_t)p.nchunks * kQ1FragBytesPerChunk) + tq;
+
+    int cell = c0 + warp, r = cell / p.blocksN, blk = cell - r * p.blocksN, slot = 0;
+    while (cell < c1) {
+        float yacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        for (int s = 0; s < spc; ++s) {
+            issue_next();
+            cp_async_wait<kQ1LStages - 1>();
+            __syncwarp();
+            lean_consume(ring + slot * kQ1LStageBytes,
+                         live ? bf_live + s * (kQ1LChunks * kQ1FragBytesPerChunk) : bf_dead,
+                         inf0 + 4 * kQ1LChunks * s, woff, soff, yacc);
+            __syncwarp();  // every lane is done with this stage before it is refilled
+            slot = slot + 1 == kQ1LStages ? 0 : slot + 1;
+        }
+        float *yr = grp.y[r] + blk * kQ1StepRows;
+        finish_cell(yacc, lane, [&](int row, float v) { yr[row] = v; });
+        cell += nw;
+        blk += nw;
         while (blk >= p.blocksN) {
             blk -= p.blocksN;
             ++r;
@@ -615,6 +776,7 @@ __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid
     for (int t = 0; t < kQ1SplitStages - 1; ++t) issue_next();
 
     pdl_wait_primary();
+    uint8_t *zero = smem + p.act_smem - kQ1ZeroBytes;
     if (ch_hi > ch_lo) {
         const int n = ch_hi - ch_lo;
         if (p.x != nullptr) {
@@ -623,25 +785,25 @@ __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid
                                                                  warp * 4 * 256);
             float2 *info = reinterpret_cast<float2 *>(smem + (size_t)n * kQ1FragBytesPerChunk);
             for (int c = warp; c < n; c += kQ1SplitWarps)
-                q1_build_chunk_warp(p.x, p.K, ch_lo + c, smem + (size_t)c * kQ1FragBytesPerChunk, info + 2 * c, lw,
+                q1_build_chunk_warp(p.x, p.K, ch_lo + c, smem + (size_t)c * kQ1FragBytesPerChunk, info + 4 * c, lw,
                                     lane);
         } else {
             stage_act(smem, p, ch_lo, n);
         }
     }
+    clear_zero_block(zero);
     __syncthreads();
 
     const LaneConst lc = lane_const(lane);
-    const uint8_t *bfrag = smem + lane * 8;
-    const float2 *sinfo = reinterpret_cast<const float2 *>(smem + (size_t)(ch_hi - ch_lo) * kQ1FragBytesPerChunk) + lc.h;
+    const float2 *sinfo = reinterpret_cast<const float2 *>(smem + (size_t)(ch_hi - ch_lo) * kQ1FragBytesPerChunk) + lc.tq;
     float yacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
     for (int s = 0; s < nsteps; ++s) {
         issue_next();
         cp_async_wait<kQ1SplitStages - 1>();
         __syncwarp();
         const int lch = s * kQ1StepChunks;
-        consume_step(ring + (s % kQ1SplitStages) * kQ1StageBytes, bfrag + lch * kQ1FragBytesPerChunk,
-                     sinfo + 2 * lch, min(kQ1StepChunks, ch_hi - ch_lo - lch), lc, yacc);
+        consume_step(ring + (s % kQ1SplitStages) * kQ1StageBytes, bfrag_base(smem, zero, lch, lc),
+                     sinfo + 4 * lch, min(kQ1StepChunks, ch_hi - ch_lo - lch), lc, yacc);
         __syncwarp();
     }
     cp_async_wait<0>();
@@ -680,6 +842,8 @@ static int num_sms()
 }
 
 struct Q1Plan {
+    bool lean;          // lean stream kernel
+    int warps;          // its warps per CTA
     bool stream;        // stream kernel (else split kernel)
     int nchunks, blocksN, L, nslices, grid_x, grid_y;
     size_t act_smem, smem;
@@ -687,7 +851,8 @@ struct Q1Plan {
     bool ok;
 };
 
-static Q1Plan q1_plan(int R, int N, int K, int sms)
+// aligned: every matrix's signs and scales start on a 16-byte boundary.
+static Q1Plan q1_plan(int R, int N, int K, int sms, bool aligned = false)
 {
     Q1Plan P = {};
     P.nchunks = (K + kQ1ChunkK - 1) / kQ1ChunkK;
@@ -697,8 +862,28 @@ static Q1Plan q1_plan(int R, int N, int K, int sms)
     P.act_bytes = align256(P.xcopy_off + (size_t)K * 2u);
     const long long units = (long long)R * P.blocksN;
     const size_t per_chunk = kQ1FragBytesPerChunk + kQ1InfoBytesPerChunk;
-    const size_t whole = ((size_t)P.nchunks * per_chunk + 15) & ~size_t(15);
+    const size_t whole = (size_t)P.nchunks * per_chunk + kQ1ZeroBytes;  // fragments, constants, zero block
     const size_t ring_stream = (size_t)kQ1Warps * kQ1WarpRing;
+    // lean stream kernel: whole 1024-k steps and 32-row blocks, as many warps
+    // (at most kQ1LMaxWarps) as fit next to the activation, >= 2 cells per warp
+    if (aligned && K % 1024 == 0 && N % kQ1StepRows == 0) {
+        const size_t per_warp = (size_t)kQ1LStages * kQ1LStageBytes;
+        const long long fit = whole < (size_t)kQ1MaxSmem ? (long long)(((size_t)kQ1MaxSmem - whole) / per_warp) : 0;
+        const int warps = (int)std::min<long long>(kQ1LMaxWarps, fit);
+        if (warps >= kQ1LMinWarps && units >= 2LL * sms * warps) {
+            P.lean = true;
+            P.stream = true;
+            P.warps = warps;
+            P.L = P.nchunks;
+            P.nslices = 1;
+            P.act_smem = whole;
+            P.smem = whole + (size_t)warps * per_warp;
+            P.grid_x = (int)std::min<long long>(sms, (units + warps - 1) / warps);
+            P.grid_y = 1;
+            P.ok = true;
+            return P;
+        }
+    }
     // stream kernel: enough 32-row blocks for >= 2 cells per warp slot, and
     // the whole activation fits next to the rings
     if (units >= 2LL * sms * 2 * kQ1Warps && whole + ring_stream <= (size_t)kQ1MaxSmem) {
@@ -725,7 +910,7 @@ static Q1Plan q1_plan(int R, int N, int K, int sms)
     while (true) {
         P.L = (P.nchunks + S - 1) / S;
         P.nslices = (P.nchunks + P.L - 1) / P.L;
-        P.act_smem = ((size_t)P.L * per_chunk + 15) & ~size_t(15);
+        P.act_smem = (size_t)P.L * per_chunk + kQ1ZeroBytes;
         P.smem = P.act_smem + ring_split + kQ1BuildScratch;
         if (P.smem <= (size_t)kQ1MaxSmem || S >= kQ1MaxCluster) break;
         S = std::min(kQ1MaxCluster, S * 2);
@@ -789,13 +974,13 @@ static lowbit_status q1m1_launch(const Q1Plan &P, const uint8_t *const *bits, co
     p.blocksN = P.blocksN;
     p.cells = (int)((long long)R * P.blocksN);
     p.act_smem = (int)P.act_smem;
-    void (*kern)(const Q1Group, const Q1Params) = P.stream ? k_q1_m1_stream : k_q1_m1_split;
+    void (*kern)(const Q1Group, const Q1Params) = P.lean ? k_q1_m1_lean : P.stream ? k_q1_m1_stream : k_q1_m1_split;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQ1MaxSmem) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(P.grid_x, P.grid_y);
-    cfg.blockDim = dim3(P.stream ? kQ1Warps * 32 : kQ1SplitWarps * 32);
+    cfg.blockDim = dim3(P.lean ? P.warps * 32 : P.stream ? kQ1Warps * 32 : kQ1SplitWarps * 32);
     cfg.dynamicSmemBytes = P.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -819,7 +1004,11 @@ lowbit_status q1m1_gemv_launch(const uint8_t *const *bits, const uint16_t *const
                                float *const *y, int R, int N, int K, cudaStream_t st)
 {
     if (use_tc(K)) return q1tc_gemv_launch(bits, scales, act, y, R, N, K, st);
-    return q1m1_launch(q1_plan(R, N, K, num_sms()), bits, scales, act, nullptr, y, R, N, K, st);
+    bool aligned = true;
+    for (int r = 0; r < R; ++r)
+        aligned = aligned && (reinterpret_cast<uintptr_t>(bits[r]) & 15u) == 0 &&
+                  (reinterpret_cast<uintptr_t>(scales[r]) & 15u) == 0;
+    return q1m1_launch(q1_plan(R, N, K, num_sms(), aligned), bits, scales, act, nullptr, y, R, N, K, st);
 }
 
 // One matrix straight from x, in one launch (the split kernel builds its
@@ -1021,7 +1210,8 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
     __shared__ float red[kStWarps];
     uint8_t *frag = smem;                                                  // 4 chunks of fragments
     float2 *info = reinterpret_cast<float2 *>(smem + kStSliceChunks * kQ1FragBytesPerChunk);
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem + kStSliceChunks * kQ1FragBytesPerChunk + 256);
+    uint8_t *zero = smem + kStSliceChunks * (kQ1FragBytesPerChunk + kQ1InfoBytesPerChunk);
+    uint16_t *xs = reinterpret_cast<uint16_t *>(zero + kQ1ZeroBytes);
     int8_t(*lwall)[256] = reinterpret_cast<int8_t(*)[256]>(reinterpret_cast<uint8_t *>(xs) + kStSliceK * 2);
     float *xsf = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(lwall) + 4 * 4 * 256);  // raw slice values
     uint8_t *rings = reinterpret_cast<uint8_t *>(xsf) + kStSliceK * 4;
@@ -1049,6 +1239,7 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
     for (int t = 0; t < kStStages - 1; ++t) issue_next();
 
     pdl_wait_primary();  // x is produced by earlier kernels
+    clear_zero_block(zero);  // ordered before its first read by the phase's barriers
     const LaneConst lc = lane_const(lane);
     StIt cs;  // consume position
     st_first(cs, p, G, c, warp, nph);
@@ -1138,13 +1329,13 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
         __syncthreads();
         if (warp < kStSliceChunks)
             q1_build_chunk_warp(xs - s * kStSliceK, q.K, s * kStSliceChunks + warp,
-                                frag + warp * kQ1FragBytesPerChunk, info + 2 * warp, lwall + 4 * warp, lane);
+                                frag + warp * kQ1FragBytesPerChunk, info + 4 * warp, lwall + 4 * warp, lane);
         __syncthreads();
 
         // ---- this warp's units of the phase ----
         float *out = p.buf + (size_t)(ph_idx % 3) * bufn;
         const int fold = (q.ph == 4 && p.rec_out == nullptr) ? q.N : 0;  // up's rows land on gate's
-        const float2 *sinfo = info + lc.h;
+        const float2 *sinfo = info + lc.tq;
         while (cs.p == ph_idx) {
             float yacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
             const int b = st_block(q, G, c, warp, cs.j);
@@ -1153,8 +1344,8 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
                 cp_async_wait<kStStages - 1>();
                 __syncwarp();
                 const int lch = t * kQ1StepChunks;
-                consume_step(ring + (ncs % kStStages) * kQ1StageBytes, frag + lane * 8 + lch * kQ1FragBytesPerChunk,
-                             sinfo + 2 * lch, kQ1StepChunks, lc, yacc);
+                consume_step(ring + (ncs % kStStages) * kQ1StageBytes, bfrag_base(frag, zero, lch, lc),
+                             sinfo + 4 * lch, kQ1StepChunks, lc, yacc);
                 __syncwarp();
                 ++ncs;
                 st_next(cs, p, G, c, warp, nph);
@@ -1192,8 +1383,8 @@ lowbit_status q1stack_launch(const uint8_t *const *bits, const uint16_t *const *
     p.H = H;
     p.F = F;
     p.eps = eps;
-    const size_t smem = kStSliceChunks * kQ1FragBytesPerChunk + 256 + kStSliceK * 2 + 4 * 4 * 256 + kStSliceK * 4 +
-                        (size_t)kStWarps * kStStages * kQ1StageBytes;
+    const size_t smem = kStSliceChunks * (kQ1FragBytesPerChunk + kQ1InfoBytesPerChunk) + kQ1ZeroBytes +
+                        kStSliceK * 2 + 4 * 4 * 256 + kStSliceK * 4 + (size_t)kStWarps * kStStages * kQ1StageBytes;
     if (cudaFuncSetAttribute(k_q1_stack_m1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
     int per_sm = 0, sms = num_sms();

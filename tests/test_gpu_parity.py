@@ -178,6 +178,34 @@ def test_q1_group_matches_oracle_and_single_calls(lb, R, N, K):
         np.testing.assert_allclose(single, host(ys[r]), rtol=0, atol=1e-5 * float(np.abs(host(ys[r])).max()))
 
 
+@pytest.mark.parametrize("R,N,K,xkind", [(40, 4096, 1024, "normal"), (148, 1024, 5120, "normal"),
+                                         (38, 4096, 17408, "normal"), (48, 4096, 2048, "extreme")])
+def test_q1_large_group(lb, R, N, K, xkind):
+    """Groups with >= 4736 32-row cells: on 148 SMs these take the persistent
+    kernel with 1024-k steps.  Sampled rows of three matrices against the
+    oracle; every output is finite and written."""
+    x = synth.bf16_normal(2700 + R, (1, K)).copy()
+    if xkind == "extreme":  # large and tiny activations in the same groups
+        x[0, ::3] = synth.to_bf16_bits(np.full(len(x[0, ::3]), 3.0e4))
+        x[0, 1::7] = synth.to_bf16_bits(np.full(len(x[0, 1::7]), 1.0e-20))
+    act = torch.zeros(lb.lowbit_q1g128_act_bytes(1, K), dtype=torch.uint8, device="cuda")
+    lb.lowbit_q1g128_prepare_act(dev(x), act)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2700 + R)
+    bits_d = [torch.randint(0, 256, (N, K // 8), generator=g, device="cuda", dtype=torch.uint8) for _ in range(R)]
+    scales_d = [(torch.randn((N, K // 128), generator=g, device="cuda") * 0.02).abs().half().view(torch.int16)
+                for _ in range(R)]
+    ys = [torch.full((1, N), float("nan"), dtype=torch.float32, device="cuda") for _ in range(R)]
+    lb.lowbit_q1g128_gemv_act_group(bits_d, scales_d, act, ys, 1)
+    _sync()
+    assert all(bool(torch.isfinite(y).all()) for y in ys)
+    for r in (0, R // 2, R - 1):
+        b, s = host(bits_d[r]), host(scales_d[r]).view(np.uint16)
+        ms, ns = sample_pairs(1, N, 96, r)
+        y64, ab = oracle.q1_gemv_at(b, s, x, ms, ns)
+        check_float(host(ys[r])[ms, ns], y64, ab, f"q1 large group R={R} N={N} K={K} r={r}")
+
+
 def test_q1_special_inputs(lb):
     N, K = 64, 512
     bits, scales, _ = _q1_problem(3000, 1, N, K)
