@@ -26,6 +26,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -249,17 +250,16 @@ def run_q1_4096(args, world, rank, local):
         scales.append(s)
     x = torch.from_numpy(synth.bf16_normal(seed, (M, K)).view(np.int16)).to(dev)
     y = torch.empty((R, M, N), dtype=torch.float32, device=dev)
-    act = torch.empty(lb.lowbit_q1g128_act_bytes(M, K), dtype=torch.uint8, device=dev)
-    ws = torch.zeros(max(16, lb.lowbit_q1g128_act_workspace_bytes(R, M, N, K)), dtype=torch.uint8, device=dev)
+    need = lb.lowbit_q1g128_group_workspace_bytes(R, M, N, K)
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev) if need else None
     stream = torch.cuda.Stream(device=dev)
 
     ys = [y[r] for r in range(R)]
 
     def step():
-        lb.lowbit_q1g128_prepare_act(x, act, stream=stream)
-        lb.lowbit_q1g128_gemv_act_group(bits, scales, act, ys, M, workspace=ws, stream=stream)
+        lb.lowbit_q1g128_gemv_group(bits, scales, x, ys, workspace=ws, stream=stream)
 
-    launches_per_step = 2
+    launches_per_step = 1 if need == 0 else 2  # one launch from x, else prepare + product
     # eager warm-up (also loads the module), then capture one step in a graph
     with torch.cuda.stream(stream):
         step()
@@ -334,7 +334,8 @@ def run_q1_4096(args, world, rank, local):
                    "weight_sets_per_step": R, "bytes_per_gemv": per,
                    "l2": f"inputs larger than L2: {R} distinct weight sets, {R * per / 2**20:.0f} MiB "
                          f"per step vs {l2 / 2**20:.0f} MiB L2",
-                   "step": "1 activation prepare + 1 grouped launch of R GEMVs, one CUDA graph",
+                   "step": ("1 grouped launch of R GEMVs from x" if launches_per_step == 1 else
+                            "1 activation prepare + 1 grouped launch of R GEMVs") + ", one CUDA graph",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
@@ -357,8 +358,10 @@ def run_q1_4096(args, world, rank, local):
 # the other workloads (one JSON line each, with their own metric)
 # ---------------------------------------------------------------------------
 
-def _graph_time(step, stream, steps, warmup):
-    """Capture step() in a CUDA graph on `stream`; return ms per replay."""
+def _graph_time(step, stream, steps, warmup, min_ms=20.0):
+    """Capture step() in a CUDA graph on `stream`; return ms per replay.
+    At least `steps` replays are timed, and more when those take under
+    min_ms, so that the launch of the first replay is a small part of it."""
     import torch
     with torch.cuda.stream(stream):
         step()
@@ -369,16 +372,24 @@ def _graph_time(step, stream, steps, warmup):
     for _ in range(warmup):
         graph.replay()
     stream.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(steps):
-            graph.replay()
-        e1.record(stream)
-    e1.synchronize()
-    ms = e0.elapsed_time(e1) / steps
+
+    def timed(n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(n):
+                graph.replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1)
+
+    n = max(1, steps)
+    total = timed(n)
+    if total < min_ms:
+        n = min(100000, int(math.ceil(n * min_ms / max(total, 1e-3))))
+        total = timed(n)
     del graph
-    return ms
+    return total / n
 
 
 def _emit(rank, line):
@@ -446,17 +457,17 @@ def run_q1_sweep(args, world, rank, local):
             ys = [torch.empty((M, N), dtype=torch.float32, device=dev) for _ in range(R)]
             stream = torch.cuda.Stream(device=dev)
             if M == 1:
-                act = torch.empty(lb.lowbit_q1g128_act_bytes(1, K), dtype=torch.uint8, device=dev)
+                need = lb.lowbit_q1g128_group_workspace_bytes(R, 1, N, K)
+                ws = torch.zeros(need, dtype=torch.uint8, device=dev) if need else None
 
                 def step():
-                    lb.lowbit_q1g128_prepare_act(x, act, stream=stream)
-                    lb.lowbit_q1g128_gemv_act_group([b for b, _ in mats], [s for _, s in mats], act, ys, 1,
-                                                    stream=stream)
+                    lb.lowbit_q1g128_gemv_group([b for b, _ in mats], [s for _, s in mats], x, ys, workspace=ws,
+                                                stream=stream)
             else:
                 def step():
                     for r in range(R):
                         lb.lowbit_q1g128_gemv(mats[r][0], mats[r][1], x, ys[r], stream=stream)
-            ms = max_over_ranks(_graph_time(step, stream, max(3, args.steps // 5), args.warmup), world)
+            ms = max_over_ranks(_graph_time(step, stream, max(20, args.steps), args.warmup), world)
             results.append({"N": N, "K": K, "M": M, "weight_sets": R,
                             "gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
                             "us_per_gemv": round(ms * 1e3 / R, 3)})
@@ -495,7 +506,7 @@ def run_int4(args, world, rank, local):
         def step():
             for r in range(R):
                 lb.lowbit_int4g64_gemm(qs[r], ss[r], x, y[r], workspace=ws, stream=stream)
-        ms = max_over_ranks(_graph_time(step, stream, max(3, args.steps // 5), args.warmup), world)
+        ms = max_over_ranks(_graph_time(step, stream, max(20, args.steps), args.warmup), world)
         results.append({"M": M, "us_per_call": round(ms * 1e3 / R, 3),
                         "weight_gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
                         "tflops": round(2.0 * M * N * K * R / (ms * 1e-3) / 1e12, 2)})

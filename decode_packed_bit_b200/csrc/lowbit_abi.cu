@@ -34,6 +34,9 @@ int q1stack_fault_flag();
 lowbit_status q1sm_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 lowbit_status q1m1_gemv_fused_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
                                      cudaStream_t);
+lowbit_status q1m1_gemv_x_group_launch(const uint8_t *const *, const uint16_t *const *, const uint16_t *,
+                                       float *const *, int, int, int, cudaStream_t);
+bool q1m1_x_group_supported(int R, int N, int K);
 lowbit_status q1m1_gemv_launch(const uint8_t *const *, const uint16_t *const *, const void *, float *const *,
                                int, int, int, cudaStream_t);
 
@@ -217,6 +220,41 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits, const u
         if (s != LOWBIT_OK) return s;
     }
     return LOWBIT_OK;
+}
+
+size_t lowbit_q1g128_group_workspace_bytes(int R, int M, int N, int K)
+{
+    if (R < 1 || q1_shape_ok(M, N, K) != LOWBIT_OK) return 0;
+    if (M == 1 && q1m1_x_group_supported(R, N, K)) return 0;
+    return al256(lowbit_q1g128_act_bytes(M, K)) + lowbit_q1g128_act_workspace_bytes(R, M, N, K);
+}
+
+lowbit_status lowbit_q1g128_gemv_group(const uint8_t *const *w_bits, const uint16_t *const *w_scales,
+                                       const uint16_t *x, float *const *y, int R, int M, int N, int K,
+                                       void *workspace, size_t workspace_bytes, void *stream)
+{
+    LB_CHECK(R >= 1 && R <= q1m1_max_group() && w_bits && w_scales && y && x, LOWBIT_ERR_INVALID_ARG);
+    lowbit_status s = q1_shape_ok(M, N, K);
+    if (s != LOWBIT_OK) return s;
+    LB_CHECK(aligned16(x), LOWBIT_ERR_MISALIGNED);
+    for (int r = 0; r < R; ++r) {
+        LB_CHECK(w_bits[r] && w_scales[r] && y[r], LOWBIT_ERR_INVALID_ARG);
+        LB_CHECK(aligned16(w_bits[r]) && aligned16(w_scales[r]) && aligned16(y[r]), LOWBIT_ERR_MISALIGNED);
+    }
+    const size_t need = lowbit_q1g128_group_workspace_bytes(R, M, N, K);
+    LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
+    cudaStream_t st = as_stream(stream);
+    if (M == 1) {
+        s = q1m1_gemv_x_group_launch(w_bits, w_scales, x, y, R, N, K, st);
+        if (s != LOWBIT_ERR_UNSUPPORTED_SHAPE) return s;
+    }
+    uint8_t *act = static_cast<uint8_t *>(workspace);
+    const size_t act_bytes = al256(lowbit_q1g128_act_bytes(M, K));
+    s = lowbit_q1g128_prepare_act(x, M, K, act, act_bytes, stream);
+    if (s != LOWBIT_OK) return s;
+    return lowbit_q1g128_gemv_act_group(w_bits, w_scales, act, y, R, M, N, K, act + act_bytes,
+                                        workspace_bytes - act_bytes, stream);
 }
 
 lowbit_status lowbit_q1g128_gemv_act(const uint8_t *w_bits, const uint16_t *w_scales, const void *act,

@@ -581,70 +581,106 @@ __device__ __forceinline__ void cp_async16_full(unsigned dst, const void *src)
 // One staged step.  woff[c]: this lane's byte offset of chunk c in row g of
 // a stage; soff: its scale offset (row g, group h of chunk 0); bf: its B
 // fragment base (bfrag_base); inf: its (c, n) pair of the step's first chunk.
+// The chunks go in groups of kQ1LInter: inside a group the bit planes are the
+// outer loop, so 2 kQ1LInter accumulator chains are in flight at once.
+#ifndef LOWBIT_Q1_LEAN_INTER
+#define LOWBIT_Q1_LEAN_INTER 2
+#endif
+constexpr int kQ1LInter = LOWBIT_Q1_LEAN_INTER;
+static_assert(kQ1LChunks % kQ1LInter == 0, "chunk groups must tile the step");
+
 __device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *bf, const float2 *inf,
                                              const int (&woff)[kQ1LChunks], int soff, float (&yacc)[2][2])
 {
 #pragma unroll
-    for (int c = 0; c < kQ1LChunks; ++c) {
-        uint2 w[2][2];  // [tile][row g / g+8]
+    for (int c0 = 0; c0 < kQ1LChunks; c0 += kQ1LInter) {
+        uint2 w[kQ1LInter][2][2];  // [chunk][tile][row g / g+8]
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
+        for (int q = 0; q < kQ1LInter; ++q)
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
-                w[t][r] = *reinterpret_cast<const uint2 *>(st + woff[c] + (16 * t + 8 * r) * kQ1LRowBytes);
-        int d[2][4];
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+                    w[q][t][r] = *reinterpret_cast<const uint2 *>(st + woff[c0 + q] + (16 * t + 8 * r) * kQ1LRowBytes);
+        int d[kQ1LInter][2][4];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const uint32_t m = 0x01010101u << i;
-            const uint2 b = *reinterpret_cast<const uint2 *>(bf + c * kQ1FragBytesPerChunk + i * 128);
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                if (i == 0)
-                    mma_u8s8_z(d[t], w[t][0].x & m, w[t][1].x & m, w[t][0].y & m, w[t][1].y & m, b.x, b.y);
-                else
-                    mma_u8s8(d[t], w[t][0].x & m, w[t][1].x & m, w[t][0].y & m, w[t][1].y & m, b.x, b.y);
+            for (int q = 0; q < kQ1LInter; ++q) {
+                const uint2 b = *reinterpret_cast<const uint2 *>(bf + (c0 + q) * kQ1FragBytesPerChunk + i * 128);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const uint2 w0 = w[q][t][0], w1 = w[q][t][1];
+                    if (i == 0)
+                        mma_u8s8_z(d[q][t], w0.x & m, w1.x & m, w0.y & m, w1.y & m, b.x, b.y);
+                    else
+                        mma_u8s8(d[q][t], w0.x & m, w1.x & m, w0.y & m, w1.y & m, b.x, b.y);
+                }
             }
         }
-        const float2 ci = inf[4 * c];
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
+        for (int q = 0; q < kQ1LInter; ++q) {
+            const int c = c0 + q;
+            const float2 ci = inf[4 * c];
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const uint16_t sc = *reinterpret_cast<const uint16_t *>(st + soff + (16 * t + 8 * r) * 16 + c * 4);
-                yacc[t][r] =
-                    fmaf(f16_bits_to_float(sc), fmaf(ci.x, limb_pair(d[t][2 * r], d[t][2 * r + 1]), ci.y), yacc[t][r]);
-            }
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const uint16_t sc =
+                        *reinterpret_cast<const uint16_t *>(st + soff + (16 * t + 8 * r) * 16 + c * 4);
+                    yacc[t][r] = fmaf(f16_bits_to_float(sc), fmaf(ci.x, limb_pair(d[q][t][2 * r], d[q][t][2 * r + 1]), ci.y),
+                                      yacc[t][r]);
+                }
+        }
     }
 }
 
+// Work split: CTA b takes the cells [c0, c1) (equal shares of R * N/32);
+// its T = (c1 - c0) * K/1024 steps are cut into equal contiguous ranges, one
+// per warp.  A cell cut between warps w and w+1 is finished through shared
+// memory, tail of w + head of w+1, in that order.  The planner gives every
+// warp at least two cells' worth of steps, so no cell has a third part.
+// With p.x set, every CTA builds the activation fragments from x itself (one
+// chunk per warp at a time, the limb scratch in the warp's idle ring slot).
 __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __grid_constant__ Q1Group grp,
                                                                      const Q1Params p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ float part[2][kQ1LMaxWarps][kQ1StepRows];  // [head / tail][warp][row] of cut cells
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int c0 = (int)((long long)blockIdx.x * p.cells / gridDim.x);
     const int c1 = (int)((long long)(blockIdx.x + 1) * p.cells / gridDim.x);
     const int spc = p.nchunks / kQ1LChunks;  // steps per cell
+    const int T = (c1 - c0) * spc;
+    const int s0 = (int)((long long)warp * T / nw), s1 = (int)((long long)(warp + 1) * T / nw);
     const size_t rowbytes = (size_t)(p.K >> 3);
     const int G = p.K >> 7;
     uint8_t *ring = smem + p.act_smem + warp * (kQ1LStages * kQ1LStageBytes);
     const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
 
-    // issue side: cell icell = (matrix ir, 32-row block iblk), step istep
+    // issue side: step is of this warp's range = cell c0 + is / spc, step is % spc
     const int rq = lane >> 3;
     const unsigned wdst = (unsigned)(rq * kQ1LRowBytes + (((lane & 7) ^ (rq << 1)) << 4));
     const unsigned sdst = (unsigned)(kQ1LStageW + lane * 16);
-    int icell = c0 + warp, ir = icell / p.blocksN, iblk = icell - ir * p.blocksN, istep = 0, islot = 0;
+    int is = s0, islot = 0;
+    int ir = 0, iblk = 0, ist = 0;  // matrix, 32-row block and step in cell of `is`
     const uint8_t *wsrc = nullptr;
     const uint16_t *ssrc = nullptr;
     auto cell_src = [&]() {
-        wsrc = grp.bits[ir] + (size_t)(iblk * kQ1StepRows + rq) * rowbytes + (lane & 7) * 16;
-        ssrc = grp.scales[ir] + (size_t)(iblk * kQ1StepRows + lane) * G;
+        wsrc = grp.bits[ir] + (size_t)(iblk * kQ1StepRows + rq) * rowbytes + (lane & 7) * 16 + ist * kQ1LRowBytes;
+        ssrc = grp.scales[ir] + (size_t)(iblk * kQ1StepRows + lane) * G + ist * 2 * kQ1LChunks;
     };
-    if (icell < c1) cell_src();
+    if (s0 < s1) {
+        const int cell = c0 + s0 / spc;
+        ir = cell / p.blocksN;
+        iblk = cell - ir * p.blocksN;
+        ist = s0 % spc;
+        cell_src();
+    }
     auto issue_next = [&]() {
-        if (icell < c1) {
+        if (is < s1) {
             const unsigned st = ring_s + islot * kQ1LStageBytes;
 #pragma unroll
             for (int u = 0; u < 8; ++u)
@@ -652,15 +688,14 @@ __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __gri
             cp_async16_full(st + sdst, ssrc);
             wsrc += kQ1LRowBytes;
             ssrc += 2 * kQ1LChunks;
-            if (++istep == spc) {
-                istep = 0;
-                icell += nw;
-                iblk += nw;
-                while (iblk >= p.blocksN) {
-                    iblk -= p.blocksN;
+            ++is;
+            if (++ist == spc) {
+                ist = 0;
+                if (++iblk == p.blocksN) {
+                    iblk = 0;
                     ++ir;
                 }
-                if (icell < c1) cell_src();
+                if (is < s1) cell_src();
             }
         }
         cp_async_commit();
@@ -669,9 +704,17 @@ __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __gri
 #pragma unroll
     for (int t = 0; t < kQ1LStages - 1; ++t) issue_next();
 
-    pdl_wait_primary();  // the activation and the outputs follow stream order from here
+    pdl_wait_primary();  // x or the activation, and the outputs, follow stream order from here
     uint8_t *zero = smem + p.act_smem - kQ1ZeroBytes;
-    if (c1 > c0) stage_act(smem, p, 0, p.nchunks);
+    float2 *info = reinterpret_cast<float2 *>(smem + (size_t)p.nchunks * kQ1FragBytesPerChunk);
+    if (p.x != nullptr) {
+        // the ring slot kQ1LStages - 1 of this warp is not in use yet
+        int8_t(*lw)[256] = reinterpret_cast<int8_t(*)[256]>(ring + (kQ1LStages - 1) * kQ1LStageBytes);
+        for (int ch = warp; ch < p.nchunks; ch += nw)
+            q1_build_chunk_warp(p.x, p.K, ch, smem + (size_t)ch * kQ1FragBytesPerChunk, info + 4 * ch, lw, lane);
+    } else if (c1 > c0) {
+        stage_act(smem, p, 0, p.nchunks);
+    }
     clear_zero_block(zero);
     __syncthreads();
 
@@ -683,31 +726,43 @@ __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __gri
     const int soff = kQ1LStageW + g * 16 + (tq >> 1) * 2;
     const bool live = (lane >> 4) == (tq >> 1);
     const uint8_t *bf_live = smem + (lane & 15) * 8, *bf_dead = zero + (lane & 15) * 8;
-    const float2 *inf0 = reinterpret_cast<const float2 *>(smem + (size_t)p.nchunks * kQ1FragBytesPerChunk) + tq;
+    const float2 *inf0 = info + tq;
 
-    int cell = c0 + warp, r = cell / p.blocksN, blk = cell - r * p.blocksN, slot = 0;
-    while (cell < c1) {
+    int s = s0, slot = 0;
+    while (s < s1) {
+        // one cell (or the part of it in [s0, s1))
+        const int cell = c0 + s / spc, st0 = s % spc;
+        const int st1 = min(spc, st0 + (s1 - s));
         float yacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-        for (int s = 0; s < spc; ++s) {
+        for (int t = st0; t < st1; ++t) {
             issue_next();
             cp_async_wait<kQ1LStages - 1>();
             __syncwarp();
             lean_consume(ring + slot * kQ1LStageBytes,
-                         live ? bf_live + s * (kQ1LChunks * kQ1FragBytesPerChunk) : bf_dead,
-                         inf0 + 4 * kQ1LChunks * s, woff, soff, yacc);
+                         live ? bf_live + t * (kQ1LChunks * kQ1FragBytesPerChunk) : bf_dead,
+                         inf0 + 4 * kQ1LChunks * t, woff, soff, yacc);
             __syncwarp();  // every lane is done with this stage before it is refilled
             slot = slot + 1 == kQ1LStages ? 0 : slot + 1;
         }
+        s += st1 - st0;
+        const int r = cell / p.blocksN, blk = cell - r * p.blocksN;
         float *yr = grp.y[r] + blk * kQ1StepRows;
-        finish_cell(yacc, lane, [&](int row, float v) { yr[row] = v; });
-        cell += nw;
-        blk += nw;
-        while (blk >= p.blocksN) {
-            blk -= p.blocksN;
-            ++r;
-        }
+        float *cut = st0 > 0 ? part[0][warp] : (st1 < spc ? part[1][warp] : nullptr);
+        finish_cell(yacc, lane, [&](int row, float v) {
+            if (cut != nullptr)
+                cut[row] = v;
+            else
+                yr[row] = v;
+        });
     }
     cp_async_wait<0>();
+    __syncthreads();
+    // cells cut between warps w and w + 1: one warp per cut, one row per lane
+    if (warp + 1 < nw && s1 % spc != 0 && s1 > s0) {
+        const int cell = c0 + s1 / spc;
+        const int r = cell / p.blocksN, blk = cell - r * p.blocksN;
+        grp.y[r][blk * kQ1StepRows + lane] = part[1][warp][lane] + part[0][warp + 1][lane];
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -868,8 +923,11 @@ static Q1Plan q1_plan(int R, int N, int K, int sms, bool aligned = false)
     // (at most kQ1LMaxWarps) as fit next to the activation, >= 2 cells per warp
     if (aligned && K % 1024 == 0 && N % kQ1StepRows == 0) {
         const size_t per_warp = (size_t)kQ1LStages * kQ1LStageBytes;
-        const long long fit = whole < (size_t)kQ1MaxSmem ? (long long)(((size_t)kQ1MaxSmem - whole) / per_warp) : 0;
+        const size_t cap = (size_t)kQ1MaxSmem - 2 * kQ1LMaxWarps * kQ1StepRows * 4;  // static cut buffers
+        const long long fit = whole < cap ? (long long)((cap - whole) / per_warp) : 0;
         const int warps = (int)std::min<long long>(kQ1LMaxWarps, fit);
+        // >= 2 warps' worth of cells per CTA keeps every warp's step range over
+        // two cells or more, so a cell is cut at most once
         if (warps >= kQ1LMinWarps && units >= 2LL * sms * warps) {
             P.lean = true;
             P.stream = true;
@@ -878,7 +936,7 @@ static Q1Plan q1_plan(int R, int N, int K, int sms, bool aligned = false)
             P.nslices = 1;
             P.act_smem = whole;
             P.smem = whole + (size_t)warps * per_warp;
-            P.grid_x = (int)std::min<long long>(sms, (units + warps - 1) / warps);
+            P.grid_x = sms;
             P.grid_y = 1;
             P.ok = true;
             return P;
@@ -975,7 +1033,7 @@ static lowbit_status q1m1_launch(const Q1Plan &P, const uint8_t *const *bits, co
     p.cells = (int)((long long)R * P.blocksN);
     p.act_smem = (int)P.act_smem;
     void (*kern)(const Q1Group, const Q1Params) = P.lean ? k_q1_m1_lean : P.stream ? k_q1_m1_stream : k_q1_m1_split;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQ1MaxSmem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
@@ -1009,6 +1067,24 @@ lowbit_status q1m1_gemv_launch(const uint8_t *const *bits, const uint16_t *const
         aligned = aligned && (reinterpret_cast<uintptr_t>(bits[r]) & 15u) == 0 &&
                   (reinterpret_cast<uintptr_t>(scales[r]) & 15u) == 0;
     return q1m1_launch(q1_plan(R, N, K, num_sms(), aligned), bits, scales, act, nullptr, y, R, N, K, st);
+}
+
+// R matrices straight from x in one launch, when the shape takes the lean
+// stream kernel (every CTA builds the activation itself); otherwise
+// LOWBIT_ERR_UNSUPPORTED_SHAPE and the caller prepares the activation first.
+lowbit_status q1m1_gemv_x_group_launch(const uint8_t *const *bits, const uint16_t *const *scales, const uint16_t *x,
+                                       float *const *y, int R, int N, int K, cudaStream_t st)
+{
+    if (use_tc(K) || R < 1 || R > kQ1MaxGroup || !q1m1_shape_supported(R, N, K)) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    const Q1Plan P = q1_plan(R, N, K, num_sms(), true);
+    if (!P.lean) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    return q1m1_launch(P, bits, scales, nullptr, x, y, R, N, K, st);
+}
+
+bool q1m1_x_group_supported(int R, int N, int K)
+{
+    return !use_tc(K) && R >= 1 && R <= kQ1MaxGroup && q1m1_shape_supported(R, N, K) &&
+           q1_plan(R, N, K, num_sms(), true).lean;
 }
 
 // One matrix straight from x, in one launch (the split kernel builds its

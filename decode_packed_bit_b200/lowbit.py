@@ -41,6 +41,8 @@ SYMBOLS = [
     ("lowbit_q1g128_prepare_act", I32, [P, I32, I32, P, SZ, P]),
     ("lowbit_q1g128_gemv_act", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
     ("lowbit_q1g128_gemv_act_group", I32, [P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
+    ("lowbit_q1g128_group_workspace_bytes", SZ, [I32, I32, I32, I32]),
+    ("lowbit_q1g128_gemv_group", I32, [P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
     ("lowbit_q1g128_gemv_noalloc", I32, [P, P, P, P, I32, I32, I32, P]),
     ("lowbit_int4g64_workspace_bytes", SZ, [I32, I32, I32]),
     ("lowbit_int4g64_gemm", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
@@ -175,6 +177,25 @@ def lowbit_q1g128_gemv_act_group(w_bits, w_scales, act, ys, M: int, workspace=No
     _check(lib().lowbit_q1g128_gemv_act_group(pb, ps, _ptr(act), py, R, M, N, K, _ptr(workspace),
                                               _nbytes(workspace), _stream(stream)),
            "lowbit_q1g128_gemv_act_group")
+
+
+def lowbit_q1g128_group_workspace_bytes(R: int, M: int, N: int, K: int) -> int:
+    return lib().lowbit_q1g128_group_workspace_bytes(R, M, N, K)
+
+
+def lowbit_q1g128_gemv_group(w_bits, w_scales, x, ys, workspace=None, stream=None):
+    """y_r = W_r x for equal-length lists of weight tensors and outputs; x [M][K]
+    bf16 bits.  workspace: lowbit_q1g128_group_workspace_bytes(R, M, N, K)
+    bytes (None when that is 0)."""
+    R = len(w_bits)
+    M, K = x.shape
+    N = w_bits[0].shape[0]
+    pb, kb = _ptr_array(w_bits)
+    ps, ks = _ptr_array(w_scales)
+    py, ky = _ptr_array(ys)
+    _check(lib().lowbit_q1g128_gemv_group(pb, ps, _ptr(x), py, R, M, N, K, _ptr(workspace), _nbytes(workspace),
+                                          _stream(stream)),
+           "lowbit_q1g128_gemv_group")
 
 
 def lowbit_q1g128_gemv_noalloc(w_bits, w_scales, x, y, stream=None):

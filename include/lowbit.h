@@ -158,6 +158,24 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits,
                                            float *const *y, int R, int M, int N, int K,
                                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* The same group product straight from x: y_r = W_r x for R matrices of one
+ * shape [N][K] that read one activation x [M][K] (bf16).
+ *   w_bits, w_scales, y: HOST arrays of R device pointers (1 <= R <= 256),
+ *   16-byte aligned; results as lowbit_q1g128_gemv_act_group.
+ * At M = 1, with K % 1024 == 0, N % 32 == 0 and at least 2 * SMs * 16
+ * (32-row block, matrix) pairs (e.g. 37 or more 4096-row matrices on 148
+ * SMs), this is one launch: every CTA turns x into the operand form itself,
+ * and no workspace is needed.  Otherwise the call prepares the activation in
+ * the workspace and runs lowbit_q1g128_gemv_act_group.
+ * Workspace: lowbit_q1g128_group_workspace_bytes(R, M, N, K) bytes (NULL
+ * allowed when 0).  Calls that share a workspace must be ordered on one
+ * stream. */
+size_t lowbit_q1g128_group_workspace_bytes(int R, int M, int N, int K);
+lowbit_status lowbit_q1g128_gemv_group(const uint8_t *const *w_bits,
+                                       const uint16_t *const *w_scales, const uint16_t *x,
+                                       float *const *y, int R, int M, int N, int K,
+                                       void *workspace, size_t workspace_bytes, void *stream);
+
 /* Allocation-free form of lowbit_q1g128_gemv.  The pages have no
  * counterpart: it exists for callers that cannot allocate device memory --
  * a plugin whose host framework owns every device allocation, a real-time or

@@ -206,6 +206,31 @@ def test_q1_large_group(lb, R, N, K, xkind):
         check_float(host(ys[r])[ms, ns], y64, ab, f"q1 large group R={R} N={N} K={K} r={r}")
 
 
+@pytest.mark.parametrize("R,M,N,K", [(40, 1, 4096, 1024), (38, 1, 4096, 17408), (160, 1, 1024, 3072),
+                                     (3, 1, 515, 1280), (2, 2, 300, 2048)])
+def test_q1_group_from_x(lb, R, M, N, K):
+    """lowbit_q1g128_gemv_group: one launch from x when the shape allows (the
+    first three cases on 148 SMs), else prepare + group product in the
+    workspace.  Sampled outputs of three matrices against the oracle."""
+    x = synth.bf16_normal(2800 + R, (M, K))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2800 + R)
+    bits_d = [torch.randint(0, 256, (N, K // 8), generator=g, device="cuda", dtype=torch.uint8) for _ in range(R)]
+    scales_d = [(torch.randn((N, K // 128), generator=g, device="cuda") * 0.02).abs().half().view(torch.int16)
+                for _ in range(R)]
+    ys = [torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda") for _ in range(R)]
+    need = lb.lowbit_q1g128_group_workspace_bytes(R, M, N, K)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda") if need else None
+    lb.lowbit_q1g128_gemv_group(bits_d, scales_d, dev(x), ys, workspace=ws)
+    _sync()
+    assert all(bool(torch.isfinite(y).all()) for y in ys)
+    for r in (0, R // 2, R - 1):
+        b, s = host(bits_d[r]), host(scales_d[r]).view(np.uint16)
+        ms, ns = sample_pairs(M, N, 96, r)
+        y64, ab = oracle.q1_gemv_at(b, s, x, ms, ns)
+        check_float(host(ys[r])[ms, ns], y64, ab, f"q1 group from x R={R} M={M} N={N} K={K} r={r}")
+
+
 def test_q1_special_inputs(lb):
     N, K = 64, 512
     bits, scales, _ = _q1_problem(3000, 1, N, K)
