@@ -507,9 +507,21 @@ def run_int4(args, world, rank, local):
             for r in range(R):
                 lb.lowbit_int4g64_gemm(qs[r], ss[r], x, y[r], workspace=ws, stream=stream)
         ms = max_over_ranks(_graph_time(step, stream, max(20, args.steps), args.warmup), world)
-        results.append({"M": M, "us_per_call": round(ms * 1e3 / R, 3),
-                        "weight_gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
-                        "tflops": round(2.0 * M * N * K * R / (ms * 1e-3) / 1e12, 2)})
+        res = {"M": M, "us_per_call": round(ms * 1e3 / R, 3),
+               "weight_gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
+               "tflops": round(2.0 * M * N * K * R / (ms * 1e-3) / 1e12, 2)}
+        if M == 1:
+            # the R weight sets read one x: one grouped launch
+            ys = [y[r] for r in range(R)]
+            gws = lb.lowbit_int4g64_group_workspace_bytes(R, M, N, K)
+            gw = torch.zeros(gws, dtype=torch.uint8, device=dev) if gws else None
+
+            def gstep():
+                lb.lowbit_int4g64_gemm_group(qs, ss, x, ys, workspace=gw, stream=stream)
+            gms = max_over_ranks(_graph_time(gstep, stream, max(20, args.steps), args.warmup), world)
+            res["group_us"] = round(gms * 1e3, 3)
+            res["group_weight_gbs"] = round(R * per / (gms * 1e-3) / 1e9, 1)
+        results.append(res)
     assert lb.lowbit_fault_flags() == 0
     _emit(rank, {"metric": "INT4_G64 11008x4096: packed-weight GB/s (M=1) and TFLOP/s (M=32, 256)",
                  "unit": "GB/s", "value": results[0]["weight_gbs"], "n_gpus": world, "higher_is_better": True,

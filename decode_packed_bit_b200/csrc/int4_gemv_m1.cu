@@ -26,6 +26,7 @@
 // thread-block cluster splits K and reduces through distributed shared memory
 // when the rows alone cannot fill the GPU.
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -334,6 +335,143 @@ __global__ void __launch_bounds__(kI4SplitWarps * 32) k_i4_m1_split(const I4Para
 }
 
 // ---------------------------------------------------------------------------
+// grouped kernel: R matrices of one shape that read one x, persistent CTAs
+// ---------------------------------------------------------------------------
+//
+// Cells are (matrix, 32-row block) over all of K, as in the Q1 persistent
+// kernel: CTA b takes the cells [c0, c1), its warps take equal contiguous
+// ranges of the cells' 128-k steps, and a cell cut between warps w and w+1
+// is finished through shared memory (tail of w + head of w+1).  Every CTA
+// builds the whole activation from x, one pair per warp at a time, with the
+// limb scratch in the warp's idle ring slot.  Requires N % 32 == 0.
+
+constexpr int kI4GMaxGroup = 256;
+#ifndef LOWBIT_I4_LEAN_STAGES
+#define LOWBIT_I4_LEAN_STAGES 3
+#endif
+#ifndef LOWBIT_I4_LEAN_WARPS
+#define LOWBIT_I4_LEAN_WARPS 16
+#endif
+constexpr int kI4LStages = LOWBIT_I4_LEAN_STAGES;
+constexpr int kI4LMaxWarps = LOWBIT_I4_LEAN_WARPS;
+constexpr int kI4LMinWarps = 8;
+static_assert(kI4LStages >= 2, "the build scratch lives in the last ring slot");
+
+struct I4Group {
+    const uint8_t *q[kI4GMaxGroup];
+    const uint16_t *scales[kI4GMaxGroup];
+    float *y[kI4GMaxGroup];
+};
+
+struct I4GParams {
+    const uint16_t *x;
+    int N, K, npairs, blocksN, cells, act_smem;
+};
+
+__global__ void __launch_bounds__(kI4LMaxWarps * 32, 1) k_i4_m1_lean(const __grid_constant__ I4Group grp,
+                                                                     const I4GParams p)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ float part[2][kI4LMaxWarps][kI4StepRows];  // [head / tail][warp][row] of cut cells
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int c0 = (int)((long long)blockIdx.x * p.cells / gridDim.x);
+    const int c1 = (int)((long long)(blockIdx.x + 1) * p.cells / gridDim.x);
+    const int spc = p.npairs;  // steps per cell
+    const int T = (c1 - c0) * spc;
+    const int s0 = (int)((long long)warp * T / nw), s1 = (int)((long long)(warp + 1) * T / nw);
+    const size_t rowbytes = (size_t)(p.K >> 1);
+    const int G = p.K >> 6;
+    uint8_t *ring = smem + p.act_smem + warp * (kI4LStages * kI4StageBytes);
+    const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
+
+    // issue side: lane L copies 16-byte column L%4 of rows L/4 + {0,8,16,24}
+    // and the scale pair of row L
+    const unsigned wdst = (unsigned)((lane >> 2) * kI4RowStride + (lane & 3) * 16);
+    const unsigned sdst = (unsigned)(kI4StageW + lane * 4);
+    int is = s0, islot = 0, ir = 0, iblk = 0, ist = 0;
+    const uint8_t *wsrc = nullptr;
+    const uint16_t *ssrc = nullptr;
+    auto cell_src = [&]() {
+        wsrc = grp.q[ir] + (size_t)(iblk * kI4StepRows + (lane >> 2)) * rowbytes + (lane & 3) * 16 + ist * 64;
+        ssrc = grp.scales[ir] + (size_t)(iblk * kI4StepRows + lane) * G + 2 * ist;
+    };
+    if (s0 < s1) {
+        const int cell = c0 + s0 / spc;
+        ir = cell / p.blocksN;
+        iblk = cell - ir * p.blocksN;
+        ist = s0 % spc;
+        cell_src();
+    }
+    auto issue_next = [&]() {
+        if (is < s1) {
+            const unsigned st = ring_s + islot * kI4StageBytes;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) i4_cp16(st + wdst + 8 * u * kI4RowStride, wsrc + (size_t)(8 * u) * rowbytes, true);
+            i4_cp4(st + sdst, ssrc, true);
+            wsrc += 64;
+            ssrc += 2;
+            ++is;
+            if (++ist == spc) {
+                ist = 0;
+                if (++iblk == p.blocksN) {
+                    iblk = 0;
+                    ++ir;
+                }
+                if (is < s1) cell_src();
+            }
+        }
+        i4_commit();
+        islot = islot + 1 == kI4LStages ? 0 : islot + 1;
+    };
+#pragma unroll
+    for (int t = 0; t < kI4LStages - 1; ++t) issue_next();
+
+    pdl_wait_primary();  // x and the outputs follow stream order from here
+    float2 *info = reinterpret_cast<float2 *>(smem + (size_t)p.npairs * kI4FragBytesPerPair);
+    {
+        int8_t(*lw)[128] = reinterpret_cast<int8_t(*)[128]>(ring + (kI4LStages - 1) * kI4StageBytes);
+        for (int pr = warp; pr < p.npairs; pr += nw)
+            i4_build_pair_warp(p.x, p.K, pr, smem + (size_t)pr * kI4FragBytesPerPair, info + 2 * pr, lw, lane);
+    }
+    __syncthreads();
+
+    const uint8_t *bfrag = smem + lane * 8;
+    const float2 *sinfo = info + ((lane & 3) >> 1);
+    int s = s0, slot = 0;
+    while (s < s1) {
+        const int cell = c0 + s / spc, st0 = s % spc;
+        const int st1 = min(spc, st0 + (s1 - s));
+        float yacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        for (int t = st0; t < st1; ++t) {
+            issue_next();
+            i4_wait<kI4LStages - 1>();
+            __syncwarp();
+            i4_consume(ring + slot * kI4StageBytes, bfrag + t * kI4FragBytesPerPair, sinfo[2 * t], lane, yacc);
+            __syncwarp();  // every lane is done with this stage before it is refilled
+            slot = slot + 1 == kI4LStages ? 0 : slot + 1;
+        }
+        s += st1 - st0;
+        const int r = cell / p.blocksN, blk = cell - r * p.blocksN;
+        float *yr = grp.y[r] + blk * kI4StepRows;
+        float *cut = st0 > 0 ? part[0][warp] : (st1 < spc ? part[1][warp] : nullptr);
+        i4_finish(yacc, lane, [&](int row, float v) {
+            if (cut != nullptr)
+                cut[row] = v;
+            else
+                yr[row] = v;
+        });
+    }
+    i4_wait<0>();
+    __syncthreads();
+    if (warp + 1 < nw && s1 % spc != 0 && s1 > s0) {
+        const int cell = c0 + s1 / spc;
+        const int r = cell / p.blocksN, blk = cell - r * p.blocksN;
+        grp.y[r][blk * kI4StepRows + lane] = part[1][warp][lane] + part[0][warp + 1][lane];
+    }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 
@@ -409,6 +547,73 @@ lowbit_status i4m1_launch(const uint8_t *q, const uint16_t *scales, const uint16
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, k_i4_m1_split, p);
+    return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
+// Grouped plan: one CTA per SM with as many warps (<= kI4LMaxWarps) as fit
+// next to the whole activation and as there are cells per SM (each warp needs
+// one cell's worth of steps); fewer than kI4LMinWarps falls back to single
+// calls.  The smaller the rings, the more of the SM's memory stays L1 for
+// the 4-byte scale copies, which is why three stages beat deeper rings.
+struct I4GPlan {
+    int npairs, blocksN, warps;
+    size_t act_smem, smem;
+    bool ok;
+};
+
+static I4GPlan i4g_plan(int R, int N, int K, int sms)
+{
+    I4GPlan P = {};
+    P.npairs = K / kI4PairK;
+    P.blocksN = N / kI4StepRows;
+    if (R < 1 || R > kI4GMaxGroup || N % kI4StepRows != 0 || K % kI4PairK != 0 || P.npairs < 1) return P;
+    P.act_smem = (size_t)P.npairs * (kI4FragBytesPerPair + kI4InfoBytesPerPair);
+    const size_t cap = (size_t)kI4MaxSmem - 2 * kI4LMaxWarps * kI4StepRows * 4;  // static cut buffers
+    const size_t per_warp = (size_t)kI4LStages * kI4StageBytes;
+    const long long fit = P.act_smem < cap ? (long long)((cap - P.act_smem) / per_warp) : 0;
+    P.warps = (int)std::min<long long>(std::min<long long>(kI4LMaxWarps, fit), (long long)R * P.blocksN / sms);
+    P.smem = P.act_smem + (size_t)P.warps * per_warp;
+    P.ok = P.warps >= kI4LMinWarps;
+    return P;
+}
+
+bool i4m1_group_supported(int R, int N, int K) { return i4g_plan(R, N, K, i4_num_sms()).ok; }
+
+lowbit_status i4m1_group_launch(const uint8_t *const *q, const uint16_t *const *scales, const uint16_t *x,
+                                float *const *y, int R, int N, int K, cudaStream_t st)
+{
+    const int sms = i4_num_sms();
+    const I4GPlan P = i4g_plan(R, N, K, sms);
+    if (!P.ok) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    static I4Group grp;  // large: kept off the stack
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int r = 0; r < R; ++r) {
+        grp.q[r] = q[r];
+        grp.scales[r] = scales[r];
+        grp.y[r] = y[r];
+    }
+    I4GParams p = {};
+    p.x = x;
+    p.N = N;
+    p.K = K;
+    p.npairs = P.npairs;
+    p.blocksN = P.blocksN;
+    p.cells = R * P.blocksN;
+    p.act_smem = (int)P.act_smem;
+    if (cudaFuncSetAttribute(k_i4_m1_lean, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) != cudaSuccess)
+        return LOWBIT_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(P.warps * 32);
+    cfg.dynamicSmemBytes = P.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_i4_m1_lean, grp, p);
     return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
 

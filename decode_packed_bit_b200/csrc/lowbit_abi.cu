@@ -34,6 +34,9 @@ int q1stack_fault_flag();
 lowbit_status q1sm_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 lowbit_status q1m1_gemv_fused_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
                                      cudaStream_t);
+bool i4m1_group_supported(int R, int N, int K);
+lowbit_status i4m1_group_launch(const uint8_t *const *, const uint16_t *const *, const uint16_t *, float *const *,
+                                int, int, int, cudaStream_t);
 lowbit_status q1m1_gemv_x_group_launch(const uint8_t *const *, const uint16_t *const *, const uint16_t *,
                                        float *const *, int, int, int, cudaStream_t);
 bool q1m1_x_group_supported(int R, int N, int K);
@@ -319,6 +322,38 @@ lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales, 
     if (M >= 2 && i4sm_supported(M, N, K)) return i4sm_launch(w_q, w_scales, x, y, M, N, K, st);
     if (i4tc_supported(M, N, K)) return i4tc_launch(w_q, w_scales, x, y, M, N, K, st);
     return int4_gemv_simt_launch(w_q, w_scales, x, y, M, N, K, st);
+}
+
+size_t lowbit_int4g64_group_workspace_bytes(int R, int M, int N, int K)
+{
+    (void)R;
+    return lowbit_int4g64_workspace_bytes(M, N, K);
+}
+
+lowbit_status lowbit_int4g64_gemm_group(const uint8_t *const *w_q, const uint16_t *const *w_scales,
+                                        const uint16_t *x, float *const *y, int R, int M, int N, int K,
+                                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    LB_CHECK(R >= 1 && R <= 256 && w_q && w_scales && y && x, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(M >= 1 && N >= 1 && K >= 1, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(K % 64 == 0 && (int64_t)N * K < kMaxElems && (int64_t)M * K < kMaxElems,
+             LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    LB_CHECK(aligned16(x), LOWBIT_ERR_MISALIGNED);
+    for (int r = 0; r < R; ++r) {
+        LB_CHECK(w_q[r] && w_scales[r] && y[r], LOWBIT_ERR_INVALID_ARG);
+        LB_CHECK(aligned16(w_q[r]) && aligned16(w_scales[r]) && aligned16(y[r]), LOWBIT_ERR_MISALIGNED);
+    }
+    const size_t need = lowbit_int4g64_group_workspace_bytes(R, M, N, K);
+    LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
+    cudaStream_t st = as_stream(stream);
+    if (M == 1 && i4m1_group_supported(R, N, K)) return i4m1_group_launch(w_q, w_scales, x, y, R, N, K, st);
+    for (int r = 0; r < R; ++r) {
+        const lowbit_status s =
+            lowbit_int4g64_gemm(w_q[r], w_scales[r], x, y[r], M, N, K, workspace, workspace_bytes, stream);
+        if (s != LOWBIT_OK) return s;
+    }
+    return LOWBIT_OK;
 }
 
 // ---------------------------------------------------------------------------

@@ -640,7 +640,7 @@ __device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *b
 // its T = (c1 - c0) * K/1024 steps are cut into equal contiguous ranges, one
 // per warp.  A cell cut between warps w and w+1 is finished through shared
 // memory, tail of w + head of w+1, in that order.  The planner gives every
-// warp at least two cells' worth of steps, so no cell has a third part.
+// warp at least one cell's worth of steps, so no cell has a third part.
 // With p.x set, every CTA builds the activation fragments from x itself (one
 // chunk per warp at a time, the limb scratch in the warp's idle ring slot).
 __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __grid_constant__ Q1Group grp,
@@ -925,10 +925,10 @@ static Q1Plan q1_plan(int R, int N, int K, int sms, bool aligned = false)
         const size_t per_warp = (size_t)kQ1LStages * kQ1LStageBytes;
         const size_t cap = (size_t)kQ1MaxSmem - 2 * kQ1LMaxWarps * kQ1StepRows * 4;  // static cut buffers
         const long long fit = whole < cap ? (long long)((cap - whole) / per_warp) : 0;
-        const int warps = (int)std::min<long long>(kQ1LMaxWarps, fit);
-        // >= 2 warps' worth of cells per CTA keeps every warp's step range over
-        // two cells or more, so a cell is cut at most once
-        if (warps >= kQ1LMinWarps && units >= 2LL * sms * warps) {
+        // >= one cell per warp keeps every warp's step range at least one
+        // cell long, so a cell is cut at most once
+        const int warps = (int)std::min<long long>(std::min<long long>(kQ1LMaxWarps, fit), units / sms);
+        if (warps >= kQ1LMinWarps) {
             P.lean = true;
             P.stream = true;
             P.warps = warps;

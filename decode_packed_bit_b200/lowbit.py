@@ -46,6 +46,8 @@ SYMBOLS = [
     ("lowbit_q1g128_gemv_noalloc", I32, [P, P, P, P, I32, I32, I32, P]),
     ("lowbit_int4g64_workspace_bytes", SZ, [I32, I32, I32]),
     ("lowbit_int4g64_gemm", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
+    ("lowbit_int4g64_group_workspace_bytes", SZ, [I32, I32, I32, I32]),
+    ("lowbit_int4g64_gemm_group", I32, [P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
     ("lowbit_q2_mlp_forward", I32, [P, P, I32, P, I32, P, P, P]),
     ("lowbit_rmsnorm_bf16", I32, [P, P, I32, I32, F32, P, P]),
     ("lowbit_q1g128_stack_workspace_bytes", SZ, [I32, I32, I32]),
@@ -221,6 +223,24 @@ def lowbit_int4g64_gemm(w_q, w_scales, x, y, workspace=None, stream=None):
                                      _ptr(workspace), wsb, _stream(stream)), "lowbit_int4g64_gemm")
 
 
+def lowbit_int4g64_group_workspace_bytes(R: int, M: int, N: int, K: int) -> int:
+    return lib().lowbit_int4g64_group_workspace_bytes(R, M, N, K)
+
+
+def lowbit_int4g64_gemm_group(w_q, w_scales, x, ys, workspace=None, stream=None):
+    """y_r = W_r x for equal-length lists of INT4_G64 weights (uint8 [N][K/2],
+    fp16 bits [N][K/64]) and fp32 outputs [M][N]; x [M][K] bf16 bits."""
+    R = len(w_q)
+    M, K = x.shape
+    N = w_q[0].shape[0]
+    pq, kq = _ptr_array(w_q)
+    ps, ks = _ptr_array(w_scales)
+    py, ky = _ptr_array(ys)
+    _check(lib().lowbit_int4g64_gemm_group(pq, ps, _ptr(x), py, R, M, N, K, _ptr(workspace), _nbytes(workspace),
+                                           _stream(stream)),
+           "lowbit_int4g64_gemm_group")
+
+
 # -- Q2 MLP -----------------------------------------------------------------------
 
 def lowbit_q2_mlp_forward(w_packed, dims, x, logits, argmax=None, stream=None):
@@ -256,3 +276,4 @@ def lowbit_q1g128_stack_step(w_bits, w_scales, x, hidden, ffn, workspace, eps=1e
     _check(lib().lowbit_q1g128_stack_step(bits, scales, n // 7, hidden, ffn, _ptr(x), float(eps), _ptr(workspace), wsb,
                                           _ptr(record_inputs), _ptr(record_outputs), _stream(stream)),
            "lowbit_q1g128_stack_step")
+

@@ -162,8 +162,8 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits,
  * shape [N][K] that read one activation x [M][K] (bf16).
  *   w_bits, w_scales, y: HOST arrays of R device pointers (1 <= R <= 256),
  *   16-byte aligned; results as lowbit_q1g128_gemv_act_group.
- * At M = 1, with K % 1024 == 0, N % 32 == 0 and at least 2 * SMs * 16
- * (32-row block, matrix) pairs (e.g. 37 or more 4096-row matrices on 148
+ * At M = 1, with K % 1024 == 0, N % 32 == 0 and at least SMs * 8
+ * (32-row block, matrix) pairs (e.g. 10 or more 4096-row matrices on 148
  * SMs), this is one launch: every CTA turns x into the operand form itself,
  * and no workspace is needed.  Otherwise the call prepares the activation in
  * the workspace and runs lowbit_q1g128_gemv_act_group.
@@ -255,6 +255,22 @@ size_t lowbit_int4g64_workspace_bytes(int M, int N, int K);
 lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales,
                                   const uint16_t *x, float *y, int M, int N, int K,
                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Group form: y_r = W_r x for R matrices of one shape [N][K] that read one
+ * activation x [M][K] (w_q, w_scales, y: HOST arrays of R device pointers,
+ * 1 <= R <= 256, 16-byte aligned).  At M = 1, with N % 32 == 0 and at least
+ * SMs * 8 (32-row block, matrix) pairs (e.g. 4 or more 11008-row matrices
+ * on 148 SMs), this is one launch of a persistent kernel: one CTA per SM
+ * builds the activation from x and streams its equal share of every matrix's
+ * weights.  Other shapes run lowbit_int4g64_gemm once per matrix.  Results
+ * equal the single calls up to fp32 summation order.
+ * workspace: lowbit_int4g64_group_workspace_bytes(R, M, N, K) bytes (0
+ * today; NULL allowed when 0). */
+size_t lowbit_int4g64_group_workspace_bytes(int R, int M, int N, int K);
+lowbit_status lowbit_int4g64_gemm_group(const uint8_t *const *w_q,
+                                        const uint16_t *const *w_scales, const uint16_t *x,
+                                        float *const *y, int R, int M, int N, int K,
+                                        void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------
  * Z80-style 2-bit integer MLP ("Show HN: Z80-uLM"), fused over all layers:

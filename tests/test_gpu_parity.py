@@ -331,6 +331,37 @@ def test_int4_11008x4096_sampled(lb, M):
     assert lb.lowbit_fault_flags() == 0
 
 
+@pytest.mark.parametrize("R,M,N,K", [(17, 1, 11008, 4096), (80, 1, 1024, 1024), (7, 1, 11008, 11008),
+                                     (40, 1, 1024, 1024), (3, 32, 300, 512), (2, 1, 300, 448)])
+def test_int4_group(lb, R, M, N, K):
+    """lowbit_int4g64_gemm_group: the persistent kernel for the first three
+    cases on 148 SMs, single calls for the rest.  Sampled outputs of three
+    matrices against the oracle, and the group equals single calls up to fp32
+    summation order."""
+    x = synth.bf16_normal(4800 + R, (M, K))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4800 + R)
+    q_d = [torch.randint(0, 256, (N, K // 2), generator=g, device="cuda", dtype=torch.uint8) for _ in range(R)]
+    s_d = [(torch.randn((N, K // 64), generator=g, device="cuda") * 0.01).abs().half().view(torch.int16)
+           for _ in range(R)]
+    ys = [torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda") for _ in range(R)]
+    x_d = dev(x)
+    lb.lowbit_int4g64_gemm_group(q_d, s_d, x_d, ys)
+    _sync()
+    assert all(bool(torch.isfinite(y).all()) for y in ys)
+    for r in (0, R // 2, R - 1):
+        q, s = host(q_d[r]), host(s_d[r]).view(np.uint16)
+        ms, ns = sample_pairs(M, N, 96, r)
+        y64, ab = oracle.int4_gemv_at(q, s, x, ms, ns)
+        check_float(host(ys[r])[ms, ns], y64, ab, f"int4 group R={R} M={M} N={N} K={K} r={r}")
+        single = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        lb.lowbit_int4g64_gemm(q_d[r], s_d[r], x_d, single)
+        _sync()
+        ref = host(ys[r])
+        np.testing.assert_allclose(host(single), ref, rtol=0, atol=1e-5 * float(np.abs(ref).max()))
+    assert lb.lowbit_fault_flags() == 0
+
+
 # ---------------------------------------------------------------------------
 # Z80-style 2-bit MLP: bit-exact
 # ---------------------------------------------------------------------------
