@@ -60,6 +60,15 @@ constexpr int kQ1ChunkK = 256;
 constexpr int kQ1FragBytesPerChunk = 1024;  // 8 mma x 16 live lanes x 8 bytes
 constexpr int kQ1InfoBytesPerChunk = 32;    // four lane quarters x (c, n) floats
 constexpr int kQ1ZeroBytes = 4096;          // zero block read by the dead lanes (covers a 4-chunk step)
+// Inside a chunk's fragments, the live entries e = 0..15 of the mmas 2j and
+// 2j+1 sit side by side (16 bytes per entry), so one 16-byte load fetches a
+// lane's B registers for two bit planes.
+#ifndef LOWBIT_Q1_BPAIR
+#define LOWBIT_Q1_BPAIR 1
+#endif
+constexpr int kQ1FragLaneStride = LOWBIT_Q1_BPAIR ? 16 : 8;  // bytes between live entries
+// offset of mma i's fragment from a lane's base (entry e at e * kQ1FragLaneStride)
+__host__ __device__ constexpr int q1_frag_plane(int i) { return LOWBIT_Q1_BPAIR ? (i >> 1) * 256 + (i & 1) * 8 : i * 128; }
 // Tuning knobs (compile-time; the defaults are the measured best).
 #ifndef LOWBIT_Q1_WARPS
 #define LOWBIT_Q1_WARPS 8
@@ -161,7 +170,8 @@ __global__ void __launch_bounds__(256) k_q1_prep_m1(const uint16_t *__restrict__
     }
     if (kk < 128) {
         const uint2 f = q1_fragment(limb, kk >> 4, kk & 15);
-        reinterpret_cast<uint2 *>(act + (size_t)ch * kQ1FragBytesPerChunk)[kk] = f;
+        const int i = kk >> 4, e = kk & 15;
+        *reinterpret_cast<uint2 *>(act + (size_t)ch * kQ1FragBytesPerChunk + e * kQ1FragLaneStride + q1_frag_plane(i)) = f;
     }
 }
 
@@ -295,7 +305,8 @@ __device__ __forceinline__ LaneConst lane_const(int lane)
 __device__ __forceinline__ const uint8_t *bfrag_base(const uint8_t *frags, const uint8_t *zero, int chunk,
                                                      const LaneConst &lc)
 {
-    return lc.live ? frags + (size_t)chunk * kQ1FragBytesPerChunk + lc.e * 8 : zero + lc.e * 8;
+    return lc.live ? frags + (size_t)chunk * kQ1FragBytesPerChunk + lc.e * kQ1FragLaneStride
+                   : zero + lc.e * kQ1FragLaneStride;
 }
 
 // D_lo + 256 D_hi of one limb pair, as a float (one rounding; |v| < 2^29).
@@ -323,7 +334,7 @@ __device__ __forceinline__ void consume_step(const uint8_t *st, const uint8_t *b
             const uint32_t m = 0x01010101u << i;
 #pragma unroll
             for (int c = 0; c < kQ1StepChunks; ++c) {
-                const uint2 b = *reinterpret_cast<const uint2 *>(bf + c * kQ1FragBytesPerChunk + i * 128);
+                const uint2 b = *reinterpret_cast<const uint2 *>(bf + c * kQ1FragBytesPerChunk + q1_frag_plane(i));
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
                     if (i == 0)
@@ -339,7 +350,7 @@ __device__ __forceinline__ void consume_step(const uint8_t *st, const uint8_t *b
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const uint32_t m = 0x01010101u << i;
-            const uint2 b = *reinterpret_cast<const uint2 *>(bf + i * 128);
+            const uint2 b = *reinterpret_cast<const uint2 *>(bf + q1_frag_plane(i));
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 if (i == 0)
@@ -388,14 +399,27 @@ __device__ __forceinline__ void clear_zero_block(uint8_t *z)
         reinterpret_cast<uint4 *>(z)[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
-constexpr int kQ1BuildScratch = kQ1SplitWarps * 4 * 256;  // limb scratch of the fused split kernel
+// Limb scratch of one warp's build: four limbs, each 256 bytes plus 4 of
+// padding (the fragment reads of the 16 live entries then fall in distinct
+// banks).  The limb of k = 32 j + 8 c + i sits at byte 32 j + 4 i + c of its
+// limb row, so the four k = 8c + i (c = 0..3) of a fragment word are one
+// aligned 32-bit word.
+constexpr int kQ1LimbStride = 260;
+constexpr int kQ1LimbScratch = 4 * kQ1LimbStride + 16;  // per warp, 16-byte multiple
+constexpr int kQ1BuildScratch = kQ1SplitWarps * kQ1LimbScratch;  // limb scratch of the fused split kernel
+
+// 2^e for -126 <= e <= 127, exactly.
+__device__ __forceinline__ float q1_pow2(int e) { return __int_as_float((e + 127) << 23); }
 
 // The work of k_q1_prep_m1 for one 256-k chunk, done by one warp: lane l
 // takes k = 256 ch + 32 j + l (j = 0..7; j < 4 is the chunk's first group),
 // so every per-group reduction is a warp shuffle.  lw: this warp's limb
-// scratch (4 x 256 bytes); info: the chunk's four (c, n) pairs.
+// scratch (kQ1LimbScratch bytes); info: the chunk's four (c, n) pairs.
+// Writes the same bytes as k_q1_prep_m1: the scaling by 2^(23-E) and the
+// constants are exact powers of two (23 - E, E - 29, E - 13 and E - 23 stay
+// within the normal exponent range for kQ1MinExp <= E <= 128).
 __device__ __forceinline__ void q1_build_chunk_warp(const uint16_t *__restrict__ x, int K, int ch, uint8_t *frag,
-                                                    float2 *info, int8_t (*lw)[256], int lane)
+                                                    float2 *info, uint8_t *lw, int lane)
 {
     float xv[8];
 #pragma unroll
@@ -413,33 +437,48 @@ __device__ __forceinline__ void q1_build_chunk_warp(const uint16_t *__restrict__
         const int e8 = (int)((__float_as_uint(mh) >> 23) & 0xFFu);
         E[h] = max(e8 == 0 ? kQ1MinExp : e8 - 126, kQ1MinExp);  // smallest E with max|x| < 2^E
     }
+    const int wpos = 4 * (lane & 7) + (lane >> 3);  // this lane's byte in each 32-k row of the scratch
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const int X = __float2int_rn(ldexpf(xv[j], 23 - E[j >> 2]));  // |X| <= 2^23
+        const int X = __float2int_rn(xv[j] * q1_pow2(23 - E[j >> 2]));  // |X| <= 2^23
         T[j >> 2] += X;
-        const int B = X * (1 << (7 - (lane & 7)));                    // k & 7 == lane & 7
+        const int B = X * (1 << (7 - (lane & 7)));                      // k & 7 == lane & 7
         const int l0 = (int)(int8_t)(B & 0xFF);
         int r = (B - l0) >> 8;
         const int l1 = (int)(int8_t)(r & 0xFF);
         r = (r - l1) >> 8;
         const int l2 = (int)(int8_t)(r & 0xFF);
-        lw[0][32 * j + lane] = (int8_t)l0;
-        lw[1][32 * j + lane] = (int8_t)l1;
-        lw[2][32 * j + lane] = (int8_t)l2;
-        lw[3][32 * j + lane] = (int8_t)((r - l2) >> 8);
+        lw[0 * kQ1LimbStride + 32 * j + wpos] = (uint8_t)l0;
+        lw[1 * kQ1LimbStride + 32 * j + wpos] = (uint8_t)l1;
+        lw[2 * kQ1LimbStride + 32 * j + wpos] = (uint8_t)l2;
+        lw[3 * kQ1LimbStride + 32 * j + wpos] = (uint8_t)((r - l2) >> 8);
     }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int Th = warp_sum_int(T[h]);  // |T| <= 2^30
-        if (lane == 0) q1_write_info(info + 2 * h, (2 * ch + h) * 128 < K, E[h], Th);
+        if (lane == 0) {
+            float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);
+            if ((2 * ch + h) * 128 < K) {
+                lo = make_float2(q1_pow2(E[h] - 29), -((float)Th * q1_pow2(E[h] - 23)));
+                hi = make_float2(q1_pow2(E[h] - 13), 0.f);
+            }
+            info[2 * h] = lo;
+            info[2 * h + 1] = hi;
+        }
     }
     __syncwarp();
     // fragment words: the same layout as k_q1_prep_m1 writes; lane l takes
-    // entry l & 15 of mmas 4 (l >> 4) .. 4 (l >> 4) + 3
+    // entry e = l & 15 (k quarter t = e & 3, limb e >> 2) of mmas
+    // 4 (l >> 4) .. 4 (l >> 4) + 3; register j of mma i holds k = 64 t + 32 j
+    // + 8 c + i, c = 0..3: one scratch word
+    const int e = lane & 15, t = e & 3;
+    const uint8_t *lrow = lw + (e >> 2) * kQ1LimbStride;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int i = 4 * (lane >> 4) + q;
-        reinterpret_cast<uint2 *>(frag)[16 * i + (lane & 15)] = q1_fragment(lw, i, lane & 15);
+        const uint32_t w0 = *reinterpret_cast<const uint32_t *>(lrow + 32 * (2 * t) + 4 * i);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(lrow + 32 * (2 * t + 1) + 4 * i);
+        *reinterpret_cast<uint2 *>(frag + e * kQ1FragLaneStride + q1_frag_plane(i)) = make_uint2(w0, w1);
     }
     __syncwarp();  // the scratch is reused for the warp's next chunk
 }
@@ -569,6 +608,7 @@ constexpr int kQ1LStageBytes = kQ1LStageW + kQ1StepRows * 16;
 #ifndef LOWBIT_Q1_LEAN_WARPS
 #define LOWBIT_Q1_LEAN_WARPS 16
 #endif
+
 constexpr int kQ1LStages = LOWBIT_Q1_LEAN_STAGES;
 constexpr int kQ1LMaxWarps = LOWBIT_Q1_LEAN_WARPS;
 constexpr int kQ1LMinWarps = 8;
@@ -604,18 +644,31 @@ __device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *b
                     w[q][t][r] = *reinterpret_cast<const uint2 *>(st + woff[c0 + q] + (16 * t + 8 * r) * kQ1LRowBytes);
         int d[kQ1LInter][2][4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t m = 0x01010101u << i;
+        for (int j = 0; j < 4; ++j) {  // bit planes 2j, 2j+1
 #pragma unroll
             for (int q = 0; q < kQ1LInter; ++q) {
-                const uint2 b = *reinterpret_cast<const uint2 *>(bf + (c0 + q) * kQ1FragBytesPerChunk + i * 128);
+                uint2 bb[2];
+#if LOWBIT_Q1_BPAIR
+                const uint4 b4 = *reinterpret_cast<const uint4 *>(bf + (c0 + q) * kQ1FragBytesPerChunk + j * 256);
+                bb[0] = make_uint2(b4.x, b4.y);
+                bb[1] = make_uint2(b4.z, b4.w);
+#else
+                bb[0] = *reinterpret_cast<const uint2 *>(bf + (c0 + q) * kQ1FragBytesPerChunk + q1_frag_plane(2 * j));
+                bb[1] = *reinterpret_cast<const uint2 *>(bf + (c0 + q) * kQ1FragBytesPerChunk + q1_frag_plane(2 * j + 1));
+#endif
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    const uint2 w0 = w[q][t][0], w1 = w[q][t][1];
-                    if (i == 0)
-                        mma_u8s8_z(d[q][t], w0.x & m, w1.x & m, w0.y & m, w1.y & m, b.x, b.y);
-                    else
-                        mma_u8s8(d[q][t], w0.x & m, w1.x & m, w0.y & m, w1.y & m, b.x, b.y);
+                for (int o = 0; o < 2; ++o) {
+                    const int i = 2 * j + o;
+                    const uint32_t m = 0x01010101u << i;
+                    const uint2 b = bb[o];
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const uint2 w0 = w[q][t][0], w1 = w[q][t][1];
+                        if (i == 0)
+                            mma_u8s8_z(d[q][t], w0.x & m, w1.x & m, w0.y & m, w1.y & m, b.x, b.y);
+                        else
+                            mma_u8s8(d[q][t], w0.x & m, w1.x & m, w0.y & m, w1.y & m, b.x, b.y);
+                    }
                 }
             }
         }
@@ -709,7 +762,7 @@ __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __gri
     float2 *info = reinterpret_cast<float2 *>(smem + (size_t)p.nchunks * kQ1FragBytesPerChunk);
     if (p.x != nullptr) {
         // the ring slot kQ1LStages - 1 of this warp is not in use yet
-        int8_t(*lw)[256] = reinterpret_cast<int8_t(*)[256]>(ring + (kQ1LStages - 1) * kQ1LStageBytes);
+        uint8_t *lw = ring + (kQ1LStages - 1) * kQ1LStageBytes;
         for (int ch = warp; ch < p.nchunks; ch += nw)
             q1_build_chunk_warp(p.x, p.K, ch, smem + (size_t)ch * kQ1FragBytesPerChunk, info + 4 * ch, lw, lane);
     } else if (c1 > c0) {
@@ -725,7 +778,7 @@ __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __gri
         woff[c] = g * kQ1LRowBytes + (((2 * c + (tq >> 1)) ^ ((g & 3) << 1)) << 4) + (tq & 1) * 8;
     const int soff = kQ1LStageW + g * 16 + (tq >> 1) * 2;
     const bool live = (lane >> 4) == (tq >> 1);
-    const uint8_t *bf_live = smem + (lane & 15) * 8, *bf_dead = zero + (lane & 15) * 8;
+    const uint8_t *bf_live = smem + (lane & 15) * kQ1FragLaneStride, *bf_dead = zero + (lane & 15) * kQ1FragLaneStride;
     const float2 *inf0 = info + tq;
 
     int s = s0, slot = 0;
@@ -836,8 +889,7 @@ __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid
         const int n = ch_hi - ch_lo;
         if (p.x != nullptr) {
             // fused: each warp turns its share of the slice's chunks of x into fragments
-            int8_t(*lw)[256] = reinterpret_cast<int8_t(*)[256]>(smem + p.act_smem + kQ1SplitWarps * kQ1SplitRing +
-                                                                 warp * 4 * 256);
+            uint8_t *lw = smem + p.act_smem + kQ1SplitWarps * kQ1SplitRing + warp * kQ1LimbScratch;
             float2 *info = reinterpret_cast<float2 *>(smem + (size_t)n * kQ1FragBytesPerChunk);
             for (int c = warp; c < n; c += kQ1SplitWarps)
                 q1_build_chunk_warp(p.x, p.K, ch_lo + c, smem + (size_t)c * kQ1FragBytesPerChunk, info + 4 * c, lw,
@@ -1288,8 +1340,8 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
     float2 *info = reinterpret_cast<float2 *>(smem + kStSliceChunks * kQ1FragBytesPerChunk);
     uint8_t *zero = smem + kStSliceChunks * (kQ1FragBytesPerChunk + kQ1InfoBytesPerChunk);
     uint16_t *xs = reinterpret_cast<uint16_t *>(zero + kQ1ZeroBytes);
-    int8_t(*lwall)[256] = reinterpret_cast<int8_t(*)[256]>(reinterpret_cast<uint8_t *>(xs) + kStSliceK * 2);
-    float *xsf = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(lwall) + 4 * 4 * 256);  // raw slice values
+    uint8_t *lwall = reinterpret_cast<uint8_t *>(xs) + kStSliceK * 2;                         // limb scratch
+    float *xsf = reinterpret_cast<float *>(lwall + kStSliceChunks * kQ1LimbScratch);           // raw slice values
     uint8_t *rings = reinterpret_cast<uint8_t *>(xsf) + kStSliceK * 4;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1405,7 +1457,8 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
         __syncthreads();
         if (warp < kStSliceChunks)
             q1_build_chunk_warp(xs - s * kStSliceK, q.K, s * kStSliceChunks + warp,
-                                frag + warp * kQ1FragBytesPerChunk, info + 4 * warp, lwall + 4 * warp, lane);
+                                frag + warp * kQ1FragBytesPerChunk, info + 4 * warp, lwall + warp * kQ1LimbScratch,
+                                lane);
         __syncthreads();
 
         // ---- this warp's units of the phase ----
@@ -1460,7 +1513,8 @@ lowbit_status q1stack_launch(const uint8_t *const *bits, const uint16_t *const *
     p.F = F;
     p.eps = eps;
     const size_t smem = kStSliceChunks * (kQ1FragBytesPerChunk + kQ1InfoBytesPerChunk) + kQ1ZeroBytes +
-                        kStSliceK * 2 + 4 * 4 * 256 + kStSliceK * 4 + (size_t)kStWarps * kStStages * kQ1StageBytes;
+                        kStSliceK * 2 + kStSliceChunks * kQ1LimbScratch + kStSliceK * 4 +
+                        (size_t)kStWarps * kStStages * kQ1StageBytes;
     if (cudaFuncSetAttribute(k_q1_stack_m1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
     int per_sm = 0, sms = num_sms();
