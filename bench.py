@@ -464,9 +464,12 @@ def run_q1_sweep(args, world, rank, local):
                     lb.lowbit_q1g128_gemv_group([b for b, _ in mats], [s for _, s in mats], x, ys, workspace=ws,
                                                 stream=stream)
             else:
+                need = lb.lowbit_q1g128_group_workspace_bytes(R, M, N, K)
+                ws = torch.zeros(need, dtype=torch.uint8, device=dev) if need else None
+
                 def step():
-                    for r in range(R):
-                        lb.lowbit_q1g128_gemv(mats[r][0], mats[r][1], x, ys[r], stream=stream)
+                    lb.lowbit_q1g128_gemv_group([b for b, _ in mats], [s for _, s in mats], x, ys, workspace=ws,
+                                                stream=stream)
             ms = max_over_ranks(_graph_time(step, stream, max(20, args.steps), args.warmup), world)
             results.append({"N": N, "K": K, "M": M, "weight_sets": R,
                             "gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
@@ -510,7 +513,7 @@ def run_int4(args, world, rank, local):
         res = {"M": M, "us_per_call": round(ms * 1e3 / R, 3),
                "weight_gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
                "tflops": round(2.0 * M * N * K * R / (ms * 1e-3) / 1e12, 2)}
-        if M == 1:
+        if M <= 32:
             # the R weight sets read one x: one grouped launch
             ys = [y[r] for r in range(R)]
             gws = lb.lowbit_int4g64_group_workspace_bytes(R, M, N, K)

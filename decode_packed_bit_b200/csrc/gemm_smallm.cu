@@ -26,6 +26,7 @@
 // shared memory in fragment order; every warp streams its rows' sign bits
 // and scales through a cp.async ring, 256 k per step.
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -504,6 +505,231 @@ lowbit_status i4sm_launch(const uint8_t *q, const uint16_t *scales, const uint16
                           cudaStream_t st)
 {
     return sm_launch(3, q, scales, x, y, M, N, K, st);
+}
+
+// ---------------------------------------------------------------------------
+// grouped persistent form: R matrices of one shape that read one x (M >= 2)
+// ---------------------------------------------------------------------------
+//
+// One CTA per SM with nw warps; every warp owns one 32-row block of one
+// matrix over all of K per round, and the rounds walk the (matrix, block)
+// list: block (j * gridDim + blockIdx) * nw + warp in round j.  The warps of
+// a CTA move through the steps of K in lockstep, so the CTA-wide x ring of
+// the single-matrix kernel serves all of them; the weights stream through
+// per-warp rings.  With all of K per warp no partial sums cross warps or
+// CTAs: a warp writes its rows' outputs after the last step of a round.
+
+constexpr int kSgMaxGroup = 256;
+constexpr int kSgMaxWarps = 16;
+constexpr int kSgMinWarps = 8;
+
+struct SmGroup {
+    const uint8_t *bits[kSgMaxGroup];
+    const uint16_t *scales[kSgMaxGroup];
+    float *y[kSgMaxGroup];
+};
+
+struct SmGParams {
+    const uint16_t *x;
+    int M, N, K, nsteps, blocksN, nblocks, rounds;
+};
+
+template <int FMT, int NT>
+__global__ void __launch_bounds__(kSgMaxWarps * 32, 1) k_smallm_grp(const __grid_constant__ SmGroup grp,
+                                                                    const SmGParams q)
+{
+    constexpr int kStepK = SmFmt<FMT>::kStepK;
+    constexpr int kK16 = kStepK / 16;
+    constexpr int kSB = SmFmt<FMT>::kStageBytes;
+    constexpr int kXFrags = kK16 * NT * 32;  // uint2 per step
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ uint2 lut[16];
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int total = q.rounds * q.nsteps;  // the CTA's lockstep sequence of (round, step)
+    uint2 *xr = reinterpret_cast<uint2 *>(smem);  // x ring: kSmStages x kXFrags
+    uint8_t *wring = smem + (size_t)kSmStages * kXFrags * 8 + warp * kSmStages * kSB;
+    const unsigned xr_s = (unsigned)__cvta_generic_to_shared(xr);
+    const unsigned wr_s = (unsigned)__cvta_generic_to_shared(wring);
+    auto blk_of = [&](int j) { return (j * (int)gridDim.x + (int)blockIdx.x) * nw + warp; };
+
+    auto issue_w = [&](int u) {
+        if (u >= total) return;
+        const int j = u / q.nsteps, s = u - j * q.nsteps, b = blk_of(j);
+        if (b >= q.nblocks) return;
+        const int r = b / q.blocksN, blk = b - r * q.blocksN;
+        SmParams pp = {};
+        pp.bits = grp.bits[r];
+        pp.scales = grp.scales[r];
+        pp.N = q.N;
+        pp.K = q.K;
+        if (FMT == 1)
+            sm_issue(wr_s + (u % kSmStages) * kSB, pp, blk, s, lane);
+        else
+            i4s_issue(wr_s + (u % kSmStages) * kSB, pp, blk, s, lane);
+    };
+    auto issue_x = [&](int u) {
+        if (u >= total) return;
+        const int s = u % q.nsteps;
+        const unsigned dst = xr_s + (unsigned)((u % kSmStages) * kXFrags) * 8u;
+        for (int i = threadIdx.x; i < kXFrags; i += blockDim.x) {
+            const int ln = i & 31, nt = (i >> 5) % NT, ks = (i >> 5) / NT;
+            const int m = 8 * nt + (ln >> 2);
+            const int k = s * kStepK + 16 * ks + 4 * (ln & 3);
+            sm_cp8(dst + 8u * i, m < q.M ? q.x + (size_t)m * q.K + k : q.x, m < q.M);
+        }
+    };
+    // weights of the first steps go out before the previous kernel ends; x after it
+#pragma unroll
+    for (int t = 0; t < kSmStages - 1; ++t) {
+        issue_w(t);
+        sm_commit();
+    }
+    if (FMT == 1 && threadIdx.x < 16) {
+        const uint32_t v = threadIdx.x;
+        auto sg = [&](int j) -> uint32_t { return ((v >> j) & 1u) ? 0x3F80u : 0xBF80u; };
+        lut[threadIdx.x] = make_uint2(sg(0) | (sg(1) << 16), sg(2) | (sg(3) << 16));
+    }
+    pdl_wait_primary();  // x is produced, and y last read, by earlier kernels
+#pragma unroll
+    for (int t = 0; t < kSmStages - 1; ++t) issue_x(t);
+    sm_commit();
+
+    float yacc[2][NT][4];
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) yacc[tt][nt][0] = yacc[tt][nt][1] = yacc[tt][nt][2] = yacc[tt][nt][3] = 0.f;
+    const int g = lane >> 2, t4 = lane & 3;
+    for (int u = 0; u < total; ++u) {
+        // as in the single-matrix kernel: the prologue's groups at u = 0, then
+        // all but the newest group, and a CTA barrier (which also frees the
+        // slot of step u - 1)
+        if (u == 0)
+            sm_wait<0>();
+        else
+            sm_wait<kSmStages - 2>();
+        __syncthreads();
+        issue_w(u + kSmStages - 1);
+        issue_x(u + kSmStages - 1);
+        sm_commit();
+        const int j = u / q.nsteps, s = u - j * q.nsteps, b = blk_of(j);
+        if (b < q.nblocks) {
+            const uint8_t *st = wring + (u % kSmStages) * kSB;
+            const uint2 *xf = xr + (u % kSmStages) * kXFrags;
+            if (FMT == 1)
+                sm_consume<NT>(st, xf, lut, lane, yacc);
+            else
+                i4s_consume<NT>(st, xf, lane, yacc);
+        }
+        if (s == q.nsteps - 1) {
+            if (b < q.nblocks) {
+                const int r = b / q.blocksN, blk = b - r * q.blocksN;
+                float *y = grp.y[r];
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int m = 8 * nt + 2 * t4 + (e & 1);
+                            const int row = blk * 32 + 16 * tt + g + 8 * (e >> 1);
+                            if (m < q.M && row < q.N) y[(size_t)m * q.N + row] = yacc[tt][nt][e];
+                        }
+            }
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    yacc[tt][nt][0] = yacc[tt][nt][1] = yacc[tt][nt][2] = yacc[tt][nt][3] = 0.f;
+        }
+    }
+    sm_wait<0>();
+}
+
+struct SgPlan {
+    int nsteps, blocksN, nblocks, warps, rounds, NT;
+    size_t smem;
+    bool ok;
+};
+
+// Warps per CTA: as many as fit (<= kSgMaxWarps), then the count in
+// [kSgMinWarps, max] whose rounds come out fullest (ties: more warps).
+static SgPlan sg_plan(int fmt, int R, int M, int N, int K, int sms)
+{
+    SgPlan P = {};
+    const int stepk = fmt == 1 ? kSmStepK : kI4sStepK, maxm = fmt == 1 ? kSmMaxM : kI4sMaxM;
+    if (R < 1 || R > kSgMaxGroup || M < 2 || M > maxm || N < 1 || K % stepk != 0 || K < stepk) return P;
+    P.NT = (M + 7) / 8;
+    P.nsteps = K / stepk;
+    P.blocksN = (N + 31) / 32;
+    P.nblocks = R * P.blocksN;
+    const size_t xring = (size_t)kSmStages * (stepk / 16) * P.NT * 32 * 8;
+    const size_t per_warp = (size_t)kSmStages * (fmt == 1 ? kSmStageBytes : kI4sStageBytes);
+    const int fit = (int)std::min<size_t>(kSgMaxWarps, ((size_t)kSmMaxSmem - xring) / per_warp);
+    double best = -1.0;
+    for (int w = fit; w >= kSgMinWarps; --w) {
+        if ((long long)P.nblocks < (long long)sms * w) continue;  // at least one full round
+        const int rounds = (int)((P.nblocks + (long long)sms * w - 1) / ((long long)sms * w));
+        const double eff = (double)P.nblocks / ((double)rounds * sms * w);
+        if (eff > best + 1e-9) {
+            best = eff;
+            P.warps = w;
+            P.rounds = rounds;
+        }
+    }
+    P.smem = xring + (size_t)P.warps * per_warp;
+    P.ok = P.warps >= kSgMinWarps;
+    return P;
+}
+
+bool smg_supported(int fmt, int R, int M, int N, int K) { return sg_plan(fmt, R, M, N, K, sm_num_sms()).ok; }
+
+lowbit_status smg_launch(int fmt, const uint8_t *const *bits, const uint16_t *const *scales, const uint16_t *x,
+                         float *const *y, int R, int M, int N, int K, cudaStream_t st)
+{
+    const int sms = sm_num_sms();
+    const SgPlan P = sg_plan(fmt, R, M, N, K, sms);
+    if (!P.ok) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    static SmGroup grp;  // large: kept off the stack
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int r = 0; r < R; ++r) {
+        grp.bits[r] = bits[r];
+        grp.scales[r] = scales[r];
+        grp.y[r] = y[r];
+    }
+    SmGParams q = {};
+    q.x = x;
+    q.M = M;
+    q.N = N;
+    q.K = K;
+    q.nsteps = P.nsteps;
+    q.blocksN = P.blocksN;
+    q.nblocks = P.nblocks;
+    q.rounds = P.rounds;
+    void (*kern)(const SmGroup, const SmGParams);
+    if (fmt == 1)
+        kern = P.NT == 1 ? k_smallm_grp<1, 1> : k_smallm_grp<1, 2>;
+    else
+        kern = P.NT == 1 ? k_smallm_grp<3, 1>
+             : P.NT == 2 ? k_smallm_grp<3, 2>
+             : P.NT == 3 ? k_smallm_grp<3, 3>
+                         : k_smallm_grp<3, 4>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) != cudaSuccess)
+        return LOWBIT_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(P.warps * 32);
+    cfg.dynamicSmemBytes = P.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, grp, q);
+    return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
 
 }  // namespace lowbit

@@ -34,6 +34,9 @@ int q1stack_fault_flag();
 lowbit_status q1sm_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 lowbit_status q1m1_gemv_fused_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
                                      cudaStream_t);
+bool smg_supported(int fmt, int R, int M, int N, int K);
+lowbit_status smg_launch(int fmt, const uint8_t *const *, const uint16_t *const *, const uint16_t *, float *const *,
+                         int R, int M, int N, int K, cudaStream_t);
 bool i4m1_group_supported(int R, int N, int K);
 lowbit_status i4m1_group_launch(const uint8_t *const *, const uint16_t *const *, const uint16_t *, float *const *,
                                 int, int, int, cudaStream_t);
@@ -229,6 +232,7 @@ size_t lowbit_q1g128_group_workspace_bytes(int R, int M, int N, int K)
 {
     if (R < 1 || q1_shape_ok(M, N, K) != LOWBIT_OK) return 0;
     if (M == 1 && q1m1_x_group_supported(R, N, K)) return 0;
+    if (M >= 2 && smg_supported(1, R, M, N, K)) return 0;
     return al256(lowbit_q1g128_act_bytes(M, K)) + lowbit_q1g128_act_workspace_bytes(R, M, N, K);
 }
 
@@ -251,6 +255,8 @@ lowbit_status lowbit_q1g128_gemv_group(const uint8_t *const *w_bits, const uint1
     if (M == 1) {
         s = q1m1_gemv_x_group_launch(w_bits, w_scales, x, y, R, N, K, st);
         if (s != LOWBIT_ERR_UNSUPPORTED_SHAPE) return s;
+    } else if (smg_supported(1, R, M, N, K)) {
+        return smg_launch(1, w_bits, w_scales, x, y, R, M, N, K, st);
     }
     uint8_t *act = static_cast<uint8_t *>(workspace);
     const size_t act_bytes = al256(lowbit_q1g128_act_bytes(M, K));
@@ -348,6 +354,7 @@ lowbit_status lowbit_int4g64_gemm_group(const uint8_t *const *w_q, const uint16_
     LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
     cudaStream_t st = as_stream(stream);
     if (M == 1 && i4m1_group_supported(R, N, K)) return i4m1_group_launch(w_q, w_scales, x, y, R, N, K, st);
+    if (M >= 2 && smg_supported(3, R, M, N, K)) return smg_launch(3, w_q, w_scales, x, y, R, M, N, K, st);
     for (int r = 0; r < R; ++r) {
         const lowbit_status s =
             lowbit_int4g64_gemm(w_q[r], w_scales[r], x, y[r], M, N, K, workspace, workspace_bytes, stream);

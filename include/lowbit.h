@@ -165,8 +165,11 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits,
  * At M = 1, with K % 1024 == 0, N % 32 == 0 and at least SMs * 8
  * (32-row block, matrix) pairs (e.g. 10 or more 4096-row matrices on 148
  * SMs), this is one launch: every CTA turns x into the operand form itself,
- * and no workspace is needed.  Otherwise the call prepares the activation in
- * the workspace and runs lowbit_q1g128_gemv_act_group.
+ * and no workspace is needed.  At 2 <= M <= 16 with K % 256 == 0 and at
+ * least SMs * 8 32-row blocks over the group, it is one launch of a
+ * persistent kernel (each warp owns a 32-row block over all of K; the warps
+ * of a CTA share x).  Otherwise the call prepares the activation in the
+ * workspace and runs lowbit_q1g128_gemv_act_group.
  * Workspace: lowbit_q1g128_group_workspace_bytes(R, M, N, K) bytes (NULL
  * allowed when 0).  Calls that share a workspace must be ordered on one
  * stream. */
@@ -262,7 +265,9 @@ lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales,
  * SMs * 8 (32-row block, matrix) pairs (e.g. 4 or more 11008-row matrices
  * on 148 SMs), this is one launch of a persistent kernel: one CTA per SM
  * builds the activation from x and streams its equal share of every matrix's
- * weights.  Other shapes run lowbit_int4g64_gemm once per matrix.  Results
+ * weights.  At 2 <= M <= 32 with K % 128 == 0 and at least SMs * 8 32-row
+ * blocks over the group, one launch of the persistent small-batch kernel
+ * (as for Q1_0_g128).  Other shapes run lowbit_int4g64_gemm once per matrix.  Results
  * equal the single calls up to fp32 summation order.
  * workspace: lowbit_int4g64_group_workspace_bytes(R, M, N, K) bytes (0
  * today; NULL allowed when 0). */

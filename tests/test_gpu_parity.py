@@ -207,11 +207,14 @@ def test_q1_large_group(lb, R, N, K, xkind):
 
 
 @pytest.mark.parametrize("R,M,N,K", [(40, 1, 4096, 1024), (38, 1, 4096, 17408), (160, 1, 1024, 3072),
+                                     (40, 4, 4096, 1024), (12, 16, 5120, 5120), (40, 9, 1000, 2048),
                                      (3, 1, 515, 1280), (2, 2, 300, 2048)])
 def test_q1_group_from_x(lb, R, M, N, K):
-    """lowbit_q1g128_gemv_group: one launch from x when the shape allows (the
-    first three cases on 148 SMs), else prepare + group product in the
-    workspace.  Sampled outputs of three matrices against the oracle."""
+    """lowbit_q1g128_gemv_group: one launch when the shape allows (the first
+    six cases on 148 SMs: the M = 1 persistent kernel, then the small-batch
+    persistent kernel with ragged rows and a partial batch tile), else
+    prepare + group product in the workspace.  Sampled outputs of three
+    matrices against the oracle."""
     x = synth.bf16_normal(2800 + R, (M, K))
     g = torch.Generator(device="cuda")
     g.manual_seed(2800 + R)
@@ -332,10 +335,12 @@ def test_int4_11008x4096_sampled(lb, M):
 
 
 @pytest.mark.parametrize("R,M,N,K", [(17, 1, 11008, 4096), (80, 1, 1024, 1024), (7, 1, 11008, 11008),
+                                     (17, 32, 11008, 4096), (40, 5, 1000, 1024), (10, 17, 4096, 512),
                                      (40, 1, 1024, 1024), (3, 32, 300, 512), (2, 1, 300, 448)])
 def test_int4_group(lb, R, M, N, K):
-    """lowbit_int4g64_gemm_group: the persistent kernel for the first three
-    cases on 148 SMs, single calls for the rest.  Sampled outputs of three
+    """lowbit_int4g64_gemm_group: the persistent kernels for the first six
+    cases on 148 SMs (M = 1, then small batches with ragged rows and partial
+    batch tiles), single calls for the rest.  Sampled outputs of three
     matrices against the oracle, and the group equals single calls up to fp32
     summation order."""
     x = synth.bf16_normal(4800 + R, (M, K))
