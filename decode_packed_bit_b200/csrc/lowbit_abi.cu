@@ -41,8 +41,8 @@ bool i4m1_group_supported(int R, int N, int K);
 lowbit_status i4m1_group_launch(const uint8_t *const *, const uint16_t *const *, const uint16_t *, float *const *,
                                 int, int, int, cudaStream_t);
 lowbit_status q1m1_gemv_x_group_launch(const uint8_t *const *, const uint16_t *const *, const uint16_t *,
-                                       float *const *, int, int, int, cudaStream_t);
-bool q1m1_x_group_supported(int R, int N, int K);
+                                       float *const *, int, int, int, int, cudaStream_t);
+bool q1m1_x_group_supported(int R, int M, int N, int K);
 lowbit_status q1m1_gemv_launch(const uint8_t *const *, const uint16_t *const *, const void *, float *const *,
                                int, int, int, cudaStream_t);
 
@@ -231,7 +231,7 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits, const u
 size_t lowbit_q1g128_group_workspace_bytes(int R, int M, int N, int K)
 {
     if (R < 1 || q1_shape_ok(M, N, K) != LOWBIT_OK) return 0;
-    if (M == 1 && q1m1_x_group_supported(R, N, K)) return 0;
+    if (q1m1_x_group_supported(R, M, N, K)) return 0;
     if (M >= 2 && smg_supported(1, R, M, N, K)) return 0;
     return al256(lowbit_q1g128_act_bytes(M, K)) + lowbit_q1g128_act_workspace_bytes(R, M, N, K);
 }
@@ -252,12 +252,9 @@ lowbit_status lowbit_q1g128_gemv_group(const uint8_t *const *w_bits, const uint1
     LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
     cudaStream_t st = as_stream(stream);
-    if (M == 1) {
-        s = q1m1_gemv_x_group_launch(w_bits, w_scales, x, y, R, N, K, st);
-        if (s != LOWBIT_ERR_UNSUPPORTED_SHAPE) return s;
-    } else if (smg_supported(1, R, M, N, K)) {
-        return smg_launch(1, w_bits, w_scales, x, y, R, M, N, K, st);
-    }
+    s = q1m1_gemv_x_group_launch(w_bits, w_scales, x, y, R, M, N, K, st);  // M <= 4: integer bit planes
+    if (s != LOWBIT_ERR_UNSUPPORTED_SHAPE) return s;
+    if (M >= 2 && smg_supported(1, R, M, N, K)) return smg_launch(1, w_bits, w_scales, x, y, R, M, N, K, st);
     uint8_t *act = static_cast<uint8_t *>(workspace);
     const size_t act_bytes = al256(lowbit_q1g128_act_bytes(M, K));
     s = lowbit_q1g128_prepare_act(x, M, K, act, act_bytes, stream);

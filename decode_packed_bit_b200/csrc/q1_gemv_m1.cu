@@ -232,6 +232,7 @@ struct Q1Params {
     const uint16_t *x;  // split kernel: build the activation from x itself (act unused)
     size_t info_off;
     int R, N, K, nchunks;
+    int M;              // lean kernel: vectors of x (<= its MV)
     int L;              // chunks per K-slice (split kernel) or nchunks (stream kernel)
     int blocksN;        // 32-row blocks per matrix
     int cells;          // stream kernel: R * blocksN
@@ -629,61 +630,81 @@ __device__ __forceinline__ void cp_async16_full(unsigned dst, const void *src)
 constexpr int kQ1LInter = LOWBIT_Q1_LEAN_INTER;
 static_assert(kQ1LChunks % kQ1LInter == 0, "chunk groups must tile the step");
 
-__device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *bf, const float2 *inf,
-                                             const int (&woff)[kQ1LChunks], int soff, float (&yacc)[2][2])
+// MV vectors: vector v's fragments at bf + v * bstride (bstride = 0 for the
+// dead lanes, which read the zero block) and its constants at inf + v *
+// istride.  A bit plane's masked weights feed one mma per vector.  With one
+// vector two chunks are interleaved (kQ1LInter); with more, one chunk at a
+// time keeps the accumulators in registers.
+template <int MV>
+__device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *bf, int bstride, const float2 *inf,
+                                             int istride, const int (&woff)[kQ1LChunks], int soff,
+                                             float (&yacc)[2][2][MV])
 {
+    constexpr int kInter = MV == 1 ? kQ1LInter : 1;
 #pragma unroll
-    for (int c0 = 0; c0 < kQ1LChunks; c0 += kQ1LInter) {
-        uint2 w[kQ1LInter][2][2];  // [chunk][tile][row g / g+8]
+    for (int c0 = 0; c0 < kQ1LChunks; c0 += kInter) {
+        uint2 w[kInter][2][2];  // [chunk][tile][row g / g+8]
 #pragma unroll
-        for (int q = 0; q < kQ1LInter; ++q)
+        for (int q = 0; q < kInter; ++q)
 #pragma unroll
             for (int t = 0; t < 2; ++t)
 #pragma unroll
                 for (int r = 0; r < 2; ++r)
                     w[q][t][r] = *reinterpret_cast<const uint2 *>(st + woff[c0 + q] + (16 * t + 8 * r) * kQ1LRowBytes);
-        int d[kQ1LInter][2][4];
+        int d[kInter][2][MV][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {  // bit planes 2j, 2j+1
 #pragma unroll
-            for (int q = 0; q < kQ1LInter; ++q) {
-                uint2 bb[2];
+            for (int q = 0; q < kInter; ++q) {
+                uint2 bb[MV][2];
+#pragma unroll
+                for (int v = 0; v < MV; ++v) {
 #if LOWBIT_Q1_BPAIR
-                const uint4 b4 = *reinterpret_cast<const uint4 *>(bf + (c0 + q) * kQ1FragBytesPerChunk + j * 256);
-                bb[0] = make_uint2(b4.x, b4.y);
-                bb[1] = make_uint2(b4.z, b4.w);
+                    const uint4 b4 = *reinterpret_cast<const uint4 *>(bf + v * bstride + (c0 + q) * kQ1FragBytesPerChunk +
+                                                                      j * 256);
+                    bb[v][0] = make_uint2(b4.x, b4.y);
+                    bb[v][1] = make_uint2(b4.z, b4.w);
 #else
-                bb[0] = *reinterpret_cast<const uint2 *>(bf + (c0 + q) * kQ1FragBytesPerChunk + q1_frag_plane(2 * j));
-                bb[1] = *reinterpret_cast<const uint2 *>(bf + (c0 + q) * kQ1FragBytesPerChunk + q1_frag_plane(2 * j + 1));
+                    bb[v][0] = *reinterpret_cast<const uint2 *>(bf + v * bstride + (c0 + q) * kQ1FragBytesPerChunk +
+                                                                q1_frag_plane(2 * j));
+                    bb[v][1] = *reinterpret_cast<const uint2 *>(bf + v * bstride + (c0 + q) * kQ1FragBytesPerChunk +
+                                                                q1_frag_plane(2 * j + 1));
 #endif
+                }
 #pragma unroll
                 for (int o = 0; o < 2; ++o) {
                     const int i = 2 * j + o;
                     const uint32_t m = 0x01010101u << i;
-                    const uint2 b = bb[o];
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
                         const uint2 w0 = w[q][t][0], w1 = w[q][t][1];
-                        if (i == 0)
-                            mma_u8s8_z(d[q][t], w0.x & m, w1.x & m, w0.y & m, w1.y & m, b.x, b.y);
-                        else
-                            mma_u8s8(d[q][t], w0.x & m, w1.x & m, w0.y & m, w1.y & m, b.x, b.y);
+                        const uint32_t a0 = w0.x & m, a1 = w1.x & m, a2 = w0.y & m, a3 = w1.y & m;
+#pragma unroll
+                        for (int v = 0; v < MV; ++v) {
+                            if (i == 0)
+                                mma_u8s8_z(d[q][t][v], a0, a1, a2, a3, bb[v][o].x, bb[v][o].y);
+                            else
+                                mma_u8s8(d[q][t][v], a0, a1, a2, a3, bb[v][o].x, bb[v][o].y);
+                        }
                     }
                 }
             }
         }
 #pragma unroll
-        for (int q = 0; q < kQ1LInter; ++q) {
+        for (int q = 0; q < kInter; ++q) {
             const int c = c0 + q;
-            const float2 ci = inf[4 * c];
 #pragma unroll
             for (int t = 0; t < 2; ++t)
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
-                    const uint16_t sc =
-                        *reinterpret_cast<const uint16_t *>(st + soff + (16 * t + 8 * r) * 16 + c * 4);
-                    yacc[t][r] = fmaf(f16_bits_to_float(sc), fmaf(ci.x, limb_pair(d[q][t][2 * r], d[q][t][2 * r + 1]), ci.y),
-                                      yacc[t][r]);
+                    const float sc = f16_bits_to_float(
+                        *reinterpret_cast<const uint16_t *>(st + soff + (16 * t + 8 * r) * 16 + c * 4));
+#pragma unroll
+                    for (int v = 0; v < MV; ++v) {
+                        const float2 ci = inf[v * istride + 4 * c];
+                        yacc[t][r][v] = fmaf(sc, fmaf(ci.x, limb_pair(d[q][t][v][2 * r], d[q][t][v][2 * r + 1]), ci.y),
+                                             yacc[t][r][v]);
+                    }
                 }
         }
     }
@@ -696,11 +717,19 @@ __device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *b
 // warp at least one cell's worth of steps, so no cell has a third part.
 // With p.x set, every CTA builds the activation fragments from x itself (one
 // chunk per warp at a time, the limb scratch in the warp's idle ring slot).
-__global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __grid_constant__ Q1Group grp,
-                                                                     const Q1Params p)
+// MV > 1: the product of MV vectors (rows of x; those at or past p.M read as
+// zero and are not written), each with its own fragments and constants:
+// vector v's fragments at v * nchunks KB, then all constants, vector-major.
+// Warps per CTA at most: the several-vector forms keep more accumulators, so
+// they run at most 12 warps (168 registers a thread).
+__host__ __device__ constexpr int q1l_max_warps(int mv) { return mv == 1 ? kQ1LMaxWarps : 12; }
+
+template <int MV>
+__global__ void __launch_bounds__(q1l_max_warps(MV) * 32, 1) k_q1_m1_lean(const __grid_constant__ Q1Group grp,
+                                                                          const Q1Params p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ float part[2][kQ1LMaxWarps][kQ1StepRows];  // [head / tail][warp][row] of cut cells
+    __shared__ float part[2][q1l_max_warps(MV)][MV][kQ1StepRows];  // [head / tail][warp][vector][row] of cut cells
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int c0 = (int)((long long)blockIdx.x * p.cells / gridDim.x);
@@ -758,15 +787,26 @@ __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __gri
     for (int t = 0; t < kQ1LStages - 1; ++t) issue_next();
 
     pdl_wait_primary();  // x or the activation, and the outputs, follow stream order from here
+    const int vfrag = p.nchunks * kQ1FragBytesPerChunk;  // bytes of one vector's fragments
     uint8_t *zero = smem + p.act_smem - kQ1ZeroBytes;
-    float2 *info = reinterpret_cast<float2 *>(smem + (size_t)p.nchunks * kQ1FragBytesPerChunk);
+    float2 *info = reinterpret_cast<float2 *>(smem + (size_t)MV * vfrag);
     if (p.x != nullptr) {
         // the ring slot kQ1LStages - 1 of this warp is not in use yet
         uint8_t *lw = ring + (kQ1LStages - 1) * kQ1LStageBytes;
-        for (int ch = warp; ch < p.nchunks; ch += nw)
-            q1_build_chunk_warp(p.x, p.K, ch, smem + (size_t)ch * kQ1FragBytesPerChunk, info + 4 * ch, lw, lane);
+        for (int idx = warp; idx < MV * p.nchunks; idx += nw) {
+            const int v = idx / p.nchunks, ch = idx - v * p.nchunks;
+            uint8_t *frag = smem + (size_t)v * vfrag + (size_t)ch * kQ1FragBytesPerChunk;
+            float2 *inf = info + 4 * (v * p.nchunks + ch);
+            if (v < p.M) {
+                q1_build_chunk_warp(p.x + (size_t)v * p.K, p.K, ch, frag, inf, lw, lane);
+            } else {
+                for (int i = lane; i < kQ1FragBytesPerChunk / 16; i += 32)
+                    reinterpret_cast<uint4 *>(frag)[i] = make_uint4(0u, 0u, 0u, 0u);
+                if (lane < 4) inf[lane] = make_float2(0.f, 0.f);
+            }
+        }
     } else if (c1 > c0) {
-        stage_act(smem, p, 0, p.nchunks);
+        stage_act(smem, p, 0, p.nchunks);  // one vector
     }
     clear_zero_block(zero);
     __syncthreads();
@@ -779,6 +819,7 @@ __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __gri
     const int soff = kQ1LStageW + g * 16 + (tq >> 1) * 2;
     const bool live = (lane >> 4) == (tq >> 1);
     const uint8_t *bf_live = smem + (lane & 15) * kQ1FragLaneStride, *bf_dead = zero + (lane & 15) * kQ1FragLaneStride;
+    const int bstride = live ? vfrag : 0;
     const float2 *inf0 = info + tq;
 
     int s = s0, slot = 0;
@@ -786,27 +827,37 @@ __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __gri
         // one cell (or the part of it in [s0, s1))
         const int cell = c0 + s / spc, st0 = s % spc;
         const int st1 = min(spc, st0 + (s1 - s));
-        float yacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        float yacc[2][2][MV];
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int v = 0; v < MV; ++v) yacc[t][r][v] = 0.f;
         for (int t = st0; t < st1; ++t) {
             issue_next();
             cp_async_wait<kQ1LStages - 1>();
             __syncwarp();
-            lean_consume(ring + slot * kQ1LStageBytes,
-                         live ? bf_live + t * (kQ1LChunks * kQ1FragBytesPerChunk) : bf_dead,
-                         inf0 + 4 * kQ1LChunks * t, woff, soff, yacc);
+            lean_consume<MV>(ring + slot * kQ1LStageBytes,
+                             live ? bf_live + t * (kQ1LChunks * kQ1FragBytesPerChunk) : bf_dead, bstride,
+                             inf0 + 4 * kQ1LChunks * t, 4 * p.nchunks, woff, soff, yacc);
             __syncwarp();  // every lane is done with this stage before it is refilled
             slot = slot + 1 == kQ1LStages ? 0 : slot + 1;
         }
         s += st1 - st0;
         const int r = cell / p.blocksN, blk = cell - r * p.blocksN;
-        float *yr = grp.y[r] + blk * kQ1StepRows;
-        float *cut = st0 > 0 ? part[0][warp] : (st1 < spc ? part[1][warp] : nullptr);
-        finish_cell(yacc, lane, [&](int row, float v) {
-            if (cut != nullptr)
-                cut[row] = v;
-            else
-                yr[row] = v;
-        });
+        const int cut = st0 > 0 ? 0 : (st1 < spc ? 1 : -1);
+#pragma unroll
+        for (int v = 0; v < MV; ++v) {
+            float yv[2][2] = {{yacc[0][0][v], yacc[0][1][v]}, {yacc[1][0][v], yacc[1][1][v]}};
+            float *yr = grp.y[r] + (size_t)v * p.N + blk * kQ1StepRows;
+            finish_cell(yv, lane, [&](int row, float val) {
+                if (cut >= 0)
+                    part[cut][warp][v][row] = val;
+                else if (v < p.M)
+                    yr[row] = val;
+            });
+        }
     }
     cp_async_wait<0>();
     __syncthreads();
@@ -814,7 +865,10 @@ __global__ void __launch_bounds__(kQ1LMaxWarps * 32, 1) k_q1_m1_lean(const __gri
     if (warp + 1 < nw && s1 % spc != 0 && s1 > s0) {
         const int cell = c0 + s1 / spc;
         const int r = cell / p.blocksN, blk = cell - r * p.blocksN;
-        grp.y[r][blk * kQ1StepRows + lane] = part[1][warp][lane] + part[0][warp + 1][lane];
+#pragma unroll
+        for (int v = 0; v < MV; ++v)
+            if (v < p.M)
+                grp.y[r][(size_t)v * p.N + blk * kQ1StepRows + lane] = part[1][warp][v][lane] + part[0][warp + 1][v][lane];
     }
 }
 
@@ -951,6 +1005,7 @@ static int num_sms()
 struct Q1Plan {
     bool lean;          // lean stream kernel
     int warps;          // its warps per CTA
+    int mv;             // its vectors (1, 2 or 4)
     bool stream;        // stream kernel (else split kernel)
     int nchunks, blocksN, L, nslices, grid_x, grid_y;
     size_t act_smem, smem;
@@ -959,7 +1014,9 @@ struct Q1Plan {
 };
 
 // aligned: every matrix's signs and scales start on a 16-byte boundary.
-static Q1Plan q1_plan(int R, int N, int K, int sms, bool aligned = false)
+// mv > 1: only the lean stream kernel for mv vectors is considered (lean =
+// false when it does not apply).
+static Q1Plan q1_plan(int R, int N, int K, int sms, bool aligned = false, int mv = 1)
 {
     Q1Plan P = {};
     P.nchunks = (K + kQ1ChunkK - 1) / kQ1ChunkK;
@@ -975,25 +1032,28 @@ static Q1Plan q1_plan(int R, int N, int K, int sms, bool aligned = false)
     // (at most kQ1LMaxWarps) as fit next to the activation, >= 2 cells per warp
     if (aligned && K % 1024 == 0 && N % kQ1StepRows == 0) {
         const size_t per_warp = (size_t)kQ1LStages * kQ1LStageBytes;
-        const size_t cap = (size_t)kQ1MaxSmem - 2 * kQ1LMaxWarps * kQ1StepRows * 4;  // static cut buffers
-        const long long fit = whole < cap ? (long long)((cap - whole) / per_warp) : 0;
+        const size_t cap = (size_t)kQ1MaxSmem - 2 * q1l_max_warps(mv) * mv * kQ1StepRows * 4;  // static cut buffers
+        const size_t whole_mv = (size_t)mv * P.nchunks * per_chunk + kQ1ZeroBytes;
+        const long long fit = whole_mv < cap ? (long long)((cap - whole_mv) / per_warp) : 0;
         // >= one cell per warp keeps every warp's step range at least one
         // cell long, so a cell is cut at most once
-        const int warps = (int)std::min<long long>(std::min<long long>(kQ1LMaxWarps, fit), units / sms);
+        const int warps = (int)std::min<long long>(std::min<long long>(q1l_max_warps(mv), fit), units / sms);
         if (warps >= kQ1LMinWarps) {
             P.lean = true;
             P.stream = true;
             P.warps = warps;
+            P.mv = mv;
             P.L = P.nchunks;
             P.nslices = 1;
-            P.act_smem = whole;
-            P.smem = whole + (size_t)warps * per_warp;
+            P.act_smem = whole_mv;
+            P.smem = whole_mv + (size_t)warps * per_warp;
             P.grid_x = sms;
             P.grid_y = 1;
             P.ok = true;
             return P;
         }
     }
+    if (mv > 1) return P;
     // stream kernel: enough 32-row blocks for >= 2 cells per warp slot, and
     // the whole activation fits next to the rings
     if (units >= 2LL * sms * 2 * kQ1Warps && whole + ring_stream <= (size_t)kQ1MaxSmem) {
@@ -1064,7 +1124,7 @@ lowbit_status q1m1_prepare_launch(const uint16_t *x, int K, void *act, cudaStrea
 
 static lowbit_status q1m1_launch(const Q1Plan &P, const uint8_t *const *bits, const uint16_t *const *scales,
                                  const void *act, const uint16_t *x, float *const *y, int R, int N, int K,
-                                 cudaStream_t st)
+                                 cudaStream_t st, int M = 1)
 {
     Q1Group grp;
     for (int r = 0; r < R; ++r) {
@@ -1084,7 +1144,12 @@ static lowbit_status q1m1_launch(const Q1Plan &P, const uint8_t *const *bits, co
     p.blocksN = P.blocksN;
     p.cells = (int)((long long)R * P.blocksN);
     p.act_smem = (int)P.act_smem;
-    void (*kern)(const Q1Group, const Q1Params) = P.lean ? k_q1_m1_lean : P.stream ? k_q1_m1_stream : k_q1_m1_split;
+    p.M = M;
+    void (*kern)(const Q1Group, const Q1Params) = k_q1_m1_split;
+    if (P.lean)
+        kern = P.mv == 1 ? k_q1_m1_lean<1> : P.mv == 2 ? k_q1_m1_lean<2> : k_q1_m1_lean<4>;
+    else if (P.stream)
+        kern = k_q1_m1_stream;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
 
@@ -1121,22 +1186,26 @@ lowbit_status q1m1_gemv_launch(const uint8_t *const *bits, const uint16_t *const
     return q1m1_launch(q1_plan(R, N, K, num_sms(), aligned), bits, scales, act, nullptr, y, R, N, K, st);
 }
 
-// R matrices straight from x in one launch, when the shape takes the lean
-// stream kernel (every CTA builds the activation itself); otherwise
-// LOWBIT_ERR_UNSUPPORTED_SHAPE and the caller prepares the activation first.
+// R matrices straight from x ([M][K], 1 <= M <= 4) in one launch, when the
+// shape takes the lean stream kernel (every CTA builds the activation
+// itself; M = 3 runs the 4-vector form with a zero vector); otherwise
+// LOWBIT_ERR_UNSUPPORTED_SHAPE and the caller takes another path.
+static int q1_mv(int M) { return M <= 1 ? 1 : M == 2 ? 2 : 4; }
+
 lowbit_status q1m1_gemv_x_group_launch(const uint8_t *const *bits, const uint16_t *const *scales, const uint16_t *x,
-                                       float *const *y, int R, int N, int K, cudaStream_t st)
+                                       float *const *y, int R, int M, int N, int K, cudaStream_t st)
 {
-    if (use_tc(K) || R < 1 || R > kQ1MaxGroup || !q1m1_shape_supported(R, N, K)) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
-    const Q1Plan P = q1_plan(R, N, K, num_sms(), true);
+    if (M < 1 || M > 4 || use_tc(K) || R < 1 || R > kQ1MaxGroup || !q1m1_shape_supported(R, N, K))
+        return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    const Q1Plan P = q1_plan(R, N, K, num_sms(), true, q1_mv(M));
     if (!P.lean) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
-    return q1m1_launch(P, bits, scales, nullptr, x, y, R, N, K, st);
+    return q1m1_launch(P, bits, scales, nullptr, x, y, R, N, K, st, M);
 }
 
-bool q1m1_x_group_supported(int R, int N, int K)
+bool q1m1_x_group_supported(int R, int M, int N, int K)
 {
-    return !use_tc(K) && R >= 1 && R <= kQ1MaxGroup && q1m1_shape_supported(R, N, K) &&
-           q1_plan(R, N, K, num_sms(), true).lean;
+    return M >= 1 && M <= 4 && !use_tc(K) && R >= 1 && R <= kQ1MaxGroup && q1m1_shape_supported(R, N, K) &&
+           q1_plan(R, N, K, num_sms(), true, q1_mv(M)).lean;
 }
 
 // One matrix straight from x, in one launch (the split kernel builds its

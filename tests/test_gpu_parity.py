@@ -207,13 +207,15 @@ def test_q1_large_group(lb, R, N, K, xkind):
 
 
 @pytest.mark.parametrize("R,M,N,K", [(40, 1, 4096, 1024), (38, 1, 4096, 17408), (160, 1, 1024, 3072),
-                                     (40, 4, 4096, 1024), (12, 16, 5120, 5120), (40, 9, 1000, 2048),
+                                     (40, 4, 4096, 1024), (40, 2, 4096, 2048), (30, 3, 4096, 1024),
+                                     (12, 16, 5120, 5120), (40, 9, 1000, 2048),
                                      (3, 1, 515, 1280), (2, 2, 300, 2048)])
 def test_q1_group_from_x(lb, R, M, N, K):
     """lowbit_q1g128_gemv_group: one launch when the shape allows (the first
-    six cases on 148 SMs: the M = 1 persistent kernel, then the small-batch
-    persistent kernel with ragged rows and a partial batch tile), else
-    prepare + group product in the workspace.  Sampled outputs of three
+    eight cases on 148 SMs: the persistent bit-plane kernel for M = 1, 4, 2
+    and 3 (four vectors, one of them zero), then the small-batch bf16 kernel
+    with ragged rows and a partial batch tile), else prepare + group product
+    in the workspace.  Sampled outputs of three
     matrices against the oracle."""
     x = synth.bf16_normal(2800 + R, (M, K))
     g = torch.Generator(device="cuda")
