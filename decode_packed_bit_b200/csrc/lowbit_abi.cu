@@ -34,6 +34,8 @@ int q1stack_fault_flag();
 lowbit_status q1sm_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 lowbit_status q1m1_gemv_fused_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
                                      cudaStream_t);
+lowbit_status quantize_launch(int fmt, const float *w, int64_t rows, int64_t cols, uint8_t *packed, uint16_t *scales,
+                              cudaStream_t st);
 bool smg_supported(int fmt, int R, int M, int N, int K);
 lowbit_status smg_launch(int fmt, const uint8_t *const *, const uint16_t *const *, const uint16_t *, float *const *,
                          int R, int M, int N, int K, cudaStream_t);
@@ -101,6 +103,19 @@ lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, 
     LB_CHECK(codes != nullptr && packed != nullptr, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(aligned16(codes) && aligned16(packed), LOWBIT_ERR_MISALIGNED);
     return pack_launch(fmt, codes, rows, cols, packed, as_stream(stream));
+}
+
+lowbit_status lowbit_quantize(lowbit_format fmt, const float *w, int64_t rows, int64_t cols, uint8_t *packed,
+                              uint16_t *scales, void *stream)
+{
+    LB_CHECK(fmt == LOWBIT_FMT_Q1_G128 || fmt == LOWBIT_FMT_INT4_G64 || fmt == LOWBIT_FMT_Q2, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(fmt != LOWBIT_FMT_Q2, LOWBIT_ERR_UNSUPPORTED_SHAPE);  // the pages give no rule for 2-bit codes
+    LB_CHECK(rows >= 0 && cols >= 0 && rows * cols < kMaxElems, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(cols % (fmt == LOWBIT_FMT_Q1_G128 ? 128 : 64) == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    if (rows == 0 || cols == 0) return LOWBIT_OK;
+    LB_CHECK(w != nullptr && packed != nullptr && scales != nullptr, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(w) && aligned16(packed) && aligned16(scales), LOWBIT_ERR_MISALIGNED);
+    return quantize_launch(fmt == LOWBIT_FMT_Q1_G128 ? 1 : 3, w, rows, cols, packed, scales, as_stream(stream));
 }
 
 lowbit_status lowbit_unpack(lowbit_format fmt, const uint8_t *packed, int64_t rows, int64_t cols,

@@ -34,6 +34,7 @@ SYMBOLS = [
     ("lowbit_fault_flags", I32, []),
     ("lowbit_pack", I32, [I32, P, I64, I64, P, P]),
     ("lowbit_unpack", I32, [I32, P, I64, I64, P, P]),
+    ("lowbit_quantize", I32, [I32, P, I64, I64, P, P, P]),
     ("lowbit_q1g128_workspace_bytes", SZ, [I32, I32, I32]),
     ("lowbit_q1g128_gemv", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
     ("lowbit_q1g128_act_bytes", SZ, [I32, I32]),
@@ -120,6 +121,13 @@ def lowbit_unpack(fmt, packed, codes, stream=None):
     rows, cols = codes.shape
     _check(lib().lowbit_unpack(_fmt(fmt), _ptr(packed), rows, cols, _ptr(codes), _stream(stream)),
            "lowbit_unpack")
+
+
+def lowbit_quantize(fmt, w, packed, scales, stream=None):
+    """float32 weights [rows][cols] -> packed codes and FP16 scale bits ("q1" or "int4")."""
+    rows, cols = w.shape
+    _check(lib().lowbit_quantize(_fmt(fmt), _ptr(w), rows, cols, _ptr(packed), _ptr(scales), _stream(stream)),
+           "lowbit_quantize")
 
 
 # -- Q1_0_g128 --------------------------------------------------------------------

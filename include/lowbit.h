@@ -100,6 +100,26 @@ int lowbit_fault_flags(void);
  * ------------------------------------------------------------------------- */
 lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, int64_t cols,
                           uint8_t *packed, void *stream);
+/* Quantisation of float weights straight into the packed layouts above.
+ *   w       [rows][cols] float32 (16-byte aligned)
+ *   packed  [rows][cols/8] (Q1_0_g128) or [rows][cols/2] (INT4_G64)
+ *   scales  [rows][cols/128] or [rows][cols/64] FP16 bit patterns
+ * Q1_0_g128 ("Bonsai-27B-gguf technical white paper digest", "technical
+ * architecture highlights" fixes one sign per weight and one FP16 scale per
+ * 128): bit = (w >= 0), so -0.0 gives +1 and NaN -1; the scale is the
+ * group's mean |w| (the d minimising sum (w - d*sign)^2).
+ * INT4_G64 ("acorn-llm 0.11.4", "int4 quantisation quality: group
+ * quantisation": round-to-nearest int4, one scale per group along the input
+ * dimension): d = max|w| / 7 per 64-group; q = w / d rounded to nearest,
+ * ties to even, clamped to [-8, 7] (-8 never occurs); q = 0 where d = 0 or w
+ * is NaN.
+ * Scales round to FP16 nearest-even; magnitudes >= 65504 saturate to 65504.
+ * Every step is an IEEE double operation in a fixed order, so the result is
+ * the same bits on every run.  LOWBIT_FMT_Q2 returns
+ * LOWBIT_ERR_UNSUPPORTED_SHAPE (the pages give no rule for its codes);
+ * cols must be a multiple of the group size; rows == 0 is a no-op. */
+lowbit_status lowbit_quantize(lowbit_format fmt, const float *w, int64_t rows, int64_t cols,
+                              uint8_t *packed, uint16_t *scales, void *stream);
 lowbit_status lowbit_unpack(lowbit_format fmt, const uint8_t *packed, int64_t rows, int64_t cols,
                             int8_t *codes, void *stream);
 

@@ -75,6 +75,11 @@ def _load():
     lib.orc_trigram_encode.restype = None
     lib.orc_rmsnorm.argtypes = [P, P, I64, I64, ctypes.c_double, P]
     lib.orc_rmsnorm.restype = None
+    lib.orc_f64_to_f16.argtypes = [ctypes.c_double]
+    lib.orc_f64_to_f16.restype = ctypes.c_uint16
+    for name in ("orc_q1_quantize", "orc_int4_quantize"):
+        getattr(lib, name).argtypes = [P, I64, I64, P, P]
+        getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -245,3 +250,32 @@ def rmsnorm(a, b=None, eps=1e-6):
         bp = _ptr(b)
     _load().orc_rmsnorm(_ptr(a), bp, M, D, eps, _ptr(r))
     return r
+
+
+def f64_to_f16(v: float) -> int:
+    """IEEE binary16 bits of v: nearest, ties to even; |v| >= 65504 saturates."""
+    return int(_load().orc_f64_to_f16(float(v)))
+
+
+def q1_quantize(w):
+    """float32 [N][K] -> (codes int8 {0,1} [N][K], fp16 scale bits [N][K/128]):
+    sign w >= 0 -> 1, scale = fp16(mean |w| over each 128-group)."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    codes = np.zeros((N, K), np.int8)
+    scales = np.zeros((N, K // 128), np.uint16)
+    if _load().orc_q1_quantize(_ptr(w), N, K, _ptr(codes), _ptr(scales)) != 0:
+        raise ValueError("oracle q1_quantize: K must be a multiple of 128")
+    return codes, scales
+
+
+def int4_quantize(w):
+    """float32 [N][K] -> (codes int8 [-8,7] [N][K], fp16 scale bits [N][K/64]):
+    d = fp16(max|w| / 7) per 64-group, q = clamp(rint(w / d), -8, 7)."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    codes = np.zeros((N, K), np.int8)
+    scales = np.zeros((N, K // 64), np.uint16)
+    if _load().orc_int4_quantize(_ptr(w), N, K, _ptr(codes), _ptr(scales)) != 0:
+        raise ValueError("oracle int4_quantize: K must be a multiple of 64")
+    return codes, scales

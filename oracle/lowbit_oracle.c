@@ -29,7 +29,7 @@
  *            the input dimension; symmetric round-to-nearest int4; the scale
  *            changes every 64 values).
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - Q1 bit polarity: bit 1 -> +1, bit 0 -> -1.
  *   - Q1 bit order: weight k of a row is bit (k % 8) of byte (k / 8), LSB first
  *     (the same LSB-first order the Z80 listing uses for its 2-bit fields).
@@ -435,4 +435,92 @@ void orc_rmsnorm(const float *a, const float *b, int64_t M, int64_t D, double ep
             r[m * D + d] = v * inv;
         }
     }
+}
+
+
+/* ------------------------------------------------------------------------
+ * Quantisers: float weights -> the packed formats' codes and FP16 scales.
+ *
+ * [BONSAI] "technical architecture highlights" fixes only the result (one
+ * sign per weight, one FP16 scale per 128 weights).  Reading: the sign is
+ * w >= 0 -> +1 (so -0.0 -> +1 and NaN -> -1), and the scale is the group's
+ * mean |w|, the value of d that minimises sum (w - d s)^2 with s = sign(w).
+ * [ACORN] "int4 quantisation quality: group quantisation": round-to-nearest
+ * int4 with one scale per group along the input dimension (64 values here).
+ * Reading: symmetric, d = max |w| / 7, q = w / d rounded to nearest with
+ * ties to even, clamped to [-8, 7] (so -8 never occurs), q = 0 where d = 0
+ * or w is NaN.
+ * Every step is an IEEE double operation in a fixed order (sums with k
+ * ascending), and FP16 rounding is to nearest, ties to even, with values at
+ * or above 65504 saturating to 65504.
+ * ---------------------------------------------------------------------- */
+
+/* double -> FP16 bits: round to nearest, ties to even; |v| >= 65504 gives
+ * +-65504 (the largest finite half); NaN gives 0. */
+uint16_t orc_f64_to_f16(double v)
+{
+    if (v != v) return 0;
+    const uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (a >= 65504.0) return (uint16_t)(sign | 0x7BFFu);
+    if (a == 0.0) return sign;
+    /* the spacing of halves near a: 2^-24 below 2^-14, else 2^(e-10) */
+    int e;
+    frexp(a, &e);           /* a = f * 2^e, 0.5 <= f < 1: a in [2^(e-1), 2^e) */
+    int ex = e - 1;         /* a in [2^ex, 2^(ex+1)) */
+    if (ex < -14) ex = -14; /* subnormal range shares the spacing of 2^-14 */
+    const double quantum = ldexp(1.0, ex - 10);
+    const double r = rint(a / quantum) * quantum; /* a / quantum is exact; rint: ties to even */
+    if (r >= 65504.0) return (uint16_t)(sign | 0x7BFFu);
+    if (r < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)(r / ldexp(1.0, -24)));
+    int er;
+    const double fr = frexp(r, &er); /* r = fr * 2^er */
+    const int exp16 = er - 1 + 15;
+    const unsigned mant = (unsigned)((fr * 2.0 - 1.0) * 1024.0);
+    return (uint16_t)(sign | ((unsigned)exp16 << 10) | mant);
+}
+
+int orc_q1_quantize(const float *w, int64_t rows, int64_t cols, int8_t *codes, uint16_t *scales)
+{
+    if (cols % 128 != 0) return 1;
+    const int64_t G = cols / 128;
+    for (int64_t n = 0; n < rows; ++n)
+        for (int64_t g = 0; g < G; ++g) {
+            double s = 0.0;
+            for (int64_t k = g * 128; k < (g + 1) * 128; ++k) {
+                const float v = w[n * cols + k];
+                s += fabs((double)v);
+                codes[n * cols + k] = (int8_t)(v >= 0.0f ? 1 : 0);
+            }
+            scales[n * G + g] = orc_f64_to_f16(s / 128.0);
+        }
+    return 0;
+}
+
+int orc_int4_quantize(const float *w, int64_t rows, int64_t cols, int8_t *codes, uint16_t *scales)
+{
+    if (cols % 64 != 0) return 1;
+    const int64_t G = cols / 64;
+    for (int64_t n = 0; n < rows; ++n)
+        for (int64_t g = 0; g < G; ++g) {
+            double amax = 0.0;
+            for (int64_t k = g * 64; k < (g + 1) * 64; ++k) {
+                const double a = fabs((double)w[n * cols + k]);
+                if (a > amax) amax = a;
+            }
+            const uint16_t dh = orc_f64_to_f16(amax / 7.0);
+            scales[n * G + g] = dh;
+            const double d = orc_f16_to_f64(dh);
+            for (int64_t k = g * 64; k < (g + 1) * 64; ++k) {
+                const double v = (double)w[n * cols + k];
+                double q = 0.0;
+                if (d > 0.0 && v == v) {
+                    q = rint(v / d);
+                    if (q < -8.0) q = -8.0;
+                    if (q > 7.0) q = 7.0;
+                }
+                codes[n * cols + k] = (int8_t)q;
+            }
+        }
+    return 0;
 }

@@ -49,6 +49,62 @@ def test_pack_unpack_bitexact(lb, fmt, per, rows, cols):
     assert np.array_equal(host(back), codes)
 
 
+def _quant_inputs(seed, rows, cols, special):
+    g = np.random.default_rng(seed)
+    w = (g.standard_normal((rows, cols)) * g.uniform(1e-3, 5.0, (rows, 1))).astype(np.float32)
+    if special:
+        w[0, :128] = 0.0                                   # a zero group
+        w[1, :8] = [-0.0, 0.0, np.nan, np.inf, -np.inf, 1e30, -1e-30, 7.0]
+        w[2, :64] = 1e-6                                   # subnormal FP16 scales
+        w[3, :64] = 3.0e5                                  # saturating scales
+    return w
+
+
+@pytest.mark.parametrize("fmt,group", [("q1", 128), ("int4", 64)])
+@pytest.mark.parametrize("rows,cols,special", [(37, 1280, False), (300, 4096, False), (8, 512, True)])
+def test_quantize_bitexact(lb, fmt, group, rows, cols, special):
+    """lowbit_quantize against the oracle's quantiser + packer: every packed
+    byte and every FP16 scale bit-exact."""
+    w = _quant_inputs(5100 + rows, rows, cols, special)
+    per = 8 if fmt == "q1" else 2
+    packed = torch.zeros((rows, cols // per), dtype=torch.uint8, device="cuda")
+    scales = torch.zeros((rows, cols // group), dtype=torch.int16, device="cuda")
+    lb.lowbit_quantize(fmt, torch.from_numpy(w).cuda(), packed, scales)
+    _sync()
+    codes, sref = oracle.q1_quantize(w) if fmt == "q1" else oracle.int4_quantize(w)
+    assert np.array_equal(host(scales).view(np.uint16), sref)
+    assert np.array_equal(host(packed), oracle.pack(fmt, codes))
+
+
+def test_quantize_then_product(lb):
+    """Quantise on the GPU, then multiply: matches the oracle's product of the
+    oracle-quantised weights (same bits in, so the float bar applies)."""
+    N, K = 256, 2048
+    w = _quant_inputs(5200, N, K, False)
+    x = synth.bf16_normal(5200, (1, K))
+    bits = torch.zeros((N, K // 8), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros((N, K // 128), dtype=torch.int16, device="cuda")
+    lb.lowbit_quantize("q1", torch.from_numpy(w).cuda(), bits, sc)
+    y = torch.zeros((1, N), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(16, lb.lowbit_q1g128_workspace_bytes(1, N, K)), dtype=torch.uint8, device="cuda")
+    lb.lowbit_q1g128_gemv(bits, sc, dev(x), y, workspace=ws)
+    _sync()
+    codes, sref = oracle.q1_quantize(w)
+    y64, ab = oracle.q1_gemv(oracle.pack("q1", codes), sref, x, want_abs=True)
+    check_float(host(y), y64, ab, "quantise then Q1 product")
+
+
+def test_quantize_rejects_q2_and_ragged(lb):
+    from decode_packed_bit_b200.lowbit import LowbitError
+    w = torch.zeros((4, 128), dtype=torch.float32, device="cuda")
+    out = torch.zeros((4, 64), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros((4, 2), dtype=torch.int16, device="cuda")
+    with pytest.raises(LowbitError):
+        lb.lowbit_quantize("q2", w, out, sc)
+    with pytest.raises(LowbitError):
+        lb.lowbit_quantize("q1", torch.zeros((4, 96), dtype=torch.float32, device="cuda"), out, sc)
+
+
 @pytest.mark.parametrize("fmt,per", [("q1", 8), ("q2", 4), ("int4", 2)])
 def test_unpack_every_byte_value(lb, fmt, per):
     allb = np.tile(np.arange(256, dtype=np.uint8), 16).reshape(16, 256)   # 16-byte aligned rows
