@@ -19,12 +19,14 @@
 // registers, and the matching B registers are simply x[m][k..k+3], one
 // 8-byte word.
 //
-// Work split (as for the M = 1 kernels): a warp owns 32 rows (two 16-row
-// tiles); a CTA of four warps 128 rows of one K-slice; the S slices of a row
-// block form a thread-block cluster and add their partial sums in rank order
-// through distributed shared memory.  The CTA stages its slice of x in
-// shared memory in fragment order; every warp streams its rows' sign bits
-// and scales through a cp.async ring, 256 k per step.
+// Work split of one product (as for the M = 1 kernels): a warp owns 32 rows
+// (two 16-row tiles); a CTA of four warps 128 rows of one K-slice; the S
+// slices of a row block form a thread-block cluster and add their partial
+// sums in rank order through distributed shared memory.  The CTA stages x in
+// shared memory in fragment order; every warp streams its rows' packed
+// weights and scales through a cp.async ring, one step (256 k for Q1_0_g128,
+// 128 k for INT4_G64) at a time.  A group of products that read one x runs in
+// one persistent launch instead (k_smallm_grp, at the end of this file).
 #include <algorithm>
 #include <mutex>
 

@@ -22,9 +22,11 @@
 //     y += d * (2^(E-27) * D - 2^(E-20) * sum_k X_k).
 //
 // Work split and weight streaming follow the Q1 kernels: a step is 32 rows
-// (two mma tiles) x one 128-k pair of groups, staged per warp by cp.async; a
-// thread-block cluster splits K and reduces through distributed shared memory
-// when the rows alone cannot fill the GPU.
+// (two mma tiles) x one 128-k pair of groups, staged per warp by cp.async.
+// One matrix: a thread-block cluster splits K and reduces through distributed
+// shared memory when the rows alone cannot fill the GPU (k_i4_m1_split).  A
+// group of matrices that read one x: one persistent CTA per SM streams an
+// equal share of every matrix's 32-row blocks over all of K (k_i4_m1_lean).
 #include <algorithm>
 #include <mutex>
 

@@ -1,6 +1,7 @@
-// q1_gemv_m1.cu -- Q1_0_g128 matrix-vector products at M = 1 on the tensor
-// cores (mma.sync m16n8k32, u8 x s8 -> s32), for one weight matrix or a
-// group of R matrices that multiply the same activation vector.
+// q1_gemv_m1.cu -- Q1_0_g128 products at M = 1 (and, in the persistent
+// kernel, M = 2..4) on the integer tensor cores (mma.sync m16n8k32, u8 x s8
+// -> s32), for one weight matrix or a group of R matrices that multiply the
+// same activation; and the one-launch decode step through a stack of them.
 //
 // What is computed ("Bonsai-27B-gguf technical white paper digest",
 // "technical architecture highlights": one sign bit per weight, one FP16
@@ -36,15 +37,19 @@
 //     the 24-bit rounding of x and the fp32 epilogue.
 //
 // Weight streaming: each warp owns a ring of shared-memory stages filled by
-// cp.async; a stage is 32 rows x 2 chunks (64 bytes of each row) plus their
-// scales, so kQ1Stages-1 stages of every warp are always in flight, and each
-// B fragment read from shared memory feeds two 16-row mma tiles.  The first stages are issued before griddepcontrol.wait, which lets
-// the weight stream of a launch overlap the tail of the previous kernel.
+// cp.async, so the stages after the one being consumed are always in flight,
+// and each B fragment read from shared memory feeds two 16-row mma tiles.
+// The first stages are issued before griddepcontrol.wait, which lets the
+// weight stream of a launch overlap the tail of the previous kernel.
 //
-// Two work splits:
-//   stream kernel (a group with many 16-row tiles): persistent CTAs take
-//     equal contiguous ranges of (matrix, 16-row tile) cells, each over all
-//     of K; the whole prepared activation sits in shared memory.
+// Work splits:
+//   persistent kernel (k_q1_m1_lean; groups with at least 8 32-row blocks
+//     per SM, K % 1024 == 0): one CTA per SM takes an equal range of (matrix,
+//     32-row block) cells over all of K, cut into equal per-warp ranges of
+//     1024-k steps; the activation of MV = 1, 2 or 4 vectors sits in shared
+//     memory, built from x by every CTA or staged from a prepared copy.
+//   stream kernel (other groups with many 32-row blocks): the older
+//     persistent form with 512-k steps and whole cells per warp.
 //   split kernel (too few tiles to fill the GPU, e.g. one matrix): K is cut
 //     into S <= 8 slices, the S CTAs of one 128-row block form a thread-block
 //     cluster, and their partial sums are added in fixed rank order through
