@@ -32,10 +32,12 @@
  *     failed launch (cudaGetLastError).  Faults inside a kernel are
  *     asynchronous and surface at the caller's next synchronisation.
  *   - The caller owns every buffer.  The library allocates no device memory
- *     and keeps no global state; entry points are safe to call from several
- *     host threads on different streams.  Kernels whose work needs scratch
- *     memory take a caller-provided workspace, sized by the matching
- *     *_workspace_bytes() query.
+ *     and keeps no state across calls besides the fault flags
+ *     (lowbit_fault_flags) and the scratch array of the allocation-free
+ *     entry point; entry points are safe to call from several host threads
+ *     on different streams.  Kernels whose work needs scratch memory take a
+ *     caller-provided workspace, sized by the matching *_workspace_bytes()
+ *     query.
  *
  * Packed layouts (one row of a matrix is packed along K):
  *   Q1_0_g128  bits   [N][K/8]:   weight k is bit (k%8) of byte k/8; bit 1
@@ -182,14 +184,16 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits,
  * shape [N][K] that read one activation x [M][K] (bf16).
  *   w_bits, w_scales, y: HOST arrays of R device pointers (1 <= R <= 256),
  *   16-byte aligned; results as lowbit_q1g128_gemv_act_group.
- * At M = 1, with K % 1024 == 0, N % 32 == 0 and at least SMs * 8
+ * At M <= 4, with K % 1024 == 0, N % 32 == 0 and at least SMs * 8
  * (32-row block, matrix) pairs (e.g. 10 or more 4096-row matrices on 148
  * SMs), this is one launch: every CTA turns x into the operand form itself,
- * and no workspace is needed.  At 2 <= M <= 16 with K % 256 == 0 and at
- * least SMs * 8 32-row blocks over the group, it is one launch of a
- * persistent kernel (each warp owns a 32-row block over all of K; the warps
- * of a CTA share x).  Otherwise the call prepares the activation in the
- * workspace and runs lowbit_q1g128_gemv_act_group.
+ * the masked sign planes feed one integer mma per vector, and no workspace is
+ * needed (at M = 2..4 while all M vectors' operands fit in shared memory:
+ * K up to about 12k at M = 3, 4).  At 2 <= M <= 16 otherwise, with
+ * K % 256 == 0 and at least SMs * 8 32-row blocks over the group, it is one
+ * launch of a persistent bf16 kernel (each warp owns a 32-row block over all
+ * of K; the warps of a CTA share x).  Other shapes prepare the activation in
+ * the workspace and run lowbit_q1g128_gemv_act_group.
  * Workspace: lowbit_q1g128_group_workspace_bytes(R, M, N, K) bytes (NULL
  * allowed when 0).  Calls that share a workspace must be ordered on one
  * stream. */
