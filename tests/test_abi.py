@@ -116,3 +116,45 @@ def test_q2_and_glue_validation(L):
     assert n(FAKE, None, 1, 12, 1e-6, FAKE, None) == 3
     assert n(FAKE, None, 1, 16, -1.0, FAKE, None) == 1
     assert n(FAKE, MIS, 1, 16, 1e-6, FAKE, None) == 2
+
+
+def test_quantize_validation(L):
+    q = L.lowbit_quantize
+    assert q(7, FAKE, 4, 128, FAKE, FAKE, None) == 1                   # bad format
+    assert q(2, FAKE, 4, 128, FAKE, FAKE, None) == 3                   # Q2: no rule on the pages
+    assert q(1, FAKE, 4, 64, FAKE, FAKE, None) == 3                    # Q1: cols % 128
+    assert q(3, FAKE, 4, 96, FAKE, FAKE, None) == 3                    # INT4: cols % 64
+    assert q(1, None, 4, 128, FAKE, FAKE, None) == 1                   # null weights
+    assert q(3, FAKE, 4, 128, FAKE, None, None) == 1                   # null scales
+    assert q(1, FAKE, 4, 128, MIS, FAKE, None) == 2                    # misaligned output
+    assert q(1, None, 0, 128, None, None, None) == 0                   # empty: no-op
+    assert q(3, FAKE, -1, 128, FAKE, FAKE, None) == 1
+
+
+def test_group_validation(L):
+    ptrs = (ctypes.c_void_p * 2)(0x10000, 0x10000)
+    pp = ctypes.cast(ptrs, ctypes.c_void_p)
+    misp = ctypes.cast((ctypes.c_void_p * 2)(0x10000, 0x10008), ctypes.c_void_p)
+    g = L.lowbit_q1g128_gemv_group
+    assert g(pp, pp, FAKE, pp, 0, 1, 16, 256, None, 0, None) == 1       # R < 1
+    assert g(pp, pp, FAKE, pp, 257, 1, 16, 256, None, 0, None) == 1     # R > 256
+    assert g(pp, pp, None, pp, 2, 1, 16, 256, None, 0, None) == 1       # null x
+    assert g(pp, pp, MIS, pp, 2, 1, 16, 256, None, 0, None) == 2        # misaligned x
+    assert g(pp, pp, FAKE, misp, 2, 1, 16, 256, None, 0, None) == 2     # misaligned y[1]
+    assert g(pp, pp, FAKE, pp, 2, 1, 16, 200, None, 0, None) == 3       # K % 128
+    assert g(pp, pp, FAKE, pp, 2, 17, 16, 256, None, 0, None) == 1      # M > 16
+    # a small group needs the prepared activation in the workspace
+    need = L.lowbit_q1g128_group_workspace_bytes(2, 1, 16, 256)
+    assert need > 0
+    assert g(pp, pp, FAKE, pp, 2, 1, 16, 256, None, need, None) == 1
+    assert g(pp, pp, FAKE, pp, 2, 1, 16, 256, FAKE, need - 1, None) == 1
+    # groups the persistent kernels take need none (148 SMs when no device is visible)
+    assert L.lowbit_q1g128_group_workspace_bytes(10, 1, 4096, 1024) == 0
+    assert L.lowbit_q1g128_group_workspace_bytes(40, 4, 4096, 1024) == 0
+    assert L.lowbit_q1g128_group_workspace_bytes(40, 16, 4096, 1024) == 0
+    i = L.lowbit_int4g64_gemm_group
+    assert i(pp, pp, FAKE, pp, 0, 1, 16, 128, None, 0, None) == 1       # R < 1
+    assert i(pp, pp, None, pp, 2, 1, 16, 128, None, 0, None) == 1       # null x
+    assert i(pp, pp, FAKE, misp, 2, 1, 16, 128, None, 0, None) == 2     # misaligned y[1]
+    assert i(pp, pp, FAKE, pp, 2, 1, 16, 96, None, 0, None) == 3        # K % 64
+    assert L.lowbit_int4g64_group_workspace_bytes(17, 1, 11008, 4096) == 0
