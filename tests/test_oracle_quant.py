@@ -157,3 +157,46 @@ def test_int4_zero_and_nan_groups():
     codes, scales = oracle.int4_quantize(w)
     assert (codes[0, :64] == 0).all() and scales[0, 0] == 0
     assert codes[0, 70] == 0 and (np.delete(codes[0, 64:], 6) == 7).all()
+
+
+# ---------------------------------------------------------------------------
+# properties over random inputs (hypothesis)
+# ---------------------------------------------------------------------------
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+_floats = st.floats(min_value=-1e4, max_value=1e4, allow_nan=False, allow_infinity=False, width=32)
+
+
+def _sse(w, s, d):
+    return float(((w - d * s) ** 2).sum())
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.lists(_floats, min_size=128, max_size=128))
+def test_q1_scale_beats_its_fp16_neighbours(vals):
+    """The squared error is a convex quadratic in d, so the fp16 scale the
+    oracle picks must do at least as well as the neighbouring fp16 values."""
+    w = np.array(vals, np.float32)[None, :]
+    codes, scales = oracle.q1_quantize(w)
+    s = np.where(codes[0] == 1, 1.0, -1.0)
+    wd = w[0].astype(np.float64)
+    h = int(scales[0, 0])
+    best = _sse(wd, s, f16(h))
+    for nb in (h - 1, h + 1):
+        if 0 <= nb <= 0x7BFF:
+            assert best <= _sse(wd, s, f16(nb)) * (1 + 1e-12) + 1e-300
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.lists(_floats, min_size=64, max_size=64))
+def test_int4_codes_are_nearest_for_their_scale(vals):
+    w = np.array(vals, np.float32)[None, :]
+    codes, scales = oracle.int4_quantize(w)
+    d = f16(int(scales[0, 0]))
+    wd = w[0].astype(np.float64)
+    allq = np.arange(-8, 8)
+    for k in range(64):
+        err = np.abs(wd[k] - allq * d).min()
+        assert abs(wd[k] - codes[0, k] * d) <= err * (1 + 1e-12) + 1e-300
+    assert codes.min() >= -7
