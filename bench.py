@@ -503,12 +503,11 @@ def run_int4(args, world, rank, local):
     for M in (1, 32, 256):
         x = torch.randn((M, K), generator=g, device=dev).bfloat16()
         y = torch.empty((R, M, N), dtype=torch.float32, device=dev)
-        ws = torch.empty(max(16, lb.lowbit_int4g64_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
         stream = torch.cuda.Stream(device=dev)
 
         def step():
             for r in range(R):
-                lb.lowbit_int4g64_gemm(qs[r], ss[r], x, y[r], workspace=ws, stream=stream)
+                lb.lowbit_int4g64_gemm(qs[r], ss[r], x, y[r], stream=stream)
         ms = max_over_ranks(_graph_time(step, stream, max(20, args.steps), args.warmup), world)
         res = {"M": M, "us_per_call": round(ms * 1e3 / R, 3),
                "weight_gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
@@ -516,11 +515,9 @@ def run_int4(args, world, rank, local):
         if M <= 32:
             # the R weight sets read one x: one grouped launch
             ys = [y[r] for r in range(R)]
-            gws = lb.lowbit_int4g64_group_workspace_bytes(R, M, N, K)
-            gw = torch.zeros(gws, dtype=torch.uint8, device=dev) if gws else None
 
             def gstep():
-                lb.lowbit_int4g64_gemm_group(qs, ss, x, ys, workspace=gw, stream=stream)
+                lb.lowbit_int4g64_gemm_group(qs, ss, x, ys, stream=stream)
             gms = max_over_ranks(_graph_time(gstep, stream, max(20, args.steps), args.warmup), world)
             res["group_us"] = round(gms * 1e3, 3)
             res["group_weight_gbs"] = round(R * per / (gms * 1e-3) / 1e9, 1)

@@ -21,7 +21,6 @@ bool i4m1_supported(int N, int K);
 bool i4tc_supported(int M, int N, int K);
 lowbit_status i4tc_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 int i4tc_fault_flag();
-int q1tc_fault_flag();
 lowbit_status i4m1_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, cudaStream_t);
 lowbit_status q1m1_prepare_launch(const uint16_t *, int, void *, cudaStream_t);
 bool q1sm_supported(int M, int N, int K);
@@ -34,6 +33,7 @@ int q1stack_fault_flag();
 lowbit_status q1sm_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 lowbit_status q1m1_gemv_fused_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
                                      cudaStream_t);
+bool q1m1_fused_supported(int N, int K);
 lowbit_status quantize_launch(int fmt, const float *w, int64_t rows, int64_t cols, uint8_t *packed, uint16_t *scales,
                               cudaStream_t st);
 bool smg_supported(int fmt, int R, int M, int N, int K);
@@ -87,9 +87,9 @@ int lowbit_version(void) { return 100; }
 
 int lowbit_fault_flags(void)
 {
-    const int f4 = i4tc_fault_flag(), f1 = q1tc_fault_flag(), fs = q1stack_fault_flag();
-    if (f4 < 0 || f1 < 0 || fs < 0) return -1;
-    return (f4 ? 1 : 0) | (f1 ? 2 : 0) | (fs ? 4 : 0);
+    const int f4 = i4tc_fault_flag(), fs = q1stack_fault_flag();
+    if (f4 < 0 || fs < 0) return -1;
+    return (f4 ? 1 : 0) | (fs ? 4 : 0);
 }
 
 lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, int64_t cols,
@@ -172,7 +172,8 @@ size_t lowbit_q1g128_workspace_bytes(int M, int N, int K)
 {
     if (M < 1 || M > kQ1MaxM || N < 1 || K < 128 || K % 128 != 0) return 0;
     if (!q1_tc_path(1, M, N, K)) return 0;
-    return al256(q1m1_act_bytes(K));  // the prepared activation
+    if (q1m1_fused_supported(N, K)) return 0;  // one launch builds the activation in shared memory
+    return al256(q1m1_act_bytes(K));           // the persistent kernel reads a prepared activation
 }
 
 lowbit_status lowbit_q1g128_gemv(const uint8_t *w_bits, const uint16_t *w_scales, const uint16_t *x,
@@ -316,25 +317,14 @@ lowbit_status lowbit_q1g128_stack_step(const uint8_t *const *w_bits, const uint1
 // INT4_G64
 // ---------------------------------------------------------------------------
 
-size_t lowbit_int4g64_workspace_bytes(int M, int N, int K)
-{
-    (void)M;
-    (void)N;
-    (void)K;
-    return 0;  // every INT4_G64 kernel builds what it needs in shared memory
-}
-
 lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales, const uint16_t *x, float *y,
-                                  int M, int N, int K, void *workspace, size_t workspace_bytes, void *stream)
+                                  int M, int N, int K, void *stream)
 {
     LB_CHECK(M >= 1 && N >= 1 && K >= 1, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(K % 64 == 0 && (int64_t)N * K < kMaxElems && (int64_t)M * K < kMaxElems,
              LOWBIT_ERR_UNSUPPORTED_SHAPE);
     LB_CHECK(w_q && w_scales && x && y, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(aligned16(w_q) && aligned16(w_scales) && aligned16(x) && aligned16(y), LOWBIT_ERR_MISALIGNED);
-    const size_t need = lowbit_int4g64_workspace_bytes(M, N, K);
-    LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
-    LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
     cudaStream_t st = as_stream(stream);
     if (M == 1 && i4m1_supported(N, K)) return i4m1_launch(w_q, w_scales, x, y, N, K, st);
     if (M >= 2 && i4sm_supported(M, N, K)) return i4sm_launch(w_q, w_scales, x, y, M, N, K, st);
@@ -342,15 +332,9 @@ lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales, 
     return int4_gemv_simt_launch(w_q, w_scales, x, y, M, N, K, st);
 }
 
-size_t lowbit_int4g64_group_workspace_bytes(int R, int M, int N, int K)
-{
-    (void)R;
-    return lowbit_int4g64_workspace_bytes(M, N, K);
-}
-
 lowbit_status lowbit_int4g64_gemm_group(const uint8_t *const *w_q, const uint16_t *const *w_scales,
                                         const uint16_t *x, float *const *y, int R, int M, int N, int K,
-                                        void *workspace, size_t workspace_bytes, void *stream)
+                                        void *stream)
 {
     LB_CHECK(R >= 1 && R <= 256 && w_q && w_scales && y && x, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(M >= 1 && N >= 1 && K >= 1, LOWBIT_ERR_INVALID_ARG);
@@ -361,15 +345,11 @@ lowbit_status lowbit_int4g64_gemm_group(const uint8_t *const *w_q, const uint16_
         LB_CHECK(w_q[r] && w_scales[r] && y[r], LOWBIT_ERR_INVALID_ARG);
         LB_CHECK(aligned16(w_q[r]) && aligned16(w_scales[r]) && aligned16(y[r]), LOWBIT_ERR_MISALIGNED);
     }
-    const size_t need = lowbit_int4g64_group_workspace_bytes(R, M, N, K);
-    LB_CHECK(workspace_bytes >= need && (need == 0 || workspace != nullptr), LOWBIT_ERR_INVALID_ARG);
-    LB_CHECK(workspace == nullptr || aligned16(workspace), LOWBIT_ERR_MISALIGNED);
     cudaStream_t st = as_stream(stream);
     if (M == 1 && i4m1_group_supported(R, N, K)) return i4m1_group_launch(w_q, w_scales, x, y, R, N, K, st);
     if (M >= 2 && smg_supported(3, R, M, N, K)) return smg_launch(3, w_q, w_scales, x, y, R, M, N, K, st);
     for (int r = 0; r < R; ++r) {
-        const lowbit_status s =
-            lowbit_int4g64_gemm(w_q[r], w_scales[r], x, y[r], M, N, K, workspace, workspace_bytes, stream);
+        const lowbit_status s = lowbit_int4g64_gemm(w_q[r], w_scales[r], x, y[r], M, N, K, stream);
         if (s != LOWBIT_OK) return s;
     }
     return LOWBIT_OK;

@@ -1096,23 +1096,12 @@ static Q1Plan q1_plan(int R, int N, int K, int sms, bool aligned = false, int mv
     return P;
 }
 
-// With LOWBIT_Q1_TC=1 at build time, K a multiple of 1024 goes to the
-// tcgen05 kernel (q1_gemv_tc.cu) instead.  It is off by default: measured on
-// B200 it streams 1.4 TB/s against 3.5 TB/s for the mma.sync kernels above,
-// because every 128-row tile needs a four-warp hand-off to the MMA warp per
-// 256 k, where the mma.sync warps run independently.
-#ifndef LOWBIT_Q1_TC
-#define LOWBIT_Q1_TC 0
-#endif
-static bool use_tc(int K) { return LOWBIT_Q1_TC && q1tc_supported(1, 1, K); }
-
-size_t q1m1_act_bytes(int K) { return use_tc(K) ? q1tc_act_bytes(K) : q1_plan(1, 1, K, 148).act_bytes; }
-size_t q1m1_xcopy_off(int K) { return use_tc(K) ? q1tc_xcopy_off(K) : q1_plan(1, 1, K, 148).xcopy_off; }
+size_t q1m1_act_bytes(int K) { return q1_plan(1, 1, K, 148).act_bytes; }
+size_t q1m1_xcopy_off(int K) { return q1_plan(1, 1, K, 148).xcopy_off; }
 int q1m1_max_group() { return kQ1MaxGroup; }
 
 bool q1m1_shape_supported(int R, int N, int K)
 {
-    if (use_tc(K)) return q1tc_supported(R, N, K);
     if ((K / 128) % 2 != 0) return false;  // scale pairs must be 4-byte aligned
     if (R < 1 || R > kQ1MaxGroup) return false;
     return q1_plan(R, N, K, num_sms()).ok;
@@ -1120,7 +1109,6 @@ bool q1m1_shape_supported(int R, int N, int K)
 
 lowbit_status q1m1_prepare_launch(const uint16_t *x, int K, void *act, cudaStream_t st)
 {
-    if (use_tc(K)) return q1tc_prepare_launch(x, K, act, st);
     const Q1Plan P = q1_plan(1, 1, K, 148);
     cudaError_t e = launch_pdl(k_q1_prep_m1, dim3(P.nchunks), dim3(256), 0, st, x, K, static_cast<uint8_t *>(act),
                                P.info_off, P.xcopy_off);
@@ -1183,7 +1171,6 @@ static lowbit_status q1m1_launch(const Q1Plan &P, const uint8_t *const *bits, co
 lowbit_status q1m1_gemv_launch(const uint8_t *const *bits, const uint16_t *const *scales, const void *act,
                                float *const *y, int R, int N, int K, cudaStream_t st)
 {
-    if (use_tc(K)) return q1tc_gemv_launch(bits, scales, act, y, R, N, K, st);
     bool aligned = true;
     for (int r = 0; r < R; ++r)
         aligned = aligned && (reinterpret_cast<uintptr_t>(bits[r]) & 15u) == 0 &&
@@ -1200,7 +1187,7 @@ static int q1_mv(int M) { return M <= 1 ? 1 : M == 2 ? 2 : 4; }
 lowbit_status q1m1_gemv_x_group_launch(const uint8_t *const *bits, const uint16_t *const *scales, const uint16_t *x,
                                        float *const *y, int R, int M, int N, int K, cudaStream_t st)
 {
-    if (M < 1 || M > 4 || use_tc(K) || R < 1 || R > kQ1MaxGroup || !q1m1_shape_supported(R, N, K))
+    if (M < 1 || M > 4 || R < 1 || R > kQ1MaxGroup || !q1m1_shape_supported(R, N, K))
         return LOWBIT_ERR_UNSUPPORTED_SHAPE;
     const Q1Plan P = q1_plan(R, N, K, num_sms(), true, q1_mv(M));
     if (!P.lean) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
@@ -1209,17 +1196,23 @@ lowbit_status q1m1_gemv_x_group_launch(const uint8_t *const *bits, const uint16_
 
 bool q1m1_x_group_supported(int R, int M, int N, int K)
 {
-    return M >= 1 && M <= 4 && !use_tc(K) && R >= 1 && R <= kQ1MaxGroup && q1m1_shape_supported(R, N, K) &&
+    return M >= 1 && M <= 4 && R >= 1 && R <= kQ1MaxGroup && q1m1_shape_supported(R, N, K) &&
            q1_plan(R, N, K, num_sms(), true, q1_mv(M)).lean;
 }
 
 // One matrix straight from x, in one launch (the split kernel builds its
-// slice of the activation itself).  LOWBIT_ERR_UNSUPPORTED_SHAPE when the
-// shape takes the stream kernel, which needs a prepared activation.
+// slice of the activation itself).  q1m1_fused_supported: the shape takes it.
+bool q1m1_fused_supported(int N, int K)
+{
+    return q1m1_shape_supported(1, N, K) && !q1_plan(1, N, K, num_sms()).stream;
+}
+
+// LOWBIT_ERR_UNSUPPORTED_SHAPE when the shape takes the stream kernel, which
+// needs a prepared activation.
 lowbit_status q1m1_gemv_fused_launch(const uint8_t *bits, const uint16_t *scales, const uint16_t *x, float *y, int N,
                                      int K, cudaStream_t st)
 {
-    if (use_tc(K) || !q1m1_shape_supported(1, N, K)) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    if (!q1m1_shape_supported(1, N, K)) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
     const Q1Plan P = q1_plan(1, N, K, num_sms());
     if (P.stream) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
     return q1m1_launch(P, &bits, &scales, nullptr, x, &y, 1, N, K, st);

@@ -45,10 +45,8 @@ SYMBOLS = [
     ("lowbit_q1g128_group_workspace_bytes", SZ, [I32, I32, I32, I32]),
     ("lowbit_q1g128_gemv_group", I32, [P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
     ("lowbit_q1g128_gemv_noalloc", I32, [P, P, P, P, I32, I32, I32, P]),
-    ("lowbit_int4g64_workspace_bytes", SZ, [I32, I32, I32]),
-    ("lowbit_int4g64_gemm", I32, [P, P, P, P, I32, I32, I32, P, SZ, P]),
-    ("lowbit_int4g64_group_workspace_bytes", SZ, [I32, I32, I32, I32]),
-    ("lowbit_int4g64_gemm_group", I32, [P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
+    ("lowbit_int4g64_gemm", I32, [P, P, P, P, I32, I32, I32, P]),
+    ("lowbit_int4g64_gemm_group", I32, [P, P, P, P, I32, I32, I32, I32, P]),
     ("lowbit_q2_mlp_forward", I32, [P, P, I32, P, I32, P, P, P]),
     ("lowbit_rmsnorm_bf16", I32, [P, P, I32, I32, F32, P, P]),
     ("lowbit_q1g128_stack_workspace_bytes", SZ, [I32, I32, I32]),
@@ -219,23 +217,14 @@ def lowbit_q1g128_gemv_noalloc(w_bits, w_scales, x, y, stream=None):
 
 # -- INT4_G64 ---------------------------------------------------------------------
 
-def lowbit_int4g64_workspace_bytes(M: int, N: int, K: int) -> int:
-    return int(lib().lowbit_int4g64_workspace_bytes(M, N, K))
-
-
-def lowbit_int4g64_gemm(w_q, w_scales, x, y, workspace=None, stream=None):
+def lowbit_int4g64_gemm(w_q, w_scales, x, y, stream=None):
     M, K = x.shape
     N = w_q.shape[0]
-    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().lowbit_int4g64_gemm(_ptr(w_q), _ptr(w_scales), _ptr(x), _ptr(y), M, N, K,
-                                     _ptr(workspace), wsb, _stream(stream)), "lowbit_int4g64_gemm")
+    _check(lib().lowbit_int4g64_gemm(_ptr(w_q), _ptr(w_scales), _ptr(x), _ptr(y), M, N, K, _stream(stream)),
+           "lowbit_int4g64_gemm")
 
 
-def lowbit_int4g64_group_workspace_bytes(R: int, M: int, N: int, K: int) -> int:
-    return lib().lowbit_int4g64_group_workspace_bytes(R, M, N, K)
-
-
-def lowbit_int4g64_gemm_group(w_q, w_scales, x, ys, workspace=None, stream=None):
+def lowbit_int4g64_gemm_group(w_q, w_scales, x, ys, stream=None):
     """y_r = W_r x for equal-length lists of INT4_G64 weights (uint8 [N][K/2],
     fp16 bits [N][K/64]) and fp32 outputs [M][N]; x [M][K] bf16 bits."""
     R = len(w_q)
@@ -244,8 +233,7 @@ def lowbit_int4g64_gemm_group(w_q, w_scales, x, ys, workspace=None, stream=None)
     pq, kq = _ptr_array(w_q)
     ps, ks = _ptr_array(w_scales)
     py, ky = _ptr_array(ys)
-    _check(lib().lowbit_int4g64_gemm_group(pq, ps, _ptr(x), py, R, M, N, K, _ptr(workspace), _nbytes(workspace),
-                                           _stream(stream)),
+    _check(lib().lowbit_int4g64_gemm_group(pq, ps, _ptr(x), py, R, M, N, K, _stream(stream)),
            "lowbit_int4g64_gemm_group")
 
 

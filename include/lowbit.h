@@ -35,9 +35,12 @@
  *     and keeps no state across calls besides the fault flags
  *     (lowbit_fault_flags) and the scratch array of the allocation-free
  *     entry point; entry points are safe to call from several host threads
- *     on different streams.  Kernels whose work needs scratch memory take a
- *     caller-provided workspace, sized by the matching *_workspace_bytes()
- *     query.
+ *     on different streams.  Only the Q1_0_g128 entry points take a
+ *     caller-provided workspace, for the shapes whose kernel reads a
+ *     prepared activation from global memory; its size comes from the
+ *     matching *_workspace_bytes() query, which returns 0 for every shape a
+ *     one-launch kernel takes (the activation is then built in shared
+ *     memory).
  *
  * Packed layouts (one row of a matrix is packed along K):
  *   Q1_0_g128  bits   [N][K/8]:   weight k is bit (k%8) of byte k/8; bit 1
@@ -83,10 +86,11 @@ int lowbit_version(void);
 
 /* Faults the kernels of the current device recorded since the last call,
  * and clears them: 0 = none; bit 0 = a bounded wait inside the INT4_G64
- * tcgen05 GEMM ran out, bit 1 = one inside the Q1_0_g128 tcgen05 product,
- * bit 2 = a grid barrier of lowbit_q1g128_stack_step (the results of that
- * call are then not valid); -1 = the flags could not be read.  Synchronises
- * with the device. */
+ * tcgen05 GEMM ran out, bit 2 = a grid barrier of lowbit_q1g128_stack_step
+ * (the results of that call are then not valid); -1 = the flags could not
+ * be read.  This is a diagnostic call, not part of any product: it reads the
+ * flags from device memory and therefore synchronises with the device (every
+ * other entry point is asynchronous). */
 int lowbit_fault_flags(void);
 
 /* ---------------------------------------------------------------------------
@@ -139,9 +143,13 @@ lowbit_status lowbit_unpack(lowbit_format fmt, const uint8_t *packed, int64_t ro
  * Activations must be finite; values below 2^-96 in magnitude count as 0 at
  * M = 1 (the tensor-core path works in per-group 24-bit fixed point).
  * workspace: device scratch of at least lowbit_q1g128_workspace_bytes(M, N,
- * K) bytes (may be NULL when that size is 0); it holds the prepared
- * activation and needs no initialisation.  Calls that share one workspace
- * must be ordered on one stream.
+ * K) bytes (may be NULL when that size is 0).  The size is 0 whenever the
+ * product is one launch (M >= 2, and at M = 1 every shape whose matrix is
+ * split across the GPU by K slices, e.g. 4096 x 4096); it is the prepared
+ * activation otherwise (M = 1 with so many rows -- above about 150k on 148
+ * SMs -- that the persistent kernel takes the product).  It needs no
+ * initialisation.  Calls that share one workspace must be ordered on one
+ * stream.
  * The weights are read before the kernel waits for the previous kernel on
  * the stream (programmatic dependent launch): a kernel that writes w_bits or
  * w_scales must not trigger its dependents early.  The library's packers
@@ -209,13 +217,17 @@ lowbit_status lowbit_q1g128_gemv_group(const uint8_t *const *w_bits,
  * embedded deployment that reserves all device memory up front, or code that
  * must not call cudaMalloc at the point where the product runs.
  *   Same arguments and result as lowbit_q1g128_gemv, without a workspace.
- *   The scratch the M = 1 path needs lives in a fixed 512 KiB array in the
- *   library's own device memory, present on every device that loads the
- *   library until the process exits; it limits K to 32768 at M = 1 (larger K
- *   returns LOWBIT_ERR_UNSUPPORTED_SHAPE).  The call allocates nothing.
- *   The first call on a device looks up that array's device address (with
- *   the device current) and caches it; make that first call before any
- *   stream capture.
+ *   Shapes that lowbit_q1g128_gemv runs in one launch need no scratch and
+ *   take that launch.  The others (M = 1 with very many rows) keep the
+ *   prepared activation in a fixed 512 KiB array in the library's own device
+ *   memory, present on every device that loads the library until the process
+ *   exits.  That array limits K to 32768 at M = 1: a larger K returns
+ *   LOWBIT_ERR_UNSUPPORTED_SHAPE for every N, before anything is enqueued.
+ *   The call allocates nothing.
+ *   The device address of the array is looked up (with the device current)
+ *   on a device's first call that needs it, and again whenever the device's
+ *   context has changed since (for example after cudaDeviceReset); make the
+ *   first call before any stream capture.
  *   All calls share the one array, so calls that overlap on the GPU (for
  *   example on two streams without ordering between them) race; order them
  *   on one stream.  Each call overwrites the part it reads, so the contents a
@@ -272,16 +284,12 @@ lowbit_status lowbit_q1g128_stack_step(const uint8_t *const *w_bits, const uint1
  * (K % 128 == 0) mma.sync on bf16 operands, q exact in bf16 and the group
  * scale applied once per group; above that a tcgen05 GEMM that dequantises
  * each weight tile into shared memory as two exact bf16 halves (hi + lo =
- * q*d) and accumulates in TMEM; other shapes a CUDA-core kernel.
- * workspace: at least lowbit_int4g64_workspace_bytes(M, N, K) bytes (NULL
- * allowed when that is 0, which it is for every shape today: each kernel
- * builds its operands in shared memory; the argument is kept so that a
- * kernel needing scratch can be added without changing the call).
+ * q*d) and accumulates in TMEM; other shapes a CUDA-core kernel.  Every
+ * kernel builds its operands in shared memory: no workspace.
  * ------------------------------------------------------------------------- */
-size_t lowbit_int4g64_workspace_bytes(int M, int N, int K);
 lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales,
                                   const uint16_t *x, float *y, int M, int N, int K,
-                                  void *workspace, size_t workspace_bytes, void *stream);
+                                  void *stream);
 
 /* Group form: y_r = W_r x for R matrices of one shape [N][K] that read one
  * activation x [M][K] (w_q, w_scales, y: HOST arrays of R device pointers,
@@ -292,14 +300,11 @@ lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales,
  * weights.  At 2 <= M <= 32 with K % 128 == 0 and at least SMs * 8 32-row
  * blocks over the group, one launch of the persistent small-batch kernel
  * (as for Q1_0_g128).  Other shapes run lowbit_int4g64_gemm once per matrix.  Results
- * equal the single calls up to fp32 summation order.
- * workspace: lowbit_int4g64_group_workspace_bytes(R, M, N, K) bytes (0
- * today; NULL allowed when 0). */
-size_t lowbit_int4g64_group_workspace_bytes(int R, int M, int N, int K);
+ * equal the single calls up to fp32 summation order. */
 lowbit_status lowbit_int4g64_gemm_group(const uint8_t *const *w_q,
                                         const uint16_t *const *w_scales, const uint16_t *x,
                                         float *const *y, int R, int M, int N, int K,
-                                        void *workspace, size_t workspace_bytes, void *stream);
+                                        void *stream);
 
 /* ---------------------------------------------------------------------------
  * Z80-style 2-bit integer MLP ("Show HN: Z80-uLM"), fused over all layers:

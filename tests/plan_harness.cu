@@ -20,22 +20,6 @@
 #include "int4_gemv_m1.cu"
 #include "gemm_smallm.cu"
 
-// The tcgen05 Q1 kernel is compiled out of the default build (the planner
-// above consults it only when it is switched on); stand-ins for its entry
-// points let the harness link without it.
-namespace lowbit {
-size_t q1tc_act_bytes(int) { return 0; }
-size_t q1tc_xcopy_off(int) { return 0; }
-bool q1tc_supported(int, int, int) { return false; }
-lowbit_status q1tc_prepare_launch(const uint16_t *, int, void *, cudaStream_t) { return LOWBIT_ERR_UNSUPPORTED_SHAPE; }
-lowbit_status q1tc_gemv_launch(const uint8_t *const *, const uint16_t *const *, const void *, float *const *, int, int,
-                               int, cudaStream_t)
-{
-    return LOWBIT_ERR_UNSUPPORTED_SHAPE;
-}
-int q1tc_fault_flag() { return 0; }
-}  // namespace lowbit
-
 using namespace lowbit;
 
 static int g_checked = 0, g_failed = 0;

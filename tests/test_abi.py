@@ -68,11 +68,23 @@ def test_q1_validation(L):
     assert g(FAKE, FAKE, FAKE, FAKE, 1, 0, 128, None, 0, None) == 1    # N < 1
     assert g(None, FAKE, FAKE, FAKE, 1, 16, 128, None, 0, None) == 1   # null
     assert g(FAKE, FAKE, MIS, FAKE, 1, 16, 128, None, 0, None) == 2    # misaligned x
-    need = L.lowbit_q1g128_workspace_bytes(1, 4096, 4096)
+    # one-launch shapes need no workspace; the persistent M = 1 kernel (very
+    # many rows, 148 SMs when no device is visible) reads a prepared activation
+    assert L.lowbit_q1g128_workspace_bytes(1, 4096, 4096) == 0
+    assert L.lowbit_q1g128_workspace_bytes(4, 4096, 4096) == 0
+    big = 2 * 148 * 2 * 8 * 32
+    need = L.lowbit_q1g128_workspace_bytes(1, big, 1024)
     assert need > 0
-    assert g(FAKE, FAKE, FAKE, FAKE, 1, 4096, 4096, FAKE, need - 1, None) == 1
-    assert g(FAKE, FAKE, FAKE, FAKE, 1, 4096, 4096, None, need, None) == 1
-    assert g(FAKE, FAKE, FAKE, FAKE, 1, 4096, 4096, MIS, need, None) == 2
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, big, 1024, FAKE, need - 1, None) == 1
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, big, 1024, None, need, None) == 1
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, big, 1024, MIS, need, None) == 2
+    # the allocation-free form: K beyond its fixed scratch is refused at M = 1
+    # for every N, before any dispatch
+    na = L.lowbit_q1g128_gemv_noalloc
+    for n in (16, 4096, big):
+        assert na(FAKE, FAKE, FAKE, FAKE, 1, n, 32768 + 128, None) == 3
+    assert na(FAKE, FAKE, FAKE, FAKE, 0, 16, 128, None) == 1
+    assert na(FAKE, FAKE, MIS, FAKE, 1, 16, 128, None) == 2
     assert L.lowbit_q1g128_workspace_bytes(1, 16, 100) == 0            # invalid shape -> 0
     assert L.lowbit_q1g128_act_bytes(1, 4096) > 0
     assert L.lowbit_q1g128_prepare_act(FAKE, 1, 100, FAKE, 1 << 20, None) == 3
@@ -91,10 +103,10 @@ def test_q1_validation(L):
 
 def test_int4_validation(L):
     g = L.lowbit_int4g64_gemm
-    assert g(FAKE, FAKE, FAKE, FAKE, 1, 16, 96, None, 0, None) == 3    # K % 64
-    assert g(FAKE, FAKE, FAKE, FAKE, 0, 16, 64, None, 0, None) == 1
-    assert g(FAKE, None, FAKE, FAKE, 1, 16, 64, None, 0, None) == 1
-    assert g(FAKE, FAKE, FAKE, MIS, 1, 16, 64, None, 0, None) == 2
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 16, 96, None) == 3    # K % 64
+    assert g(FAKE, FAKE, FAKE, FAKE, 0, 16, 64, None) == 1
+    assert g(FAKE, None, FAKE, FAKE, 1, 16, 64, None) == 1
+    assert g(FAKE, FAKE, FAKE, MIS, 1, 16, 64, None) == 2
 
 
 def test_q2_and_glue_validation(L):
@@ -153,8 +165,7 @@ def test_group_validation(L):
     assert L.lowbit_q1g128_group_workspace_bytes(40, 4, 4096, 1024) == 0
     assert L.lowbit_q1g128_group_workspace_bytes(40, 16, 4096, 1024) == 0
     i = L.lowbit_int4g64_gemm_group
-    assert i(pp, pp, FAKE, pp, 0, 1, 16, 128, None, 0, None) == 1       # R < 1
-    assert i(pp, pp, None, pp, 2, 1, 16, 128, None, 0, None) == 1       # null x
-    assert i(pp, pp, FAKE, misp, 2, 1, 16, 128, None, 0, None) == 2     # misaligned y[1]
-    assert i(pp, pp, FAKE, pp, 2, 1, 16, 96, None, 0, None) == 3        # K % 64
-    assert L.lowbit_int4g64_group_workspace_bytes(17, 1, 11008, 4096) == 0
+    assert i(pp, pp, FAKE, pp, 0, 1, 16, 128, None) == 1       # R < 1
+    assert i(pp, pp, None, pp, 2, 1, 16, 128, None) == 1       # null x
+    assert i(pp, pp, FAKE, misp, 2, 1, 16, 128, None) == 2     # misaligned y[1]
+    assert i(pp, pp, FAKE, pp, 2, 1, 16, 96, None) == 3        # K % 64

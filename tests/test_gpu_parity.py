@@ -342,9 +342,7 @@ def test_q1_layer_shapes_sampled(lb, shape, M):
 def _run_int4(lb, q, scales, x, N):
     M, K = x.shape
     y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
-    nws = lb.lowbit_int4g64_workspace_bytes(M, N, K)
-    ws = torch.zeros(nws, dtype=torch.uint8, device="cuda") if nws else None
-    lb.lowbit_int4g64_gemm(dev(q), dev(scales), dev(x), y, workspace=ws)
+    lb.lowbit_int4g64_gemm(dev(q), dev(scales), dev(x), y)
     _sync()
     return host(y)
 

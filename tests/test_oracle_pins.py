@@ -194,6 +194,57 @@ def test_int4_gemv_matches_numpy_matmul():
     np.testing.assert_allclose(ab, np.abs(xf) @ np.abs(W).T, rtol=1e-12)
 
 
+def _int4_numpy_weights(q, scales, K):
+    """Weights decoded with numpy alone: low nibble = even k, high = odd k,
+    sign-extended by arithmetic shifts; times the fp16 scale of k // 64."""
+    lo = (q.astype(np.int8) << 4) >> 4
+    hi = q.astype(np.int8) >> 4
+    codes = np.stack([lo, hi], axis=-1).reshape(q.shape[0], K).astype(np.float64)
+    return codes * np.repeat(scales.view(np.float16).astype(np.float64), 64, axis=1)
+
+
+def test_int4_gemv_at_matches_numpy_at_every_element():
+    """The sampled-output form checks the INT4 parity tests at full size: at
+    every (m, n) of a small product it must equal a numpy matmul of weights
+    decoded independently of the oracle (so a wrong row, batch or scale
+    index in it fails here)."""
+    M, N, K = 3, 13, 448
+    q = synth.rng(12, 0).integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    scales = synth.int4_scales(12, N, K)
+    x = synth.bf16_normal(12, (M, K))
+    W = _int4_numpy_weights(q, scales, K)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    ref = xf @ W.T
+    mm, nn = np.meshgrid(np.arange(M), np.arange(N), indexing="ij")
+    ys, ab = oracle.int4_gemv_at(q, scales, x, mm.ravel(), nn.ravel())
+    np.testing.assert_allclose(ys, ref.ravel(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ab, (np.abs(xf) @ np.abs(W).T).ravel(), rtol=1e-12)
+    # the same elements in the reverse order: no state carried between them
+    ys_rev, _ = oracle.int4_gemv_at(q, scales, x, mm.ravel()[::-1], nn.ravel()[::-1])
+    assert np.array_equal(ys_rev, ys[::-1])
+
+
+def test_int4_gemv_at_hand_computed_element():
+    """One output worked by hand: row 1 holds q = +3 at k = 0 (low nibble),
+    q = -2 at k = 65 (high nibble of byte 32, second group) and 0 elsewhere;
+    scales 0.5 and 0.25; x = 1.0 at k = 0 and 2.0 at k = 65, batch row 1.
+    y[1][1] = 3 * 0.5 * 1 + (-2) * 0.25 * 2 = 0.5."""
+    N, K = 2, 128
+    q = np.zeros((N, K // 2), np.uint8)
+    q[1, 0] = 0x03            # k = 0: +3
+    q[1, 32] = 0xE0           # k = 65: high nibble 0xE = -2
+    q[0, :] = 0x77            # row 0: +7 everywhere (must not leak into row 1)
+    scales = np.array([[0x3C00, 0x3C00], [0x3800, 0x3400]], np.uint16)   # 1, 1 | 0.5, 0.25
+    x = np.zeros((2, K), np.uint16)
+    x[1, 0] = 0x3F80          # 1.0
+    x[1, 65] = 0x4000         # 2.0
+    x[0, :] = 0x3F80          # batch row 0: all ones (must not leak into batch row 1)
+    ys, ab = oracle.int4_gemv_at(q, scales, x, np.array([1, 0, 1]), np.array([1, 0, 0]))
+    assert ys[0] == 0.5 and ab[0] == 2.5
+    assert ys[1] == 7 * 128                       # row 0, all-ones x: 7 per weight, scale 1
+    assert ys[2] == 7 * 1.0 + 7 * 2.0             # row 0 against batch row 1
+
+
 def test_int4_group_isolation_probe():
     # Only group g has a non-zero scale: y must equal d * sum over that group.
     N, K = 3, 256
