@@ -6,20 +6,25 @@ M=1 (fp16 scale per 128 weights, bf16 activations, fp32 output).  Metric:
 packed-weight bytes (sign bits + scales) streamed per second, and that rate
 as a fraction of the measured HBM bandwidth.
 
-One step = one activation vector x prepared once, then multiplied by R
-distinct 4096x4096 weight matrices (y_r = W_r x) in one grouped launch --
-the way the projections that read one hidden state are applied in a decode
-step.  The R weight sets total more than 3x the L2 cache, so every matrix
-streams from HBM (no L2 flush is needed).  The step is one CUDA graph
-replay on the launching stream; it is timed with CUDA events over exactly
---steps replays after --warmup untimed ones.
+A launch multiplies one activation vector x by R distinct 4096x4096 weight
+matrices (y_r = W_r x) in one grouped call -- the way the projections that
+read one hidden state are applied in a decode step.  The R weight sets total
+more than 3x the L2 cache, so every matrix streams from HBM (no L2 flush is
+needed).  One step is --launches-per-step such launches (one CUDA graph
+replay each), so that the timed region of --steps steps lasts about a second
+and the sampled clocks cover it; exactly --steps steps are timed with CUDA
+events after --warmup untimed ones.  The other four workloads (layer-shape
+sweep, 64-layer stack, INT4_G64, 2-bit MLP) are measured after the headline
+and reported in the same line under "workloads" (--headline-only skips them).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload q1_4096|q1_sweep|q1_stack|int4|q2_mlp]
 
-With N > 1 (under torchrun) every rank runs the same workload on its own GPU
-with its own weights (independent problems, no collective on the data path);
-the time is the max over ranks and the value the sum of all ranks' bytes.
+With N > 1 (under torchrun) every weight matrix is split by rows across the
+ranks (each rank holds N/G rows of each of R*G matrices, so the bytes per GPU
+stay those of R matrices: weak scaling), x is replicated, each rank computes
+its rows, and one NCCL all-gather per launch gives every rank all of y.  The
+time is the max over ranks and the value the sum of all ranks' bytes.
 `--impl reference` times the CPU oracle instead (rank 0 only).
 """
 from __future__ import annotations
@@ -40,6 +45,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "packed-weight GB/s streamed & % of B200 HBM peak (Q1_0_g128 GEMV, M=1)"
 FALLBACK_HBM_GBS = 6650.0
+KERNEL_DTYPE = "u8xs8->s32 (tensor core), f32 epilogue"
+DEFAULT_LAUNCHES_PER_STEP = 600
 
 
 def measured_peaks():
@@ -51,8 +58,35 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def measured_bf16_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured burst bf16_tflops (cuBLAS)"
+    return 1590.0, "fallback burst bf16"
+
+
 def q1_bytes(N, K):
     return N * K // 8 + 2 * N * (K // 128)
+
+
+def int4_bytes(N, K):
+    return N * K // 2 + 2 * N * (K // 64)
+
+
+def q1_4096_sets(l2_bytes):
+    """Weight sets of the headline launch: at least 3x L2 of distinct bytes."""
+    return max(8, -(-3 * l2_bytes // q1_bytes(4096, 4096)))
+
+
+def rotation(per_bytes, l2_bytes):
+    """Distinct weight sets that total at least 3x L2."""
+    return max(4, -(-3 * l2_bytes // per_bytes))
+
+
+def sweep_sets(N, K, l2_bytes):
+    return min(256, rotation(q1_bytes(N, K), l2_bytes))
 
 
 # ---------------------------------------------------------------------------
@@ -67,12 +101,13 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.lines = []
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
@@ -82,7 +117,7 @@ class ClockSampler:
     def __exit__(self, *exc):
         self.lines = []
         if self.proc is not None:
-            time.sleep(0.25)
+            time.sleep(0.15)
             self.proc.terminate()
             try:
                 out, _ = self.proc.communicate(timeout=5)
@@ -108,10 +143,10 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(name)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        loaded = [s for s in sm if smax and s > 0.5 * smax] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "samples_under_load": 0}
+        loaded = [s for s in sm if smax and s > 0.5 * smax]
+        return {"sm_mhz": statistics.median(loaded or sm), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded)}
 
 
 # ---------------------------------------------------------------------------
@@ -155,32 +190,82 @@ def max_over_ranks(v, world):
 
 
 # ---------------------------------------------------------------------------
-# CPU baseline: the oracle as it stands, single-threaded, bounded sample
+# CPU baseline: the oracle as it stands, single-threaded, on one pinned core
 # ---------------------------------------------------------------------------
 
-def oracle_q1_rate(seconds=10.0, rows=1024, max_reps=1000):
-    """Time the oracle's Q1 GEMV on row samples of the 4096x4096 workload
-    until `seconds` have passed.  Returns (GB/s of packed weights, sample)."""
-    import oracle
-    import synth
-    seed = synth.SEED_BASE + synth.W_Q1_4096
-    N, K = 4096, 4096
-    bits = synth.q1_packed_random(seed, N, K, tag=7)
-    scales = synth.q1_scales(seed, N, K, tag=7)
-    x = synth.bf16_normal(seed, (1, K))
-    oracle.q1_gemv(bits[:8], scales[:8], x)           # build + warm
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+class PinnedCore:
+    """Run the enclosed host code on one core (the lowest this process may
+    use), restoring the previous affinity afterwards."""
+
+    def __enter__(self):
+        self.prev = None
+        self.core = None
+        if hasattr(os, "sched_getaffinity"):
+            try:
+                self.prev = os.sched_getaffinity(0)
+                self.core = min(self.prev)
+                os.sched_setaffinity(0, {self.core})
+            except OSError:
+                self.prev = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            os.sched_setaffinity(0, self.prev)
+        return False
+
+
+def cpu_info(pin):
+    n = os.cpu_count() or 1
+    return {"cores": 1, "nproc": n, "cpu_model": cpu_model(),
+            "pinned_core": pin.core, "note": f"1 of {n} cores used"}
+
+
+def _timed_loop(fn, seconds, max_reps):
+    fn(0)  # build + warm
     t0 = time.perf_counter()
-    reps, done = 0, 0
+    reps = 0
     while reps < max_reps:
-        r0 = (reps * rows) % N
-        oracle.q1_gemv(bits[r0:r0 + rows], scales[r0:r0 + rows], x)
+        fn(reps)
         reps += 1
-        done += q1_bytes(rows, K)
         if time.perf_counter() - t0 >= seconds:
             break
-    dt = time.perf_counter() - t0
-    sample = f"{reps} oracle GEMVs of {rows} rows x {K} of the 4096x4096 M=1 workload ({dt:.1f} s)"
-    return done / dt / 1e9, sample
+    return reps, time.perf_counter() - t0
+
+
+def oracle_q1_rate(seconds=10.0, rows=1024, max_reps=1000, N=4096, K=4096, seed_index=None, tag=7):
+    """The oracle's Q1 GEMV on row samples of an N x K M=1 workload until
+    `seconds` have passed, on one pinned core.  Returns (cpu_baseline dict
+    with value in GB/s of packed weights)."""
+    import oracle
+    import synth
+    seed = synth.SEED_BASE + (synth.W_Q1_4096 if seed_index is None else seed_index)
+    bits = synth.q1_packed_random(seed, N, K, tag=tag)
+    scales = synth.q1_scales(seed, N, K, tag=tag)
+    x = synth.bf16_normal(seed, (1, K))
+    rows = min(rows, N)
+
+    def one(i):
+        r0 = (i * rows) % (N - rows + 1)
+        oracle.q1_gemv(bits[r0:r0 + rows], scales[r0:r0 + rows], x)
+
+    with PinnedCore() as pin:
+        reps, dt = _timed_loop(one, seconds, max_reps)
+    v = reps * q1_bytes(rows, K) / dt / 1e9
+    return dict(value=round(v, 5), unit="GB/s", kind="oracle",
+                sample=f"{reps} oracle GEMVs of {rows} rows x {K} of the {N}x{K} M=1 workload ({dt:.1f} s)",
+                **cpu_info(pin))
 
 
 def run_reference(args, world, rank):
@@ -200,12 +285,13 @@ def run_reference(args, world, rank):
         r0 = (i * rows) % N
         oracle.q1_gemv(bits[r0:r0 + rows], scales[r0:r0 + rows], x)
 
-    for i in range(args.warmup):
-        step(i)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        step(args.warmup + i)
-    dt = time.perf_counter() - t0
+    with PinnedCore() as pin:
+        for i in range(args.warmup):
+            step(i)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            step(args.warmup + i)
+        dt = time.perf_counter() - t0
     per_step = q1_bytes(rows, K)
     value = per_step * args.steps / dt / 1e9
     sample = f"each step: oracle GEMV over {rows} of the 4096 rows (K=4096, M=1), single thread"
@@ -216,8 +302,7 @@ def run_reference(args, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "Q1_0_g128 GEMV 4096x4096, M=1", "N": 4096, "K": 4096, "M": 1,
                    "rows_per_step": rows},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": dict(value=round(value, 4), unit="GB/s", kind="oracle", sample=sample, **cpu_info(pin)),
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -226,149 +311,26 @@ def run_reference(args, world, rank):
 
 
 # ---------------------------------------------------------------------------
-# the GPU arm: Q1 4096x4096 M=1
+# timing helpers
 # ---------------------------------------------------------------------------
 
-def run_q1_4096(args, world, rank, local):
+def _capture(step, stream):
     import torch
-    import synth
-    from decode_packed_bit_b200 import build as lb_build
-    lb_build.build()
-    from decode_packed_bit_b200 import lowbit as lb
-
-    N = K = 4096
-    M = 1
-    dev = torch.device("cuda", local)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    per = q1_bytes(N, K)
-    R = max(8, -(-3 * l2 // per))                      # >= 3x L2 of distinct weights
-    seed = synth.SEED_BASE + synth.W_Q1_4096 + 1000 * rank
-    bits, scales = [], []
-    for r in range(R):
-        b, s = synth.torch_q1_layer(seed, N, K, r, dev)
-        bits.append(b)
-        scales.append(s)
-    x = torch.from_numpy(synth.bf16_normal(seed, (M, K)).view(np.int16)).to(dev)
-    y = torch.empty((R, M, N), dtype=torch.float32, device=dev)
-    need = lb.lowbit_q1g128_group_workspace_bytes(R, M, N, K)
-    ws = torch.zeros(need, dtype=torch.uint8, device=dev) if need else None
-    stream = torch.cuda.Stream(device=dev)
-
-    ys = [y[r] for r in range(R)]
-
-    def step():
-        lb.lowbit_q1g128_gemv_group(bits, scales, x, ys, workspace=ws, stream=stream)
-
-    launches_per_step = 1 if need == 0 else 2  # one launch from x, else prepare + product
-    # eager warm-up (also loads the module), then capture one step in a graph
     with torch.cuda.stream(stream):
         step()
     stream.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         step()
-    for _ in range(args.warmup):
-        graph.replay()
-    stream.synchronize()
+    return graph
 
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(args.steps):
-                graph.replay()
-            e1.record(stream)
-        e1.synchronize()
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    ms = e0.elapsed_time(e1)
-    ms_max = max_over_ranks(ms, world)
-
-    bytes_step = R * per
-    value = bytes_step * args.steps * world / (ms_max * 1e-3) / 1e9
-    peak, peak_kind = measured_peaks()
-    achieved = bytes_step * args.steps / (ms * 1e-3) / 1e9   # this rank's stream rate
-
-    # end to end through the C ABI with host buffers: x in from pinned host
-    # memory, all R outputs back to pinned host memory, inside the timed region
-    x_host = x.cpu().pin_memory()
-    y_host = torch.empty((R, M, N), dtype=torch.float32).pin_memory()
-    for _ in range(2):
-        with torch.cuda.stream(stream):
-            x.copy_(x_host, non_blocking=True)
-            graph.replay()
-            y_host.copy_(y, non_blocking=True)
-        stream.synchronize()
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(1, min(args.steps, 50))
-    with torch.cuda.stream(stream):
-        t0.record(stream)
-        for _ in range(e2e_steps):
-            x.copy_(x_host, non_blocking=True)
-            graph.replay()
-            y_host.copy_(y, non_blocking=True)
-        t1.record(stream)
-    t1.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world)
-    e2e_value = bytes_step * e2e_steps * world / (e2e_ms * 1e-3) / 1e9
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, sample = oracle_q1_rate(seconds=args.cpu_seconds)
-        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample}
-
-    traffic = load_traffic("q1_gemv")
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": KERNEL_DTYPE, "data": "synthetic",
-        "config": {"workload": "Q1_0_g128 GEMV 4096x4096, M=1", "N": N, "K": K, "M": M,
-                   "weight_sets_per_step": R, "bytes_per_gemv": per,
-                   "l2": f"inputs larger than L2: {R} distinct weight sets, {R * per / 2**20:.0f} MiB "
-                         f"per step vs {l2 / 2**20:.0f} MiB L2",
-                   "step": ("1 grouped launch of R GEMVs from x" if launches_per_step == 1 else
-                            "1 activation prepare + 1 grouped launch of R GEMVs") + ", one CUDA graph",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)"},
-        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
-                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
-        "cpu_baseline": cpu,
-    }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    del graph
-    return 0
-
-
-# ---------------------------------------------------------------------------
-# the other workloads (one JSON line each, with their own metric)
-# ---------------------------------------------------------------------------
 
 def _graph_time(step, stream, steps, warmup, min_ms=20.0):
     """Capture step() in a CUDA graph on `stream`; return ms per replay.
     At least `steps` replays are timed, and more when those take under
     min_ms, so that the launch of the first replay is a small part of it."""
     import torch
-    with torch.cuda.stream(stream):
-        step()
-    stream.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        step()
+    graph = _capture(step, stream)
     for _ in range(warmup):
         graph.replay()
     stream.synchronize()
@@ -392,109 +354,286 @@ def _graph_time(step, stream, steps, warmup, min_ms=20.0):
     return total / n
 
 
+def load_traffic(kernel):
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel code (comments and layout do not count), else null."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        from decode_packed_bit_b200 import build as lb_build
+        ent = d.get(kernel)
+        if ent and ent.get("kernel_sha1") == lb_build.kernel_digest():
+            return ent.get("dram_bytes_per_launch")
+    except Exception:
+        return None
+    return None
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm: Q1 4096x4096 M=1
+# ---------------------------------------------------------------------------
+
+def run_q1_4096(args, world, rank, local):
+    import torch
+    import synth
+    from decode_packed_bit_b200 import build as lb_build
+    lb_build.build()
+    from decode_packed_bit_b200 import lowbit as lb
+    from decode_packed_bit_b200.shard import RowShardedGroup, row_shard
+
+    N = K = 4096
+    M = 1
+    dev = torch.device("cuda", local)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per = q1_bytes(N, K)
+    R = q1_4096_sets(l2)
+    L = max(1, args.launches_per_step)
+    seed = synth.SEED_BASE + synth.W_Q1_4096
+    x = torch.from_numpy(synth.bf16_normal(seed, (M, K)).view(np.int16)).to(dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    if world == 1:
+        bits, scales = [], []
+        for r in range(R):
+            b, s = synth.torch_q1_layer(seed, N, K, r, dev)
+            bits.append(b)
+            scales.append(s)
+        y = torch.empty((R, M, N), dtype=torch.float32, device=dev)
+        ys = [y[r] for r in range(R)]
+        need = lb.lowbit_q1g128_group_workspace_bytes(R, M, N, K)
+        ws = torch.zeros(need, dtype=torch.uint8, device=dev) if need else None
+
+        def launch():
+            lb.lowbit_q1g128_gemv_group(bits, scales, x, ys, workspace=ws, stream=stream)
+        calls_per_launch = 1 if need == 0 else 2   # one launch from x, else prepare + product
+        bytes_launch = R * per
+        gather = None
+        out_host_shape = (R, M, N)
+        out_dev = y
+    else:
+        # row-sharded: R*world matrices, rows [n0, n1) of each on this rank
+        n0, n1 = row_shard(N, world, rank)
+        Rt = R * world
+        bits, scales = [], []
+        for r in range(Rt):
+            b, s = synth.torch_q1_layer(seed + 7919 * rank, n1 - n0, K, r, dev)
+            bits.append(b)
+            scales.append(s)
+        grp = RowShardedGroup("q1", bits, scales, N, K, M, device=dev, stream=stream)
+
+        def launch():
+            grp.compute(x)
+        calls_per_launch = 1 if grp.workspace is None else 2
+        bytes_launch = Rt * q1_bytes(n1 - n0, K)
+        gather = grp.gather
+        out_host_shape = (grp.gathered.numel(),)
+        out_dev = grp.gathered
+
+    # one launch per graph replay; a step is L replays (plus, with several
+    # ranks, the all-gather of each launch's outputs)
+    graph = _capture(launch, stream)
+
+    def run_steps(n):
+        with torch.cuda.stream(stream):
+            for _ in range(n):
+                for _ in range(L):
+                    graph.replay()
+                    if gather is not None:
+                        gather()
+
+    run_steps(args.warmup)
+    stream.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+        run_steps(args.steps)
+        with torch.cuda.stream(stream):
+            e1.record(stream)
+        e1.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms, world)
+    launches = L * args.steps
+
+    bytes_step = bytes_launch * L
+    value = bytes_step * args.steps * world / (ms_max * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    achieved = bytes_launch * launches / (ms * 1e-3) / 1e9   # this rank's stream rate per launch
+
+    # end to end through the C ABI with host buffers: per call, x in from
+    # pinned host memory and all outputs back to pinned host memory, inside
+    # the timed region
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(out_host_shape, dtype=torch.float32).pin_memory()
+
+    def e2e_call():
+        x.copy_(x_host, non_blocking=True)
+        graph.replay()
+        if gather is not None:
+            gather()
+        y_host.copy_(out_dev.view(out_host_shape), non_blocking=True)
+
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            e2e_call()
+        stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    e2e_calls = 200
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(e2e_calls):
+            e2e_call()
+        t1.record(stream)
+    t1.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    e2e_value = bytes_launch * e2e_calls * world / (e2e_ms * 1e-3) / 1e9
+
+    # the single-matrix call (lowbit_q1g128_gemv), R separate calls in one graph
+    single = None
+    if world == 1:
+        yone = torch.empty((M, N), dtype=torch.float32, device=dev)
+        nws1 = lb.lowbit_q1g128_workspace_bytes(M, N, K)
+        ws1 = torch.zeros(nws1, dtype=torch.uint8, device=dev) if nws1 else None
+
+        def singles():
+            for r in range(R):
+                lb.lowbit_q1g128_gemv(bits[r], scales[r], x, yone, workspace=ws1, stream=stream)
+        sms = _graph_time(singles, stream, 20, 3)
+        single = {"call": "lowbit_q1g128_gemv, one 4096x4096 matrix per call", "calls_per_replay": R,
+                  "us_per_call": round(sms * 1e3 / R, 3), "gbs": round(R * per / (sms * 1e-3) / 1e9, 1),
+                  "frac_of_peak": round(R * per / (sms * 1e-3) / 1e9 / peak, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_q1_rate(seconds=args.cpu_seconds)
+
+    traffic = load_traffic("q1_gemv")
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": KERNEL_DTYPE, "data": "synthetic",
+        "config": {"workload": "Q1_0_g128 GEMV 4096x4096, M=1", "N": N, "K": K, "M": M,
+                   "weight_sets_per_launch": R * world, "bytes_per_gemv": per,
+                   "launches_per_step": L,
+                   "l2": f"inputs larger than L2: {R} distinct weight sets per GPU, "
+                         f"{bytes_launch / 2**20:.0f} MiB per launch vs {l2 / 2**20:.0f} MiB L2",
+                   "step": f"{L} grouped launches of R GEMVs from x (one CUDA graph replay each)"
+                           + (", each followed by an NCCL all-gather of y" if world > 1 else ""),
+                   "parallelism": (f"row-shard x{world}: each GPU holds N/{world} rows of every matrix, "
+                                   "all-gather of y") if world > 1 else "single GPU"},
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_bytes_per_launch": bytes_launch,
+                     "us_per_launch": round(ms * 1e3 / launches, 3),
+                     "kernel": "k_q1_m1_lean<1>",
+                     "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)"},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
+                "note": "one grouped call per step: x in from pinned host, all outputs out"},
+        "single_call": single,
+        "gpu_launches": calls_per_launch * launches,
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    del graph
+    if world == 1 and not args.headline_only and args.workload == "q1_4096":
+        del bits, scales
+        torch.cuda.empty_cache()
+        line["workloads"] = run_other_workloads(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the other workloads
+# ---------------------------------------------------------------------------
+
 def _emit(rank, line):
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
-def run_q1_stack(args, world, rank, local):
-    """64-layer Q1_0_g128 projection stack, one decode step per replay."""
-    import torch
-    import synth
-    from decode_packed_bit_b200 import build as lb_build
-    lb_build.build()
-    from decode_packed_bit_b200.stack import Q1Layer, Q1Stack
-    dev = torch.device("cuda", local)
-    seed = synth.SEED_BASE + synth.W_Q1_STACK + 1000 * rank
-    layers = [Q1Layer({name: synth.torch_q1_layer(seed, n, k, li * 16 + pi, dev)
-                       for pi, (name, n, k) in enumerate(synth.STACK_PROJ)})
-              for li in range(synth.STACK_LAYERS)]
-    M = args.m
-    st = Q1Stack(layers, synth.STACK_HIDDEN, synth.STACK_FFN, M, dev)
-    st.x.copy_(torch.from_numpy(synth.bf16_normal(seed, (M, synth.STACK_HIDDEN)).view(np.int16))
-               .view(torch.bfloat16).to(dev))
-    stream = torch.cuda.Stream(device=dev)
-    fused = st.fused_supported()  # M = 1: the whole step is one launch
-    with ClockSampler(local) as clk:
-        ms = _graph_time(lambda: (st.step_fused if fused else st.step)(stream=stream), stream, args.steps, args.warmup)
-    ms = max_over_ranks(ms, world)
-    gbs = st.bytes_per_step / (ms * 1e-3) / 1e9
-    _emit(rank, {"metric": f"decode tokens/s through the 64-layer Q1 stack (M={M})",
-                 "value": round(M * world * 1e3 / ms, 2), "unit": "tokens/s", "n_gpus": world,
-                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-                 "higher_is_better": True, "scaling": "weak", "dtype": KERNEL_DTYPE if M == 1 else "bf16xsign->f32",
-                 "data": "synthetic",
-                 "config": {"workload": "Q1_0_g128 64-layer stack, hidden 5120, ffn 17408", "M": M,
-                            "bytes_per_step": st.bytes_per_step, "l2": "inputs larger than L2 (3.35 GB)"},
-                 "weight_gbs": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / measured_peaks()[0], 2),
-                 "gpu_launches": (1 if fused else st.launches_per_step()) * args.steps,
-                 "step": "one cooperative launch (lowbit_q1g128_stack_step)" if fused else "one launch per product "
-                         "and per normalisation", "clocks": clk.summary()})
-    return 0
-
-
-def _rotation(per_bytes, l2):
-    return max(4, -(-3 * l2 // per_bytes))
-
-
-def run_q1_sweep(args, world, rank, local):
-    """Q1_0_g128 at the three layer shapes and M in {1, 4, 16}."""
-    import torch
-    import synth
+def _lib():
     from decode_packed_bit_b200 import build as lb_build
     lb_build.build()
     from decode_packed_bit_b200 import lowbit as lb
+    return lb
+
+
+def sweep_results(args, world, rank, local, cpu=True):
+    """Q1_0_g128 at the three layer shapes and M in {1, 4, 16}, grouped."""
+    import torch
+    import synth
+    lb = _lib()
     dev = torch.device("cuda", local)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    peak = measured_peaks()[0]
     seed = synth.SEED_BASE + synth.W_Q1_SWEEP + 1000 * rank
     results = []
     for (N, K) in synth.Q1_SWEEP_SHAPES:
         per = q1_bytes(N, K)
-        R = min(256, _rotation(per, l2))
+        R = sweep_sets(N, K, l2)
         mats = [synth.torch_q1_layer(seed, N, K, r, dev) for r in range(R)]
         for M in (1, 4, 16):
             x = torch.from_numpy(synth.bf16_normal(seed, (M, K), tag=M).view(np.int16)).to(dev)
             ys = [torch.empty((M, N), dtype=torch.float32, device=dev) for _ in range(R)]
             stream = torch.cuda.Stream(device=dev)
-            if M == 1:
-                need = lb.lowbit_q1g128_group_workspace_bytes(R, 1, N, K)
-                ws = torch.zeros(need, dtype=torch.uint8, device=dev) if need else None
+            need = lb.lowbit_q1g128_group_workspace_bytes(R, M, N, K)
+            ws = torch.zeros(need, dtype=torch.uint8, device=dev) if need else None
 
-                def step():
-                    lb.lowbit_q1g128_gemv_group([b for b, _ in mats], [s for _, s in mats], x, ys, workspace=ws,
-                                                stream=stream)
-            else:
-                need = lb.lowbit_q1g128_group_workspace_bytes(R, M, N, K)
-                ws = torch.zeros(need, dtype=torch.uint8, device=dev) if need else None
-
-                def step():
-                    lb.lowbit_q1g128_gemv_group([b for b, _ in mats], [s for _, s in mats], x, ys, workspace=ws,
-                                                stream=stream)
+            def step():
+                lb.lowbit_q1g128_gemv_group([b for b, _ in mats], [s for _, s in mats], x, ys, workspace=ws,
+                                            stream=stream)
             ms = max_over_ranks(_graph_time(step, stream, max(20, args.steps), args.warmup), world)
-            results.append({"N": N, "K": K, "M": M, "weight_sets": R,
-                            "gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
-                            "us_per_gemv": round(ms * 1e3 / R, 3)})
+            gbs = R * per / (ms * 1e-3) / 1e9
+            results.append({"N": N, "K": K, "M": M, "weight_sets": R, "gbs": round(gbs, 1),
+                            "frac_of_peak": round(gbs / peak, 4), "us_per_gemv": round(ms * 1e3 / R, 3)})
         del mats
-    _emit(rank, {"metric": "packed-weight GB/s, Q1_0_g128 layer-shape sweep", "unit": "GB/s",
-                 "value": results[0]["gbs"], "n_gpus": world, "higher_is_better": True, "data": "synthetic",
-                 "config": {"workload": "Q1_0_g128 (5120,5120),(17408,5120),(5120,17408) x M in {1,4,16}",
-                            "l2": "inputs larger than L2 (rotating weight sets)"},
-                 "results": results})
-    return 0
+        torch.cuda.empty_cache()
+    out = {"metric": "packed-weight GB/s, Q1_0_g128 layer-shape sweep (grouped launches)", "unit": "GB/s",
+           "config": {"workload": "Q1_0_g128 (5120,5120),(17408,5120),(5120,17408) x M in {1,4,16}",
+                      "l2": "inputs larger than L2 (rotating weight sets)"},
+           "results": results}
+    if cpu and rank == 0 and not args.no_cpu_baseline:
+        base = []
+        for (N, K) in synth.Q1_SWEEP_SHAPES:
+            b = oracle_q1_rate(seconds=args.cpu_seconds / 3, rows=256, N=N, K=K,
+                               seed_index=synth.W_Q1_SWEEP, tag=N + K)
+            base.append({"N": N, "K": K, "M": 1, "gbs": b["value"], "sample": b["sample"]})
+        out["cpu_baseline"] = {"kind": "oracle", "unit": "GB/s", "per_shape": base,
+                               **{k: v for k, v in b.items() if k in ("cores", "nproc", "cpu_model",
+                                                                      "pinned_core", "note")}}
+    return out
 
 
-def run_int4(args, world, rank, local):
+def int4_results(args, world, rank, local, cpu=True):
     """INT4_G64 11008 x 4096 at M in {1, 32, 256}."""
     import torch
     import synth
-    from decode_packed_bit_b200 import build as lb_build
-    lb_build.build()
-    from decode_packed_bit_b200 import lowbit as lb
+    lb = _lib()
     dev = torch.device("cuda", local)
     N, K = synth.INT4_N, synth.INT4_K
-    per = N * K // 2 + 2 * N * (K // 64)
+    per = int4_bytes(N, K)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    R = _rotation(per, l2)
+    peak = measured_peaks()[0]
+    tpeak, tkind = measured_bf16_peak()
+    R = rotation(per, l2)
     g = torch.Generator(device=dev)
     g.manual_seed(synth.SEED_BASE + synth.W_INT4 + 1000 * rank)
     qs = [torch.randint(0, 256, (N, K // 2), generator=g, device=dev, dtype=torch.uint8) for _ in range(R)]
@@ -509,11 +648,12 @@ def run_int4(args, world, rank, local):
             for r in range(R):
                 lb.lowbit_int4g64_gemm(qs[r], ss[r], x, y[r], stream=stream)
         ms = max_over_ranks(_graph_time(step, stream, max(20, args.steps), args.warmup), world)
+        tf = 2.0 * M * N * K * R / (ms * 1e-3) / 1e12
         res = {"M": M, "us_per_call": round(ms * 1e3 / R, 3),
                "weight_gbs": round(R * per / (ms * 1e-3) / 1e9, 1),
-               "tflops": round(2.0 * M * N * K * R / (ms * 1e-3) / 1e12, 2)}
+               "frac_of_hbm_peak": round(R * per / (ms * 1e-3) / 1e9 / peak, 4),
+               "tflops": round(tf, 2), "frac_of_bf16_peak": round(tf / tpeak, 4)}
         if M <= 32:
-            # the R weight sets read one x: one grouped launch
             ys = [y[r] for r in range(R)]
 
             def gstep():
@@ -521,24 +661,42 @@ def run_int4(args, world, rank, local):
             gms = max_over_ranks(_graph_time(gstep, stream, max(20, args.steps), args.warmup), world)
             res["group_us"] = round(gms * 1e3, 3)
             res["group_weight_gbs"] = round(R * per / (gms * 1e-3) / 1e9, 1)
+            res["group_frac_of_hbm_peak"] = round(R * per / (gms * 1e-3) / 1e9 / peak, 4)
         results.append(res)
     assert lb.lowbit_fault_flags() == 0
-    _emit(rank, {"metric": "INT4_G64 11008x4096: packed-weight GB/s (M=1) and TFLOP/s (M=32, 256)",
-                 "unit": "GB/s", "value": results[0]["weight_gbs"], "n_gpus": world, "higher_is_better": True,
-                 "data": "synthetic",
-                 "config": {"workload": "INT4_G64 N=11008 K=4096 M in {1,32,256}", "weight_sets": R,
-                            "l2": "inputs larger than L2 (rotating weight sets)"},
-                 "results": results})
-    return 0
+    out = {"metric": "INT4_G64 11008x4096: packed-weight GB/s (M=1, 32) and TFLOP/s (M=256)",
+           "unit": "GB/s",
+           "config": {"workload": "INT4_G64 N=11008 K=4096 M in {1,32,256}", "weight_sets": R,
+                      "l2": "inputs larger than L2 (rotating weight sets)", "tensor_peak_source": tkind},
+           "results": results}
+    if cpu and rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        q = synth.rng(synth.SEED_BASE + synth.W_INT4, 0).integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+        s = synth.int4_scales(synth.SEED_BASE + synth.W_INT4, N, K)
+        rows = 128
+        base = []
+        for M in (1, 32, 256):
+            xm = synth.bf16_normal(synth.SEED_BASE + synth.W_INT4, (M, K), tag=M)
+
+            def one(i):
+                r0 = (i * rows) % (N - rows)
+                oracle.int4_gemv(q[r0:r0 + rows], s[r0:r0 + rows], xm)
+            with PinnedCore() as pin:
+                reps, dt = _timed_loop(one, args.cpu_seconds / 3, 100000)
+            base.append({"M": M, "weight_gbs": round(reps * int4_bytes(rows, K) / dt / 1e9, 6),
+                         "gflops": round(reps * 2.0 * M * rows * K / dt / 1e9, 4),
+                         "sample": f"{reps} oracle products of {rows} rows x {K} at M={M} ({dt:.1f} s)"})
+        out["cpu_baseline"] = {"kind": "oracle", "per_m": base, **cpu_info(pin)}
+    del qs, ss
+    torch.cuda.empty_cache()
+    return out
 
 
-def run_q2_mlp(args, world, rank, local):
+def q2_results(args, world, rank, local, cpu=True):
     """The 2-bit integer MLP (256->192->128->40) over 1024 and 1M vectors."""
     import torch
     import synth
-    from decode_packed_bit_b200 import build as lb_build
-    lb_build.build()
-    from decode_packed_bit_b200 import lowbit as lb
+    lb = _lib()
     dev = torch.device("cuda", local)
     seed = synth.SEED_BASE + synth.W_Q2_MLP + 1000 * rank
     dims = synth.Q2_DIMS
@@ -560,46 +718,106 @@ def run_q2_mlp(args, world, rank, local):
                                         stream, args.steps, args.warmup), world)
         results.append({"batch": batch, "us": round(ms * 1e3, 3), "vectors_per_s": round(batch / (ms * 1e-3), 1),
                         "gmac_per_s": round(batch * macs / (ms * 1e-3) / 1e9, 2)})
-    _emit(rank, {"metric": "2-bit integer MLP vectors/s (256->192->128->40)", "unit": "vectors/s",
-                 "value": results[0]["vectors_per_s"], "n_gpus": world, "higher_is_better": True,
-                 "dtype": "int16 wrap / int32", "data": "synthetic",
-                 "config": {"workload": "Z80-style 2-bit MLP, 1024 and 1048576 vectors", "macs_per_vector": macs},
-                 "results": results})
-    return 0
+    out = {"metric": "2-bit integer MLP vectors/s (256->192->128->40)", "unit": "vectors/s",
+           "dtype": "int16 wrap / int32",
+           "config": {"workload": "Z80-style 2-bit MLP, 1024 and 1048576 vectors", "macs_per_vector": macs},
+           "results": results}
+    if cpu and rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        packed = [oracle.pack("q2", c) for c in synth.q2_codes(synth.SEED_BASE + synth.W_Q2_MLP, dims)]
+        xb = synth.q2_inputs(synth.SEED_BASE + synth.W_Q2_MLP, 1024)
+        with PinnedCore() as pin:
+            reps, dt = _timed_loop(lambda i: oracle.q2_mlp_forward(packed, dims, xb), args.cpu_seconds / 3, 1000)
+        vps = reps * 1024 / dt
+        out["cpu_baseline"] = {"kind": "oracle", "value": round(vps, 1), "unit": "vectors/s",
+                               "gmac_per_s": round(vps * macs / 1e9, 4),
+                               "sample": f"{reps} oracle passes over the 1024 vectors ({dt:.1f} s)", **cpu_info(pin)}
+    return out
 
 
-OTHER_WORKLOADS = {"q1_stack": run_q1_stack, "q1_sweep": run_q1_sweep, "int4": run_int4, "q2_mlp": run_q2_mlp}
+def stack_results(args, world, rank, local, Ms=(1, 8), cpu=True):
+    """64-layer Q1_0_g128 projection stack, one decode step per replay."""
+    import torch
+    import synth
+    _lib()
+    from decode_packed_bit_b200.stack import Q1Layer, Q1Stack
+    dev = torch.device("cuda", local)
+    seed = synth.SEED_BASE + synth.W_Q1_STACK + 1000 * rank
+    layers = [Q1Layer({name: synth.torch_q1_layer(seed, n, k, li * 16 + pi, dev)
+                       for pi, (name, n, k) in enumerate(synth.STACK_PROJ)})
+              for li in range(synth.STACK_LAYERS)]
+    peak = measured_peaks()[0]
+    results = []
+    for M in Ms:
+        st = Q1Stack(layers, synth.STACK_HIDDEN, synth.STACK_FFN, M, dev)
+        st.x.copy_(torch.from_numpy(synth.bf16_normal(seed, (M, synth.STACK_HIDDEN)).view(np.int16))
+                   .view(torch.bfloat16).to(dev))
+        stream = torch.cuda.Stream(device=dev)
+        fused = st.fused_supported()
+        ms = _graph_time(lambda: (st.step_fused if fused else st.step)(stream=stream), stream, max(5, args.steps),
+                         args.warmup)
+        ms = max_over_ranks(ms, world)
+        gbs = st.bytes_per_step / (ms * 1e-3) / 1e9
+        results.append({"M": M, "tokens_per_s": round(M * 1e3 / ms, 2), "ms_per_step": round(ms, 4),
+                        "weight_gbs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / peak, 4),
+                        "launches_per_step": 1 if fused else st.launches_per_step(),
+                        "step": "one launch (lowbit_q1g128_stack_step)" if fused else
+                                "one launch per product and per normalisation"})
+        del st
+    out = {"metric": "decode tokens/s through the 64-layer Q1 stack", "unit": "tokens/s",
+           "config": {"workload": "Q1_0_g128 64-layer stack, hidden 5120, ffn 17408",
+                      "bytes_per_step": 3350200320, "l2": "inputs larger than L2 (3.35 GB)"},
+           "results": results}
+    if cpu and rank == 0 and not args.no_cpu_baseline:
+        b = oracle_q1_rate(seconds=args.cpu_seconds / 3, rows=64, N=17408, K=5120,
+                           seed_index=synth.W_Q1_STACK, tag=3)
+        steps_per_s = b["value"] * 1e9 / 3350200320
+        out["cpu_baseline"] = dict(b, value=round(steps_per_s, 8), unit="tokens/s (M=1)",
+                                   weight_gbs=b["value"],
+                                   sample=b["sample"] + "; tokens/s = that weight rate / 3.35 GB per step "
+                                                        "(extrapolated, not a timed full step)")
+    del layers
+    torch.cuda.empty_cache()
+    return out
 
 
-KERNEL_DTYPE = "u8xs8->s32 (tensor core), f32 epilogue"
+def run_other_workloads(args, world, rank, local):
+    out = {}
+    for name, fn in (("q1_sweep", sweep_results), ("int4", int4_results), ("q2_mlp", q2_results),
+                     ("q1_stack", stack_results)):
+        try:
+            out[name] = fn(args, world, rank, local)
+        except Exception as e:  # a failing side workload must not hide the headline
+            out[name] = {"error": f"{type(e).__name__}: {e}"}
+    return out
 
 
-def load_traffic(kernel):
-    """dram bytes per launch from the committed ncu summary, if it matches
-    the current kernel sources (else null)."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
-        return None
-    try:
-        with open(p) as f:
-            d = json.load(f)
-        from decode_packed_bit_b200 import build as lb_build
-        ent = d.get(kernel)
-        if ent and ent.get("sources_sha1") == lb_build.digest():
-            return ent.get("dram_bytes_per_launch")
-    except Exception:
-        return None
-    return None
+def _single(fn, key):
+    def run(args, world, rank, local):
+        line = fn(args, world, rank, local)
+        line.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                     "data": "synthetic", "scaling": "weak"})
+        _emit(rank, line)
+        return 0
+    return run
+
+
+OTHER_WORKLOADS = {"q1_stack": _single(lambda a, w, r, l: stack_results(a, w, r, l, Ms=(a.m,)), "q1_stack"),
+                   "q1_sweep": _single(sweep_results, "q1_sweep"), "int4": _single(int4_results, "int4"),
+                   "q2_mlp": _single(q2_results, "q2_mlp")}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="q1_4096",
                     choices=["q1_4096", "q1_sweep", "q1_stack", "int4", "q2_mlp"])
+    ap.add_argument("--launches-per-step", type=int, default=DEFAULT_LAUNCHES_PER_STEP,
+                    help="grouped launches per headline step")
+    ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--m", type=int, default=1, help="batch rows for --workload q1_stack")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -11,6 +11,7 @@ import argparse
 import glob
 import hashlib
 import os
+import re
 import subprocess
 import sys
 from concurrent.futures import ThreadPoolExecutor
@@ -43,17 +44,46 @@ def digest() -> str:
     return h.hexdigest()
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    d = digest()
-    if not force and os.path.exists(LIB) and os.path.exists(STAMP):
-        with open(STAMP) as f:
+def _strip_c_comments(text: str) -> str:
+    """C/C++ source with comments removed and whitespace runs collapsed (a
+    string literal holding a comment marker would be cut too; the sources
+    have none that matter for code identity)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def kernel_digest() -> str:
+    """SHA-1 of the CUDA sources' code alone (comments and layout stripped)
+    and the compile flags: the key under which measured counters of a kernel
+    (profiles/traffic.json) stay valid.  Editing documentation does not
+    change it; editing code does."""
+    h = hashlib.sha1()
+    for p in sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))):
+        h.update(os.path.basename(p).encode())
+        with open(p, encoding="utf-8") as f:
+            h.update(_strip_c_comments(f.read()).encode())
+    h.update(" ".join(ARCH + CFLAGS).encode())
+    return h.hexdigest()
+
+
+def build(force: bool = False, verbose: bool = False, out: str | None = None, defines=()) -> str:
+    """Compile every csrc/*.cu and link liblowbit.so.  `out` and `defines`
+    (extra -D flags) build a variant elsewhere, e.g. for a tuning sweep; the
+    default is the in-tree library."""
+    lib = out or LIB
+    stamp = STAMP if out is None else out + ".sha1"
+    objdir = OBJDIR if out is None else out + ".objs"
+    d = digest() + "".join(" -D" + x for x in defines)
+    if not force and os.path.exists(lib) and os.path.exists(stamp):
+        with open(stamp) as f:
             if f.read().strip() == d:
-                return LIB
-    os.makedirs(OBJDIR, exist_ok=True)
-    extra = ["-Xptxas", "-v"] if verbose else []
+                return lib
+    os.makedirs(objdir, exist_ok=True)
+    extra = (["-Xptxas", "-v"] if verbose else []) + ["-D" + x for x in defines]
 
     def compile_one(src):
-        obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [NVCC, *ARCH, *CFLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -64,15 +94,15 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, sources()))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc link failed:\n{r.stderr}")
-    os.replace(tmp, LIB)
-    with open(STAMP, "w") as f:
+    os.replace(tmp, lib)
+    with open(stamp, "w") as f:
         f.write(d + "\n")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":

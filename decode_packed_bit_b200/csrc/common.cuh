@@ -71,7 +71,11 @@ __device__ __forceinline__ void pdl_wait_primary()
 
 // Launch with the programmatic-stream-serialisation attribute so that a
 // kernel which calls pdl_wait_primary() before touching dependent memory may
-// overlap its prologue with the tail of the previous kernel.
+// overlap its prologue with the tail of the previous kernel.  LOWBIT_PDL=0
+// at build time launches without it (plain stream order; for measurement).
+#ifndef LOWBIT_PDL
+#define LOWBIT_PDL 1
+#endif
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t st, Args... args)
@@ -83,7 +87,7 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = LOWBIT_PDL;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);

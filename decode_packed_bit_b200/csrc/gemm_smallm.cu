@@ -486,7 +486,7 @@ static lowbit_status sm_launch(int fmt, const uint8_t *bits, const uint16_t *sca
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = LOWBIT_PDL;
     attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = P.S;
     attr[1].val.clusterDim.y = 1;
@@ -727,7 +727,7 @@ lowbit_status smg_launch(int fmt, const uint8_t *const *bits, const uint16_t *co
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = LOWBIT_PDL;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, grp, q);

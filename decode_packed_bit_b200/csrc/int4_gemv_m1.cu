@@ -541,7 +541,7 @@ lowbit_status i4m1_launch(const uint8_t *q, const uint16_t *scales, const uint16
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = LOWBIT_PDL;
     attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = P.nslices;
     attr[1].val.clusterDim.y = 1;
@@ -612,7 +612,7 @@ lowbit_status i4m1_group_launch(const uint8_t *const *q, const uint16_t *const *
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = LOWBIT_PDL;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, k_i4_m1_lean, grp, p);

@@ -1153,7 +1153,7 @@ static lowbit_status q1m1_launch(const Q1Plan &P, const uint8_t *const *bits, co
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = LOWBIT_PDL;
     int na = 1;
     if (!P.stream) {
         attr[1].id = cudaLaunchAttributeClusterDimension;

@@ -498,3 +498,69 @@ def test_rmsnorm_bf16_within_half_ulp(lb, M, D, two):
     # plus the fp32 error of the normalisation itself
     tol = 0.5 * _bf16_ulp(r64) + 1e-6 * np.abs(r64) + 1e-30
     assert (np.abs(got - r64) <= tol).all()
+
+
+# ---------------------------------------------------------------------------
+# the launches bench.py times, in its exact configuration
+# ---------------------------------------------------------------------------
+
+def _bench_sets_check(lb, mats, x, ys, what):
+    """Sampled outputs of the first, middle and last matrix against the
+    oracle; every output of every matrix written and finite."""
+    assert all(bool(torch.isfinite(y).all()) for y in ys), f"{what}: an output was not written"
+    M = x.shape[0]
+    R = len(mats)
+    for r in (0, R // 2, R - 1):
+        b, s = host(mats[r][0]), host(mats[r][1]).view(np.uint16)
+        N = b.shape[0]
+        ms, ns = sample_pairs(M, N, 128, 9000 + r)
+        y64, ab = oracle.q1_gemv_at(b, s, x, ms, ns)
+        check_float(host(ys[r])[ms, ns], y64, ab, f"{what} r={r}")
+
+
+def test_bench_headline_launch(lb):
+    """The headline launch: R = bench.q1_4096_sets(L2) (169 on B200)
+    4096x4096 matrices drawn as the bench draws them, one grouped call from
+    x, with the workspace the bench passes."""
+    import bench
+    N = K = 4096
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    R = bench.q1_4096_sets(l2)
+    seed = synth.SEED_BASE + synth.W_Q1_4096
+    mats = [synth.torch_q1_layer(seed, N, K, r, torch.device("cuda")) for r in range(R)]
+    x = synth.bf16_normal(seed, (1, K))
+    ys = [torch.full((1, N), float("nan"), dtype=torch.float32, device="cuda") for _ in range(R)]
+    need = lb.lowbit_q1g128_group_workspace_bytes(R, 1, N, K)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda") if need else None
+    lb.lowbit_q1g128_gemv_group([b for b, _ in mats], [s for _, s in mats], dev(x), ys, workspace=ws)
+    _sync()
+    _bench_sets_check(lb, mats, x, ys, f"bench headline R={R}")
+    # the single-call figure's launch: lowbit_q1g128_gemv on one of the matrices
+    y1 = torch.full((1, N), float("nan"), dtype=torch.float32, device="cuda")
+    nws = lb.lowbit_q1g128_workspace_bytes(1, N, K)
+    lb.lowbit_q1g128_gemv(mats[R - 1][0], mats[R - 1][1], dev(x), y1,
+                          workspace=torch.zeros(nws, dtype=torch.uint8, device="cuda") if nws else None)
+    _sync()
+    _bench_sets_check(lb, [mats[R - 1]], x, [y1], "bench single call")
+
+
+@pytest.mark.parametrize("shape", synth.Q1_SWEEP_SHAPES)
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_bench_sweep_launch(lb, shape, M):
+    """The layer-shape sweep's grouped launches (108 sets of 5120x5120, 32 of
+    the FFN shapes on B200), drawn and sized as the bench does."""
+    import bench
+    N, K = shape
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    R = bench.sweep_sets(N, K, l2)
+    seed = synth.SEED_BASE + synth.W_Q1_SWEEP
+    mats = [synth.torch_q1_layer(seed, N, K, r, torch.device("cuda")) for r in range(R)]
+    x = synth.bf16_normal(seed, (M, K), tag=M)
+    ys = [torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda") for _ in range(R)]
+    need = lb.lowbit_q1g128_group_workspace_bytes(R, M, N, K)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda") if need else None
+    lb.lowbit_q1g128_gemv_group([b for b, _ in mats], [s for _, s in mats], dev(x), ys, workspace=ws)
+    _sync()
+    _bench_sets_check(lb, mats, x, ys, f"bench sweep {shape} M={M} R={R}")
+    del mats, ys
+    torch.cuda.empty_cache()
