@@ -71,6 +71,8 @@ def _load():
     lib.orc_argmax16.restype = ctypes.c_int32
     lib.orc_q2_mlp_forward.argtypes = [P, P, ctypes.c_int, P, I64, P, P, ctypes.c_int]
     lib.orc_q2_mlp_forward.restype = ctypes.c_int
+    lib.orc_z80_generate.argtypes = [P, P, ctypes.c_int, P, I64, I64, P, I64, P, P]
+    lib.orc_z80_generate.restype = ctypes.c_int
     lib.orc_trigram_encode.argtypes = [ctypes.c_char_p, P]
     lib.orc_trigram_encode.restype = None
     lib.orc_rmsnorm.argtypes = [P, P, I64, I64, ctypes.c_double, P]
@@ -229,6 +231,25 @@ def q2_mlp_forward(packed_layers, dims, x, muladd16=False):
 def argmax16(v) -> int:
     v = _c(v, np.int16)
     return int(_load().orc_argmax16(_ptr(v), len(v)))
+
+
+def z80_generate(packed_layers, dims, queries, charset, max_new):
+    """Autoregressive replies: queries uint8 [batch][qlen] (0-padded text),
+    charset uint8 [dims[-1]] (byte 0 = end of reply).  Returns (replies uint8
+    [batch][max_new], 0 past each end; lengths int32 [batch])."""
+    layers = [_c(p, np.uint8) for p in packed_layers]
+    dims_a = _c(dims, np.int32)
+    queries = _c(queries, np.uint8)
+    charset = _c(charset, np.uint8)
+    batch, qlen = queries.shape
+    ptrs = (ctypes.c_void_p * len(layers))(*[p.ctypes.data for p in layers])
+    reply = np.zeros((batch, max_new), np.uint8)
+    lens = np.zeros(batch, np.int32)
+    rc = _load().orc_z80_generate(ctypes.cast(ptrs, ctypes.c_void_p), _ptr(dims_a), len(layers), _ptr(queries),
+                                  batch, qlen, _ptr(charset), max_new, _ptr(reply), _ptr(lens))
+    if rc != 0:
+        raise ValueError("oracle z80_generate rejected its sizes")
+    return reply, lens
 
 
 def trigram_encode(text: str) -> np.ndarray:

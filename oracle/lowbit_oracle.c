@@ -524,3 +524,56 @@ int orc_int4_quantize(const float *w, int64_t rows, int64_t cols, int8_t *codes,
         }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Autoregressive reply loop [Z80]: architecture list (128 query + 128
+ * context trigram buckets in, one output neuron per character of the
+ * character set, ReLU between hidden layers) and feature list (autoregressive
+ * generation, one character at a time).
+ *
+ * Reading (the page names the loop but not its state): the query buckets are
+ * the trigram encoding of the user's text; the context buckets are the
+ * trigram encoding of the reply generated so far in this turn (empty at the
+ * start).  Each step feeds [query, context] through the network, takes the
+ * argmax output, and maps it through the character set; the character-set
+ * byte 0 marks the end of the reply.  A reply also ends after max_new
+ * characters.  Every step re-encodes the whole reply from its text.
+ *
+ *   queries  [batch][qlen] bytes; a query ends at its first 0 byte or at qlen
+ *   charset  [dims[n_layers]] bytes
+ *   reply    [batch][max_new] bytes written; bytes past a reply's end are 0
+ *   reply_len[batch]
+ * dims[0] must be 256; max_new at most 250 (so no reply word is longer than
+ * the encoder's 255-character word limit).  Returns 0, or -1 on bad sizes.
+ * ---------------------------------------------------------------------- */
+int orc_z80_generate(const uint8_t *const *packed_layers, const int32_t *dims, int n_layers,
+                     const uint8_t *queries, int64_t batch, int64_t qlen, const uint8_t *charset,
+                     int64_t max_new, uint8_t *reply, int32_t *reply_len)
+{
+    static char qtext[4097];
+    static char rtext[251];
+    int16_t x[256], logit[4096];
+    int32_t am = 0;
+    if (n_layers < 1 || dims[0] != 256 || qlen < 1 || qlen > 4096 || max_new < 0 || max_new > 250) return -1;
+    for (int64_t b = 0; b < batch; b++) {
+        memcpy(qtext, queries + b * qlen, (size_t)qlen);
+        qtext[qlen] = 0;                        /* the query ends at its first 0 byte */
+        int16_t qb[128];
+        orc_trigram_encode(qtext, qb);
+        int64_t t = 0;
+        rtext[0] = 0;
+        for (; t < max_new; t++) {
+            orc_trigram_encode(rtext, x + 128);  /* context: the reply so far */
+            memcpy(x, qb, sizeof qb);
+            if (orc_q2_mlp_forward(packed_layers, dims, n_layers, x, 1, logit, &am, 0) != 0) return -1;
+            const uint8_t ch = charset[am];
+            if (ch == 0) break;                  /* end of reply */
+            reply[b * max_new + t] = ch;
+            rtext[t] = (char)ch;
+            rtext[t + 1] = 0;
+        }
+        reply_len[b] = (int32_t)t;
+        for (int64_t i = t; i < max_new; i++) reply[b * max_new + i] = 0;
+    }
+    return 0;
+}

@@ -417,3 +417,107 @@ def test_rmsnorm_matches_numpy_and_closed_forms():
     np.testing.assert_allclose(oracle.rmsnorm(c), 3.0 / np.sqrt(9.0 + 1e-6), rtol=1e-15)
     r = oracle.rmsnorm(a * 1000.0)
     np.testing.assert_allclose(r, oracle.rmsnorm(a), rtol=1e-5)
+
+
+# ---------------------------------------------------------------------------
+# the autoregressive reply loop
+# ---------------------------------------------------------------------------
+
+# index 0 ends a reply; then space, A-Z, 0-9, '?', '!' (40 outputs)
+CHARSET = np.frombuffer(b"\0 ABCDEFGHIJKLMNOPQRSTUVWXYZ0123456789?!", np.uint8)
+
+
+def _queries(texts, qlen=32):
+    q = np.zeros((len(texts), qlen), np.uint8)
+    for i, t in enumerate(texts):
+        b = t.encode()
+        q[i, :len(b)] = np.frombuffer(b, np.uint8)
+    return q
+
+
+def _counting_net():
+    """256 -> 4 -> 40.  Hidden units 0 and 1 sum the 128 context buckets,
+    unit 2 the 128 query buckets (weight +1 = code 3; every other weight is
+    0 = code 2).  Output 0 (end of reply) adds units 0 and 1, output 2 ('A')
+    reads unit 2.  With n query trigrams and a reply of t letters 'A' (one
+    word: t trigrams), every trigram adds 32, so after the shifts
+    logit[end] = 4 t and logit['A'] = 2 n: the reply is 'A' * ceil(n / 2)."""
+    dims = (256, 4, 40)
+    c1 = np.full((4, 256), 2, np.int8)
+    c1[0, 128:] = 3
+    c1[1, 128:] = 3
+    c1[2, :128] = 3
+    c2 = np.full((40, 4), 2, np.int8)
+    c2[0, 0] = 3
+    c2[0, 1] = 3
+    c2[2, 2] = 3
+    return dims, [oracle.pack("q2", c1), oracle.pack("q2", c2)]
+
+
+def test_reply_loop_closed_form_on_a_counting_network():
+    dims, packed = _counting_net()
+    texts = ["hi", "hello there", "do you dream", "are you a robot", "x", "abcdefghijklmnopq"]
+    reply, lens = oracle.z80_generate(packed, dims, _queries(texts), CHARSET, 40)
+    for i, t in enumerate(texts):
+        n = sum(len(w) for w in t.split())            # one trigram per letter of a padded word
+        want = -(-n // 2)
+        assert lens[i] == want, (t, lens[i], want)
+        assert bytes(reply[i, :want]) == b"A" * want
+        assert not reply[i, want:].any()
+    # a cap shorter than the natural length stops the reply there
+    reply, lens = oracle.z80_generate(packed, dims, _queries(["abcdefghijklmnopq"]), CHARSET, 3)
+    assert lens[0] == 3 and bytes(reply[0]) == b"AAA"
+
+
+def test_reply_loop_word_order_invariance_from_page():
+    """The page: reordered words give the same bucket vector, so the same
+    reply; the query's last byte may be used without a terminator."""
+    dims = synth.Q2_DIMS
+    packed = [oracle.pack("q2", c) for c in synth.q2_codes(31, dims)]
+    a = _queries(["hello there", "there hello", "are you a robot", "robot a you are"], qlen=16)
+    r, n = oracle.z80_generate(packed, dims, a, CHARSET, 24)
+    assert np.array_equal(r[0], r[1]) and n[0] == n[1]
+    assert np.array_equal(r[2], r[3]) and n[2] == n[3]
+    full = _queries(["abcdefghijklmnop"], qlen=16)      # no terminating 0 inside the row
+    r2, n2 = oracle.z80_generate(packed, dims, full, CHARSET, 8)
+    r3, n3 = oracle.z80_generate(packed, dims, _queries(["abcdefghijklmnop"], qlen=20), CHARSET, 8)
+    assert np.array_equal(r2, r3) and np.array_equal(n2, n3)
+
+
+def test_reply_loop_degenerate_cases():
+    dims = (256, 8, 40)
+    zero = [oracle.pack("q2", np.full((8, 256), 2, np.int8)), oracle.pack("q2", np.full((40, 8), 2, np.int8))]
+    q = _queries(["hello"])
+    # all logits 0: the argmax is output 0, the end symbol: empty reply
+    r, n = oracle.z80_generate(zero, dims, q, CHARSET, 10)
+    assert n[0] == 0 and not r.any()
+    # with no end symbol at index 0, the same network repeats charset[0]
+    cs = CHARSET.copy()
+    cs[0] = ord("Z")
+    r, n = oracle.z80_generate(zero, dims, q, cs, 10)
+    assert n[0] == 10 and bytes(r[0]) == b"Z" * 10
+    r, n = oracle.z80_generate(zero, dims, q, cs, 0)
+    assert r.shape == (1, 0) and n[0] == 0
+    with pytest.raises(ValueError):
+        oracle.z80_generate(zero, (128, 8, 40), q, CHARSET, 4)   # the input must be 128 + 128 buckets
+
+
+def test_reply_loop_matches_stepwise_recomposition():
+    """The loop against the same steps driven from Python through the
+    separately pinned pieces (trigram encoder, network, argmax)."""
+    dims = synth.Q2_DIMS
+    packed = [oracle.pack("q2", c) for c in synth.q2_codes(32, dims)]
+    texts = ["hello", "what is your name", "ok", "r u human", "tell me a joke", ""]
+    q = _queries(texts)
+    r, n = oracle.z80_generate(packed, dims, q, CHARSET, 30)
+    for i, t in enumerate(texts):
+        qb = oracle.trigram_encode(t)
+        out = ""
+        for _ in range(30):
+            x = np.concatenate([qb, oracle.trigram_encode(out)])[None, :]
+            _, am = oracle.q2_mlp_forward(packed, dims, x)
+            ch = int(CHARSET[am[0]])
+            if ch == 0:
+                break
+            out += chr(ch)
+        assert n[i] == len(out) and bytes(r[i, :n[i]]) == out.encode(), (t, out)
