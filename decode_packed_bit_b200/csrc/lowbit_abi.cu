@@ -12,6 +12,9 @@ lowbit_status int4_gemv_simt_launch(const uint8_t *, const uint16_t *, const uin
 lowbit_status q2_mlp_launch(const uint8_t *const *, const int32_t *, int, const int16_t *, int, int16_t *,
                             int32_t *, cudaStream_t);
 int q2_weight_bytes_padded(const int32_t *, int);
+size_t z80_smem_bytes(const int32_t *dims, int n_layers);
+lowbit_status z80_generate_launch(const uint8_t *const *, const int32_t *, int, const uint8_t *, int, int,
+                                  const uint8_t *, int, uint8_t *, int32_t *, cudaStream_t);
 lowbit_status rmsnorm_launch(const float *, const float *, int, int, float, uint16_t *, cudaStream_t);
 size_t q1m1_act_bytes(int K);
 bool q1m1_shape_supported(int R, int N, int K);
@@ -377,6 +380,29 @@ lowbit_status lowbit_q2_mlp_forward(const uint8_t *const *w_packed, const int32_
     LB_CHECK(aligned16(x) && aligned16(logits) && (argmax == nullptr || aligned16(argmax)),
              LOWBIT_ERR_MISALIGNED);
     return q2_mlp_launch(w_packed, dims, n_layers, x, batch, logits, argmax, as_stream(stream));
+}
+
+lowbit_status lowbit_z80_generate(const uint8_t *const *w_packed, const int32_t *dims, int n_layers,
+                                  const uint8_t *queries, int batch, int qlen, const uint8_t *charset, int max_new,
+                                  uint8_t *reply, int32_t *reply_len, void *stream)
+{
+    LB_CHECK(w_packed && dims && charset && n_layers >= 1 && n_layers <= 8 && batch >= 0, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(qlen >= 1 && qlen <= 4096 && max_new >= 0 && max_new <= 250, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(dims[0] == 256, LOWBIT_ERR_UNSUPPORTED_SHAPE);  // 128 query + 128 context buckets
+    for (int l = 0; l < n_layers; ++l) {
+        LB_CHECK(dims[l] >= 4 && dims[l] <= 256 && dims[l] % 4 == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+        LB_CHECK(w_packed[l] != nullptr, LOWBIT_ERR_INVALID_ARG);
+        LB_CHECK(aligned16(w_packed[l]), LOWBIT_ERR_MISALIGNED);
+    }
+    LB_CHECK(dims[n_layers] >= 1 && dims[n_layers] <= 256, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    const size_t smem = z80_smem_bytes(dims, n_layers);
+    LB_CHECK(smem > 0 && smem <= 226u * 1024u, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    if (batch == 0) return LOWBIT_OK;
+    LB_CHECK(queries && reply_len && (reply || max_new == 0), LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(aligned16(queries) && aligned16(reply_len) && (reply == nullptr || aligned16(reply)),
+             LOWBIT_ERR_MISALIGNED);
+    return z80_generate_launch(w_packed, dims, n_layers, queries, batch, qlen, charset, max_new, reply, reply_len,
+                               as_stream(stream));
 }
 
 // ---------------------------------------------------------------------------

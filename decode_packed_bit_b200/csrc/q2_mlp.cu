@@ -157,21 +157,18 @@ __device__ __forceinline__ void imma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1,
                  : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(kQ2tThreads) k_q2_mlp_tc(const Q2TNet net, const int16_t *__restrict__ x,
-                                                           int batch, int16_t *__restrict__ logits,
-                                                           int32_t *__restrict__ argmax)
-{
-    extern __shared__ __align__(16) uint8_t smem[];
-    int8_t *wsm = reinterpret_cast<int8_t *>(smem);
-    // activation limbs: [buffer 2][limb 2][vector 32][kQ2tMaxDim + pad]
-    constexpr int kAStride = kQ2tMaxDim + kQ2tPad;
-    uint8_t *abuf = smem + net.wbytes;
-    auto limb = [&](int buf, int l, int v) { return abuf + ((size_t)(buf * 2 + l) * kQ2tVecs + v) * kAStride; };
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+constexpr int kAStride = kQ2tMaxDim + kQ2tPad;
 
-    pdl_launch_dependents();
-    pdl_wait_primary();
-    // expand the codes once: weight (c - 2) as a signed byte; padding is 0
+// Activation limb row of vector v: [buffer 2][limb 2][vector 32][kAStride].
+__device__ __forceinline__ uint8_t *q2t_limb(uint8_t *abuf, int buf, int l, int v)
+{
+    return abuf + ((size_t)(buf * 2 + l) * kQ2tVecs + v) * kAStride;
+}
+
+// Expand every layer's codes once into signed bytes (c - 2) in shared
+// memory; padding rows and columns are 0.  Ends with a CTA barrier.
+__device__ __forceinline__ void q2t_expand_weights(const Q2TNet &net, int8_t *wsm)
+{
     for (int i = threadIdx.x; i < net.wbytes / 16; i += kQ2tThreads)
         reinterpret_cast<uint4 *>(wsm)[i] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
@@ -214,6 +211,80 @@ __global__ void __launch_bounds__(kQ2tThreads) k_q2_mlp_tc(const Q2TNet net, con
         }
     }
     __syncthreads();
+}
+
+// Every layer for the 32 vectors whose input limbs are in buffer 0 (columns
+// past dims[0] zero).  Returns the buffer whose first bytes hold the int16
+// logits, vector v's at [v * kAStride + o].  Ends with a CTA barrier.
+__device__ __forceinline__ int q2t_forward(const Q2TNet &net, const int8_t *wsm, uint8_t *abuf)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+    int cur = 0;
+    for (int l = 0; l < net.n_layers; ++l) {
+        const bool hidden = l < net.n_layers - 1;
+        const int mts = net.rows[l] / 16, kcs = net.cols[l] / 32, wcols = net.cols[l] + kQ2tPad;
+        const int8_t *wl = wsm + net.woff[l];
+        // (16-row tile, 8-vector tile) pairs, round-robin over the warps
+        for (int pr = warp; pr < mts * (kQ2tVecs / 8); pr += kQ2tThreads / 32) {
+            const int mt = pr / (kQ2tVecs / 8), nt = pr - mt * (kQ2tVecs / 8);
+            int dlo[4] = {0, 0, 0, 0}, dhi[4] = {0, 0, 0, 0};
+            const int8_t *wa = wl + (size_t)(mt * 16 + g) * wcols + 4 * t;
+            const uint8_t *blo = q2t_limb(abuf, cur, 0, nt * 8 + g) + 4 * t;
+            const uint8_t *bhi = q2t_limb(abuf, cur, 1, nt * 8 + g) + 4 * t;
+            for (int kc = 0; kc < kcs; ++kc) {
+                const int k0 = 32 * kc;
+                const uint32_t a0 = *reinterpret_cast<const uint32_t *>(wa + k0);
+                const uint32_t a1 = *reinterpret_cast<const uint32_t *>(wa + 8 * wcols + k0);
+                const uint32_t a2 = *reinterpret_cast<const uint32_t *>(wa + k0 + 16);
+                const uint32_t a3 = *reinterpret_cast<const uint32_t *>(wa + 8 * wcols + k0 + 16);
+                imma_s8u8(dlo, a0, a1, a2, a3, *reinterpret_cast<const uint32_t *>(blo + k0),
+                          *reinterpret_cast<const uint32_t *>(blo + k0 + 16));
+                imma_s8s8(dhi, a0, a1, a2, a3, *reinterpret_cast<const uint32_t *>(bhi + k0),
+                          *reinterpret_cast<const uint32_t *>(bhi + k0 + 16));
+            }
+            // d[j]: row mt*16 + g + 8 (j >> 1), vector nt*8 + 2t + (j & 1)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int acc = dlo[j] + 256 * dhi[j];                         // exact: |acc| < 2^27
+                const int16_t wrapped = (int16_t)(uint16_t)(uint32_t)acc;      // mod 2^16
+                int16_t z = (int16_t)(wrapped >> 2);                           // arithmetic shift
+                if (hidden && z < 0) z = 0;
+                const int o = mt * 16 + g + 8 * (j >> 1), v = nt * 8 + 2 * t + (j & 1);
+                if (hidden) {
+                    q2t_limb(abuf, cur ^ 1, 0, v)[o] = (uint8_t)(z & 0xFF);
+                    q2t_limb(abuf, cur ^ 1, 1, v)[o] = (uint8_t)(int8_t)(z >> 8);
+                } else if (o < net.dims[l + 1]) {
+                    // logits as int16: vector v's row spans both limb regions of the buffer
+                    reinterpret_cast<int16_t *>(q2t_limb(abuf, cur ^ 1, 0, 0))[v * kAStride + o] = z;
+                }
+            }
+        }
+        __syncthreads();
+        cur ^= 1;
+    }
+    return cur;
+}
+
+// Smallest index of the largest of n int16 values.
+__device__ __forceinline__ int q2t_argmax(const int16_t *a, int n)
+{
+    int best = 0;
+    for (int c = 1; c < n; ++c)
+        if (a[c] > a[best]) best = c;  // strict: the lowest index wins ties
+    return best;
+}
+
+__global__ void __launch_bounds__(kQ2tThreads) k_q2_mlp_tc(const Q2TNet net, const int16_t *__restrict__ x,
+                                                           int batch, int16_t *__restrict__ logits,
+                                                           int32_t *__restrict__ argmax)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    int8_t *wsm = reinterpret_cast<int8_t *>(smem);
+    uint8_t *abuf = smem + net.wbytes;
+
+    pdl_launch_dependents();
+    pdl_wait_primary();
+    q2t_expand_weights(net, wsm);
 
     const int ntiles = (batch + kQ2tVecs - 1) / kQ2tVecs;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -223,68 +294,236 @@ __global__ void __launch_bounds__(kQ2tThreads) k_q2_mlp_tc(const Q2TNet net, con
         for (int i = threadIdx.x; i < kQ2tVecs * net.cols[0]; i += kQ2tThreads) {
             const int v = i / net.cols[0], k = i - v * net.cols[0];
             const int a = (v < nv && k < d0) ? (int)x[(int64_t)(v0 + v) * d0 + k] : 0;
-            limb(0, 0, v)[k] = (uint8_t)(a & 0xFF);
-            limb(0, 1, v)[k] = (uint8_t)(int8_t)(a >> 8);
+            q2t_limb(abuf, 0, 0, v)[k] = (uint8_t)(a & 0xFF);
+            q2t_limb(abuf, 0, 1, v)[k] = (uint8_t)(int8_t)(a >> 8);
         }
         __syncthreads();
-        int cur = 0;
-        for (int l = 0; l < net.n_layers; ++l) {
-            const bool hidden = l < net.n_layers - 1;
-            const int mts = net.rows[l] / 16, kcs = net.cols[l] / 32, wcols = net.cols[l] + kQ2tPad;
-            const int8_t *wl = wsm + net.woff[l];
-            // (16-row tile, 8-vector tile) pairs, round-robin over the warps
-            for (int pr = warp; pr < mts * (kQ2tVecs / 8); pr += kQ2tThreads / 32) {
-                const int mt = pr / (kQ2tVecs / 8), nt = pr - mt * (kQ2tVecs / 8);
-                int dlo[4] = {0, 0, 0, 0}, dhi[4] = {0, 0, 0, 0};
-                const int8_t *wa = wl + (size_t)(mt * 16 + g) * wcols + 4 * t;
-                const uint8_t *blo = limb(cur, 0, nt * 8 + g) + 4 * t, *bhi = limb(cur, 1, nt * 8 + g) + 4 * t;
-                for (int kc = 0; kc < kcs; ++kc) {
-                    const int k0 = 32 * kc;
-                    const uint32_t a0 = *reinterpret_cast<const uint32_t *>(wa + k0);
-                    const uint32_t a1 = *reinterpret_cast<const uint32_t *>(wa + 8 * wcols + k0);
-                    const uint32_t a2 = *reinterpret_cast<const uint32_t *>(wa + k0 + 16);
-                    const uint32_t a3 = *reinterpret_cast<const uint32_t *>(wa + 8 * wcols + k0 + 16);
-                    imma_s8u8(dlo, a0, a1, a2, a3, *reinterpret_cast<const uint32_t *>(blo + k0),
-                              *reinterpret_cast<const uint32_t *>(blo + k0 + 16));
-                    imma_s8s8(dhi, a0, a1, a2, a3, *reinterpret_cast<const uint32_t *>(bhi + k0),
-                              *reinterpret_cast<const uint32_t *>(bhi + k0 + 16));
-                }
-                // d[j]: row mt*16 + g + 8 (j >> 1), vector nt*8 + 2t + (j & 1)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int acc = dlo[j] + 256 * dhi[j];                         // exact: |acc| < 2^27
-                    const int16_t wrapped = (int16_t)(uint16_t)(uint32_t)acc;      // mod 2^16
-                    int16_t z = (int16_t)(wrapped >> 2);                           // arithmetic shift
-                    if (hidden && z < 0) z = 0;
-                    const int o = mt * 16 + g + 8 * (j >> 1), v = nt * 8 + 2 * t + (j & 1);
-                    if (hidden) {
-                        limb(cur ^ 1, 0, v)[o] = (uint8_t)(z & 0xFF);
-                        limb(cur ^ 1, 1, v)[o] = (uint8_t)(int8_t)(z >> 8);
-                    } else if (o < net.dims[l + 1]) {
-                        // logits as int16: vector v's row spans both limb regions of the buffer
-                        reinterpret_cast<int16_t *>(limb(cur ^ 1, 0, 0))[v * kAStride + o] = z;
-                    }
-                }
-            }
-            __syncthreads();
-            cur ^= 1;
-        }
+        const int cur = q2t_forward(net, wsm, abuf);
         // logits (int16, in the last buffer) and argmax
         const int dl = net.dims[net.n_layers];
-        const int16_t *lg = reinterpret_cast<const int16_t *>(limb(cur, 0, 0));
+        const int16_t *lg = reinterpret_cast<const int16_t *>(q2t_limb(abuf, cur, 0, 0));
         for (int i = threadIdx.x; i < nv * dl; i += kQ2tThreads) {
             const int v = i / dl, c = i - v * dl;
             logits[(int64_t)(v0 + v) * dl + c] = lg[v * kAStride + c];
         }
-        if (argmax != nullptr && threadIdx.x < nv) {
-            const int16_t *a = lg + threadIdx.x * kAStride;
-            int best = 0;
-            for (int c = 1; c < dl; ++c)
-                if (a[c] > a[best]) best = c;  // strict: the lowest index wins ties
-            argmax[v0 + threadIdx.x] = best;
-        }
+        if (argmax != nullptr && threadIdx.x < nv) argmax[v0 + threadIdx.x] = q2t_argmax(lg + threadIdx.x * kAStride, dl);
         __syncthreads();  // the buffers are reused by the next tile
     }
+}
+
+// ---------------------------------------------------------------------------
+// the autoregressive reply loop of "Show HN: Z80-uLM" (architecture and
+// feature lists): 128 query + 128 context trigram buckets in, one output per
+// character, one character per step.  The context buckets hold the trigram
+// encoding of the reply so far (the library's reading; the page names the
+// loop, not its state), and the character-set byte 0 ends a reply.
+// ---------------------------------------------------------------------------
+//
+// A CTA keeps 32 conversations on the SM for their whole reply: their bucket
+// vectors (int16 [32][256]) stay in shared memory, each step runs the network
+// on all 32 (q2t_forward), and thread v then takes conversation v's argmax,
+// writes its character and updates its context buckets in place.  Appending
+// a letter c to a word whose last two characters are a, b (a = ' ' at the
+// word start) changes three trigrams of the padded word: "ab " leaves, "abc"
+// and "bc " arrive; a letter after a space starts a word " c "; a space
+// changes nothing.  So the buckets after t characters equal the encoding of
+// the t-character reply, which is what the definition re-encodes each step.
+
+constexpr int kZ80MaxReply = 250;  // replies stay under the encoder's 255-character word limit
+constexpr int kZ80Buckets = 128;
+
+struct Z80Params {
+    const uint8_t *queries;  // [batch][qlen]
+    uint8_t *reply;          // [batch][max_new]
+    int32_t *reply_len;      // [batch]
+    int batch, qlen, max_new, nchars;
+    uint8_t charset[kQ2tMaxDim];
+};
+
+__device__ __forceinline__ uint32_t z80_lower(uint32_t c) { return (c >= 'A' && c <= 'Z') ? c - 'A' + 'a' : c; }
+
+// FNV-1a (32-bit) of three bytes, reduced to one of the 128 buckets.
+__device__ __forceinline__ int z80_bucket(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t h = 2166136261u;
+    h = (h ^ a) * 16777619u;
+    h = (h ^ b) * 16777619u;
+    h = (h ^ c) * 16777619u;
+    return (int)(h & (kZ80Buckets - 1));
+}
+
+// Trigram buckets of one text (one thread): words are the runs between
+// spaces, lower-cased, padded with one space on each side, at most 255
+// characters kept per word; every 3-byte window adds 32 to its bucket.
+__device__ void z80_encode(const uint8_t *__restrict__ text, int n, int16_t *buckets)
+{
+    for (int i = 0; i < kZ80Buckets; ++i) buckets[i] = 0;
+    int i = 0;
+    while (i < n) {
+        while (i < n && text[i] == ' ') ++i;
+        uint32_t x = 0, y = ' ';
+        int len = 0;
+        while (i < n && text[i] != ' ') {
+            if (len < 255) {
+                const uint32_t c = z80_lower(text[i]);
+                if (len > 0) buckets[z80_bucket(x, y, c)] += 32;
+                x = y;
+                y = c;
+                ++len;
+            }
+            ++i;
+        }
+        if (len == 0) break;
+        buckets[z80_bucket(x, y, ' ')] += 32;
+    }
+}
+
+__global__ void __launch_bounds__(kQ2tThreads) k_z80_generate(const Q2TNet net, const Z80Params p)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    int8_t *wsm = reinterpret_cast<int8_t *>(smem);
+    uint8_t *abuf = smem + net.wbytes;
+    int16_t *bk = reinterpret_cast<int16_t *>(abuf + 4 * kQ2tVecs * kAStride);  // [32][256]: query, context
+    __shared__ int s_len[kQ2tVecs];
+
+    pdl_launch_dependents();
+    pdl_wait_primary();
+    q2t_expand_weights(net, wsm);
+
+    const int ntiles = (p.batch + kQ2tVecs - 1) / kQ2tVecs;
+    const int dl = net.dims[net.n_layers];
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int v0 = tile * kQ2tVecs, nv = min(kQ2tVecs, p.batch - v0);
+        const int v = threadIdx.x;
+        // per-conversation state (thread v < 32): the last two characters of
+        // the reply (lower-cased; ' ' before the first) and whether it ended
+        uint32_t a = ' ', b = ' ';
+        bool live = false;
+        if (v < kQ2tVecs) {
+            int16_t *row = bk + v * 2 * kZ80Buckets;
+            if (v < nv) {
+                const uint8_t *q = p.queries + (int64_t)(v0 + v) * p.qlen;
+                int n = 0;
+                while (n < p.qlen && q[n] != 0) ++n;   // the query ends at its first 0 byte
+                z80_encode(q, n, row);
+                live = true;
+            } else {
+                for (int i = 0; i < kZ80Buckets; ++i) row[i] = 0;
+            }
+            for (int i = 0; i < kZ80Buckets; ++i) row[kZ80Buckets + i] = 0;  // empty reply
+            s_len[v] = 0;
+        }
+        __syncthreads();
+        for (int t = 0; t < p.max_new; ++t) {
+            // input limbs from the bucket vectors
+            for (int i = threadIdx.x; i < kQ2tVecs * 2 * kZ80Buckets; i += kQ2tThreads) {
+                const int u = i >> 8, k = i & 255;
+                const int val = bk[i];
+                q2t_limb(abuf, 0, 0, u)[k] = (uint8_t)(val & 0xFF);
+                q2t_limb(abuf, 0, 1, u)[k] = (uint8_t)(int8_t)(val >> 8);
+            }
+            __syncthreads();
+            const int cur = q2t_forward(net, wsm, abuf);
+            const int16_t *lg = reinterpret_cast<const int16_t *>(q2t_limb(abuf, cur, 0, 0));
+            if (v < kQ2tVecs && live) {
+                const uint32_t ch = p.charset[q2t_argmax(lg + v * kAStride, dl)];
+                if (ch == 0) {
+                    live = false;                          // end of reply
+                } else {
+                    p.reply[(int64_t)(v0 + v) * p.max_new + t] = (uint8_t)ch;
+                    s_len[v] = t + 1;
+                    int16_t *ctx = bk + v * 2 * kZ80Buckets + kZ80Buckets;
+                    const uint32_t c = z80_lower(ch);
+                    if (c != ' ') {
+                        if (b == ' ') {
+                            ctx[z80_bucket(' ', c, ' ')] += 32;   // a new word " c "
+                        } else {
+                            ctx[z80_bucket(a, b, ' ')] -= 32;     // "ab " leaves
+                            ctx[z80_bucket(a, b, c)] += 32;       // "abc" and "bc " arrive
+                            ctx[z80_bucket(b, c, ' ')] += 32;
+                        }
+                    }
+                    a = b;
+                    b = c;
+                }
+            }
+            // every thread has read the logits; stop when no reply of the tile goes on
+            if (!__syncthreads_or(v < kQ2tVecs && live)) break;
+        }
+        if (v < nv) {
+            const int len = s_len[v];
+            p.reply_len[v0 + v] = len;
+            uint8_t *r = p.reply + (int64_t)(v0 + v) * p.max_new;
+            for (int i = len; i < p.max_new; ++i) r[i] = 0;
+        }
+        __syncthreads();  // shared state is reused by the next tile
+    }
+}
+
+// Network description for the tensor-core kernels (all widths <= 256);
+// false when a width is larger.
+static bool q2t_describe(const uint8_t *const *w_packed, const int32_t *dims, int n_layers, Q2TNet &tn)
+{
+    tn = Q2TNet{};
+    tn.n_layers = n_layers;
+    bool fits = true;
+    int toff = 0;
+    for (int l = 0; l <= n_layers; ++l) {
+        tn.dims[l] = dims[l];
+        fits = fits && dims[l] <= kQ2tMaxDim;
+    }
+    for (int l = 0; l < n_layers && fits; ++l) {
+        tn.w[l] = w_packed[l];
+        tn.rows[l] = (dims[l + 1] + 15) / 16 * 16;
+        tn.cols[l] = (dims[l] + 31) / 32 * 32;
+        tn.woff[l] = toff;
+        toff += tn.rows[l] * (tn.cols[l] + kQ2tPad);
+    }
+    tn.wbytes = (toff + 15) & ~15;
+    return fits;
+}
+
+static int num_sms_q2()
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+constexpr size_t kZ80MaxSmem = 226u * 1024u;
+
+size_t z80_smem_bytes(const int32_t *dims, int n_layers)
+{
+    Q2TNet tn;
+    const uint8_t *none[kQ2MaxLayers] = {};
+    if (n_layers < 1 || n_layers > kQ2MaxLayers || !q2t_describe(none, dims, n_layers, tn)) return 0;
+    return (size_t)tn.wbytes + 4u * kQ2tVecs * kAStride + (size_t)kQ2tVecs * 2 * kZ80Buckets * 2;
+}
+
+lowbit_status z80_generate_launch(const uint8_t *const *w_packed, const int32_t *dims, int n_layers,
+                                  const uint8_t *queries, int batch, int qlen, const uint8_t *charset, int max_new,
+                                  uint8_t *reply, int32_t *reply_len, cudaStream_t st)
+{
+    Q2TNet tn;
+    if (!q2t_describe(w_packed, dims, n_layers, tn)) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    const size_t smem = z80_smem_bytes(dims, n_layers);
+    if (smem == 0 || smem > kZ80MaxSmem) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
+    Z80Params p = {};
+    p.queries = queries;
+    p.reply = reply;
+    p.reply_len = reply_len;
+    p.batch = batch;
+    p.qlen = qlen;
+    p.max_new = max_new;
+    p.nchars = dims[n_layers];
+    for (int i = 0; i < dims[n_layers]; ++i) p.charset[i] = charset[i];
+    if (cudaFuncSetAttribute(k_z80_generate, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kZ80MaxSmem) !=
+        cudaSuccess)
+        return LOWBIT_ERR_CUDA;
+    const int tiles = (batch + kQ2tVecs - 1) / kQ2tVecs;
+    dim3 grid(std::min(tiles, num_sms_q2())), block(kQ2tThreads);
+    cudaError_t e = launch_pdl(k_z80_generate, grid, block, smem, st, tn, p);
+    return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
 
 lowbit_status q2_mlp_launch(const uint8_t *const *w_packed, const int32_t *dims, int n_layers,
@@ -303,34 +542,19 @@ lowbit_status q2_mlp_launch(const uint8_t *const *w_packed, const int32_t *dims,
     net.wbytes = off;
     if (batch == 0) return LOWBIT_OK;
     {
-        Q2TNet tn = {};
-        tn.n_layers = n_layers;
-        bool fits = true;
-        int toff = 0;
-        for (int l = 0; l <= n_layers; ++l) {
-            tn.dims[l] = dims[l];
-            fits = fits && dims[l] <= kQ2tMaxDim;
-        }
-        for (int l = 0; l < n_layers && fits; ++l) {
-            tn.w[l] = w_packed[l];
-            tn.rows[l] = (dims[l + 1] + 15) / 16 * 16;
-            tn.cols[l] = (dims[l] + 31) / 32 * 32;
-            tn.woff[l] = toff;
-            toff += tn.rows[l] * (tn.cols[l] + kQ2tPad);
-        }
-        tn.wbytes = (toff + 15) & ~15;
-        const size_t tsmem = (size_t)tn.wbytes + 4u * kQ2tVecs * (kQ2tMaxDim + kQ2tPad);
+        Q2TNet tn;
+        const bool fits = q2t_describe(w_packed, dims, n_layers, tn);
+        const size_t tsmem = (size_t)tn.wbytes + 4u * kQ2tVecs * kAStride;
         if (fits && tsmem <= 200u * 1024u) {
             if (cudaFuncSetAttribute(k_q2_mlp_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
                 cudaSuccess)
                 return LOWBIT_ERR_CUDA;
-            int dev = 0, sms = 148, per_sm = 1;
-            if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            int per_sm = 1;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_q2_mlp_tc, kQ2tThreads, tsmem) != cudaSuccess ||
                 per_sm < 1)
                 per_sm = 1;
             const int tiles = (batch + kQ2tVecs - 1) / kQ2tVecs;
-            dim3 tgrid(std::min(tiles, per_sm * sms)), tblock(kQ2tThreads);  // persistent: every CTA resident
+            dim3 tgrid(std::min(tiles, per_sm * num_sms_q2())), tblock(kQ2tThreads);  // persistent: every CTA resident
             cudaError_t e = launch_pdl(k_q2_mlp_tc, tgrid, tblock, tsmem, st, tn, x, batch, logits, argmax);
             return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
         }

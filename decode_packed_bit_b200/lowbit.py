@@ -48,6 +48,7 @@ SYMBOLS = [
     ("lowbit_int4g64_gemm", I32, [P, P, P, P, I32, I32, I32, P]),
     ("lowbit_int4g64_gemm_group", I32, [P, P, P, P, I32, I32, I32, I32, P]),
     ("lowbit_q2_mlp_forward", I32, [P, P, I32, P, I32, P, P, P]),
+    ("lowbit_z80_generate", I32, [P, P, I32, P, I32, I32, P, I32, P, P, P]),
     ("lowbit_rmsnorm_bf16", I32, [P, P, I32, I32, F32, P, P]),
     ("lowbit_q1g128_stack_workspace_bytes", SZ, [I32, I32, I32]),
     ("lowbit_q1g128_stack_step", I32, [P, P, I32, I32, I32, P, F32, P, SZ, P, P, P]),
@@ -246,6 +247,23 @@ def lowbit_q2_mlp_forward(w_packed, dims, x, logits, argmax=None, stream=None):
     _check(lib().lowbit_q2_mlp_forward(ctypes.cast(ptrs, ctypes.c_void_p), ctypes.cast(dims_c, ctypes.c_void_p),
                                        n_layers, _ptr(x), x.shape[0], _ptr(logits), _ptr(argmax),
                                        _stream(stream)), "lowbit_q2_mlp_forward")
+
+
+def lowbit_z80_generate(w_packed, dims, queries, charset, reply, reply_len, stream=None):
+    """Autoregressive replies: queries uint8 [batch][qlen] (0-padded text),
+    charset: bytes or a uint8 sequence of dims[-1] entries (0 = end of reply),
+    reply uint8 [batch][max_new], reply_len int32 [batch]."""
+    n_layers = len(w_packed)
+    ptrs = (ctypes.c_void_p * n_layers)(*[w.data_ptr() for w in w_packed])
+    dims_c = (ctypes.c_int32 * (n_layers + 1))(*[int(d) for d in dims])
+    cs = bytes(bytearray(int(c) for c in charset))
+    cs_c = ctypes.create_string_buffer(cs, len(cs))
+    batch, qlen = queries.shape
+    max_new = reply.shape[1]
+    _check(lib().lowbit_z80_generate(ctypes.cast(ptrs, ctypes.c_void_p), ctypes.cast(dims_c, ctypes.c_void_p),
+                                     n_layers, _ptr(queries), batch, qlen, ctypes.cast(cs_c, ctypes.c_void_p),
+                                     max_new, _ptr(reply), _ptr(reply_len), _stream(stream)),
+           "lowbit_z80_generate")
 
 
 # -- glue -------------------------------------------------------------------------

@@ -330,6 +330,42 @@ lowbit_status lowbit_q2_mlp_forward(const uint8_t *const *w_packed, const int32_
                                     int16_t *logits, int32_t *argmax, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * Autoregressive replies of the 2-bit network ("Show HN: Z80-uLM",
+ * architecture list: 128 query + 128 context trigram buckets in, one output
+ * neuron per character; feature list: autoregressive generation, one
+ * character at a time; "trigram hash encoding": text hashed into 128
+ * buckets, word order does not matter).  For every conversation b:
+ *     q = buckets(query b);  reply = ""
+ *     repeat up to max_new times:
+ *         logits = network([q, buckets(reply)])   (as lowbit_q2_mlp_forward)
+ *         c = charset[argmax(logits)];  stop if c == 0;  reply += c
+ * buckets(text): the text is split into words at spaces; each word (at most
+ * 255 characters kept), lower-cased (A-Z only) and padded with one space on
+ * each side, adds 32 to bucket FNV-1a-32(w) mod 128 for every 3-byte window
+ * w.  The page shows the buckets and the loop but not the hash, the per-
+ * trigram value or how the context is kept; these are this library's
+ * readings (the context is the encoding of the reply so far, and charset
+ * byte 0 ends a reply).  The kernel updates the context buckets in place as
+ * characters arrive; the result equals the re-encoding above exactly.
+ *
+ *   w_packed, dims, n_layers: the network as for lowbit_q2_mlp_forward, with
+ *             dims[0] == 256 and every width <= 256
+ *   queries   [batch][qlen] bytes; a query ends at its first 0 byte or at
+ *             qlen (1 <= qlen <= 4096)
+ *   charset   HOST array of dims[n_layers] bytes: output index -> character;
+ *             the byte 0 ends a reply
+ *   reply     [batch][max_new] bytes (0 <= max_new <= 250); bytes after a
+ *             reply's end are set to 0 (may be NULL when max_new == 0)
+ *   reply_len [batch] int32: characters in each reply
+ * The weights of all layers, expanded to bytes, must fit in shared memory
+ * (about 190 KB; the 256->192->128->40 network takes 85 KB), else
+ * LOWBIT_ERR_UNSUPPORTED_SHAPE.  Bit-exact: integer arithmetic throughout.
+ * ------------------------------------------------------------------------- */
+lowbit_status lowbit_z80_generate(const uint8_t *const *w_packed, const int32_t *dims, int n_layers,
+                                  const uint8_t *queries, int batch, int qlen, const uint8_t *charset,
+                                  int max_new, uint8_t *reply, int32_t *reply_len, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Glue between the projections of a layer stack: RMS normalisation with unit
  * gain, rounded to bf16.
  *     v[m][d] = a[m][d] (+ b[m][d] when b is not NULL)

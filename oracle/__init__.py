@@ -48,17 +48,19 @@ def _load():
     lib.orc_bf16_to_f64.argtypes = [ctypes.c_uint16]
     lib.orc_bf16_to_f64.restype = ctypes.c_double
     for name in ("orc_q1_pack", "orc_q1_unpack", "orc_int4_pack", "orc_int4_unpack",
-                 "orc_q2_pack", "orc_q2_unpack"):
+                 "orc_q2_pack", "orc_q2_unpack", "orc_t3_pack", "orc_t3_unpack"):
         getattr(lib, name).argtypes = [P, I64, I64, P]
         getattr(lib, name).restype = ctypes.c_int
-    for name in ("orc_q1_gemv", "orc_int4_gemv"):
+    for name in ("orc_q1_gemv", "orc_int4_gemv", "orc_t3_gemv"):
         getattr(lib, name).argtypes = [P, P, P, I64, I64, I64, P, P]
         getattr(lib, name).restype = ctypes.c_int
-    for name in ("orc_q1_gemv_at", "orc_int4_gemv_at"):
+    for name in ("orc_q1_gemv_at", "orc_int4_gemv_at", "orc_t3_gemv_at"):
         getattr(lib, name).argtypes = [P, P, P, I64, P, P, I64, P, P]
         getattr(lib, name).restype = ctypes.c_int
     lib.orc_q1_weight.argtypes = [P, P, I64, I64, I64]
     lib.orc_q1_weight.restype = ctypes.c_double
+    lib.orc_t3_weight.argtypes = [P, P, I64, I64, I64]
+    lib.orc_t3_weight.restype = ctypes.c_double
     lib.orc_int4_weight.argtypes = [P, P, I64, I64, I64]
     lib.orc_int4_weight.restype = ctypes.c_double
     lib.orc_q2_weight.argtypes = [P, I64, I64, I64]
@@ -109,15 +111,24 @@ def bf16_to_f64(bits: int) -> float:
 
 _PACK = {"q1": ("orc_q1_pack", "orc_q1_unpack", 8),
          "q2": ("orc_q2_pack", "orc_q2_unpack", 4),
-         "int4": ("orc_int4_pack", "orc_int4_unpack", 2)}
+         "int4": ("orc_int4_pack", "orc_int4_unpack", 2),
+         "t3": ("orc_t3_pack", "orc_t3_unpack", None)}
+
+
+def packed_cols(fmt: str, cols: int) -> int:
+    """Bytes of one packed row: cols / per_byte, or 26 per 128 for ternary."""
+    per = _PACK[fmt][2]
+    return 26 * (cols // 128) if per is None else cols // per
 
 
 def pack(fmt: str, codes: np.ndarray) -> np.ndarray:
-    """codes int8 [rows][cols] -> packed uint8 [rows][cols/per_byte]."""
+    """codes int8 [rows][cols] -> packed uint8 [rows][packed_cols(fmt, cols)]."""
     fn, _, per = _PACK[fmt]
     codes = _c(codes, np.int8)
     rows, cols = codes.shape
-    out = np.zeros((rows, cols // per), np.uint8)
+    if per is None and cols % 128 != 0:
+        raise ValueError(f"oracle {fn}: cols must be a multiple of 128")
+    out = np.zeros((rows, packed_cols(fmt, cols)), np.uint8)
     rc = getattr(_load(), fn)(_ptr(codes), rows, cols, _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle {fn} rejected the codes (shape {codes.shape})")
@@ -193,6 +204,37 @@ def int4_gemv_at(q, scales, x, ms, ns):
     if rc != 0:
         raise ValueError("oracle int4_gemv_at: K must be a multiple of 64")
     return y, ab
+
+
+def t3_gemv(packed, scales, x, want_abs=False):
+    """packed uint8 [N][26 K/128], scales uint16 (fp16 bits) [N][K/128], x bf16 bits [M][K]."""
+    packed, scales, x = _c(packed, np.uint8), _c(scales, np.uint16), _c(x, np.uint16)
+    M, K = x.shape
+    N = packed.shape[0]
+    y = np.zeros((M, N), np.float64)
+    ab = np.zeros((M, N), np.float64)
+    rc = _load().orc_t3_gemv(_ptr(packed), _ptr(scales), _ptr(x), M, N, K, _ptr(y), _ptr(ab))
+    if rc != 0:
+        raise ValueError("oracle t3_gemv: K must be a multiple of 128")
+    return (y, ab) if want_abs else y
+
+
+def t3_gemv_at(packed, scales, x, ms, ns):
+    packed, scales, x = _c(packed, np.uint8), _c(scales, np.uint16), _c(x, np.uint16)
+    ms, ns = _c(ms, np.int64), _c(ns, np.int64)
+    K = x.shape[1]
+    y = np.zeros(len(ms), np.float64)
+    ab = np.zeros(len(ms), np.float64)
+    rc = _load().orc_t3_gemv_at(_ptr(packed), _ptr(scales), _ptr(x), K, _ptr(ms), _ptr(ns),
+                                len(ms), _ptr(y), _ptr(ab))
+    if rc != 0:
+        raise ValueError("oracle t3_gemv_at: K must be a multiple of 128")
+    return y, ab
+
+
+def t3_weight(packed, scales, K, n, k) -> float:
+    packed, scales = _c(packed, np.uint8), _c(scales, np.uint16)
+    return _load().orc_t3_weight(_ptr(packed), _ptr(scales), K, n, k)
 
 
 def int4_weight(q, scales, K, n, k) -> float:

@@ -577,3 +577,107 @@ int orc_z80_generate(const uint8_t *const *packed_layers, const int32_t *dims, i
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Ternary weights with an FP16 scale per 128 ("Bonsai-27B-gguf technical
+ * white paper digest", section on intelligence density: the ternary model of
+ * the same 27B network is 5.9 GB where the 1-bit Q1_0_g128 one is 3.79 GB).
+ * The page gives no layout.  Reading: weights w in {-1, 0, +1}, one FP16
+ * scale per 128 consecutive weights of a row (as Q1_0_g128), and the 128
+ * trits t = w + 1 of a group packed five per byte in base 3 -- byte j < 25
+ * holds k = 5j .. 5j+4 of the group as sum_i t_i 3^i, byte 25 holds
+ * k = 125..127 as t_0 + 3 t_1 + 9 t_2 -- so a group is 26 bytes plus 2 of
+ * scale: 1.75 bits per weight, and 3.79 GB x 1.75 / 1.125 = 5.90 GB.
+ * Row n's packed bytes are [n][26 * K/128], its scales [n][K/128].
+ * Decoding takes digit i of a byte b as floor(b / 3^i) mod 3 (i < 5, or
+ * i < 3 in byte 25); the packer only writes bytes below 243 (below 27 in
+ * byte 25).
+ * ---------------------------------------------------------------------- */
+
+static int64_t t3_byte_of(int64_t k, int *digit)
+{
+    int64_t g = k / 128, r = k % 128;
+    *digit = (int)(r % 5);
+    return 26 * g + r / 5;     /* r = 125..127 -> byte 25, digits 0..2 */
+}
+
+int orc_t3_pack(const int8_t *codes, int64_t rows, int64_t cols, uint8_t *packed)
+{
+    if (cols % 128 != 0) return -1;
+    const int64_t rb = 26 * (cols / 128);
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t j = 0; j < rb; j++) packed[r * rb + j] = 0;
+        for (int64_t k = 0; k < cols; k++) {
+            int8_t c = codes[r * cols + k];
+            if (c < -1 || c > 1) return -1;
+            int digit;
+            int64_t j = t3_byte_of(k, &digit);
+            int p = 1;
+            for (int i = 0; i < digit; i++) p *= 3;
+            packed[r * rb + j] = (uint8_t)(packed[r * rb + j] + (c + 1) * p);
+        }
+    }
+    return 0;
+}
+
+/* Weight value (-1, 0 or +1) of column k of a packed row. */
+static int t3_code(const uint8_t *row, int64_t k)
+{
+    int digit;
+    int64_t j = t3_byte_of(k, &digit);
+    int v = row[j];
+    for (int i = 0; i < digit; i++) v /= 3;
+    return v % 3 - 1;
+}
+
+int orc_t3_unpack(const uint8_t *packed, int64_t rows, int64_t cols, int8_t *codes)
+{
+    if (cols % 128 != 0) return -1;
+    const int64_t rb = 26 * (cols / 128);
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t k = 0; k < cols; k++) codes[r * cols + k] = (int8_t)t3_code(packed + r * rb, k);
+    return 0;
+}
+
+/* w[n][k] = code * d[n][k/128]. */
+double orc_t3_weight(const uint8_t *packed, const uint16_t *scales, int64_t K, int64_t n, int64_t k)
+{
+    return (double)t3_code(packed + n * 26 * (K / 128), k) * orc_f16_to_f64(scales[n * (K / 128) + k / 128]);
+}
+
+int orc_t3_gemv(const uint8_t *packed, const uint16_t *scales, const uint16_t *x,
+                int64_t M, int64_t N, int64_t K, double *y, double *absdot)
+{
+    if (K % 128 != 0) return -1;
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                double p = orc_t3_weight(packed, scales, K, n, k) * orc_bf16_to_f64(x[m * K + k]);
+                acc += p;
+                aacc += fabs(p);
+            }
+            y[m * N + n] = acc;
+            if (absdot) absdot[m * N + n] = aacc;
+        }
+    }
+    return 0;
+}
+
+int orc_t3_gemv_at(const uint8_t *packed, const uint16_t *scales, const uint16_t *x,
+                   int64_t K, const int64_t *ms, const int64_t *ns, int64_t count,
+                   double *y, double *absdot)
+{
+    if (K % 128 != 0) return -1;
+    for (int64_t i = 0; i < count; i++) {
+        double acc = 0.0, aacc = 0.0;
+        for (int64_t k = 0; k < K; k++) {
+            double p = orc_t3_weight(packed, scales, K, ns[i], k) * orc_bf16_to_f64(x[ms[i] * K + k]);
+            acc += p;
+            aacc += fabs(p);
+        }
+        y[i] = acc;
+        if (absdot) absdot[i] = aacc;
+    }
+    return 0;
+}

@@ -126,3 +126,29 @@ def torch_q1_layer(seed: int, N: int, K: int, tag: int, device):
     bits = torch.randint(0, 256, (N, K // 8), generator=g, device=device, dtype=torch.uint8)
     scales = (torch.randn((N, K // 128), generator=g, device=device) * 0.02).abs().half()
     return bits, scales
+
+
+# -- chat prompts for the reply loop ---------------------------------------------------
+
+# Output index -> character of the 40-output network: 0 ends a reply, then
+# space, A-Z, 0-9, '?', '!'.
+CHARSET = b"\0 ABCDEFGHIJKLMNOPQRSTUVWXYZ0123456789?!"
+
+
+def chat_queries(seed: int, batch: int, qlen: int = 32, words=(1, 5), wlen=(1, 8)) -> np.ndarray:
+    """Prompts as 0-padded bytes [batch][qlen]: `words` words of `wlen`
+    letters each (a-z, a quarter of them upper-case, an occasional '?'),
+    separated by one or two spaces and cut to qlen bytes."""
+    g = rng(seed, S_ROWS)
+    out = np.zeros((batch, qlen), np.uint8)
+    letters = np.frombuffer(b"abcdefghijklmnopqrstuvwxyz", np.uint8)
+    for b in range(batch):
+        parts = []
+        for _ in range(int(g.integers(words[0], words[1] + 1))):
+            w = letters[g.integers(0, 26, size=int(g.integers(wlen[0], wlen[1] + 1)))].copy()
+            up = g.random(len(w)) < 0.25
+            w[up] -= 32
+            parts.append(bytes(w) + (b"?" if g.random() < 0.1 else b""))
+        text = b"".join(p + (b"  " if g.random() < 0.2 else b" ") for p in parts).rstrip(b" ")[:qlen]
+        out[b, :len(text)] = np.frombuffer(text, np.uint8)
+    return out

@@ -169,3 +169,23 @@ def test_group_validation(L):
     assert i(pp, pp, None, pp, 2, 1, 16, 128, None) == 1       # null x
     assert i(pp, pp, FAKE, misp, 2, 1, 16, 128, None) == 2     # misaligned y[1]
     assert i(pp, pp, FAKE, pp, 2, 1, 16, 96, None) == 3        # K % 64
+
+
+def test_z80_generate_validation(L):
+    layers = (ctypes.c_void_p * 3)(0x10000, 0x10000, 0x10000)
+    lp = ctypes.cast(layers, ctypes.c_void_p)
+    dims = (ctypes.c_int32 * 4)(256, 192, 128, 40)
+    dp = ctypes.cast(dims, ctypes.c_void_p)
+    cs = ctypes.create_string_buffer(40)
+    csp = ctypes.cast(cs, ctypes.c_void_p)
+    f = L.lowbit_z80_generate
+    assert f(lp, dp, 3, FAKE, 0, 32, csp, 8, FAKE, FAKE, None) == 0         # no conversations: no-op
+    assert f(lp, dp, 3, FAKE, 4, 32, None, 8, FAKE, FAKE, None) == 1        # no character set
+    assert f(lp, dp, 3, FAKE, 4, 0, csp, 8, FAKE, FAKE, None) == 1          # qlen < 1
+    assert f(lp, dp, 3, FAKE, 4, 32, csp, 251, FAKE, FAKE, None) == 1       # max_new > 250
+    assert f(lp, dp, 3, FAKE, 4, 32, csp, 8, None, FAKE, None) == 1         # null reply
+    assert f(lp, dp, 3, MIS, 4, 32, csp, 8, FAKE, FAKE, None) == 2          # misaligned queries
+    bad = (ctypes.c_int32 * 4)(128, 192, 128, 40)                           # input is not 256 buckets
+    assert f(lp, ctypes.cast(bad, ctypes.c_void_p), 3, FAKE, 4, 32, csp, 8, FAKE, FAKE, None) == 3
+    wide = (ctypes.c_int32 * 4)(256, 512, 128, 40)                          # a width above 256
+    assert f(lp, ctypes.cast(wide, ctypes.c_void_p), 3, FAKE, 4, 32, csp, 8, FAKE, FAKE, None) == 3

@@ -521,3 +521,98 @@ def test_reply_loop_matches_stepwise_recomposition():
                 break
             out += chr(ch)
         assert n[i] == len(out) and bytes(r[i, :n[i]]) == out.encode(), (t, out)
+
+
+# ---------------------------------------------------------------------------
+# ternary, FP16 scale per 128 (base-3 bytes)
+# ---------------------------------------------------------------------------
+
+def _np_t3_codes(packed, K):
+    """Codes decoded with numpy alone: group g's byte j < 25 holds k = 5j..5j+4
+    as base-3 digits (least significant first), byte 25 holds k = 125..127."""
+    N = packed.shape[0]
+    G = K // 128
+    b = packed.reshape(N, G, 26).astype(np.int64)
+    digits = np.stack([(b // 3 ** i) % 3 for i in range(5)], axis=-1)   # [N][G][26][5]
+    flat = digits.reshape(N, G, 130)[:, :, :128]                          # byte 25 keeps 3 digits
+    return (flat - 1).reshape(N, K).astype(np.int8)
+
+
+def test_t3_size_matches_the_page():
+    g = {r[0]: float(r[1]) for r in read_golden("ternary_size.txt")}
+    N, K = 4, 1024
+    codes = synth.rng(40, 0).integers(-1, 2, size=(N, K), dtype=np.int8)
+    packed = oracle.pack("t3", codes)
+    bpw = 8 * (packed.nbytes + 2 * N * K // int(g["group_size"])) / (N * K)
+    assert bpw == 1.75
+    assert round(g["q1_model_gb"] * bpw / g["q1_bits_per_weight"], 1) == g["ternary_model_gb"]
+    # the 2-bit alternative would not fit the page's figure
+    two_bit = 2 + g["scale_bits"] / g["group_size"]
+    assert round(g["q1_model_gb"] * two_bit / g["q1_bits_per_weight"], 1) != g["ternary_model_gb"]
+
+
+def test_t3_every_byte_value_decodes_like_numpy_base3():
+    # one group per row; byte 7 of row v takes the value v (k = 35..39)
+    rows = 243
+    packed = np.full((rows, 26), 121, np.uint8)   # 121 = 11111 in base 3: all zero weights
+    packed[:, 25] = 13                            # 111 in base 3
+    packed[:, 7] = np.arange(rows, dtype=np.uint8)
+    got = oracle.unpack("t3", packed, 128)
+    assert np.array_equal(got, _np_t3_codes(packed, 128))
+    assert not got[:, :35].any() and not got[:, 40:].any()
+    # all 3^5 patterns appear once: the byte is a bijection onto {-1,0,1}^5
+    assert len({tuple(r) for r in got[:, 35:40]}) == 243
+    assert np.array_equal(oracle.pack("t3", got), packed)
+    # the last byte of a group: 27 values, three weights
+    last = np.full((27, 26), 121, np.uint8)
+    last[:, 25] = np.arange(27, dtype=np.uint8)
+    got = oracle.unpack("t3", last, 128)
+    assert len({tuple(r) for r in got[:, 125:128]}) == 27 and not got[:, :125].any()
+    assert np.array_equal(oracle.pack("t3", got), last)
+
+
+def test_t3_pack_roundtrip_and_range():
+    codes = synth.rng(41, 0).integers(-1, 2, size=(9, 640), dtype=np.int8)
+    p = oracle.pack("t3", codes)
+    assert p.shape == (9, 26 * 5) and p.max() < 243
+    assert np.array_equal(oracle.unpack("t3", p, 640), codes)
+    assert np.array_equal(_np_t3_codes(p, 640), codes)
+    with pytest.raises(ValueError):
+        oracle.pack("t3", np.full((1, 128), 2, np.int8))
+    with pytest.raises(ValueError):
+        oracle.pack("t3", np.zeros((1, 96), np.int8))
+
+
+def test_t3_gemv_matches_numpy_at_every_element():
+    M, N, K = 3, 21, 384
+    codes = synth.rng(42, 0).integers(-1, 2, size=(N, K), dtype=np.int8)
+    packed = oracle.pack("t3", codes)
+    scales = synth.q1_scales(42, N, K)
+    x = synth.bf16_normal(42, (M, K))
+    W = _np_t3_codes(packed, K).astype(np.float64) * np.repeat(scales.view(np.float16).astype(np.float64), 128, 1)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    y, ab = oracle.t3_gemv(packed, scales, x, want_abs=True)
+    np.testing.assert_allclose(y, xf @ W.T, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ab, np.abs(xf) @ np.abs(W).T, rtol=1e-12)
+    mm, nn = np.meshgrid(np.arange(M), np.arange(N), indexing="ij")
+    ys, _ = oracle.t3_gemv_at(packed, scales, x, mm.ravel(), nn.ravel())
+    np.testing.assert_allclose(ys, (xf @ W.T).ravel(), rtol=1e-12, atol=1e-12)
+
+
+def test_t3_bruteforce_one_byte_patterns():
+    # x_k = 4^i on k = 5 + i (byte 1 of the group), 0 elsewhere: sum_i w_i 4^i
+    # identifies the pattern; every pattern is reached by some byte value
+    K = 128
+    x = np.zeros((1, K), np.uint16)
+    x[0, 5:10] = synth.to_bf16_bits(4.0 ** np.arange(5))
+    scales = np.full((1, 1), 0x3C00, np.uint16)
+    seen = set()
+    for v in range(243):
+        packed = np.full((1, 26), 121, np.uint8)
+        packed[0, 25] = 13
+        packed[0, 1] = v
+        y = oracle.t3_gemv(packed, scales, x)[0, 0]
+        want = sum((((v // 3 ** i) % 3) - 1) * 4 ** i for i in range(5))
+        assert y == want
+        seen.add(y)
+    assert len(seen) == 243
