@@ -4,6 +4,13 @@
 
 namespace lowbit {
 lowbit_status pack_launch(lowbit_format, const int8_t *, int64_t, int64_t, uint8_t *, cudaStream_t);
+lowbit_status t3_pack_launch(const int8_t *, int64_t, int64_t, uint8_t *, cudaStream_t);
+lowbit_status t3_unpack_launch(const uint8_t *, int64_t, int64_t, int8_t *, cudaStream_t);
+bool t3_fast_supported(int R, int N, int K);
+lowbit_status t3_group_launch(const uint8_t *const *, const uint16_t *const *, const uint16_t *, float *const *, int,
+                              int, int, cudaStream_t);
+lowbit_status t3_simt_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int,
+                             cudaStream_t);
 lowbit_status unpack_launch(lowbit_format, const uint8_t *, int64_t, int64_t, int8_t *, cudaStream_t);
 lowbit_status q1_gemv_simt_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
                                   int, cudaStream_t);
@@ -68,6 +75,7 @@ static int per_byte(lowbit_format f)
     case LOWBIT_FMT_Q1_G128: return 8;
     case LOWBIT_FMT_Q2: return 4;
     case LOWBIT_FMT_INT4_G64: return 2;
+    case LOWBIT_FMT_TERNARY_G128: return -1;  // 26 bytes per 128 columns
     default: return 0;
     }
 }
@@ -101,18 +109,22 @@ lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, 
     const int per = per_byte(fmt);
     LB_CHECK(per != 0, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(rows >= 0 && cols >= 0 && rows * cols < kMaxElems, LOWBIT_ERR_INVALID_ARG);
-    LB_CHECK(cols % per == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    LB_CHECK(cols % (per > 0 ? per : 128) == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
     if (rows == 0 || cols == 0) return LOWBIT_OK;
     LB_CHECK(codes != nullptr && packed != nullptr, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(aligned16(codes) && aligned16(packed), LOWBIT_ERR_MISALIGNED);
+    if (per < 0) return t3_pack_launch(codes, rows, cols, packed, as_stream(stream));
     return pack_launch(fmt, codes, rows, cols, packed, as_stream(stream));
 }
 
 lowbit_status lowbit_quantize(lowbit_format fmt, const float *w, int64_t rows, int64_t cols, uint8_t *packed,
                               uint16_t *scales, void *stream)
 {
-    LB_CHECK(fmt == LOWBIT_FMT_Q1_G128 || fmt == LOWBIT_FMT_INT4_G64 || fmt == LOWBIT_FMT_Q2, LOWBIT_ERR_INVALID_ARG);
-    LB_CHECK(fmt != LOWBIT_FMT_Q2, LOWBIT_ERR_UNSUPPORTED_SHAPE);  // the pages give no rule for 2-bit codes
+    LB_CHECK(fmt == LOWBIT_FMT_Q1_G128 || fmt == LOWBIT_FMT_INT4_G64 || fmt == LOWBIT_FMT_Q2 ||
+                 fmt == LOWBIT_FMT_TERNARY_G128,
+             LOWBIT_ERR_INVALID_ARG);
+    // the pages give no rule for 2-bit or ternary codes
+    LB_CHECK(fmt != LOWBIT_FMT_Q2 && fmt != LOWBIT_FMT_TERNARY_G128, LOWBIT_ERR_UNSUPPORTED_SHAPE);
     LB_CHECK(rows >= 0 && cols >= 0 && rows * cols < kMaxElems, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(cols % (fmt == LOWBIT_FMT_Q1_G128 ? 128 : 64) == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
     if (rows == 0 || cols == 0) return LOWBIT_OK;
@@ -127,10 +139,11 @@ lowbit_status lowbit_unpack(lowbit_format fmt, const uint8_t *packed, int64_t ro
     const int per = per_byte(fmt);
     LB_CHECK(per != 0, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(rows >= 0 && cols >= 0 && rows * cols < kMaxElems, LOWBIT_ERR_INVALID_ARG);
-    LB_CHECK(cols % per == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    LB_CHECK(cols % (per > 0 ? per : 128) == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
     if (rows == 0 || cols == 0) return LOWBIT_OK;
     LB_CHECK(codes != nullptr && packed != nullptr, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(aligned16(codes) && aligned16(packed), LOWBIT_ERR_MISALIGNED);
+    if (per < 0) return t3_unpack_launch(packed, rows, cols, codes, as_stream(stream));
     return unpack_launch(fmt, packed, rows, cols, codes, as_stream(stream));
 }
 
@@ -356,6 +369,43 @@ lowbit_status lowbit_int4g64_gemm_group(const uint8_t *const *w_q, const uint16_
         if (s != LOWBIT_OK) return s;
     }
     return LOWBIT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// ternary, FP16 scale per 128
+// ---------------------------------------------------------------------------
+
+static lowbit_status t3_shape_ok(int M, int N, int K)
+{
+    LB_CHECK(M >= 1 && M <= 16 && N >= 1 && K >= 1, LOWBIT_ERR_INVALID_ARG);
+    LB_CHECK(K % 128 == 0 && (int64_t)N * K < kMaxElems, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    return LOWBIT_OK;
+}
+
+lowbit_status lowbit_t3g128_gemv_group(const uint8_t *const *w, const uint16_t *const *w_scales, const uint16_t *x,
+                                       float *const *y, int R, int M, int N, int K, void *stream)
+{
+    LB_CHECK(R >= 1 && R <= 256 && w && w_scales && y && x, LOWBIT_ERR_INVALID_ARG);
+    lowbit_status s = t3_shape_ok(M, N, K);
+    if (s != LOWBIT_OK) return s;
+    LB_CHECK(aligned16(x), LOWBIT_ERR_MISALIGNED);
+    for (int r = 0; r < R; ++r) {
+        LB_CHECK(w[r] && w_scales[r] && y[r], LOWBIT_ERR_INVALID_ARG);
+        LB_CHECK(aligned16(w[r]) && aligned16(w_scales[r]) && aligned16(y[r]), LOWBIT_ERR_MISALIGNED);
+    }
+    cudaStream_t st = as_stream(stream);
+    if (M == 1 && t3_fast_supported(R, N, K)) return t3_group_launch(w, w_scales, x, y, R, N, K, st);
+    for (int r = 0; r < R; ++r) {
+        s = t3_simt_launch(w[r], w_scales[r], x, y[r], M, N, K, st);
+        if (s != LOWBIT_OK) return s;
+    }
+    return LOWBIT_OK;
+}
+
+lowbit_status lowbit_t3g128_gemv(const uint8_t *w, const uint16_t *w_scales, const uint16_t *x, float *y, int M, int N,
+                                 int K, void *stream)
+{
+    return lowbit_t3g128_gemv_group(&w, &w_scales, x, &y, 1, M, N, K, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -24,7 +24,8 @@ LOWBIT_ERR_CUDA = 4
 LOWBIT_FMT_Q1_G128 = 1
 LOWBIT_FMT_Q2 = 2
 LOWBIT_FMT_INT4_G64 = 3
-FORMATS = {"q1": LOWBIT_FMT_Q1_G128, "q2": LOWBIT_FMT_Q2, "int4": LOWBIT_FMT_INT4_G64}
+LOWBIT_FMT_TERNARY_G128 = 4
+FORMATS = {"q1": LOWBIT_FMT_Q1_G128, "q2": LOWBIT_FMT_Q2, "int4": LOWBIT_FMT_INT4_G64, "t3": LOWBIT_FMT_TERNARY_G128}
 
 # (name, restype, argtypes) of every symbol include/lowbit.h declares.
 P, I32, I64, SZ, F32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -47,6 +48,8 @@ SYMBOLS = [
     ("lowbit_q1g128_gemv_noalloc", I32, [P, P, P, P, I32, I32, I32, P]),
     ("lowbit_int4g64_gemm", I32, [P, P, P, P, I32, I32, I32, P]),
     ("lowbit_int4g64_gemm_group", I32, [P, P, P, P, I32, I32, I32, I32, P]),
+    ("lowbit_t3g128_gemv", I32, [P, P, P, P, I32, I32, I32, P]),
+    ("lowbit_t3g128_gemv_group", I32, [P, P, P, P, I32, I32, I32, I32, P]),
     ("lowbit_q2_mlp_forward", I32, [P, P, I32, P, I32, P, P, P]),
     ("lowbit_z80_generate", I32, [P, P, I32, P, I32, I32, P, I32, P, P, P]),
     ("lowbit_rmsnorm_bf16", I32, [P, P, I32, I32, F32, P, P]),
@@ -236,6 +239,27 @@ def lowbit_int4g64_gemm_group(w_q, w_scales, x, ys, stream=None):
     py, ky = _ptr_array(ys)
     _check(lib().lowbit_int4g64_gemm_group(pq, ps, _ptr(x), py, R, M, N, K, _stream(stream)),
            "lowbit_int4g64_gemm_group")
+
+
+# -- ternary, FP16 scale per 128 ---------------------------------------------------
+
+def lowbit_t3g128_gemv(w, w_scales, x, y, stream=None):
+    """w uint8 [N][26 K/128], w_scales fp16 bits [N][K/128], x bf16 [M][K], y fp32 [M][N]."""
+    M, K = x.shape
+    N = w.shape[0]
+    _check(lib().lowbit_t3g128_gemv(_ptr(w), _ptr(w_scales), _ptr(x), _ptr(y), M, N, K, _stream(stream)),
+           "lowbit_t3g128_gemv")
+
+
+def lowbit_t3g128_gemv_group(w, w_scales, x, ys, stream=None):
+    R = len(w)
+    M, K = x.shape
+    N = w[0].shape[0]
+    pw, kw = _ptr_array(w)
+    ps, ks = _ptr_array(w_scales)
+    py, ky = _ptr_array(ys)
+    _check(lib().lowbit_t3g128_gemv_group(pw, ps, _ptr(x), py, R, M, N, K, _stream(stream)),
+           "lowbit_t3g128_gemv_group")
 
 
 # -- Q2 MLP -----------------------------------------------------------------------

@@ -53,6 +53,15 @@
  *                                 high nibble (k odd) of byte k/2, a 4-bit
  *                                 two's-complement value in [-8, 7].
  *              scales [N][K/64]:  fp16; scale g covers k in [64g, 64g+64).
+ *   TERNARY_G128 bytes [N][26*K/128]: weights w in {-1, 0, +1}; the trits
+ *                                 t = w + 1 of group g (k in [128g, 128g+128))
+ *                                 fill its 26 bytes five per byte in base 3:
+ *                                 byte 26g + j (j < 25) = sum_i t[128g+5j+i]
+ *                                 3^i, byte 26g + 25 = sum_{i<3}
+ *                                 t[128g+125+i] 3^i.  A byte b holds digits
+ *                                 floor(b / 3^i) mod 3; the packer writes
+ *                                 only b < 243 (b < 27 in the last byte).
+ *              scales [N][K/128]: fp16.  1.75 bits per weight.
  */
 #ifndef LOWBIT_H
 #define LOWBIT_H
@@ -75,7 +84,8 @@ typedef enum {
 typedef enum {
     LOWBIT_FMT_Q1_G128 = 1,
     LOWBIT_FMT_Q2 = 2,
-    LOWBIT_FMT_INT4_G64 = 3
+    LOWBIT_FMT_INT4_G64 = 3,
+    LOWBIT_FMT_TERNARY_G128 = 4
 } lowbit_format;
 
 /* Static string for a status code (never NULL). */
@@ -98,10 +108,13 @@ int lowbit_fault_flags(void);
  *
  * lowbit_pack: codes int8 [rows][cols] -> packed uint8 [rows][cols/per_byte]
  * with per_byte = 8 (Q1_0_g128; codes 0 or 1), 4 (Q2; codes 0..3) or 2
- * (INT4_G64; codes -8..7).  Codes outside the format's range are masked to
- * the field width (the packer does not read the data on the host to check).
- * lowbit_unpack is the exact inverse, for every packed byte value.
- * cols must be a multiple of per_byte, else LOWBIT_ERR_UNSUPPORTED_SHAPE.
+ * (INT4_G64; codes -8..7); TERNARY_G128 (codes -1..1) writes 26 bytes per
+ * 128 columns.  Codes outside the format's range are masked to the field
+ * width (clamped to [-1, 1] for TERNARY_G128; the packer does not read the
+ * data on the host to check).  lowbit_unpack is the exact inverse, and
+ * decodes every packed byte value as the layout above defines.
+ * cols must be a multiple of per_byte (of 128 for TERNARY_G128), else
+ * LOWBIT_ERR_UNSUPPORTED_SHAPE.
  * rows == 0 is a no-op that returns LOWBIT_OK.
  * ------------------------------------------------------------------------- */
 lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, int64_t cols,
@@ -305,6 +318,34 @@ lowbit_status lowbit_int4g64_gemm_group(const uint8_t *const *w_q,
                                         const uint16_t *const *w_scales, const uint16_t *x,
                                         float *const *y, int R, int M, int N, int K,
                                         void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Ternary product with an FP16 scale per 128 ("Bonsai-27B-gguf technical
+ * white paper digest": the ternary 27B model is 5.9 GB where the 1.125-bit
+ * one is 3.79 GB, about 1.75 bits per weight; the page gives no layout, the
+ * TERNARY_G128 layout above is this library's reading, and it stores exactly
+ * 1.75 bits per weight):
+ *     y[m][n] = sum_g d[n][g] * sum_{k in group g} w[n][k] * x[m][k]
+ * with w in {-1, 0, +1}, groups of 128, fp32 accumulate.
+ *   w        [N][26*K/128] packed trits
+ *   w_scales [N][K/128]    fp16 scales
+ *   x        [M][K]        bf16
+ *   y        [M][N]        fp32
+ * Shapes: 1 <= M <= 16, N >= 1, K % 128 == 0.  At M = 1 with K % 1024 == 0
+ * the product streams 32 rows per warp (x as per-group 22-bit fixed point,
+ * exact int32 group sums), writing y directly, or, when the group has too
+ * few 32-row blocks to fill the GPU, adding K-slice partial sums into y
+ * after zeroing it (fp32 atomics: the last bits may differ run to run).
+ * Other shapes run a plain CUDA-core kernel.  Packed bytes >= 243 are not
+ * part of the format and give unspecified products.
+ * Group form: R matrices of one shape that read one x (HOST arrays of R
+ * device pointers, 1 <= R <= 256).
+ * ------------------------------------------------------------------------- */
+lowbit_status lowbit_t3g128_gemv(const uint8_t *w, const uint16_t *w_scales, const uint16_t *x,
+                                 float *y, int M, int N, int K, void *stream);
+lowbit_status lowbit_t3g128_gemv_group(const uint8_t *const *w, const uint16_t *const *w_scales,
+                                       const uint16_t *x, float *const *y, int R, int M, int N,
+                                       int K, void *stream);
 
 /* ---------------------------------------------------------------------------
  * Z80-style 2-bit integer MLP ("Show HN: Z80-uLM"), fused over all layers:

@@ -152,3 +152,29 @@ def chat_queries(seed: int, batch: int, qlen: int = 32, words=(1, 5), wlen=(1, 8
         text = b"".join(p + (b"  " if g.random() < 0.2 else b" ") for p in parts).rstrip(b" ")[:qlen]
         out[b, :len(text)] = np.frombuffer(text, np.uint8)
     return out
+
+
+# -- ternary, FP16 scale per 128 ---------------------------------------------------
+
+def t3_codes(seed: int, N: int, K: int, tag: int = 0, p_zero: float = 1 / 3) -> np.ndarray:
+    """Codes in {-1, 0, +1} [N][K]: 0 with probability p_zero, else a fair sign."""
+    g = rng(seed, S_CODES, tag)
+    z = g.random((N, K)) < p_zero
+    s = g.integers(0, 2, size=(N, K), dtype=np.int8) * 2 - 1
+    return np.where(z, 0, s).astype(np.int8)
+
+
+def torch_t3_layer(seed: int, N: int, K: int, tag: int, device):
+    """(packed base-3 bytes uint8 [N][26 K/128], fp16 scales [N][K/128]) drawn
+    on `device`: every byte uniform over the 243 valid values (each of its
+    five trits uniform and independent), the last byte of a group over its
+    27; scales |N(0, 0.02)|."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed((seed * 1000033 + tag) & 0x7FFFFFFFFFFFFFFF)
+    G = K // 128
+    b = torch.randint(0, 243, (N, G, 26), generator=g, device=device, dtype=torch.int16)
+    b[:, :, 25] = torch.randint(0, 27, (N, G), generator=g, device=device, dtype=torch.int16)
+    packed = b.to(torch.uint8).reshape(N, 26 * G).contiguous()
+    scales = (torch.randn((N, G), generator=g, device=device) * 0.02).abs().half()
+    return packed, scales
