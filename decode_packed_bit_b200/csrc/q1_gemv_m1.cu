@@ -721,7 +721,8 @@ __device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *b
 // memory, tail of w + head of w+1, in that order.  The planner gives every
 // warp at least one cell's worth of steps, so no cell has a third part.
 // With p.x set, every CTA builds the activation fragments from x itself (one
-// chunk per warp at a time, the limb scratch in the warp's idle ring slot).
+// chunk per warp at a time, in a limb scratch of its own after the rings, so
+// that every ring slot is already streaming weights during the build).
 // MV > 1: the product of MV vectors (rows of x; those at or past p.M read as
 // zero and are not written), each with its own fragments and constants:
 // vector v's fragments at v * nchunks KB, then all constants, vector-major.
@@ -788,16 +789,18 @@ __global__ void __launch_bounds__(q1l_max_warps(MV) * 32, 1) k_q1_m1_lean(const 
         cp_async_commit();
         islot = islot + 1 == kQ1LStages ? 0 : islot + 1;
     };
+    // every ring slot starts filling before the wait: while the activation is
+    // built, all of this warp's stages are in flight
 #pragma unroll
-    for (int t = 0; t < kQ1LStages - 1; ++t) issue_next();
+    for (int t = 0; t < kQ1LStages; ++t) issue_next();
 
     pdl_wait_primary();  // x or the activation, and the outputs, follow stream order from here
     const int vfrag = p.nchunks * kQ1FragBytesPerChunk;  // bytes of one vector's fragments
     uint8_t *zero = smem + p.act_smem - kQ1ZeroBytes;
     float2 *info = reinterpret_cast<float2 *>(smem + (size_t)MV * vfrag);
     if (p.x != nullptr) {
-        // the ring slot kQ1LStages - 1 of this warp is not in use yet
-        uint8_t *lw = ring + (kQ1LStages - 1) * kQ1LStageBytes;
+        // this warp's limb scratch, after every warp's ring
+        uint8_t *lw = smem + p.act_smem + (size_t)nw * (kQ1LStages * kQ1LStageBytes) + (size_t)warp * kQ1LimbScratch;
         for (int idx = warp; idx < MV * p.nchunks; idx += nw) {
             const int v = idx / p.nchunks, ch = idx - v * p.nchunks;
             uint8_t *frag = smem + (size_t)v * vfrag + (size_t)ch * kQ1FragBytesPerChunk;
@@ -840,13 +843,13 @@ __global__ void __launch_bounds__(q1l_max_warps(MV) * 32, 1) k_q1_m1_lean(const 
 #pragma unroll
                 for (int v = 0; v < MV; ++v) yacc[t][r][v] = 0.f;
         for (int t = st0; t < st1; ++t) {
-            issue_next();
-            cp_async_wait<kQ1LStages - 1>();
+            cp_async_wait<kQ1LStages - 1>();  // the oldest of the kQ1LStages stages in flight has landed
             __syncwarp();
             lean_consume<MV>(ring + slot * kQ1LStageBytes,
                              live ? bf_live + t * (kQ1LChunks * kQ1FragBytesPerChunk) : bf_dead, bstride,
                              inf0 + 4 * kQ1LChunks * t, 4 * p.nchunks, woff, soff, yacc);
             __syncwarp();  // every lane is done with this stage before it is refilled
+            issue_next();  // refill the slot just consumed
             slot = slot + 1 == kQ1LStages ? 0 : slot + 1;
         }
         s += st1 - st0;
@@ -1036,7 +1039,7 @@ static Q1Plan q1_plan(int R, int N, int K, int sms, bool aligned = false, int mv
     // lean stream kernel: whole 1024-k steps and 32-row blocks, as many warps
     // (at most kQ1LMaxWarps) as fit next to the activation, >= 2 cells per warp
     if (aligned && K % 1024 == 0 && N % kQ1StepRows == 0) {
-        const size_t per_warp = (size_t)kQ1LStages * kQ1LStageBytes;
+        const size_t per_warp = (size_t)kQ1LStages * kQ1LStageBytes + kQ1LimbScratch;  // ring + build scratch
         const size_t cap = (size_t)kQ1MaxSmem - 2 * q1l_max_warps(mv) * mv * kQ1StepRows * 4;  // static cut buffers
         const size_t whole_mv = (size_t)mv * P.nchunks * per_chunk + kQ1ZeroBytes;
         const long long fit = whole_mv < cap ? (long long)((cap - whole_mv) / per_warp) : 0;
