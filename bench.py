@@ -13,12 +13,13 @@ more than 3x the L2 cache, so every matrix streams from HBM (no L2 flush is
 needed).  One step is --launches-per-step such launches (one CUDA graph
 replay each), so that the timed region of --steps steps lasts about a second
 and the sampled clocks cover it; exactly --steps steps are timed with CUDA
-events after --warmup untimed ones.  The other four workloads (layer-shape
-sweep, 64-layer stack, INT4_G64, 2-bit MLP) are measured after the headline
-and reported in the same line under "workloads" (--headline-only skips them).
+events after --warmup untimed ones.  The other workloads (layer-shape sweep,
+64-layer stack, INT4_G64, 2-bit MLP, ternary format, reply loop) are measured
+after the headline and reported in the same line under "workloads"
+(--headline-only skips them).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload q1_4096|q1_sweep|q1_stack|int4|q2_mlp]
+                  [--workload q1_4096|q1_sweep|q1_stack|int4|q2_mlp|ternary|z80_reply]
 
 With N > 1 (under torchrun) every weight matrix is split by rows across the
 ranks (each rank holds N/G rows of each of R*G matrices, so the bytes per GPU
@@ -128,7 +129,7 @@ class ClockSampler:
         return False
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
+        sm, pw, smax, reasons = [], [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for l in self.lines:
             f = [c.strip() for c in l.split(",")]
@@ -139,6 +140,10 @@ class ClockSampler:
                 smax = float(f[2])
             except ValueError:
                 continue
+            try:
+                pw.append(float(f[3]))
+            except ValueError:
+                pass
             for name, v in zip(names, f[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(name)
@@ -146,7 +151,8 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "samples_under_load": 0}
         loaded = [s for s in sm if smax and s > 0.5 * smax]
         return {"sm_mhz": statistics.median(loaded or sm), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded)}
+                "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded),
+                "power_w_median": statistics.median(pw) if pw else None}
 
 
 # ---------------------------------------------------------------------------
@@ -781,10 +787,119 @@ def stack_results(args, world, rank, local, Ms=(1, 8), cpu=True):
     return out
 
 
+def t3_bytes(N, K):
+    return N * 26 * (K // 128) + 2 * N * (K // 128)
+
+
+def t3_results(args, world, rank, local, cpu=True):
+    """Ternary weights (FP16 scale per 128, base-3 bytes), 4096 x 4096, M = 1:
+    grouped launches over weight sets larger than L2, and single calls."""
+    import torch
+    import synth
+    lb = _lib()
+    dev = torch.device("cuda", local)
+    N = K = 4096
+    per = t3_bytes(N, K)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    peak = measured_peaks()[0]
+    R = min(256, rotation(per, l2))
+    seed = synth.SEED_BASE + synth.W_T3 + 1000 * rank
+    mats = [synth.torch_t3_layer(seed, N, K, r, dev) for r in range(R)]
+    w = [m for m, _ in mats]
+    sc = [s for _, s in mats]
+    x = torch.from_numpy(synth.bf16_normal(seed, (1, K)).view(np.int16)).to(dev)
+    ys = [torch.empty((1, N), dtype=torch.float32, device=dev) for _ in range(R)]
+    stream = torch.cuda.Stream(device=dev)
+    gms = max_over_ranks(_graph_time(lambda: lb.lowbit_t3g128_gemv_group(w, sc, x, ys, stream=stream), stream,
+                                     max(20, args.steps), args.warmup), world)
+    sms_ = max_over_ranks(_graph_time(lambda: [lb.lowbit_t3g128_gemv(w[r], sc[r], x, ys[r], stream=stream)
+                                               for r in range(R)], stream, max(20, args.steps), args.warmup), world)
+    g_gbs = R * per / (gms * 1e-3) / 1e9
+    s_gbs = R * per / (sms_ * 1e-3) / 1e9
+    out = {"metric": "packed-weight GB/s, ternary (FP16 scale per 128, 1.75 bits per weight) 4096x4096 M=1",
+           "unit": "GB/s", "config": {"workload": "ternary 4096x4096, M=1", "weight_sets": R, "bytes_per_gemv": per,
+                                      "l2": "inputs larger than L2 (rotating weight sets)"},
+           "results": [{"call": "lowbit_t3g128_gemv_group (one launch)", "us": round(gms * 1e3, 3),
+                        "gbs": round(g_gbs, 1), "frac_of_hbm_peak": round(g_gbs / peak, 4)},
+                       {"call": "lowbit_t3g128_gemv, one call per matrix", "us_per_call": round(sms_ * 1e3 / R, 3),
+                        "gbs": round(s_gbs, 1), "frac_of_hbm_peak": round(s_gbs / peak, 4)}]}
+    if cpu and rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        pk = mats[0][0][:1024].cpu().numpy()
+        sk = mats[0][1][:1024].cpu().view(torch.int16).numpy().view(np.uint16)
+        xh = synth.bf16_normal(seed, (1, K))
+        rows = 256
+
+        def one(i):
+            r0 = (i * rows) % (1024 - rows + 1)
+            oracle.t3_gemv(pk[r0:r0 + rows], sk[r0:r0 + rows], xh)
+        with PinnedCore() as pin:
+            reps, dt = _timed_loop(one, args.cpu_seconds / 3, 100000)
+        out["cpu_baseline"] = {"kind": "oracle", "value": round(reps * t3_bytes(rows, K) / dt / 1e9, 6), "unit": "GB/s",
+                               "sample": f"{reps} oracle products of {rows} rows x {K} ({dt:.1f} s)", **cpu_info(pin)}
+    del mats, w, sc
+    torch.cuda.empty_cache()
+    return out
+
+
+def z80_results(args, world, rank, local, cpu=True):
+    """The Z80-uLM reply loop: 4096 conversations, up to 32 characters each,
+    on the 256->192->128->40 network."""
+    import torch
+    import synth
+    lb = _lib()
+    dev = torch.device("cuda", local)
+    seed = synth.SEED_BASE + synth.W_Q2_MLP + 1000 * rank
+    dims = synth.Q2_DIMS
+    w = []
+    for c in synth.q2_codes(seed, dims):
+        codes = torch.from_numpy(c).to(dev)
+        packed = torch.empty((c.shape[0], c.shape[1] // 4), dtype=torch.uint8, device=dev)
+        lb.lowbit_pack("q2", codes, packed)
+        w.append(packed)
+    batch, max_new, qlen = 4096, 32, 32
+    q = torch.from_numpy(synth.chat_queries(seed, batch, qlen)).to(dev)
+    reply = torch.empty((batch, max_new), dtype=torch.uint8, device=dev)
+    lens = torch.empty((batch,), dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    ms = max_over_ranks(_graph_time(lambda: lb.lowbit_z80_generate(w, dims, q, synth.CHARSET, reply, lens,
+                                                                   stream=stream), stream, args.steps, args.warmup),
+                        world)
+    chars = int(lens.sum().item())
+    macs = sum(dims[i] * dims[i + 1] for i in range(len(dims) - 1))
+    out = {"metric": "Z80-uLM reply loop: characters/s (4096 conversations, up to 32 characters)",
+           "unit": "characters/s",
+           "config": {"workload": "reply loop, 256->192->128->40 2-bit network, 4096 prompts of 1-5 words",
+                      "max_new": max_new, "characters_generated": chars},
+           "results": [{"us_per_batch": round(ms * 1e3, 3), "characters_per_s": round(chars / (ms * 1e-3), 1),
+                        "conversations_per_s": round(batch / (ms * 1e-3), 1),
+                        "gmac_per_s": round(chars * macs / (ms * 1e-3) / 1e9, 2)}]}
+    if cpu and rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        packed = [oracle.pack("q2", c) for c in synth.q2_codes(synth.SEED_BASE + synth.W_Q2_MLP, dims)]
+        qh = synth.chat_queries(synth.SEED_BASE + synth.W_Q2_MLP, 64, qlen)
+        with PinnedCore() as pin:
+            t0 = time.perf_counter()
+            n_done = 0
+            total_chars = 0
+            while n_done < 64:
+                _, ln = oracle.z80_generate(packed, dims, qh[n_done:n_done + 8], np.frombuffer(synth.CHARSET, np.uint8),
+                                            max_new)
+                total_chars += int(ln.sum())
+                n_done += 8
+                if time.perf_counter() - t0 > args.cpu_seconds / 3:
+                    break
+            dt = time.perf_counter() - t0
+        out["cpu_baseline"] = {"kind": "oracle", "value": round(total_chars / dt, 2), "unit": "characters/s",
+                               "sample": f"{n_done} oracle replies ({total_chars} characters, {dt:.1f} s)",
+                               **cpu_info(pin)}
+    return out
+
+
 def run_other_workloads(args, world, rank, local):
     out = {}
     for name, fn in (("q1_sweep", sweep_results), ("int4", int4_results), ("q2_mlp", q2_results),
-                     ("q1_stack", stack_results)):
+                     ("q1_stack", stack_results), ("ternary", t3_results), ("z80_reply", z80_results)):
         try:
             out[name] = fn(args, world, rank, local)
         except Exception as e:  # a failing side workload must not hide the headline
@@ -804,7 +919,8 @@ def _single(fn, key):
 
 OTHER_WORKLOADS = {"q1_stack": _single(lambda a, w, r, l: stack_results(a, w, r, l, Ms=(a.m,)), "q1_stack"),
                    "q1_sweep": _single(sweep_results, "q1_sweep"), "int4": _single(int4_results, "int4"),
-                   "q2_mlp": _single(q2_results, "q2_mlp")}
+                   "q2_mlp": _single(q2_results, "q2_mlp"), "ternary": _single(t3_results, "ternary"),
+                   "z80_reply": _single(z80_results, "z80_reply")}
 
 
 def main():
@@ -814,7 +930,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="q1_4096",
-                    choices=["q1_4096", "q1_sweep", "q1_stack", "int4", "q2_mlp"])
+                    choices=["q1_4096", "q1_sweep", "q1_stack", "int4", "q2_mlp", "ternary", "z80_reply"])
     ap.add_argument("--launches-per-step", type=int, default=DEFAULT_LAUNCHES_PER_STEP,
                     help="grouped launches per headline step")
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")

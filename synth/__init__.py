@@ -19,8 +19,9 @@ SEED_BASE = 0x5EED0000
 # Sub-stream ids, one per tensor role.
 S_CODES, S_SCALES, S_X, S_BUCKETS, S_VALUES, S_ROWS = range(6)
 
-# Workload indices (the order the five workloads are listed in).
-W_Q2_MLP, W_Q1_4096, W_Q1_SWEEP, W_Q1_STACK, W_INT4 = range(5)
+# Workload indices (the order the five workloads are listed in, then the
+# ternary format).
+W_Q2_MLP, W_Q1_4096, W_Q1_SWEEP, W_Q1_STACK, W_INT4, W_T3 = range(6)
 
 Q2_DIMS = (256, 192, 128, 40)
 Q1_SWEEP_SHAPES = ((5120, 5120), (17408, 5120), (5120, 17408))
