@@ -92,23 +92,38 @@ __device__ __forceinline__ uint4 q8_to_bf16(uint32_t word)
 }
 
 // One thread's row of a finished group: 32 * NCH TMEM columns (BM / 2),
-// read 16 at a time (fewer live registers next to the 128 accumulators), and
-// acc += d * D.
+// read 16 at a time, LOWBIT_I4TC_DRAIN loads in flight before each wait
+// (fewer live registers than one 32-column load next to the 128
+// accumulators), and acc += d * D.
+#ifndef LOWBIT_I4TC_DRAIN
+#define LOWBIT_I4TC_DRAIN 2
+#endif
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+
 template <int NCH>  // 32-column chunks a thread drains (BM / 64)
 __device__ __forceinline__ void drain_group(uint32_t taddr, float d, float (&acc)[128])
 {
+    constexpr int D = LOWBIT_I4TC_DRAIN;
 #pragma unroll
-    for (int c = 0; c < 2 * NCH; ++c) {
-        uint32_t v[16];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-              "=r"(v[15])
-            : "r"(taddr + 16u * c));
+    for (int c0 = 0; c0 < 2 * NCH; c0 += D) {
+        uint32_t v[D][16];
+#pragma unroll
+        for (int u = 0; u < D; ++u)
+            if (c0 + u < 2 * NCH) tmem_ld16(taddr + 16u * (c0 + u), v[u]);
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(d, __uint_as_float(v[i]), acc[16 * c + i]);
+        for (int u = 0; u < D; ++u)
+            if (c0 + u < 2 * NCH)
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    acc[16 * (c0 + u) + i] = fmaf(d, __uint_as_float(v[u][i]), acc[16 * (c0 + u) + i]);
     }
 }
 
