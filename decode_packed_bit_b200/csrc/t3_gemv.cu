@@ -231,7 +231,12 @@ __device__ __forceinline__ void t3_byte(uint32_t b, const uint32_t *lut_lane, co
     acc[2] = dp4a_us(t, ta.z, acc[2]);
 }
 
-__global__ void __launch_bounds__(256, 1) k_t3_m1(const __grid_constant__ T3Group grp, const T3Params p)
+#ifndef LOWBIT_T3_MAX_WARPS
+#define LOWBIT_T3_MAX_WARPS 12
+#endif
+constexpr int kT3MaxWarps = LOWBIT_T3_MAX_WARPS;
+
+__global__ void __launch_bounds__(kT3MaxWarps * 32, 1) k_t3_m1(const __grid_constant__ T3Group grp, const T3Params p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
@@ -302,26 +307,29 @@ __global__ void __launch_bounds__(256, 1) k_t3_m1(const __grid_constant__ T3Grou
             t3_wait(S - 1);
             __syncwarp();
             const uint8_t *st = ring + slot * kT3StageBytes;
-            // this lane's row: 52 words, 8 fp16 scales
-            uint32_t wv[52];
-#pragma unroll
-            for (int c = 0; c < 13; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(st + lane * kT3UnitBytes + 16 * c);
-                wv[4 * c] = v.x;
-                wv[4 * c + 1] = v.y;
-                wv[4 * c + 2] = v.z;
-                wv[4 * c + 3] = v.w;
-            }
+            // this lane's row: 8 fp16 scales, then one group pair (52 bytes)
+            // at a time from the 16-word window that holds it
+            const uint8_t *row = st + lane * kT3UnitBytes;
             const uint4 sc4 = *reinterpret_cast<const uint4 *>(st + kT3StageW + lane * 16);
             const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
-            __syncwarp();   // the stage may be refilled from here
             const int p0 = u * kT3UnitBytes;    // first byte position of the unit in the row
 #pragma unroll
             for (int q = 0; q < 4; ++q) {       // group pairs 2q, 2q + 1
+                constexpr int kBase[4] = {0, 12, 24, 36};   // 16-byte aligned window of words 13q .. 13q+12
+                uint32_t wv[16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(row + 4 * kBase[q] + 16 * c);
+                    wv[4 * c] = v.x;
+                    wv[4 * c + 1] = v.y;
+                    wv[4 * c + 2] = v.z;
+                    wv[4 * c + 3] = v.w;
+                }
+                const int off = 13 * q - kBase[q];
                 int accA[3] = {0, 0, 0}, accB[3] = {0, 0, 0};
 #pragma unroll
                 for (int w = 0; w < 13; ++w) {
-                    const uint32_t word = wv[13 * q + w];
+                    const uint32_t word = wv[off + w];
                     const int pw = p0 + 52 * q + 4 * w;           // position of the word's first byte
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
@@ -363,6 +371,7 @@ __global__ void __launch_bounds__(256, 1) k_t3_m1(const __grid_constant__ T3Grou
                 yacc = fmaf(da * ga.x, (float)va, yacc);
                 yacc = fmaf(db * gb.x, (float)vb, yacc);
             }
+            __syncwarp();   // every lane is done with the stage before it is refilled
             slot = slot + 1 == S ? 0 : slot + 1;
         }
         const int n = blk * kT3StepRows + lane;
@@ -441,9 +450,10 @@ static T3Plan t3_plan(int R, int N, int K, int sms)
     P.gtab_off = P.tabB_off + 16 * (Pn / 4);
     P.ring_off = (int)align256((size_t)P.gtab_off + 12u * G);
     const size_t left = P.ring_off < kT3MaxSmem ? kT3MaxSmem - P.ring_off : 0;
-    // as many warps as fit with three stages each, then two
-    for (int st = 3; st >= 2 && !P.ok; --st)
-        for (int w = 8; w >= 4; --w)
+    // as many warps as fit (at most kT3MaxWarps), each with three stages if
+    // they fit, else two
+    for (int w = kT3MaxWarps; w >= 4 && !P.ok; --w)
+        for (int st = 3; st >= 2; --st)
             if ((size_t)w * st * kT3StageBytes <= left) {
                 P.warps = w;
                 P.stages = st;
