@@ -371,7 +371,7 @@ def load_traffic(kernel):
             d = json.load(f)
         from decode_packed_bit_b200 import build as lb_build
         ent = d.get(kernel)
-        if ent and ent.get("kernel_sha1") == lb_build.kernel_digest():
+        if ent and ent.get("kernel_sha1") == lb_build.kernel_digest(ent.get("sources")):
             return ent.get("dram_bytes_per_launch")
     except Exception:
         return None

@@ -53,13 +53,17 @@ def _strip_c_comments(text: str) -> str:
     return " ".join(text.split())
 
 
-def kernel_digest() -> str:
-    """SHA-1 of the CUDA sources' code alone (comments and layout stripped)
-    and the compile flags: the key under which measured counters of a kernel
-    (profiles/traffic.json) stay valid.  Editing documentation does not
-    change it; editing code does."""
+def kernel_digest(files=None) -> str:
+    """SHA-1 of CUDA sources' code alone (comments and layout stripped) and
+    the compile flags: the key under which measured counters of a kernel
+    (profiles/traffic.json) stay valid.  `files`: the csrc file names a
+    kernel is compiled from (default: all of them).  Editing documentation
+    does not change it; editing the code of those files does."""
     h = hashlib.sha1()
-    for p in sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))):
+    paths = sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh")))
+    if files is not None:
+        paths = [os.path.join(CSRC, f) for f in files]
+    for p in paths:
         h.update(os.path.basename(p).encode())
         with open(p, encoding="utf-8") as f:
             h.update(_strip_c_comments(f.read()).encode())

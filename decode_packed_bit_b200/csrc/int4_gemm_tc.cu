@@ -50,7 +50,10 @@ constexpr int kTcThreads = (kTcProdWarps + 2) * 32;
 constexpr int kTcATile = kTcBN * kTcBK * 2;        // 16 KiB of bf16
 constexpr int kTcBTile = 256 * kTcBK * 2;          // 32 KiB of bf16 (BM <= 256)
 constexpr int kTcStageBytes = kTcATile + kTcBTile;
-constexpr int kTcSmemBytes = kTcStages * kTcStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kTcPf = 4;                           // groups of packed weights copied ahead
+constexpr int kTcPfBuf = kTcPf + 1;
+constexpr int kTcPfBytes = kTcBN * 32;             // one group's packed nibbles of the tile (4 KiB)
+constexpr int kTcSmemBytes = kTcStages * kTcStageBytes + kTcPfBuf * kTcPfBytes + 1024 /*align*/ + 256 /*barriers*/;
 constexpr int kTcTmemCols = 512;       // two accumulators of up to 256 columns
 
 __device__ unsigned g_tc_fault;  // set when a bounded wait ran out
@@ -136,7 +139,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
     constexpr int BM = 64 * NCH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full_a = reinterpret_cast<uint64_t *>(smem + kTcStages * kTcStageBytes);
+    uint8_t *pfbuf = smem + kTcStages * kTcStageBytes;     // packed weights copied ahead (cp.async)
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(pfbuf + kTcPfBuf * kTcPfBytes);
     uint64_t *full_b = full_a + kTcStages;
     uint64_t *empty = full_b + kTcStages;
     uint64_t *tfull = empty + kTcStages;    // [2]: a group's MMAs have completed in TMEM buffer b
@@ -183,9 +187,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
 #pragma unroll
         for (int i = 0; i < 128; ++i) acc[i] = 0.f;
 
+        // this thread's 16 bytes of packed nibbles of group it, copied kTcPf
+        // groups ahead into a ring of its own (it reads back only what it
+        // copied, so its own cp.async wait is all the ordering needed)
+        const unsigned pf_s = (unsigned)__cvta_generic_to_shared(pfbuf) + (unsigned)(t * 16);
+        auto prefetch = [&](int it) {
+            if (valid && it < ngroups)
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(pf_s + (unsigned)((it % kTcPfBuf) * kTcPfBytes)),
+                             "l"(qrow + (size_t)it * 32)
+                             : "memory");
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
         auto produce = [&](int it) -> bool {   // dequantise group it into stage it % S
             const int s = it % kTcStages, j = it / kTcStages;
-            const uint4 pk = valid ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)it * 32))
+            prefetch(it + kTcPf);
+            asm volatile("cp.async.wait_group %0;" ::"n"(kTcPf) : "memory");
+            const uint4 pk = valid ? *reinterpret_cast<const uint4 *>(pfbuf + (it % kTcPfBuf) * kTcPfBytes + t * 16)
                                    : make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
             if (it >= kTcStages && !mbar_wait(empty + s, (j - 1) & 1, &g_tc_fault)) return false;
             uint8_t *a = smem + s * kTcStageBytes;
@@ -200,6 +217,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
             if (lane == 0) mbar_arrive(full_a + s);
             return true;
         };
+        for (int it = 0; it < kTcPf; ++it) prefetch(it);
         // rows past N dequantise nibble 8 (q = 0): zero weights
         for (int it = 0; it < kTcStages - 1 && it < ngroups && ok; ++it) ok = produce(it);
         float dnext = ne < N ? f16_bits_to_float(__ldg(srow)) : 0.f;
@@ -221,6 +239,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + b);
         }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
         pdl_wait_primary();  // y may still be read by an earlier kernel
         if (ok && ne < N) {
 #pragma unroll
