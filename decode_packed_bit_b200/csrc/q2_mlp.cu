@@ -213,10 +213,13 @@ __device__ __forceinline__ void q2t_expand_weights(const Q2TNet &net, int8_t *ws
     __syncthreads();
 }
 
-// Every layer for the 32 vectors whose input limbs are in buffer 0 (columns
-// past dims[0] zero).  Returns the buffer whose first bytes hold the int16
-// logits, vector v's at [v * kAStride + o].  Ends with a CTA barrier.
-__device__ __forceinline__ int q2t_forward(const Q2TNet &net, const int8_t *wsm, uint8_t *abuf)
+// Every layer for 32 vectors.  The input limbs (columns past dims[0] zero)
+// are read from `in`, laid out as one buffer ([limb 2][vector 32][kAStride]):
+// buffer 0 of abuf, or a buffer of the caller's that the layers never write.
+// The layers alternate between abuf's buffers 1 and 0.  Returns the buffer
+// whose first bytes hold the int16 logits, vector v's at [v * kAStride + o].
+// Ends with a CTA barrier.
+__device__ __forceinline__ int q2t_forward(const Q2TNet &net, const int8_t *wsm, uint8_t *abuf, const uint8_t *in)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
     int cur = 0;
@@ -229,8 +232,9 @@ __device__ __forceinline__ int q2t_forward(const Q2TNet &net, const int8_t *wsm,
             const int mt = pr / (kQ2tVecs / 8), nt = pr - mt * (kQ2tVecs / 8);
             int dlo[4] = {0, 0, 0, 0}, dhi[4] = {0, 0, 0, 0};
             const int8_t *wa = wl + (size_t)(mt * 16 + g) * wcols + 4 * t;
-            const uint8_t *blo = q2t_limb(abuf, cur, 0, nt * 8 + g) + 4 * t;
-            const uint8_t *bhi = q2t_limb(abuf, cur, 1, nt * 8 + g) + 4 * t;
+            const uint8_t *blo = (l == 0 ? in + (size_t)(nt * 8 + g) * kAStride : q2t_limb(abuf, cur, 0, nt * 8 + g)) + 4 * t;
+            const uint8_t *bhi =
+                (l == 0 ? in + (size_t)(kQ2tVecs + nt * 8 + g) * kAStride : q2t_limb(abuf, cur, 1, nt * 8 + g)) + 4 * t;
             for (int kc = 0; kc < kcs; ++kc) {
                 const int k0 = 32 * kc;
                 const uint32_t a0 = *reinterpret_cast<const uint32_t *>(wa + k0);
@@ -298,7 +302,7 @@ __global__ void __launch_bounds__(kQ2tThreads) k_q2_mlp_tc(const Q2TNet net, con
             q2t_limb(abuf, 0, 1, v)[k] = (uint8_t)(int8_t)(a >> 8);
         }
         __syncthreads();
-        const int cur = q2t_forward(net, wsm, abuf);
+        const int cur = q2t_forward(net, wsm, abuf, q2t_limb(abuf, 0, 0, 0));
         // logits (int16, in the last buffer) and argmax
         const int dl = net.dims[net.n_layers];
         const int16_t *lg = reinterpret_cast<const int16_t *>(q2t_limb(abuf, cur, 0, 0));
@@ -320,9 +324,11 @@ __global__ void __launch_bounds__(kQ2tThreads) k_q2_mlp_tc(const Q2TNet net, con
 // ---------------------------------------------------------------------------
 //
 // A CTA keeps 32 conversations on the SM for their whole reply: their bucket
-// vectors (int16 [32][256]) stay in shared memory, each step runs the network
-// on all 32 (q2t_forward), and thread v then takes conversation v's argmax,
-// writes its character and updates its context buckets in place.  Appending
+// vectors (int16 [32][256]) and the network's input limbs stay in shared
+// memory, each step runs the network on all 32 (q2t_forward; the layers never
+// write the input limbs), eight threads per conversation take its argmax, and
+// one of them writes the character and updates the context buckets, and the
+// limbs of the buckets that changed, in place.  Appending
 // a letter c to a word whose last two characters are a, b (a = ' ' at the
 // word start) changes three trigrams of the padded word: "ab " leaves, "abc"
 // and "bc " arrive; a letter after a space starts a word " c "; a space
@@ -383,7 +389,8 @@ __global__ void __launch_bounds__(kQ2tThreads) k_z80_generate(const Q2TNet net, 
     extern __shared__ __align__(16) uint8_t smem[];
     int8_t *wsm = reinterpret_cast<int8_t *>(smem);
     uint8_t *abuf = smem + net.wbytes;
-    int16_t *bk = reinterpret_cast<int16_t *>(abuf + 4 * kQ2tVecs * kAStride);  // [32][256]: query, context
+    uint8_t *inb = abuf + 4 * kQ2tVecs * kAStride;                 // input limbs: [limb 2][vector 32][kAStride]
+    int16_t *bk = reinterpret_cast<int16_t *>(inb + 2 * kQ2tVecs * kAStride);  // [32][256]: query, context
     __shared__ int s_len[kQ2tVecs];
 
     pdl_launch_dependents();
@@ -392,14 +399,20 @@ __global__ void __launch_bounds__(kQ2tThreads) k_z80_generate(const Q2TNet net, 
 
     const int ntiles = (p.batch + kQ2tVecs - 1) / kQ2tVecs;
     const int dl = net.dims[net.n_layers];
+    // conversation v of a tile belongs to the 8 threads 8v .. 8v+7; thread 8v
+    // keeps its state (the last two characters of the reply, lower-cased, ' '
+    // before the first; whether it goes on)
+    const int v = threadIdx.x >> 3, part = threadIdx.x & 7;
+    const bool owner = part == 0;
+    auto set_input = [&](int u, int k, int val) {   // bucket k of conversation u -> its two limbs
+        inb[(size_t)u * kAStride + k] = (uint8_t)(val & 0xFF);
+        inb[(size_t)(kQ2tVecs + u) * kAStride + k] = (uint8_t)(int8_t)(val >> 8);
+    };
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int v0 = tile * kQ2tVecs, nv = min(kQ2tVecs, p.batch - v0);
-        const int v = threadIdx.x;
-        // per-conversation state (thread v < 32): the last two characters of
-        // the reply (lower-cased; ' ' before the first) and whether it ended
         uint32_t a = ' ', b = ' ';
         bool live = false;
-        if (v < kQ2tVecs) {
+        if (owner) {
             int16_t *row = bk + v * 2 * kZ80Buckets;
             if (v < nv) {
                 const uint8_t *q = p.queries + (int64_t)(v0 + v) * p.qlen;
@@ -414,19 +427,31 @@ __global__ void __launch_bounds__(kQ2tThreads) k_z80_generate(const Q2TNet net, 
             s_len[v] = 0;
         }
         __syncthreads();
+        // the input limbs once per tile; afterwards only changed buckets are rewritten
+        for (int i = threadIdx.x; i < kQ2tVecs * 2 * kZ80Buckets; i += kQ2tThreads) set_input(i >> 8, i & 255, bk[i]);
+        __syncthreads();
         for (int t = 0; t < p.max_new; ++t) {
-            // input limbs from the bucket vectors
-            for (int i = threadIdx.x; i < kQ2tVecs * 2 * kZ80Buckets; i += kQ2tThreads) {
-                const int u = i >> 8, k = i & 255;
-                const int val = bk[i];
-                q2t_limb(abuf, 0, 0, u)[k] = (uint8_t)(val & 0xFF);
-                q2t_limb(abuf, 0, 1, u)[k] = (uint8_t)(int8_t)(val >> 8);
+            const int cur = q2t_forward(net, wsm, abuf, inb);
+            const int16_t *lg = reinterpret_cast<const int16_t *>(q2t_limb(abuf, cur, 0, 0)) + v * kAStride;
+            // argmax: each of the 8 threads scans every 8th logit, then the
+            // largest value wins, the lowest index among equals
+            int best = part < dl ? part : 0;
+            int bv = part < dl ? lg[best] : -32768 - 1;
+            for (int c = part + 8; c < dl; c += 8)
+                if (lg[c] > bv) {
+                    bv = lg[c];
+                    best = c;
+                }
+#pragma unroll
+            for (int o = 4; o > 0; o >>= 1) {
+                const int ov = __shfl_xor_sync(0xffffffffu, bv, o), oc = __shfl_xor_sync(0xffffffffu, best, o);
+                if (ov > bv || (ov == bv && oc < best)) {
+                    bv = ov;
+                    best = oc;
+                }
             }
-            __syncthreads();
-            const int cur = q2t_forward(net, wsm, abuf);
-            const int16_t *lg = reinterpret_cast<const int16_t *>(q2t_limb(abuf, cur, 0, 0));
-            if (v < kQ2tVecs && live) {
-                const uint32_t ch = p.charset[q2t_argmax(lg + v * kAStride, dl)];
+            if (owner && live) {
+                const uint32_t ch = p.charset[best];
                 if (ch == 0) {
                     live = false;                          // end of reply
                 } else {
@@ -434,13 +459,17 @@ __global__ void __launch_bounds__(kQ2tThreads) k_z80_generate(const Q2TNet net, 
                     s_len[v] = t + 1;
                     int16_t *ctx = bk + v * 2 * kZ80Buckets + kZ80Buckets;
                     const uint32_t c = z80_lower(ch);
+                    auto bump = [&](int k, int d) {
+                        ctx[k] += d;
+                        set_input(v, kZ80Buckets + k, ctx[k]);
+                    };
                     if (c != ' ') {
                         if (b == ' ') {
-                            ctx[z80_bucket(' ', c, ' ')] += 32;   // a new word " c "
+                            bump(z80_bucket(' ', c, ' '), 32);   // a new word " c "
                         } else {
-                            ctx[z80_bucket(a, b, ' ')] -= 32;     // "ab " leaves
-                            ctx[z80_bucket(a, b, c)] += 32;       // "abc" and "bc " arrive
-                            ctx[z80_bucket(b, c, ' ')] += 32;
+                            bump(z80_bucket(a, b, ' '), -32);    // "ab " leaves
+                            bump(z80_bucket(a, b, c), 32);       // "abc" and "bc " arrive
+                            bump(z80_bucket(b, c, ' '), 32);
                         }
                     }
                     a = b;
@@ -448,9 +477,9 @@ __global__ void __launch_bounds__(kQ2tThreads) k_z80_generate(const Q2TNet net, 
                 }
             }
             // every thread has read the logits; stop when no reply of the tile goes on
-            if (!__syncthreads_or(v < kQ2tVecs && live)) break;
+            if (!__syncthreads_or(owner && live)) break;
         }
-        if (v < nv) {
+        if (owner && v < nv) {
             const int len = s_len[v];
             p.reply_len[v0 + v] = len;
             uint8_t *r = p.reply + (int64_t)(v0 + v) * p.max_new;
@@ -497,7 +526,7 @@ size_t z80_smem_bytes(const int32_t *dims, int n_layers)
     Q2TNet tn;
     const uint8_t *none[kQ2MaxLayers] = {};
     if (n_layers < 1 || n_layers > kQ2MaxLayers || !q2t_describe(none, dims, n_layers, tn)) return 0;
-    return (size_t)tn.wbytes + 4u * kQ2tVecs * kAStride + (size_t)kQ2tVecs * 2 * kZ80Buckets * 2;
+    return (size_t)tn.wbytes + 6u * kQ2tVecs * kAStride + (size_t)kQ2tVecs * 2 * kZ80Buckets * 2;
 }
 
 lowbit_status z80_generate_launch(const uint8_t *const *w_packed, const int32_t *dims, int n_layers,
