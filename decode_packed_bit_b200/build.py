@@ -67,7 +67,8 @@ def kernel_digest(files=None) -> str:
         h.update(os.path.basename(p).encode())
         with open(p, encoding="utf-8") as f:
             h.update(_strip_c_comments(f.read()).encode())
-    h.update(" ".join(ARCH + CFLAGS).encode())
+    # the flags without include paths, which depend on where the tree lives
+    h.update(" ".join(ARCH + [f for f in CFLAGS if not f.startswith("-I")]).encode())
     return h.hexdigest()
 
 

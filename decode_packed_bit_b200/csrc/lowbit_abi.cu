@@ -60,6 +60,13 @@ lowbit_status q1m1_gemv_launch(const uint8_t *const *, const uint16_t *const *, 
 
 constexpr int64_t kMaxElems = int64_t(1) << 40;
 constexpr int kQ1MaxM = 16;
+// INT4_G64 single calls with 2 <= M <= this take the mma.sync small-batch
+// kernel; larger M (from 16 up, where the tensor-core GEMM applies) the
+// tcgen05 GEMM.
+#ifndef LOWBIT_I4_SMALLM_MAX
+#define LOWBIT_I4_SMALLM_MAX 32
+#endif
+constexpr int kI4SmallMMax = LOWBIT_I4_SMALLM_MAX;
 }  // namespace lowbit
 
 using namespace lowbit;
@@ -343,7 +350,7 @@ lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales, 
     LB_CHECK(aligned16(w_q) && aligned16(w_scales) && aligned16(x) && aligned16(y), LOWBIT_ERR_MISALIGNED);
     cudaStream_t st = as_stream(stream);
     if (M == 1 && i4m1_supported(N, K)) return i4m1_launch(w_q, w_scales, x, y, N, K, st);
-    if (M >= 2 && i4sm_supported(M, N, K)) return i4sm_launch(w_q, w_scales, x, y, M, N, K, st);
+    if (M >= 2 && M <= kI4SmallMMax && i4sm_supported(M, N, K)) return i4sm_launch(w_q, w_scales, x, y, M, N, K, st);
     if (i4tc_supported(M, N, K)) return i4tc_launch(w_q, w_scales, x, y, M, N, K, st);
     return int4_gemv_simt_launch(w_q, w_scales, x, y, M, N, K, st);
 }
