@@ -450,6 +450,24 @@ def run_q1_4096(args, world, rank, local):
                     if gather is not None:
                         gather()
 
+    # context only: 20 launches right after the capture, before the board
+    # has run long enough to reach its power limit
+    burst = None
+    if world == 1:
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                graph.replay()
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0.record(stream)
+            for _ in range(20):
+                graph.replay()
+            b1.record(stream)
+        b1.synchronize()
+        bus = b0.elapsed_time(b1) * 1e3 / 20
+        burst = {"launches": 20, "us_per_launch": round(bus, 3),
+                 "gbs": round(bytes_launch / (bus * 1e-6) / 1e9, 1),
+                 "frac": round(bytes_launch / (bus * 1e-6) / 1e9 / measured_peaks()[0], 4),
+                 "note": "not the bench value: timed before the sustained region, too short for clock samples"}
     run_steps(args.warmup)
     stream.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
@@ -552,6 +570,7 @@ def run_q1_4096(args, world, rank, local):
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
                 "note": "one grouped call per step: x in from pinned host, all outputs out"},
         "single_call": single,
+        "burst": burst,
         "gpu_launches": calls_per_launch * launches,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
