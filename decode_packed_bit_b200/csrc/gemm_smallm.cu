@@ -31,6 +31,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace lowbit {
 
@@ -513,17 +514,60 @@ lowbit_status i4sm_launch(const uint8_t *q, const uint16_t *scales, const uint16
 // grouped persistent form: R matrices of one shape that read one x (M >= 2)
 // ---------------------------------------------------------------------------
 //
-// One CTA per SM with nw warps; every warp owns one 32-row block of one
-// matrix over all of K per round, and the rounds walk the (matrix, block)
-// list: block (j * gridDim + blockIdx) * nw + warp in round j.  The warps of
-// a CTA move through the steps of K in lockstep, so the CTA-wide x ring of
-// the single-matrix kernel serves all of them; the weights stream through
-// per-warp rings.  With all of K per warp no partial sums cross warps or
-// CTAs: a warp writes its rows' outputs after the last step of a round.
+// One CTA per SM: nw consumer warps and one producer warp.  Every consumer
+// warp owns one 32-row block of one matrix over all of K per round, and the
+// rounds walk the (matrix, block) list: block (j * gridDim + blockIdx) * nw +
+// warp in round j.  Weights stream through a cp.async ring per warp, so a
+// warp waits only for its own copies.  x is shared through two rings:
+//   raw ring (kSgRaw slots, Q1_0_g128 only): one thread of the producer
+//     warp loads each step's slice of x (M rows x one step of k, one 2-D
+//     tensor copy) several steps ahead;
+//   x ring (kSgSlots slots): the producer warp rewrites each raw slice once,
+//     in the k order the A operands below want (INT4_G64: the tensor copy
+//     itself fills the slot), and signals the slot's `full` mbarrier; each
+//     consumer warp signals `empty` once it has read it.
+// Warps may drift apart by up to kSgSlots steps without waiting for one
+// another.
+//
+// A operands are built in registers:
+//   Q1_0_g128, no table: for a 32-bit word w of a row's signs (bits j <->
+//     k0 + j), w * 2^(15-j) has bit j at bit 15 and bit j+16 at bit 31, so
+//     one LOP3 (~v & 0x80008000 | 0x3F803F80) gives the bf16 pair
+//     {s(j), s(j+16)}.  In MMA step sigma of a 32-k unit, lane t's slots
+//     2t, 2t+1 take j = 4t + 2 sigma (and j + 16), slots 2t+8, 2t+9 take
+//     j + 1 (and j + 17); x is stored as pairs P[i] = {x[k0+i], x[k0+i+16]},
+//     so the B registers of both steps are one 16-byte load, P[4t .. 4t+3].
+//     The multipliers come from shared memory, which keeps the products on
+//     the integer multiply-add pipe and the ALU pipe free for the LOP3s.
+//   INT4_G64: as in the single-matrix kernel (i4_pair_bf16), lane t's slots
+//     are k 4t .. 4t+3 of a 16-k step and B is x[m][k .. k+3], so x needs no
+//     rewrite: the producer's tensor copy lands it in the x ring directly,
+//     each row one step of k plus 16 more (read past the step, or zero fill
+//     past K), which puts rows 288 bytes (32 mod 128) apart and keeps a half
+//     warp's 8-byte reads of four rows free of bank conflicts.  No raw ring.
+// The sums are exact products accumulated in fp32, one accumulator per
+// group (the group's first MMA starts from zero); the group's scale is
+// applied once per (row, group, vector).
 
 constexpr int kSgMaxGroup = 256;
-constexpr int kSgMaxWarps = 16;
+constexpr int kSgMaxWarps = 15;  // consumer warps (16 warps with the producer: 128 registers each)
 constexpr int kSgMinWarps = 8;
+// Ring depths (compile-time knobs; the defaults are the measured best).
+#ifndef LOWBIT_SG_SLOTS
+#define LOWBIT_SG_SLOTS 6
+#endif
+#ifndef LOWBIT_SG_RAW
+#define LOWBIT_SG_RAW 3
+#endif
+#ifndef LOWBIT_SG_WSTAGES
+#define LOWBIT_SG_WSTAGES 3
+#endif
+constexpr int kSgSlots = LOWBIT_SG_SLOTS;      // x ring depth, in steps
+constexpr int kSgRaw = LOWBIT_SG_RAW;          // raw ring depth, in steps
+constexpr int kSgWStages = LOWBIT_SG_WSTAGES;  // weight ring depth per warp, in steps
+constexpr int kSgThreadsMax = (kSgMaxWarps + 1) * 32;
+
+__device__ unsigned g_sg_fault;  // set when a bounded wait ran out
 
 struct SmGroup {
     const uint8_t *bits[kSgMaxGroup];
@@ -532,70 +576,387 @@ struct SmGroup {
 };
 
 struct SmGParams {
-    const uint16_t *x;
     int M, N, K, nsteps, blocksN, nblocks, rounds;
 };
 
-template <int FMT, int NT>
-__global__ void __launch_bounds__(kSgMaxWarps * 32, 1) k_smallm_grp(const __grid_constant__ SmGroup grp,
-                                                                    const SmGParams q)
-{
-    constexpr int kStepK = SmFmt<FMT>::kStepK;
-    constexpr int kK16 = kStepK / 16;
-    constexpr int kSB = SmFmt<FMT>::kStageBytes;
-    constexpr int kXFrags = kK16 * NT * 32;  // uint2 per step
-    extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ uint2 lut[16];
-    pdl_launch_dependents();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const int total = q.rounds * q.nsteps;  // the CTA's lockstep sequence of (round, step)
-    uint2 *xr = reinterpret_cast<uint2 *>(smem);  // x ring: kSmStages x kXFrags
-    uint8_t *wring = smem + (size_t)kSmStages * kXFrags * 8 + warp * kSmStages * kSB;
-    const unsigned xr_s = (unsigned)__cvta_generic_to_shared(xr);
-    const unsigned wr_s = (unsigned)__cvta_generic_to_shared(wring);
-    auto blk_of = [&](int j) { return (j * (int)gridDim.x + (int)blockIdx.x) * nw + warp; };
+// Bytes of one row of an x slot.  Q1_0_g128 (rewritten order): 64 per 32-k
+// unit plus 64, so that rows sit 64 bytes (mod 128) apart and a quarter
+// warp's 16-byte reads of two rows are free of bank conflicts.  INT4_G64
+// (natural order, filled by the tensor copy): the step's k plus 16 more.
+__host__ __device__ constexpr int sg_xrow(int fmt, int stepk) { return fmt == 1 ? stepk * 2 + 64 : (stepk + 16) * 2; }
 
-    auto issue_w = [&](int u) {
-        if (u >= total) return;
-        const int j = u / q.nsteps, s = u - j * q.nsteps, b = blk_of(j);
-        if (b >= q.nblocks) return;
-        const int r = b / q.blocksN, blk = b - r * q.blocksN;
-        SmParams pp = {};
-        pp.bits = grp.bits[r];
-        pp.scales = grp.scales[r];
-        pp.N = q.N;
-        pp.K = q.K;
-        if (FMT == 1)
-            sm_issue(wr_s + (u % kSmStages) * kSB, pp, blk, s, lane);
-        else
-            i4s_issue(wr_s + (u % kSmStages) * kSB, pp, blk, s, lane);
-    };
-    auto issue_x = [&](int u) {
-        if (u >= total) return;
-        const int s = u % q.nsteps;
-        const unsigned dst = xr_s + (unsigned)((u % kSmStages) * kXFrags) * 8u;
-        for (int i = threadIdx.x; i < kXFrags; i += blockDim.x) {
-            const int ln = i & 31, nt = (i >> 5) % NT, ks = (i >> 5) / NT;
-            const int m = 8 * nt + (ln >> 2);
-            const int k = s * kStepK + 16 * ks + 4 * (ln & 3);
-            sm_cp8(dst + 8u * i, m < q.M ? q.x + (size_t)m * q.K + k : q.x, m < q.M);
+template <int FMT>
+struct SgFmt;
+template <>
+struct SgFmt<1> {
+    static constexpr int kStepK = kSmStepK, kStageBytes = kSmStageBytes, kRowStride = kSmRowStride,
+                         kStageW = kSmStageW;
+};
+template <>
+struct SgFmt<3> {
+    static constexpr int kStepK = kI4sStepK, kStageBytes = kI4sStageBytes, kRowStride = kI4sRowStride,
+                         kStageW = kI4sStageW;
+};
+
+// Shared memory of the grouped kernel, in order: raw ring, x ring (both
+// written by tensor copies, which want 128-byte aligned destinations: every
+// slot size below is a multiple of 128), the warps' weight rings.
+__host__ __device__ constexpr size_t sg_raw_bytes(int fmt, int stepk, int M)
+{
+    return fmt == 1 ? (size_t)kSgRaw * M * stepk * 2 : 0;
+}
+__host__ __device__ constexpr size_t sg_xring_bytes(int fmt, int stepk, int NT)
+{
+    return (size_t)kSgSlots * 8 * NT * sg_xrow(fmt, stepk);
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// Wait until the phase with parity `parity` of `bar` has completed; false
+// (and the fault word set) after kTcWaitNs.  The clock is read once per 16
+// tests.
+__device__ __forceinline__ bool sg_wait(uint64_t *bar, unsigned parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kTcWaitNs) {
+            atomicExch(&g_sg_fault, 1u);
+            return false;
         }
+    }
+}
+
+// bf16 pair {s(j), s(j+16)} of sign word w, m = 2^(15-j): one LOP3 computing
+// (~(w m) & 0x80008000) | 0x3F803F80
+__device__ __forceinline__ uint32_t sg_sign_pair(uint32_t w, uint32_t m)
+{
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xAE;" : "=r"(r) : "r"(w * m), "r"(0x80008000u), "r"(0x3F803F80u));
+    return r;
+}
+
+// the MMA of hmma() with a zero accumulator input
+__device__ __forceinline__ void hmma0(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                      uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%10,%10,%10,%10};"
+                 : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+template <int NT>
+__device__ __forceinline__ void sg_mma(bool first, float (&acc)[NT][4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                       uint32_t a3, const uint4 (&bx)[NT], int sg)
+{
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t b0 = sg ? bx[nt].z : bx[nt].x, b1 = sg ? bx[nt].w : bx[nt].y;
+        if (first)
+            hmma0(acc[nt], a0, a1, a2, a3, b0, b1);
+        else
+            hmma(acc[nt], a0, a1, a2, a3, b0, b1);
+    }
+}
+
+// One staged Q1_0_g128 step of a warp (two groups), x slot `xs`.
+// mul[i] = 2^(15 - 4t - i).
+template <int NT>
+__device__ __forceinline__ void sg_consume_q1(const uint8_t *stage, const uint8_t *xs, int lane, const uint32_t (&mul)[4],
+                                           float (&yacc)[2][NT][4])
+{
+    constexpr int kXR = sg_xrow(1, kSmStepK);
+    constexpr int kRS = kSmRowStride;
+    constexpr int kSW = kSmStageW;
+    constexpr int kUnits = kSmStepK / 64;  // 32-k units per group
+    const int g = lane >> 2, t = lane & 3;
+    const uint8_t *xl = xs + g * kXR + 16 * t;
+    // both groups' scales of rows 16 tt + g (+8): one 32-bit word per row
+    uint32_t dw[2][2];
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) dw[tt][r] = *reinterpret_cast<const uint32_t *>(stage + kSW + (16 * tt + 8 * r + g) * 4);
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp) {
+        float acc[2][NT][4];
+        uint4 w4[2][2];  // the group's 16 bytes of signs of rows 16 tt + g (+8)
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+                w4[tt][r] = *reinterpret_cast<const uint4 *>(stage + (16 * tt + 8 * r + g) * kRS + 16 * grp);
+#pragma unroll
+        for (int cu = 0; cu < kUnits; ++cu) {
+            const int c = kUnits * grp + cu;  // 32-k unit within the step
+            uint4 bx[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                bx[nt] = *reinterpret_cast<const uint4 *>(xl + 8 * nt * kXR + 64 * c);
+#pragma unroll
+                for (int sg = 0; sg < 2; ++sg) {
+#pragma unroll
+                    for (int tt = 0; tt < 2; ++tt) {
+                        const uint32_t w0 = cu == 0 ? w4[tt][0].x : cu == 1 ? w4[tt][0].y : cu == 2 ? w4[tt][0].z : w4[tt][0].w;
+                        const uint32_t w1 = cu == 0 ? w4[tt][1].x : cu == 1 ? w4[tt][1].y : cu == 2 ? w4[tt][1].z : w4[tt][1].w;
+                        const uint32_t a0 = sg_sign_pair(w0, mul[2 * sg]), a2 = sg_sign_pair(w0, mul[2 * sg + 1]);
+                        const uint32_t a1 = sg_sign_pair(w1, mul[2 * sg]), a3 = sg_sign_pair(w1, mul[2 * sg + 1]);
+                        sg_mma<NT>(cu == 0 && sg == 0, acc[tt], a0, a1, a2, a3, bx, sg);
+                    }
+                }
+        }
+        // scale: rows g and g+8 of each tile
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+            const float d0 = f16_bits_to_float((uint16_t)(dw[tt][0] >> (16 * grp)));
+            const float d1 = f16_bits_to_float((uint16_t)(dw[tt][1] >> (16 * grp)));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                yacc[tt][nt][0] = fmaf(d0, acc[tt][nt][0], yacc[tt][nt][0]);
+                yacc[tt][nt][1] = fmaf(d0, acc[tt][nt][1], yacc[tt][nt][1]);
+                yacc[tt][nt][2] = fmaf(d1, acc[tt][nt][2], yacc[tt][nt][2]);
+                yacc[tt][nt][3] = fmaf(d1, acc[tt][nt][3], yacc[tt][nt][3]);
+            }
+        }
+    }
+}
+
+// One staged INT4_G64 step of a warp (two groups), x slot `xs` in natural
+// order (rows sg_xrow apart): the body of i4s_consume with the B fragments
+// read straight from the slot.
+template <int NT>
+__device__ __forceinline__ void sg_consume_i4(const uint8_t *stage, const uint8_t *xs, int lane, float (&yacc)[2][NT][4])
+{
+    constexpr int kXR = sg_xrow(3, kI4sStepK);
+    const int g = lane >> 2, t = lane & 3;
+    const uint8_t *xl = xs + g * kXR + 8 * t;
+    const uint32_t s0 = 2u * (t & 1);
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp) {
+        float acc[2][NT][4];
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const int ks = 4 * grp + s;  // 16-k step within the stage: bytes 8 ks .. 8 ks + 7 of a row
+            uint2 b[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) b[nt] = *reinterpret_cast<const uint2 *>(xl + 8 * nt * kXR + 32 * ks);
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                uint32_t a[2][2];  // [row g / g+8][k 4t..4t+1 / 4t+2..4t+3]
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    // this lane's two bytes: 2t, 2t+1 of the step's 8
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(
+                        stage + (16 * tt + 8 * r + g) * kI4sRowStride + 8 * ks + 4 * (t >> 1));
+                    a[r][0] = i4_pair_bf16(w, s0);
+                    a[r][1] = i4_pair_bf16(w, s0 + 1u);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (s == 0)
+                        hmma0(acc[tt][nt], a[0][0], a[1][0], a[0][1], a[1][1], b[nt].x, b[nt].y);
+                    else
+                        hmma(acc[tt][nt], a[0][0], a[1][0], a[0][1], a[1][1], b[nt].x, b[nt].y);
+                }
+            }
+        }
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+            const float d0 = f16_bits_to_float(
+                *reinterpret_cast<const uint16_t *>(stage + kI4sStageW + (16 * tt + g) * 4 + 2 * grp));
+            const float d1 = f16_bits_to_float(
+                *reinterpret_cast<const uint16_t *>(stage + kI4sStageW + (16 * tt + 8 + g) * 4 + 2 * grp));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                yacc[tt][nt][0] = fmaf(d0, acc[tt][nt][0], yacc[tt][nt][0]);
+                yacc[tt][nt][1] = fmaf(d0, acc[tt][nt][1], yacc[tt][nt][1]);
+                yacc[tt][nt][2] = fmaf(d1, acc[tt][nt][2], yacc[tt][nt][2]);
+                yacc[tt][nt][3] = fmaf(d1, acc[tt][nt][3], yacc[tt][nt][3]);
+            }
+        }
+    }
+}
+
+// Producer task (Q1_0_g128): output chunk q (0..3) of a 32-k unit, from
+// the unit's 64 raw bytes at `src` (natural order), to `dst`.  Chunk q =
+// P[4q .. 4q+3], P[i] = {x[i], x[i+16]}: words 2q, 2q+1 of the low half and
+// the same words 8 later, i.e. 16-byte chunks q/2 and q/2 + 2 of the unit.
+__device__ __forceinline__ void sg_rewrite(const uint8_t *src, uint8_t *dst, int q)
+{
+    const uint4 L = *reinterpret_cast<const uint4 *>(src + 16 * (q >> 1));
+    const uint4 H = *reinterpret_cast<const uint4 *>(src + 16 * (q >> 1) + 32);
+    const uint32_t l0 = (q & 1) ? L.z : L.x, l1 = (q & 1) ? L.w : L.y;
+    const uint32_t h0 = (q & 1) ? H.z : H.x, h1 = (q & 1) ? H.w : H.y;
+    *reinterpret_cast<uint4 *>(dst) =
+        make_uint4(prmt(l0, h0, 0x5410u), prmt(l0, h0, 0x7632u), prmt(l1, h1, 0x5410u), prmt(l1, h1, 0x7632u));
+}
+
+template <int FMT, int NT>
+__global__ void __launch_bounds__(kSgThreadsMax, 1) k_smallm_grp(const __grid_constant__ SmGroup grp,
+                                                                 const __grid_constant__ CUtensorMap xmap,
+                                                                 const SmGParams q)
+{
+    constexpr int kStepK = SgFmt<FMT>::kStepK;
+    constexpr int kSB = SgFmt<FMT>::kStageBytes;
+    constexpr int kXR = sg_xrow(FMT, kStepK);
+    constexpr int kXSlot = 8 * NT * kXR;
+    constexpr int kUnitsStep = kStepK / 32;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    // the tensor copies into the raw ring want a 128-byte aligned destination
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    __shared__ __align__(8) uint64_t bars[2 * kSgSlots + kSgRaw];  // full[s], empty[s], raw[s]
+    __shared__ uint32_t multab[4][4];
+    uint64_t *full = bars, *empty = bars + kSgSlots, *rawbar = bars + 2 * kSgSlots;
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x >> 5) - 1;
+    const int total = q.rounds * q.nsteps;  // (round, step) sequence of every warp
+    const int rawslot = q.M * kStepK * 2;
+    uint8_t *raw = smem;
+    uint8_t *xring = smem + sg_raw_bytes(FMT, kStepK, q.M);
+
+    // rows M .. 8 NT - 1 of every x slot stay zero; barriers; multipliers
+    {
+        const int zrows = 8 * NT - q.M;
+        for (int i = threadIdx.x; i < kSgSlots * zrows * (kXR / 16); i += blockDim.x) {
+            const int sl = i / (zrows * (kXR / 16)), rem = i - sl * zrows * (kXR / 16);
+            const int row = q.M + rem / (kXR / 16), col = rem % (kXR / 16);
+            *reinterpret_cast<uint4 *>(xring + sl * kXSlot + row * kXR + 16 * col) = make_uint4(0, 0, 0, 0);
+        }
+        if (threadIdx.x < 16) multab[threadIdx.x >> 2][threadIdx.x & 3] = 1u << (15 - 4 * (threadIdx.x >> 2) - (threadIdx.x & 3));
+        if (threadIdx.x == 0) {
+            for (int s = 0; s < kSgSlots; ++s) {
+                mbar_init(full + s, FMT == 1 ? 32 : 1);  // the rewriting lanes, or the copying thread
+                mbar_init(empty + s, (unsigned)nw);
+            }
+            for (int s = 0; s < kSgRaw; ++s) mbar_init(rawbar + s, 1);
+            mbar_fence_init();
+        }
+        __syncthreads();
+    }
+
+    if (warp == nw) {
+        pdl_wait_primary();  // x is produced by earlier kernels
+        if (FMT == 3) {
+            // ---- producer (INT4_G64): one tensor copy per step straight into the x ring
+            if (lane == 0) {
+                const unsigned bytes = (unsigned)(q.M * kXR);
+                for (int u = 0; u < total; ++u) {
+                    const int sl = u % kSgSlots;
+                    if (u >= kSgSlots && !sg_wait(empty + sl, ((u / kSgSlots) - 1) & 1)) break;
+                    mbar_arrive_expect_tx(full + sl, bytes);
+                    tma_load_2d(xring + sl * kXSlot, &xmap, (u % q.nsteps) * kStepK, 0, full + sl);
+                }
+            }
+            return;
+        }
+        // ---- producer (Q1_0_g128): raw slices by tensor copy, rewritten once into the x ring
+        auto copy_raw = [&](int v) {  // lane 0: step v of the sequence into raw slot v % kSgRaw
+            if (v >= total) return;
+            uint64_t *bar = rawbar + v % kSgRaw;
+            mbar_arrive_expect_tx(bar, (unsigned)rawslot);
+            tma_load_2d(raw + (v % kSgRaw) * rawslot, &xmap, (v % q.nsteps) * kStepK, 0, bar);
+        };
+        if (lane == 0)
+            for (int v = 0; v < kSgRaw; ++v) copy_raw(v);
+        // task T = (unit item T/4 = (row n, unit c), output chunk T%4); a
+        // quarter warp covers two adjacent units: 128 contiguous bytes each way
+        const int tasks = q.M * kUnitsStep * 4;
+        constexpr int kUn = 4;
+        for (int u = 0; u < total; ++u) {
+            const int sl = u % kSgSlots, rs = u % kSgRaw;
+            bool ok = u < kSgSlots || sg_wait(empty + sl, ((u / kSgSlots) - 1) & 1);
+            ok = ok && sg_wait(rawbar + rs, (u / kSgRaw) & 1);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const uint8_t *rsrc = raw + rs * rawslot;
+            uint8_t *xdst = xring + sl * kXSlot;
+            for (int base = 0; base < tasks; base += 32 * kUn) {
+#pragma unroll
+                for (int i = 0; i < kUn; ++i) {
+                    const int T = base + 32 * i + lane;
+                    if (T < tasks) {
+                        const int item = T >> 2, n = item / kUnitsStep, c = item - n * kUnitsStep;
+                        sg_rewrite(rsrc + n * kStepK * 2 + 64 * c, xdst + n * kXR + 64 * c + 16 * (T & 3), T & 3);
+                    }
+                }
+            }
+            mbar_arrive(full + sl);
+            // the raw slot's reads are done: it may be refilled (async proxy)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) copy_raw(u + kSgRaw);
+        }
+        return;
+    }
+
+    // ---- consumers
+    uint8_t *wring = xring + sg_xring_bytes(FMT, kStepK, NT) + (size_t)warp * kSgWStages * kSB;
+    const unsigned wr_s = (unsigned)__cvta_generic_to_shared(wring);
+    uint32_t mul[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mul[i] = multab[lane & 3][i];
+
+    // Copy cursor: the (round, step) whose weights go out next and this
+    // lane's sources for it.  Q1_0_g128: 16-byte half L%2 of rows L/2 and
+    // L/2 + 16; INT4_G64: 16-byte column L%4 of rows L/4 + {0, 8, 16, 24};
+    // both: the scale pair of row L.  Rows past N copy nothing (zero fill).
+    constexpr int kCopies = FMT == 1 ? 2 : 4;
+    constexpr int kStepBytes = kStepK / (FMT == 1 ? 8 : 2);  // packed bytes of a row per step
+    const int rowbytes = q.K / (FMT == 1 ? 8 : 2), G = q.K / (FMT == 1 ? 128 : 64);
+    // copy c lands kDstStride * c bytes after copy 0 within a stage
+    constexpr unsigned kDstStride = FMT == 1 ? 16 * kSmRowStride : 8 * kI4sRowStride;
+    const unsigned wdst0 = FMT == 1 ? (unsigned)((lane >> 1) * kSmRowStride + (lane & 1) * 16)
+                                    : (unsigned)((lane >> 2) * kI4sRowStride + (lane & 3) * 16);
+    const unsigned sdst = (unsigned)(SgFmt<FMT>::kStageW + lane * 4);
+    int cj = 0, cs = 0, cstage = 0;  // copy cursor: round, step, ring stage
+    bool clive = false;
+    const uint8_t *csrc = nullptr;  // copy 0's row; copy c reads c * cstride bytes further
+    const uint16_t *cscale = nullptr;
+    const unsigned cstride = (unsigned)((FMT == 1 ? 16 : 8) * rowbytes);
+    unsigned cok = 0;  // bit c: copy c reads a row < N; bit kCopies: the scale row
+    auto set_round = [&](int j) {
+        cj = j;
+        cs = 0;
+        const int b = (j * (int)gridDim.x + (int)blockIdx.x) * nw + warp;
+        clive = j < q.rounds && b < q.nblocks;
+        if (!clive) return;
+        const int r = b / q.blocksN, blk = b - r * q.blocksN;
+        const int r0 = blk * 32 + (FMT == 1 ? (lane >> 1) : (lane >> 2));
+        cok = 0;
+#pragma unroll
+        for (int c = 0; c < kCopies; ++c) cok |= (r0 + (FMT == 1 ? 16 : 8) * c < q.N ? 1u : 0u) << c;
+        csrc = grp.bits[r] + (size_t)r0 * rowbytes + (lane & (FMT == 1 ? 1 : 3)) * 16;
+        const int srow = blk * 32 + lane;
+        cok |= (srow < q.N ? 1u : 0u) << kCopies;
+        cscale = grp.scales[r] + (srow < q.N ? (size_t)srow * G : 0);
     };
-    // weights of the first steps go out before the previous kernel ends; x after it
+    auto issue_next = [&]() {  // one commit group per call, empty past the end
+        if (clive) {
+            const unsigned st = wr_s + cstage * kSB;
 #pragma unroll
-    for (int t = 0; t < kSmStages - 1; ++t) {
-        issue_w(t);
+            for (int c = 0; c < kCopies; ++c) {
+                const bool ok = (cok >> c) & 1u;
+                sm_cp16(st + wdst0 + kDstStride * c, ok ? csrc + c * cstride + cs * kStepBytes : grp.bits[0], ok);
+            }
+            const bool sok = (cok >> kCopies) & 1u;
+            sm_cp4(st + sdst, sok ? cscale + 2 * cs : cscale, sok);
+        }
         sm_commit();
-    }
-    if (FMT == 1 && threadIdx.x < 16) {
-        const uint32_t v = threadIdx.x;
-        auto sg = [&](int j) -> uint32_t { return ((v >> j) & 1u) ? 0x3F80u : 0xBF80u; };
-        lut[threadIdx.x] = make_uint2(sg(0) | (sg(1) << 16), sg(2) | (sg(3) << 16));
-    }
-    pdl_wait_primary();  // x is produced, and y last read, by earlier kernels
+        cstage = cstage + 1 == kSgWStages ? 0 : cstage + 1;
+        if (++cs == q.nsteps) set_round(cj + 1);
+    };
+    set_round(0);
 #pragma unroll
-    for (int t = 0; t < kSmStages - 1; ++t) issue_x(t);
-    sm_commit();
+    for (int t = 0; t < kSgWStages - 1; ++t) issue_next();
+    pdl_wait_primary();  // y was last read by earlier kernels
 
     float yacc[2][NT][4];
 #pragma unroll
@@ -603,28 +964,28 @@ __global__ void __launch_bounds__(kSgMaxWarps * 32, 1) k_smallm_grp(const __grid
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) yacc[tt][nt][0] = yacc[tt][nt][1] = yacc[tt][nt][2] = yacc[tt][nt][3] = 0.f;
     const int g = lane >> 2, t4 = lane & 3;
+    int sl = 0, stage = 0, s = 0, j = 0;
+    unsigned phase = 0;
+    int b = blockIdx.x * nw + warp;  // block of round j
     for (int u = 0; u < total; ++u) {
-        // as in the single-matrix kernel: the prologue's groups at u = 0, then
-        // all but the newest group, and a CTA barrier (which also frees the
-        // slot of step u - 1)
-        if (u == 0)
-            sm_wait<0>();
-        else
-            sm_wait<kSmStages - 2>();
-        __syncthreads();
-        issue_w(u + kSmStages - 1);
-        issue_x(u + kSmStages - 1);
-        sm_commit();
-        const int j = u / q.nsteps, s = u - j * q.nsteps, b = blk_of(j);
+        issue_next();
+        if (!__all_sync(0xffffffffu, sg_wait(full + sl, phase))) break;
+        sm_wait<kSgWStages - 1>();  // this lane's copies of step u landed
+        __syncwarp();               // ... and every lane's
         if (b < q.nblocks) {
-            const uint8_t *st = wring + (u % kSmStages) * kSB;
-            const uint2 *xf = xr + (u % kSmStages) * kXFrags;
             if (FMT == 1)
-                sm_consume<NT>(st, xf, lut, lane, yacc);
+                sg_consume_q1<NT>(wring + stage * kSB, xring + sl * kXSlot, lane, mul, yacc);
             else
-                i4s_consume<NT>(st, xf, lane, yacc);
+                sg_consume_i4<NT>(wring + stage * kSB, xring + sl * kXSlot, lane, yacc);
         }
-        if (s == q.nsteps - 1) {
+        __syncwarp();  // every lane has read the slot and the stage
+        if (lane == 0) mbar_arrive(empty + sl);
+        if (++sl == kSgSlots) {
+            sl = 0;
+            phase ^= 1u;
+        }
+        stage = stage + 1 == kSgWStages ? 0 : stage + 1;
+        if (++s == q.nsteps) {
             if (b < q.nblocks) {
                 const int r = b / q.blocksN, blk = b - r * q.blocksN;
                 float *y = grp.y[r];
@@ -644,6 +1005,9 @@ __global__ void __launch_bounds__(kSgMaxWarps * 32, 1) k_smallm_grp(const __grid
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
                     yacc[tt][nt][0] = yacc[tt][nt][1] = yacc[tt][nt][2] = yacc[tt][nt][3] = 0.f;
+            s = 0;
+            ++j;
+            b += (int)gridDim.x * nw;
         }
     }
     sm_wait<0>();
@@ -655,7 +1019,7 @@ struct SgPlan {
     bool ok;
 };
 
-// Warps per CTA: as many as fit (<= kSgMaxWarps), then the count in
+// Consumer warps per CTA: as many as fit (<= kSgMaxWarps), then the count in
 // [kSgMinWarps, max] whose rounds come out fullest (ties: more warps).
 static SgPlan sg_plan(int fmt, int R, int M, int N, int K, int sms)
 {
@@ -666,9 +1030,10 @@ static SgPlan sg_plan(int fmt, int R, int M, int N, int K, int sms)
     P.nsteps = K / stepk;
     P.blocksN = (N + 31) / 32;
     P.nblocks = R * P.blocksN;
-    const size_t xring = (size_t)kSmStages * (stepk / 16) * P.NT * 32 * 8;
-    const size_t per_warp = (size_t)kSmStages * (fmt == 1 ? kSmStageBytes : kI4sStageBytes);
-    const int fit = (int)std::min<size_t>(kSgMaxWarps, ((size_t)kSmMaxSmem - xring) / per_warp);
+    const size_t xring = sg_raw_bytes(fmt, stepk, M) + sg_xring_bytes(fmt, stepk, P.NT);
+    const size_t per_warp = (size_t)kSgWStages * (fmt == 1 ? kSmStageBytes : kI4sStageBytes);
+    if (128 + xring + kSgMinWarps * per_warp > (size_t)kSmMaxSmem) return P;
+    const int fit = (int)std::min<size_t>(kSgMaxWarps, ((size_t)kSmMaxSmem - 128 - xring) / per_warp);
     double best = -1.0;
     for (int w = fit; w >= kSgMinWarps; --w) {
         if ((long long)P.nblocks < (long long)sms * w) continue;  // at least one full round
@@ -680,7 +1045,7 @@ static SgPlan sg_plan(int fmt, int R, int M, int N, int K, int sms)
             P.rounds = rounds;
         }
     }
-    P.smem = xring + (size_t)P.warps * per_warp;
+    P.smem = 128 /*alignment*/ + xring + (size_t)P.warps * per_warp;
     P.ok = P.warps >= kSgMinWarps;
     return P;
 }
@@ -701,8 +1066,21 @@ lowbit_status smg_launch(int fmt, const uint8_t *const *bits, const uint16_t *co
         grp.scales[r] = scales[r];
         grp.y[r] = y[r];
     }
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return LOWBIT_ERR_CUDA;
+    // x [M][K] bf16; one box = the M rows of one step of k (Q1_0_g128, into
+    // the raw ring) or of one step plus 16 (INT4_G64, the x ring's row
+    // stride), rows dense in shared memory; k past K reads as zero
+    CUtensorMap xmap;
+    const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)(fmt == 1 ? kSmStepK : sg_xrow(3, kI4sStepK) / 2), (cuuint32_t)M};
+    const cuuint32_t estride[2] = {1, 1};
+    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), gdim, gstride, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return LOWBIT_ERR_CUDA;
     SmGParams q = {};
-    q.x = x;
     q.M = M;
     q.N = N;
     q.K = K;
@@ -710,7 +1088,7 @@ lowbit_status smg_launch(int fmt, const uint8_t *const *bits, const uint16_t *co
     q.blocksN = P.blocksN;
     q.nblocks = P.nblocks;
     q.rounds = P.rounds;
-    void (*kern)(const SmGroup, const SmGParams);
+    void (*kern)(const SmGroup, const CUtensorMap, const SmGParams);
     if (fmt == 1)
         kern = P.NT == 1 ? k_smallm_grp<1, 1> : k_smallm_grp<1, 2>;
     else
@@ -722,7 +1100,7 @@ lowbit_status smg_launch(int fmt, const uint8_t *const *bits, const uint16_t *co
         return LOWBIT_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sms);
-    cfg.blockDim = dim3(P.warps * 32);
+    cfg.blockDim = dim3((P.warps + 1) * 32);
     cfg.dynamicSmemBytes = P.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -730,8 +1108,17 @@ lowbit_status smg_launch(int fmt, const uint8_t *const *bits, const uint16_t *co
     attr[0].val.programmaticStreamSerializationAllowed = LOWBIT_PDL;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, grp, q);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, grp, xmap, q);
     return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
+// Read and clear the fault flag of the current device.
+int smg_fault_flag()
+{
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_sg_fault, sizeof(v)) != cudaSuccess) return -1;
+    cudaMemcpyToSymbol(g_sg_fault, &zero, sizeof(zero));
+    return v != 0;
 }
 
 }  // namespace lowbit

@@ -40,6 +40,7 @@ lowbit_status q1stack_launch(const uint8_t *const *, const uint16_t *const *, in
                              uint16_t *, float *, cudaStream_t);
 size_t q1stack_workspace_bytes(int F);
 int q1stack_fault_flag();
+int smg_fault_flag();
 lowbit_status q1sm_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int, int, cudaStream_t);
 lowbit_status q1m1_gemv_fused_launch(const uint8_t *, const uint16_t *, const uint16_t *, float *, int, int,
                                      cudaStream_t);
@@ -105,9 +106,9 @@ int lowbit_version(void) { return 100; }
 
 int lowbit_fault_flags(void)
 {
-    const int f4 = i4tc_fault_flag(), fs = q1stack_fault_flag();
-    if (f4 < 0 || fs < 0) return -1;
-    return (f4 ? 1 : 0) | (fs ? 4 : 0);
+    const int f4 = i4tc_fault_flag(), fs = q1stack_fault_flag(), fg = smg_fault_flag();
+    if (f4 < 0 || fs < 0 || fg < 0) return -1;
+    return (f4 ? 1 : 0) | (fs ? 4 : 0) | (fg ? 8 : 0);
 }
 
 lowbit_status lowbit_pack(lowbit_format fmt, const int8_t *codes, int64_t rows, int64_t cols,

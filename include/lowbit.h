@@ -96,8 +96,10 @@ int lowbit_version(void);
 
 /* Faults the kernels of the current device recorded since the last call,
  * and clears them: 0 = none; bit 0 = a bounded wait inside the INT4_G64
- * tcgen05 GEMM ran out, bit 2 = a grid barrier of lowbit_q1g128_stack_step
- * (the results of that call are then not valid); -1 = the flags could not
+ * tcgen05 GEMM ran out, bit 2 = a grid barrier of lowbit_q1g128_stack_step,
+ * bit 3 = a wait on the shared activation ring of the grouped small-batch
+ * kernel (groups at M >= 2; the results of such a call are then not
+ * valid); -1 = the flags could not
  * be read.  This is a diagnostic call, not part of any product: it reads the
  * flags from device memory and therefore synchronises with the device (every
  * other entry point is asynchronous). */

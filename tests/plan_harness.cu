@@ -11,7 +11,8 @@
 //     of cells into per-CTA ranges and of steps into per-warp ranges, every
 //     warp's range is at least one cell long, so a cell cut between two
 //     warps has exactly two parts (the kernels combine exactly two);
-//   - the small-batch persistent kernel: its rounds cover every 32-row block
+//   - the small-batch persistent kernel: its consumer warps and the producer
+//     warp fit the launch bound, and its rounds cover every 32-row block
 //     exactly once.
 #include <cstdio>
 #include <vector>
@@ -112,6 +113,7 @@ int main()
                         const SgPlan G = sg_plan(fmt, R, M, N, K, kSms);
                         if (G.ok) {
                             CHECK(G.warps >= kSgMinWarps && G.warps <= kSgMaxWarps, "grouped smallm warps %d", G.warps);
+                            CHECK((G.warps + 1) * 32 <= kSgThreadsMax, "grouped smallm threads (%d warps)", G.warps);
                             CHECK(G.smem + 128 <= kCtaSmem && G.smem <= (size_t)kSmMaxSmem, "grouped smallm smem %zu",
                                   G.smem);
                             // round j, CTA b, warp w takes block (j*grid + b)*nw + w: all blocks, once
