@@ -113,7 +113,7 @@ int main()
                         const SgPlan G = sg_plan(fmt, R, M, N, K, kSms);
                         if (G.ok) {
                             CHECK(G.warps >= kSgMinWarps && G.warps <= kSgMaxWarps, "grouped smallm warps %d", G.warps);
-                            CHECK((G.warps + 1) * 32 <= kSgThreadsMax, "grouped smallm threads (%d warps)", G.warps);
+                            CHECK(G.warps <= sg_max_warps(fmt, G.NT), "grouped smallm warps %d above the launch bound", G.warps);
                             CHECK(G.smem + 128 <= kCtaSmem && G.smem <= (size_t)kSmMaxSmem, "grouped smallm smem %zu",
                                   G.smem);
                             // round j, CTA b, warp w takes block (j*grid + b)*nw + w: all blocks, once
