@@ -49,8 +49,9 @@
 // sets the fault word and the warp leaves its loop).
 //
 // Work split.  k_smallm: a CTA of four consumer warps takes 128 rows of one
-// K-slice; the S slices of a row block form a thread-block cluster and add
-// their partial sums in rank order through distributed shared memory.
+// K-slice of one of up to 8 matrices that read the same x; the S slices of a
+// row block form a thread-block cluster and add their partial sums in rank
+// order through distributed shared memory.
 // k_smallm_grp: one CTA per SM; every consumer warp owns one 32-row block
 // of one matrix over all of K per round, and the rounds walk the group's
 // (matrix, block) list; warps may drift apart by up to SLOTS steps.
@@ -582,18 +583,21 @@ constexpr int kSmMaxCluster = 8;
 // two for the INT4_G64 instances with three or four batch tiles (170)
 __host__ __device__ constexpr int sm_min_blocks(int fmt, int NT) { return fmt == 3 && NT >= 3 ? 2 : 3; }
 
+constexpr int kSmMaxR = 8;                  // matrices of one launch
+
 struct SmParams {
-    const uint8_t *bits;
-    const uint16_t *scales;
-    float *y;
+    const uint8_t *bits[kSmMaxR];
+    const uint16_t *scales[kSmMaxR];
+    float *y[kSmMaxR];
     int M, N, K;
     int nsteps;  // K / step
     int L;       // steps per K-slice
+    int blocks;  // 128-row blocks per matrix
 };
 
 template <int FMT, int NT>
 __global__ void __launch_bounds__(kSmThreads, sm_min_blocks(FMT, NT)) k_smallm(const __grid_constant__ CUtensorMap xmap,
-                                                                           const SmParams p)
+                                                                           const __grid_constant__ SmParams p)
 {
     constexpr int kSB = SgFmt<FMT>::kStageBytes;
     constexpr int kXSlot = 8 * NT * sg_xrow(FMT);
@@ -604,7 +608,10 @@ __global__ void __launch_bounds__(kSmThreads, sm_min_blocks(FMT, NT)) k_smallm(c
     uint64_t *full = bars, *empty = bars + kSmSlots;
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int slice = blockIdx.x, nsl = gridDim.x, rb = blockIdx.y;
+    const int slice = blockIdx.x, nsl = gridDim.x;
+    const int mat = blockIdx.y / p.blocks, rb = blockIdx.y - mat * p.blocks;
+    const uint8_t *bits = p.bits[mat];
+    float *yout = p.y[mat];
     const int s_lo = slice * p.L, s_hi = min(p.nsteps, s_lo + p.L);
     const int ns = max(0, s_hi - s_lo);  // steps of this CTA
     // x arrives by direct tensor copies (no raw ring): a CTA has few steps
@@ -626,10 +633,10 @@ __global__ void __launch_bounds__(kSmThreads, sm_min_blocks(FMT, NT)) k_smallm(c
 #pragma unroll
         for (int i = 0; i < 4; ++i) mul[i] = multab[lane & 3][i];
         SgCopy<FMT> cp;
-        if (rows) cp.set(p.bits, p.scales, blk, p.N, p.K, lane);
+        if (rows) cp.set(bits, p.scales[mat], blk, p.N, p.K, lane);
         int cs = 0, cstage = 0;  // next step to copy, its stage
         auto issue_next = [&]() {
-            if (rows && cs < ns) cp.issue(wr_s + cstage * kSB, s_lo + cs, p.bits);
+            if (rows && cs < ns) cp.issue(wr_s + cstage * kSB, s_lo + cs, bits);
             sm_commit();
             ++cs;
             cstage = cstage + 1 == kSmWStages ? 0 : cstage + 1;
@@ -683,7 +690,7 @@ __global__ void __launch_bounds__(kSmThreads, sm_min_blocks(FMT, NT)) k_smallm(c
         __syncthreads();
         for (int i = threadIdx.x; i < p.M * kSmRows; i += blockDim.x) {
             const int m = i / kSmRows, row = rb * kSmRows + (i - m * kSmRows);
-            if (row < p.N) p.y[(size_t)m * p.N + row] = part[i];
+            if (row < p.N) yout[(size_t)m * p.N + row] = part[i];
         }
         return;
     }
@@ -698,7 +705,7 @@ __global__ void __launch_bounds__(kSmThreads, sm_min_blocks(FMT, NT)) k_smallm(c
 #pragma unroll
         for (int q = 0; q < kSmMaxCluster; ++q) sum += v[q];
         const int m = i / kSmRows, row = rb * kSmRows + (i - m * kSmRows);
-        if (row < p.N) p.y[(size_t)m * p.N + row] = sum;
+        if (row < p.N) yout[(size_t)m * p.N + row] = sum;
     }
     sm_cluster_sync();  // peers keep their shared memory until every rank has read it
 }
@@ -709,15 +716,16 @@ struct SmPlan {
     bool ok;
 };
 
-// fmt: 1 = Q1_0_g128 (256 k per step), 3 = INT4_G64 (128 k per step)
-static SmPlan sm_plan(int fmt, int M, int N, int K, int sms)
+// fmt: 1 = Q1_0_g128 (256 k per step), 3 = INT4_G64 (128 k per step); R
+// matrices of one launch (blocks counts the row blocks of all of them)
+static SmPlan sm_plan(int fmt, int M, int N, int K, int sms, int R = 1)
 {
     SmPlan P = {};
     const int stepk = fmt == 1 ? kSmStepK : kI4sStepK, maxm = fmt == 1 ? kSmMaxM : kI4sMaxM;
     P.NT = (M + 7) / 8;
     P.nsteps = K / stepk;
-    P.blocks = (N + kSmRows - 1) / kSmRows;
-    if (M < 2 || M > maxm || N < 1 || K % stepk != 0 || P.nsteps < 1) return P;  // ok = false
+    P.blocks = (N + kSmRows - 1) / kSmRows * R;
+    if (M < 2 || M > maxm || N < 1 || K % stepk != 0 || P.nsteps < 1 || R < 1 || R > kSmMaxR) return P;
     const size_t ring = (size_t)kSmWarps * kSmWStages * (fmt == 1 ? kSmStageBytes : kI4sStageBytes);
     P.smem = 128 /*alignment*/ + sg_xring_bytes(fmt, kSmSlots, P.NT) + ring + (size_t)M * kSmRows * 4;
     // CTAs resident per SM (shared memory, with 1 KB reserved per CTA, and registers)
@@ -735,22 +743,26 @@ static SmPlan sm_plan(int fmt, int M, int N, int K, int sms)
 bool q1sm_supported(int M, int N, int K) { return sm_plan(1, M, N, K, sm_num_sms()).ok; }
 bool i4sm_supported(int M, int N, int K) { return sm_plan(3, M, N, K, sm_num_sms()).ok; }
 
-static lowbit_status sm_launch(int fmt, const uint8_t *bits, const uint16_t *scales, const uint16_t *x, float *y,
-                               int M, int N, int K, cudaStream_t st)
+// R <= kSmMaxR matrices of one shape that read one x, one launch
+static lowbit_status sm_launch(int fmt, const uint8_t *const *bits, const uint16_t *const *scales, const uint16_t *x,
+                               float *const *y, int R, int M, int N, int K, cudaStream_t st)
 {
-    const SmPlan P = sm_plan(fmt, M, N, K, sm_num_sms());
+    const SmPlan P = sm_plan(fmt, M, N, K, sm_num_sms(), R);
     if (!P.ok) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
     CUtensorMap xmap;
     if (!sg_xmap(&xmap, fmt, true, x, M, K)) return LOWBIT_ERR_CUDA;
     SmParams p = {};
-    p.bits = bits;
-    p.scales = scales;
-    p.y = y;
+    for (int r = 0; r < R; ++r) {
+        p.bits[r] = bits[r];
+        p.scales[r] = scales[r];
+        p.y[r] = y[r];
+    }
     p.M = M;
     p.N = N;
     p.K = K;
     p.nsteps = P.nsteps;
     p.L = P.L;
+    p.blocks = P.blocks / R;
     void (*kern)(const CUtensorMap, const SmParams);
     if (fmt == 1)
         kern = P.NT == 1 ? k_smallm<1, 1> : k_smallm<1, 2>;
@@ -779,13 +791,25 @@ static lowbit_status sm_launch(int fmt, const uint8_t *bits, const uint16_t *sca
 lowbit_status q1sm_launch(const uint8_t *bits, const uint16_t *scales, const uint16_t *x, float *y, int M, int N,
                           int K, cudaStream_t st)
 {
-    return sm_launch(1, bits, scales, x, y, M, N, K, st);
+    return sm_launch(1, &bits, &scales, x, &y, 1, M, N, K, st);
 }
 
 lowbit_status i4sm_launch(const uint8_t *q, const uint16_t *scales, const uint16_t *x, float *y, int M, int N, int K,
                           cudaStream_t st)
 {
-    return sm_launch(3, q, scales, x, y, M, N, K, st);
+    return sm_launch(3, &q, &scales, x, &y, 1, M, N, K, st);
+}
+
+// R matrices in launches of up to kSmMaxR
+lowbit_status smr_launch(int fmt, const uint8_t *const *bits, const uint16_t *const *scales, const uint16_t *x,
+                         float *const *y, int R, int M, int N, int K, cudaStream_t st)
+{
+    for (int r0 = 0; r0 < R; r0 += kSmMaxR) {
+        const lowbit_status s =
+            sm_launch(fmt, bits + r0, scales + r0, x, y + r0, std::min(kSmMaxR, R - r0), M, N, K, st);
+        if (s != LOWBIT_OK) return s;
+    }
+    return LOWBIT_OK;
 }
 
 // ---------------------------------------------------------------------------

@@ -48,6 +48,8 @@ bool q1m1_fused_supported(int N, int K);
 lowbit_status quantize_launch(int fmt, const float *w, int64_t rows, int64_t cols, uint8_t *packed, uint16_t *scales,
                               cudaStream_t st);
 bool smg_supported(int fmt, int R, int M, int N, int K);
+lowbit_status smr_launch(int fmt, const uint8_t *const *, const uint16_t *const *, const uint16_t *, float *const *,
+                         int R, int M, int N, int K, cudaStream_t);
 lowbit_status smg_launch(int fmt, const uint8_t *const *, const uint16_t *const *, const uint16_t *, float *const *,
                          int R, int M, int N, int K, cudaStream_t);
 bool i4m1_group_supported(int R, int N, int K);
@@ -272,7 +274,7 @@ size_t lowbit_q1g128_group_workspace_bytes(int R, int M, int N, int K)
 {
     if (R < 1 || q1_shape_ok(M, N, K) != LOWBIT_OK) return 0;
     if (q1m1_x_group_supported(R, M, N, K)) return 0;
-    if (M >= 2 && smg_supported(1, R, M, N, K)) return 0;
+    if (M >= 2 && (smg_supported(1, R, M, N, K) || q1sm_supported(M, N, K))) return 0;
     return al256(lowbit_q1g128_act_bytes(M, K)) + lowbit_q1g128_act_workspace_bytes(R, M, N, K);
 }
 
@@ -295,6 +297,8 @@ lowbit_status lowbit_q1g128_gemv_group(const uint8_t *const *w_bits, const uint1
     s = q1m1_gemv_x_group_launch(w_bits, w_scales, x, y, R, M, N, K, st);  // M <= 4: integer bit planes
     if (s != LOWBIT_ERR_UNSUPPORTED_SHAPE) return s;
     if (M >= 2 && smg_supported(1, R, M, N, K)) return smg_launch(1, w_bits, w_scales, x, y, R, M, N, K, st);
+    // too few row blocks for the persistent kernel: up to 8 matrices per split-K launch
+    if (M >= 2 && q1sm_supported(M, N, K)) return smr_launch(1, w_bits, w_scales, x, y, R, M, N, K, st);
     uint8_t *act = static_cast<uint8_t *>(workspace);
     const size_t act_bytes = al256(lowbit_q1g128_act_bytes(M, K));
     s = lowbit_q1g128_prepare_act(x, M, K, act, act_bytes, stream);
@@ -372,6 +376,8 @@ lowbit_status lowbit_int4g64_gemm_group(const uint8_t *const *w_q, const uint16_
     cudaStream_t st = as_stream(stream);
     if (M == 1 && i4m1_group_supported(R, N, K)) return i4m1_group_launch(w_q, w_scales, x, y, R, N, K, st);
     if (M >= 2 && smg_supported(3, R, M, N, K)) return smg_launch(3, w_q, w_scales, x, y, R, M, N, K, st);
+    if (M >= 2 && M <= kI4SmallMMax && i4sm_supported(M, N, K))
+        return smr_launch(3, w_q, w_scales, x, y, R, M, N, K, st);
     for (int r = 0; r < R; ++r) {
         const lowbit_status s = lowbit_int4g64_gemm(w_q[r], w_scales[r], x, y[r], M, N, K, stream);
         if (s != LOWBIT_OK) return s;

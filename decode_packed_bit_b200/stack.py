@@ -57,6 +57,8 @@ class Q1Stack:
         self.act = torch.empty(max(lb.lowbit_q1g128_act_bytes(M, hidden), 256), dtype=torch.uint8, device=dev)
         gws = lb.lowbit_q1g128_act_workspace_bytes(2, M, ffn, hidden)
         self.gws = torch.empty(max(gws, 256), dtype=torch.uint8, device=dev)
+        grp = lb.lowbit_q1g128_group_workspace_bytes(2, M, ffn, hidden)
+        self.grp_ws = torch.empty(grp, dtype=torch.uint8, device=dev) if grp else None
 
     @property
     def bytes_per_step(self) -> int:
@@ -67,9 +69,10 @@ class Q1Stack:
         return total
 
     def launches_per_step(self) -> int:
-        # per layer: 5 one-shot products (prepare + product), 1 prepare + 1
-        # grouped product for gate/up, 6 normalisations
-        per = 5 * 2 + 2 + 6 if self.M == 1 else 7 + 6
+        # per layer, M = 1: 5 one-shot products (prepare + product), 1 prepare
+        # + 1 grouped product for gate/up, 6 normalisations; M > 1: 5 products,
+        # 1 grouped product for gate/up, 6 normalisations
+        per = 5 * 2 + 2 + 6 if self.M == 1 else 6 + 6
         return per * len(self.layers)
 
     def fused_supported(self) -> bool:
@@ -137,8 +140,8 @@ class Q1Stack:
                 lb.lowbit_q1g128_gemv_act_group([gb, ub], [gs, us], self.act, [self.tg, self.tu], M,
                                                 workspace=self.gws, stream=stream)
             else:
-                lb.lowbit_q1g128_gemv(gb, gs, src, self.tg, workspace=self.ws, stream=stream)
-                lb.lowbit_q1g128_gemv(ub, us, src, self.tu, workspace=self.ws, stream=stream)
+                lb.lowbit_q1g128_gemv_group([gb, ub], [gs, us], src, [self.tg, self.tu],
+                                            workspace=self.grp_ws, stream=stream)
             if record is not None and (record.want(li, "gate") or record.want(li, "up")):
                 record.outputs[(li, "gate")] = self.tg.clone()
                 record.outputs[(li, "up")] = self.tu.clone()

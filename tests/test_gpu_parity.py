@@ -265,14 +265,17 @@ def test_q1_large_group(lb, R, N, K, xkind):
 @pytest.mark.parametrize("R,M,N,K", [(40, 1, 4096, 1024), (38, 1, 4096, 17408), (160, 1, 1024, 3072),
                                      (40, 4, 4096, 1024), (40, 2, 4096, 2048), (30, 3, 4096, 1024),
                                      (12, 16, 5120, 5120), (40, 9, 1000, 2048),
-                                     (3, 1, 515, 1280), (2, 2, 300, 2048)])
+                                     (3, 1, 515, 1280), (2, 2, 300, 2048), (10, 8, 256, 1024),
+                                     (3, 13, 1100, 512)])
 def test_q1_group_from_x(lb, R, M, N, K):
     """lowbit_q1g128_gemv_group: one launch when the shape allows (the first
     eight cases on 148 SMs: the persistent bit-plane kernel for M = 1, 4, 2
-    and 3 (four vectors, one of them zero), then the small-batch bf16 kernel
-    with ragged rows and a partial batch tile), else prepare + group product
-    in the workspace.  Sampled outputs of three
-    matrices against the oracle."""
+    and 3 (four vectors, one of them zero), then the persistent small-batch
+    bf16 kernel with ragged rows and a partial batch tile); groups with too
+    few row blocks for it at M >= 2 run the split-K kernel, up to 8 matrices
+    per launch (the last three cases: 2, 8 + 2 and 3 matrices, ragged rows);
+    M = 1 otherwise: prepare + group product in the workspace.  Sampled
+    outputs of three matrices against the oracle."""
     x = synth.bf16_normal(2800 + R, (M, K))
     g = torch.Generator(device="cuda")
     g.manual_seed(2800 + R)
@@ -392,11 +395,14 @@ def test_int4_11008x4096_sampled(lb, M):
 
 @pytest.mark.parametrize("R,M,N,K", [(17, 1, 11008, 4096), (80, 1, 1024, 1024), (7, 1, 11008, 11008),
                                      (17, 32, 11008, 4096), (40, 5, 1000, 1024), (10, 17, 4096, 512),
-                                     (40, 1, 1024, 1024), (3, 32, 300, 512), (2, 1, 300, 448)])
+                                     (40, 1, 1024, 1024), (3, 32, 300, 512), (2, 1, 300, 448),
+                                     (10, 8, 256, 512), (9, 24, 1000, 256)])
 def test_int4_group(lb, R, M, N, K):
     """lowbit_int4g64_gemm_group: the persistent kernels for the first six
     cases on 148 SMs (M = 1, then small batches with ragged rows and partial
-    batch tiles), single calls for the rest.  Sampled outputs of three
+    batch tiles); at 2 <= M <= 32 groups with too few row blocks run the
+    split-K kernel, up to 8 matrices per launch (3, 8 + 2 and 8 + 1 matrices
+    here); single calls for the rest.  Sampled outputs of three
     matrices against the oracle, and the group equals single calls up to fp32
     summation order."""
     x = synth.bf16_normal(4800 + R, (M, K))
