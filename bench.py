@@ -494,30 +494,68 @@ def run_q1_4096(args, world, rank, local):
 
     # end to end through the C ABI with host buffers: per call, x in from
     # pinned host memory and all outputs back to pinned host memory, inside
-    # the timed region
+    # the timed region.  One GPU: two buffer sets, so that the outputs of
+    # call i travel to the host on a second stream while call i+1 runs (each
+    # call waits for the copy that last read its buffer set).  Several ranks:
+    # one call at a time (the all-gather owns the output buffer).
     x_host = x.cpu().pin_memory()
-    y_host = torch.empty(out_host_shape, dtype=torch.float32).pin_memory()
+    e2e_calls = 200
+    if world == 1:
+        x2 = torch.empty_like(x)
+        y2 = torch.empty_like(y)
+        ys2 = [y2[r] for r in range(R)]
 
-    def e2e_call():
-        x.copy_(x_host, non_blocking=True)
-        graph.replay()
-        if gather is not None:
-            gather()
-        y_host.copy_(out_dev.view(out_host_shape), non_blocking=True)
+        def launch2():
+            lb.lowbit_q1g128_gemv_group(bits, scales, x2, ys2, workspace=ws, stream=stream)
+        graph2 = _capture(launch2, stream)
+        sets = [(graph, x, y), (graph2, x2, y2)]
+        hosts = [torch.empty(out_host_shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+        y_host = hosts[0]
+        copy_stream = torch.cuda.Stream(device=dev)
+        done = [torch.cuda.Event() for _ in range(2)]
+        copied = [torch.cuda.Event() for _ in range(2)]
 
-    for _ in range(3):
-        with torch.cuda.stream(stream):
-            e2e_call()
-        stream.synchronize()
+        def e2e_run(n):
+            for i in range(n):
+                b = i % 2
+                g_b, x_b, y_b = sets[b]
+                with torch.cuda.stream(stream):
+                    if i >= 2:
+                        stream.wait_event(copied[b])
+                    x_b.copy_(x_host, non_blocking=True)
+                    g_b.replay()
+                    done[b].record(stream)
+                with torch.cuda.stream(copy_stream):
+                    copy_stream.wait_event(done[b])
+                    hosts[b].copy_(y_b.view(out_host_shape), non_blocking=True)
+                    copied[b].record(copy_stream)
+            stream.wait_event(copied[(n - 1) % 2])
+            if n >= 2:
+                stream.wait_event(copied[(n - 2) % 2])
+        e2e_note = ("x in from pinned host, all outputs out, every call; two buffer sets: the outputs of "
+                    "one call copy out on a second stream during the next call")
+    else:
+        y_host = torch.empty(out_host_shape, dtype=torch.float32).pin_memory()
+
+        def e2e_run(n):
+            with torch.cuda.stream(stream):
+                for _ in range(n):
+                    x.copy_(x_host, non_blocking=True)
+                    graph.replay()
+                    gather()
+                    y_host.copy_(out_dev.view(out_host_shape), non_blocking=True)
+        e2e_note = "one grouped call per step: x in from pinned host, all outputs out"
+
+    e2e_run(3)
+    stream.synchronize()
     barrier(world)
     torch.cuda.synchronize(dev)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    e2e_calls = 200
     with torch.cuda.stream(stream):
         t0.record(stream)
-        for _ in range(e2e_calls):
-            e2e_call()
+    e2e_run(e2e_calls)
+    with torch.cuda.stream(stream):
         t1.record(stream)
     t1.synchronize()
     barrier(world)
@@ -568,7 +606,7 @@ def run_q1_4096(args, world, rank, local):
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
-                "note": "one grouped call per step: x in from pinned host, all outputs out"},
+                "note": e2e_note},
         "single_call": single,
         "burst": burst,
         "gpu_launches": calls_per_launch * launches,

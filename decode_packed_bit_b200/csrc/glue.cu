@@ -1,7 +1,13 @@
 // glue.cu -- the normalisation step between consecutive projections of a
 // layer stack: out = bf16_rne(v / sqrt(mean(v^2) + eps)), v = a (+ b), fp32.
-// One CTA per row; the row is read twice (sum of squares, then scale), which
-// costs nothing next to the weight stream of the projections around it.
+//
+// A row is spread over a cluster of kNormCluster CTAs, which keep their part
+// of v in registers: each CTA sums its squares (thread, then warp and CTA
+// trees), the cluster adds the kNormCluster partial sums in rank order
+// through distributed shared memory (every CTA the same way, so the result
+// does not depend on timing), and each CTA scales and rounds its part.
+// Rows too long for the registers take the one-CTA kernel, which reads the
+// row twice.
 #include "common.cuh"
 
 namespace lowbit {
@@ -55,10 +61,111 @@ __global__ void __launch_bounds__(kNormThreads) k_rmsnorm_bf16(const float *__re
     }
 }
 
+constexpr int kNormCluster = 8;
+constexpr int kNormCThreads = 256;
+constexpr int kNormPer = 8;  // float4 of v per thread at most
+constexpr int kNormMaxD = 4 * kNormPer * kNormCThreads * kNormCluster;
+
+__device__ __forceinline__ float norm_ld_peer(const float *local, unsigned rank)
+{
+    unsigned ra;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"((unsigned)__cvta_generic_to_shared(local)),
+                 "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void norm_cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// grid (kNormCluster, M), cluster (kNormCluster, 1, 1): CTA q of a row takes
+// its float4 range [q n4 / C, (q+1) n4 / C)
+__global__ void __launch_bounds__(kNormCThreads) k_rmsnorm_bf16_cl(const float *__restrict__ a,
+                                                                   const float *__restrict__ b, int D, float eps,
+                                                                   uint16_t *__restrict__ out)
+{
+    __shared__ float red[kNormCThreads / 32];
+    __shared__ float part;
+    pdl_launch_dependents();
+    pdl_wait_primary();
+    const unsigned q = blockIdx.x;
+    const int64_t row = blockIdx.y;
+    const int n4 = D / 4, lo = (int)((int64_t)q * n4 / kNormCluster), hi = (int)((int64_t)(q + 1) * n4 / kNormCluster);
+    const float4 *a4 = reinterpret_cast<const float4 *>(a + row * D);
+    const float4 *b4 = b ? reinterpret_cast<const float4 *>(b + row * D) : nullptr;
+    float4 v[kNormPer];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < kNormPer; ++j) {
+        const int i = lo + (int)threadIdx.x + j * kNormCThreads;
+        v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < hi) {
+            v[j] = a4[i];
+            if (b4) {
+                const float4 w = b4[i];
+                v[j].x += w.x; v[j].y += w.y; v[j].z += w.z; v[j].w += w.w;
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kNormPer; ++j) {
+        ss = fmaf(v[j].x, v[j].x, ss);
+        ss = fmaf(v[j].y, v[j].y, ss);
+        ss = fmaf(v[j].z, v[j].z, ss);
+        ss = fmaf(v[j].w, v[j].w, ss);
+    }
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float t = threadIdx.x < kNormCThreads / 32 ? red[threadIdx.x] : 0.f;
+        t = warp_sum(t);
+        if (threadIdx.x == 0) part = t;
+    }
+    norm_cluster_sync();  // every CTA's partial sum is in its shared memory
+    float tot = 0.f;
+#pragma unroll
+    for (int r = 0; r < kNormCluster; ++r) tot += norm_ld_peer(&part, (unsigned)r);
+    const float inv = 1.0f / sqrtf(tot / (float)D + eps);
+    uint2 *o = reinterpret_cast<uint2 *>(out + row * D);
+#pragma unroll
+    for (int j = 0; j < kNormPer; ++j) {
+        const int i = lo + (int)threadIdx.x + j * kNormCThreads;
+        if (i < hi) {
+            const uint32_t l = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[j].x * inv)) |
+                               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[j].y * inv)) << 16);
+            const uint32_t h = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[j].z * inv)) |
+                               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[j].w * inv)) << 16);
+            o[i] = make_uint2(l, h);
+        }
+    }
+    norm_cluster_sync();  // peers keep their shared memory until every CTA has read it
+}
+
 lowbit_status rmsnorm_launch(const float *a, const float *b, int M, int D, float eps, uint16_t *out,
                              cudaStream_t st)
 {
-    cudaError_t e = launch_pdl(k_rmsnorm_bf16, dim3(M), dim3(kNormThreads), 0, st, a, b, D, eps, out);
+    if (D > kNormMaxD || M > 65535) {
+        cudaError_t e = launch_pdl(k_rmsnorm_bf16, dim3(M), dim3(kNormThreads), 0, st, a, b, D, eps, out);
+        return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kNormCluster, M);
+    cfg.blockDim = dim3(kNormCThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = LOWBIT_PDL;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = kNormCluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_rmsnorm_bf16_cl, a, b, D, eps, out);
     return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
 
