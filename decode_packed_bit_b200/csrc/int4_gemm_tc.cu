@@ -21,12 +21,15 @@
 // 136 from both halves (bf16x2, exact) leaves q.
 //
 // CTA tile: 128 weight rows (the MMA's M) x BM batch rows (its N, <= 256),
-// K in steps of one 64-k group, three shared-memory stages, two TMEM
-// accumulators of BM columns:
+// one of S slices of K (whole 64-k groups) when there are too few tiles to
+// fill the SMs (S picked to minimise waves x groups per CTA; the slices add
+// their sums into y, zeroed first, with fp32 reductions), in steps of one
+// group, three shared-memory stages, two TMEM accumulators of BM columns:
 //   warps 0-7  dequantise a stage's packed weights into the A tile (K-major,
 //              128-byte swizzle), then drain the finished group's TMEM buffer
 //              (warp w reads TMEM lanes 32 (w % 4).., columns of half w / 4)
-//              and keep the scaled sums in registers; at the end they store y;
+//              and keep the scaled sums in registers; at the end they store
+//              (one slice) or add (several) them to y;
 //   warp 8     loads the x tile of a stage with TMA (128-byte swizzle);
 //   warp 9     allocates TMEM, and one of its lanes issues a group's four
 //              K = 16 MMAs and commits them to the stage's "empty" barrier
@@ -98,6 +101,10 @@ __device__ __forceinline__ uint4 q8_to_bf16(uint32_t word)
 // read 16 at a time, LOWBIT_I4TC_DRAIN loads in flight before each wait
 // (fewer live registers than one 32-column load next to the 128
 // accumulators), and acc += d * D.
+// fixed cost of a wave of CTAs, in groups, for the choice of K slices
+#ifndef LOWBIT_I4TC_SLICE_COST
+#define LOWBIT_I4TC_SLICE_COST 8
+#endif
 #ifndef LOWBIT_I4TC_DRAIN
 #define LOWBIT_I4TC_DRAIN 2
 #endif
@@ -150,7 +157,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kTcBN, m0 = blockIdx.y * BM;
-    const int ngroups = K / kTcBK;
+    // this CTA's groups [g0, g0 + ngroups) of K: slice blockIdx.z of gridDim.z
+    const int gall = K / kTcBK;
+    const int g0 = gall * blockIdx.z / gridDim.z, ngroups = gall * (blockIdx.z + 1) / gridDim.z - g0;
+    const bool sliced = gridDim.z > 1;
     pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
@@ -178,10 +188,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
         const int t = threadIdx.x, r = t >> 1, hf = t & 1;
         const int n = n0 + r;
         const bool valid = n < N;
-        const uint8_t *qrow = q + (size_t)(valid ? n : 0) * (K / 2) + hf * 16;
+        const uint8_t *qrow = q + (size_t)(valid ? n : 0) * (K / 2) + (size_t)g0 * 32 + hf * 16;
         const int quarter = warp & 3, half = warp >> 2;
         const int ne = n0 + quarter * 32 + lane;            // this thread's output row in the epilogue
-        const uint16_t *srow = scales + (size_t)(ne < N ? ne : 0) * (K / 64);
+        const uint16_t *srow = scales + (size_t)(ne < N ? ne : 0) * (K / 64) + g0;
         const uint32_t tlane = (uint32_t)(quarter * 32) << 16;
         float acc[128];
 #pragma unroll
@@ -242,10 +252,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         pdl_wait_primary();  // y may still be read by an earlier kernel
         if (ok && ne < N) {
+            if (sliced) {
 #pragma unroll
-            for (int i = 0; i < 32 * NCH; ++i) {
-                const int m = m0 + half * (BM / 2) + i;
-                if (m < M) y[(size_t)m * N + ne] = acc[i];
+                for (int i = 0; i < 32 * NCH; ++i) {
+                    const int m = m0 + half * (BM / 2) + i;
+                    if (m < M) atomicAdd(y + (size_t)m * N + ne, acc[i]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32 * NCH; ++i) {
+                    const int m = m0 + half * (BM / 2) + i;
+                    if (m < M) y[(size_t)m * N + ne] = acc[i];
+                }
             }
         }
     } else if (warp == kTcTmaWarp) {
@@ -256,7 +274,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
                 const int s = it % kTcStages, j = it / kTcStages;
                 if (it >= kTcStages && !mbar_wait(empty + s, (j - 1) & 1, &g_tc_fault)) break;
                 mbar_arrive_expect_tx(full_b + s, (unsigned)(BM * kTcBK * 2));
-                tma_load_2d(smem + s * kTcStageBytes + kTcATile, &tmap_x, it * kTcBK, m0, full_b + s);
+                tma_load_2d(smem + s * kTcStageBytes + kTcATile, &tmap_x, (g0 + it) * kTcBK, m0, full_b + s);
                 ++issued;
             }
             // the copies still in flight land before the CTA may exit (they
@@ -336,7 +354,24 @@ lowbit_status i4tc_launch(const uint8_t *q, const uint16_t *scales, const uint16
         BM == 64 ? k_i4_tc_gemm<1> : BM == 128 ? k_i4_tc_gemm<2> : BM == 192 ? k_i4_tc_gemm<3> : k_i4_tc_gemm<4>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
-    dim3 grid((N + kTcBN - 1) / kTcBN, (M + BM - 1) / BM);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int tiles = ((N + kTcBN - 1) / kTcBN) * ((M + BM - 1) / BM), gall = K / kTcBK;
+    // K slices: fewest waves x groups per CTA, plus a fixed cost of about
+    // kTcSliceCost groups per wave (setup, pipeline fill, the final stores)
+    constexpr int kTcMaxSlices = 8, kTcSliceCost = LOWBIT_I4TC_SLICE_COST;
+    int S = 1;
+    long long best = -1;
+    for (int c = 1; c <= std::min(kTcMaxSlices, gall); ++c) {
+        const long long waves = ((long long)tiles * c + sms - 1) / sms;
+        const long long cost = waves * ((gall + c - 1) / c + kTcSliceCost);
+        if (best < 0 || cost < best) {
+            best = cost;
+            S = c;
+        }
+    }
+    if (S > 1 && cudaMemsetAsync(y, 0, (size_t)M * N * sizeof(float), st) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    dim3 grid((N + kTcBN - 1) / kTcBN, (M + BM - 1) / BM, S);
     cudaError_t e = launch_pdl(kern, grid, dim3(kTcThreads), kTcSmemBytes, st, map, q, scales, y, M, N, K);
     return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
