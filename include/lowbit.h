@@ -97,9 +97,9 @@ int lowbit_version(void);
 /* Faults the kernels of the current device recorded since the last call,
  * and clears them: 0 = none; bit 0 = a bounded wait inside the INT4_G64
  * tcgen05 GEMM ran out, bit 2 = a grid barrier of lowbit_q1g128_stack_step,
- * bit 3 = a wait on the shared activation ring of the grouped small-batch
- * kernel (groups at M >= 2; the results of such a call are then not
- * valid); -1 = the flags could not
+ * bit 3 = a wait on the shared activation ring of a small-batch kernel
+ * (Q1_0_g128 at 2 <= M <= 16, INT4_G64 at 2 <= M <= 32; the results of such
+ * a call are then not valid); -1 = the flags could not
  * be read.  This is a diagnostic call, not part of any product: it reads the
  * flags from device memory and therefore synchronises with the device (every
  * other entry point is asynchronous). */
@@ -215,8 +215,9 @@ lowbit_status lowbit_q1g128_gemv_act_group(const uint8_t *const *w_bits,
  * K up to about 12k at M = 3, 4).  At 2 <= M <= 16 otherwise, with
  * K % 256 == 0 and at least SMs * 8 32-row blocks over the group, it is one
  * launch of a persistent bf16 kernel (each warp owns a 32-row block over all
- * of K; the warps of a CTA share x).  Other shapes prepare the activation in
- * the workspace and run lowbit_q1g128_gemv_act_group.
+ * of K; the warps of a CTA share x); with fewer blocks, one split-K launch
+ * per 8 matrices.  Neither needs a workspace.  Other shapes (M = 1) prepare
+ * the activation in the workspace and run lowbit_q1g128_gemv_act_group.
  * Workspace: lowbit_q1g128_group_workspace_bytes(R, M, N, K) bytes (NULL
  * allowed when 0).  Calls that share a workspace must be ordered on one
  * stream. */
@@ -298,9 +299,11 @@ lowbit_status lowbit_q1g128_stack_step(const uint8_t *const *w_bits, const uint1
  * (mma.sync on the packed nibbles, integer limbs of x); for 2 <= M <= 32
  * (K % 128 == 0) mma.sync on bf16 operands, q exact in bf16 and the group
  * scale applied once per group; above that a tcgen05 GEMM that dequantises
- * each weight tile into shared memory as two exact bf16 halves (hi + lo =
- * q*d) and accumulates in TMEM; other shapes a CUDA-core kernel.  Every
- * kernel builds its operands in shared memory: no workspace.
+ * each weight tile into shared memory as exact bf16 integers q, accumulates
+ * each 64-k group in TMEM and applies the group scale in fp32 (with few
+ * 128-row tiles, K is cut into slices whose sums are added into y, which the
+ * call zeroes first with a memset on the stream); other shapes a CUDA-core
+ * kernel.  Every kernel builds its operands on chip: no workspace.
  * ------------------------------------------------------------------------- */
 lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales,
                                   const uint16_t *x, float *y, int M, int N, int K,
@@ -314,8 +317,9 @@ lowbit_status lowbit_int4g64_gemm(const uint8_t *w_q, const uint16_t *w_scales,
  * builds the activation from x and streams its equal share of every matrix's
  * weights.  At 2 <= M <= 32 with K % 128 == 0 and at least SMs * 8 32-row
  * blocks over the group, one launch of the persistent small-batch kernel
- * (as for Q1_0_g128).  Other shapes run lowbit_int4g64_gemm once per matrix.  Results
- * equal the single calls up to fp32 summation order. */
+ * (as for Q1_0_g128); with fewer blocks, one split-K launch per 8 matrices.
+ * Other shapes run lowbit_int4g64_gemm once per matrix.  Results equal the
+ * single calls up to fp32 summation order. */
 lowbit_status lowbit_int4g64_gemm_group(const uint8_t *const *w_q,
                                         const uint16_t *const *w_scales, const uint16_t *x,
                                         float *const *y, int R, int M, int N, int K,
