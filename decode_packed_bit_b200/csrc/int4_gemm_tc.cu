@@ -228,16 +228,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_i4_tc_gemm(const __grid_const
             return true;
         };
         for (int it = 0; it < kTcPf; ++it) prefetch(it);
-        // rows past N dequantise nibble 8 (q = 0): zero weights
+        // rows past N dequantise nibble 8 (q = -8); their outputs are not stored
         for (int it = 0; it < kTcStages - 1 && it < ngroups && ok; ++it) ok = produce(it);
-        float dnext = ne < N ? f16_bits_to_float(__ldg(srow)) : 0.f;
+        // the raw fp16 scales of the next two groups, converted only when used
+        // (converting right after the load would wait out its latency)
+        uint16_t d0 = ne < N ? __ldg(srow) : (uint16_t)0, d1 = ne < N && 1 < ngroups ? __ldg(srow + 1) : (uint16_t)0;
         for (int g = 0; g < ngroups && ok; ++g) {
             if (g + kTcStages - 1 < ngroups && !produce(g + kTcStages - 1)) {
                 ok = false;
                 break;
             }
-            const float d = dnext;
-            if (g + 1 < ngroups && ne < N) dnext = f16_bits_to_float(__ldg(srow + g + 1));
+            const uint16_t dbits = d0;
+            d0 = d1;
+            d1 = g + 2 < ngroups && ne < N ? __ldg(srow + g + 2) : (uint16_t)0;
+            const float d = f16_bits_to_float(dbits);
             const int b = g & 1;
             if (!mbar_wait_warp(tfull + b, (g >> 1) & 1, &g_tc_fault)) {
                 ok = false;
