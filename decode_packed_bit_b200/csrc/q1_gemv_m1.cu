@@ -1293,45 +1293,69 @@ struct StIt {
     int p, j, t;
 };
 
-// Block of unit j of warp `warp` of CTA `c` in phase q, or -1.
-__device__ __forceinline__ int st_block(const StPhase &q, int G, int c, int warp, int j)
+// This CTA's K slice s, its rank rk among the CTAs of that slice and their
+// count cps, for inputs of width H (index 0) and F (index 1): fixed for the
+// launch, so computed once (divisions by a run-time count are long chains
+// of dependent integer instructions).
+struct StCta {
+    int s[2], rk[2], cps[2];
+};
+
+__device__ __forceinline__ StCta st_cta(const StackP &p, int G, int c)
 {
-    const int S = q.K / kStSliceK;
-    const int s = c % S, rk = c / S;
-    const int cps = (G - 1 - s) / S + 1;  // CTAs that work on slice s
-    const int b = rk + cps * (warp + j * kStWarps);
+    StCta t;
+    const int Ks[2] = {p.H, p.F};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int S = Ks[i] / kStSliceK;
+        t.s[i] = c % S;
+        t.rk[i] = c / S;
+        t.cps[i] = (G - 1 - t.s[i]) / S + 1;  // CTAs that work on slice s
+    }
+    return t;
+}
+
+// Block of unit j of warp `warp` in phase q, or -1.
+__device__ __forceinline__ int st_block(const StPhase &q, const StCta &ct, int warp, int j)
+{
+    const int f = q.ph == 5;  // down reads the ffn-wide vector
+    const int b = ct.rk[f] + ct.cps[f] * (warp + j * kStWarps);
     return b < q.nblocks ? b : -1;
 }
 
 // Move to the next step that exists (or past the last phase).
-__device__ __forceinline__ void st_next(StIt &it, const StackP &p, int G, int c, int warp, int nph)
+__device__ __forceinline__ void st_next(StIt &it, const StackP &p, const StCta &ct, int warp, int nph)
 {
     if (++it.t < kStSliceChunks / kQ1StepChunks) return;
     it.t = 0;
     ++it.j;
-    while (it.p < nph && st_block(st_phase(p, it.p), G, c, warp, it.j) < 0) {
+    while (it.p < nph && st_block(st_phase(p, it.p), ct, warp, it.j) < 0) {
         ++it.p;
         it.j = 0;
     }
 }
 
-__device__ __forceinline__ void st_first(StIt &it, const StackP &p, int G, int c, int warp, int nph)
+__device__ __forceinline__ void st_first(StIt &it, const StackP &p, const StCta &ct, int warp, int nph)
 {
     it.p = 0;
     it.j = 0;
     it.t = 0;
-    while (it.p < nph && st_block(st_phase(p, it.p), G, c, warp, 0) < 0) ++it.p;
+    while (it.p < nph && st_block(st_phase(p, it.p), ct, warp, 0) < 0) ++it.p;
 }
 
-// Copy one step: 32 rows x 2 chunks of one matrix (all rows and chunks exist).
-__device__ __forceinline__ void st_issue(unsigned stage, const StackW &W, const StackP &p, const StIt &it, int G,
-                                         int c, int warp, int lane)
+// Copy one step: 32 rows x 2 chunks of one matrix (all rows and chunks
+// exist).  W: the projections' pointers, copied to shared memory at the
+// start (a run-time index into the parameter block is a constant-cache
+// load that can miss).
+__device__ __forceinline__ void st_issue(unsigned stage, const StackW &W, const StackP &p, const StIt &it,
+                                         const StCta &ct, int warp, int lane)
 {
     const StPhase q = st_phase(p, it.p);
-    const int b = st_block(q, G, c, warp, it.j);
-    const int mat = b / (q.N / 32), row0 = (b % (q.N / 32)) * 32;
+    const int b = st_block(q, ct, warp, it.j);
+    const int nb = q.N / 32;  // blocks per matrix (a power-of-two division)
+    const int mat = b >= nb ? 1 : 0, row0 = (b - mat * nb) * 32;
     const int pi = st_proj(q, mat);
-    const int ch0 = (c % (q.K / kStSliceK)) * kStSliceChunks + it.t * kQ1StepChunks;
+    const int ch0 = ct.s[q.ph == 5] * kStSliceChunks + it.t * kQ1StepChunks;
     const int rowbytes = q.K >> 3, G16 = q.K >> 7;
     const int col = lane & 3;
     const uint8_t *bsrc = W.bits[pi] + (size_t)(row0 + (lane >> 2)) * rowbytes + ch0 * 32 + col * 16;
@@ -1406,6 +1430,12 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
 {
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ float red[kStWarps];
+    __shared__ StackW Ws;  // the projections' pointers
+    for (int i = threadIdx.x; i < 7 * p.L; i += blockDim.x) {
+        Ws.bits[i] = W.bits[i];
+        Ws.scales[i] = W.scales[i];
+    }
+    __syncthreads();
     uint8_t *frag = smem;                                                  // 4 chunks of fragments
     float2 *info = reinterpret_cast<float2 *>(smem + kStSliceChunks * kQ1FragBytesPerChunk);
     uint8_t *zero = smem + kStSliceChunks * (kQ1FragBytesPerChunk + kQ1InfoBytesPerChunk);
@@ -1421,14 +1451,15 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
     uint8_t *ring = rings + warp * kStStages * kQ1StageBytes;
     const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
 
-    for (int ph = 0; ph < kStPrefetchAhead; ++ph) st_prefetch_l2(W, p, ph, G, c);
+    for (int ph = 0; ph < kStPrefetchAhead; ++ph) st_prefetch_l2(Ws, p, ph, G, c);
+    const StCta ct = st_cta(p, G, c);
     StIt is;  // issue position (runs up to kStStages - 1 steps ahead)
-    st_first(is, p, G, c, warp, nph);
+    st_first(is, p, ct, warp, nph);
     int nis = 0;
     auto issue_next = [&]() {
         if (is.p < nph) {
-            st_issue(ring_s + (nis % kStStages) * kQ1StageBytes, W, p, is, G, c, warp, lane);
-            st_next(is, p, G, c, warp, nph);
+            st_issue(ring_s + (nis % kStStages) * kQ1StageBytes, Ws, p, is, ct, warp, lane);
+            st_next(is, p, ct, warp, nph);
         }
         ++nis;
         cp_async_commit();
@@ -1440,11 +1471,11 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
     clear_zero_block(zero);  // ordered before its first read by the phase's barriers
     const LaneConst lc = lane_const(lane);
     StIt cs;  // consume position
-    st_first(cs, p, G, c, warp, nph);
+    st_first(cs, p, ct, warp, nph);
     int ncs = 0;
 
     for (int ph_idx = 0; ph_idx <= nph; ++ph_idx) {
-        st_prefetch_l2(W, p, ph_idx + kStPrefetchAhead, G, c);
+        st_prefetch_l2(Ws, p, ph_idx + kStPrefetchAhead, G, c);
         // ---- input of this phase: normalise the previous output (or take x) ----
         const bool last = ph_idx == nph;
         const StPhase q = st_phase(p, last ? nph - 1 : ph_idx);
@@ -1454,7 +1485,7 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
         // the gate+up phase adds both into one vector
         const bool two = !last && q.ph == 5 && p.rec_out != nullptr;
         float inv = 1.f;
-        const int S = q.K / kStSliceK, s = c % S;
+        const int S = q.K / kStSliceK, s = ct.s[q.ph == 5];
         if (prev != nullptr) {
             // sum of squares of the whole input, 16 loads in flight per thread;
             // this CTA's slice is kept on the way (raw, scaled once inv is known)
@@ -1537,7 +1568,7 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
         const float2 *sinfo = info + lc.tq;
         while (cs.p == ph_idx) {
             float yacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-            const int b = st_block(q, G, c, warp, cs.j);
+            const int b = st_block(q, ct, warp, cs.j);
             for (int t = 0; t < kStSliceChunks / kQ1StepChunks; ++t) {
                 issue_next();
                 cp_async_wait<kStStages - 1>();
@@ -1547,7 +1578,7 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
                              sinfo + 4 * lch, kQ1StepChunks, lc, yacc);
                 __syncwarp();
                 ++ncs;
-                st_next(cs, p, G, c, warp, nph);
+                st_next(cs, p, ct, warp, nph);
             }
             finish_cell(yacc, lane, [&](int row, float v) {
                 size_t o = (size_t)b * 32 + row;
