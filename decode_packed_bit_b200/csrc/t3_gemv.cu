@@ -251,15 +251,17 @@ __global__ void __launch_bounds__(kT3MaxWarps * 32, 1) k_t3_m1(const __grid_cons
     const size_t rowbytes = (size_t)26 * (p.K >> 7);
     const int G = p.K >> 7;
     const int upc = p.units / p.slices;          // units per work item
-    const long long items = (long long)p.cells * p.slices;
-    const long long gw = (long long)blockIdx.x * nw + warp, gstride = (long long)gridDim.x * nw;
+    // 32-bit item indices (the planner keeps cells * slices below 2^31): a
+    // 64-bit division per step is a long software routine
+    const int items = p.cells * p.slices;
+    const int gw = blockIdx.x * nw + warp, gstride = gridDim.x * nw;
 
     // issue side: step s of this warp's items, in order
-    long long is_item = gw;
+    int is_item = gw;
     int is_u = 0, is_slot = 0;
     auto issue_next = [&]() {
         if (is_item < items) {
-            const int cell = (int)(is_item / p.slices), sl = (int)(is_item - (long long)cell * p.slices);
+            const int cell = is_item / p.slices, sl = is_item - cell * p.slices;
             const int r = cell / p.blocksN, blk = cell - r * p.blocksN;
             const int u = sl * upc + is_u;
             const unsigned st = ring_s + is_slot * kT3StageBytes;
@@ -297,8 +299,8 @@ __global__ void __launch_bounds__(kT3MaxWarps * 32, 1) k_t3_m1(const __grid_cons
 
     const uint32_t *lut_lane = lut + lane;
     int slot = 0;
-    for (long long item = gw; item < items; item += gstride) {
-        const int cell = (int)(item / p.slices), sl = (int)(item - (long long)cell * p.slices);
+    for (int item = gw; item < items; item += gstride) {
+        const int cell = item / p.slices, sl = item - cell * p.slices;
         const int r = cell / p.blocksN, blk = cell - r * p.blocksN;
         float yacc = 0.f;
         for (int uu = 0; uu < upc; ++uu) {
@@ -469,6 +471,7 @@ static T3Plan t3_plan(int R, int N, int K, int sms)
     while (cells * S < 2 * warps_total && S * 2 <= K / 1024 && (K / 1024) % (S * 2) == 0) S *= 2;
     P.slices = S;
     P.grid = (int)std::min<long long>(sms, (cells * S + P.warps - 1) / P.warps);
+    if (cells * S >= (1LL << 31)) P.ok = false;  // the kernel indexes items with 32-bit ints
     return P;
 }
 
