@@ -51,11 +51,15 @@ __device__ __forceinline__ float warp_max(float v)
     return v;
 }
 
-__device__ __forceinline__ int warp_sum_int(int v)
+// Integer sum over the warp in one reduction instruction (wraps mod 2^32
+// like a chain of adds).
+__device__ __forceinline__ int warp_sum_int(int v) { return __reduce_add_sync(0xffffffffu, v); }
+
+// Maximum of non-negative finite floats over the warp in one reduction:
+// their bit patterns order like unsigned integers.
+__device__ __forceinline__ float warp_max_nonneg(float v)
 {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
+    return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(v)));
 }
 
 // Programmatic dependent launch: let the next kernel on the stream start its

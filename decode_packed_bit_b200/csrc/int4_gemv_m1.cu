@@ -182,7 +182,7 @@ __device__ __forceinline__ void i4_build_pair_warp(const uint16_t *__restrict__ 
     int E[2], T[2] = {0, 0};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const float mh = warp_max(fmaxf(fabsf(xv[2 * h]), fabsf(xv[2 * h + 1])));
+        const float mh = warp_max_nonneg(fmaxf(0.f, fmaxf(fabsf(xv[2 * h]), fabsf(xv[2 * h + 1]))));
         const int e8 = (int)((__float_as_uint(mh) >> 23) & 0xFFu);
         E[h] = max(e8 == 0 ? kI4MinExp : e8 - 126, kI4MinExp);  // smallest E with max|x| < 2^E
     }

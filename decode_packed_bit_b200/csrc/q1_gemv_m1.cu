@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(256) k_q1_prep_m1(const uint16_t *__restrict__
     const uint16_t xb = k < K ? x[k] : (uint16_t)0;
     if (k < K) reinterpret_cast<uint16_t *>(act + xcopy_off)[k] = xb;
     const float xv = bf16_bits_to_float(xb);
-    const float wm = warp_max(fabsf(xv));
+    const float wm = warp_max_nonneg(fmaxf(0.f, fabsf(xv)));
     if (lane == 0) smax[warp] = wm;
     __syncthreads();
     const float m = fmaxf(fmaxf(smax[4 * h], smax[4 * h + 1]), fmaxf(smax[4 * h + 2], smax[4 * h + 3]));
@@ -439,7 +439,7 @@ __device__ __forceinline__ void q1_build_chunk_warp(const uint16_t *__restrict__
     int E[2], T[2] = {0, 0};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const float mh = warp_max(m[h]);
+        const float mh = warp_max_nonneg(m[h]);
         const int e8 = (int)((__float_as_uint(mh) >> 23) & 0xFFu);
         E[h] = max(e8 == 0 ? kQ1MinExp : e8 - 126, kQ1MinExp);  // smallest E with max|x| < 2^E
     }

@@ -163,7 +163,7 @@ __device__ void t3_build_tables(const uint16_t *__restrict__ x, int K, uint4 *ta
             v[q] = bf16_bits_to_float(x[128 * g + 32 * q + lane]);
             m = fmaxf(m, fabsf(v[q]));
         }
-        m = warp_max(m);
+        m = warp_max_nonneg(m);
         const int e8 = (int)((__float_as_uint(m) >> 23) & 0xFFu);
         const int E = max(e8 == 0 ? kT3MinExp : e8 - 125, kT3MinExp);   // 2^(E-2) <= m < 2^(E-1)
         int s = 0;
