@@ -129,3 +129,35 @@ def test_stack_m1_one_launch_teacher_forced(stack_weights):
     got = synth.bf16_bits_to_f32(host(st.x.view(torch.int16)).view(np.uint16)).astype(np.float64)
     tol = 0.5 * _bf16_ulp(r64) + 1e-6 * np.abs(r64) + 1e-30
     assert (np.abs(got - r64) <= tol).all()
+
+
+@pytest.mark.parametrize("hidden,ffn,n_layers", [(1024, 8192, 2), (2048, 3072, 3)])
+def test_stack_one_launch_other_widths(cuda_device, hidden, ffn, n_layers):
+    """The one-launch step at widths whose K-slice counts (1 and 8, 2 and
+    3 slices of 1024) differ from the 5120/17408 stack's, so every CTA's
+    slice, rank and share of the blocks take other values; checked
+    teacher-forced like the full stack, plus the step output."""
+    from decode_packed_bit_b200 import build
+    build.build()
+    from decode_packed_bit_b200 import lowbit as lb
+    from decode_packed_bit_b200.stack import Q1Layer, Q1Stack, StackRecord
+    seed = synth.SEED_BASE + synth.W_Q1_STACK + 7 * hidden + ffn
+    shapes = [("q", hidden, hidden), ("k", hidden, hidden), ("v", hidden, hidden), ("o", hidden, hidden),
+              ("gate", ffn, hidden), ("up", ffn, hidden), ("down", hidden, ffn)]
+    layers = [Q1Layer({name: synth.torch_q1_layer(seed, n, k, li * 16 + pi, cuda_device)
+                       for pi, (name, n, k) in enumerate(shapes)}) for li in range(n_layers)]
+    st = Q1Stack(layers, hidden, ffn, 1, "cuda")
+    assert st.fused_supported()
+    x0 = synth.bf16_normal(seed, (1, hidden), tag=1)
+    st.x.copy_(torch.from_numpy(x0.view(np.int16)).view(torch.bfloat16).cuda())
+    rec = StackRecord(which=None)
+    st.step_fused(record=rec)
+    torch.cuda.synchronize()
+    assert lb.lowbit_fault_flags() == 0
+    assert len(rec.outputs) == 7 * n_layers
+    _check_projections(layers, rec, 1, rows_per_proj=16, seed=17)
+    _check_glue(rec, 1)
+    r64 = oracle.rmsnorm(host(rec.norm_in[(n_layers - 1, "down")]), None, eps=1e-6)
+    got = synth.bf16_bits_to_f32(host(st.x.view(torch.int16)).view(np.uint16)).astype(np.float64)
+    tol = 0.5 * _bf16_ulp(r64) + 1e-6 * np.abs(r64) + 1e-30
+    assert (np.abs(got - r64) <= tol).all()
