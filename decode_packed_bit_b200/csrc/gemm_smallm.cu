@@ -160,6 +160,16 @@ __device__ __forceinline__ float sm_ld_peer(const float *local, unsigned rank)
     return v;
 }
 
+// Store a float into rank `rank`'s shared memory, at the address `local`
+// has in this CTA.
+__device__ __forceinline__ void sm_st_peer(float *local, unsigned rank, float v)
+{
+    unsigned ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"((unsigned)__cvta_generic_to_shared(local)),
+                 "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 {
     uint32_t r;
@@ -593,6 +603,7 @@ struct SmParams {
     int nsteps;  // K / step
     int L;       // steps per K-slice
     int blocks;  // 128-row blocks per matrix
+    int push;    // split-K partial sums pushed to their owner before one cluster barrier
 };
 
 template <int FMT, int NT>
@@ -694,9 +705,32 @@ __global__ void __launch_bounds__(kSmThreads, sm_min_blocks(FMT, NT)) k_smallm(c
         }
         return;
     }
-    sm_cluster_sync();  // every slice's partial sums are in its CTA's shared memory
-    // rank q adds up entries [q*per, (q+1)*per) over all ranks, in rank order
+    // rank q owns entries [q*per, (q+1)*per) of part and adds them up over
+    // all ranks, in rank order.
     const int tot = p.M * kSmRows, per = (tot + nsl - 1) / nsl;
+    if (p.push) {
+        // every slice pushes its partial sums of q's share into rank q's
+        // recv[slice] before one cluster barrier (release / acquire); nothing
+        // reads another CTA's shared memory after it, so each CTA may then
+        // finish on its own
+        float *recv = part + p.M * kSmRows;
+        __syncthreads();  // part[] is complete
+        for (int q = 0; q < nsl; ++q)
+            for (int j = threadIdx.x; j < per && q * per + j < tot; j += blockDim.x)
+                sm_st_peer(recv + slice * per + j, (unsigned)q, part[q * per + j]);
+        sm_cluster_sync();
+        for (int j = threadIdx.x; j < per && slice * per + j < tot; j += blockDim.x) {
+            float sum = 0.f;
+            for (int q = 0; q < nsl; ++q) sum += recv[q * per + j];
+            const int i = slice * per + j, m = i / kSmRows, row = rb * kSmRows + (i - m * kSmRows);
+            if (row < p.N) yout[(size_t)m * p.N + row] = sum;
+        }
+        return;
+    }
+    // otherwise (the receive buffer would cost residency) rank q reads the
+    // peers' part[] after one barrier, and a second keeps it alive until all
+    // ranks have read it
+    sm_cluster_sync();
     for (int i = slice * per + threadIdx.x; i < min(tot, (slice + 1) * per); i += blockDim.x) {
         float v[kSmMaxCluster];
 #pragma unroll
@@ -707,11 +741,12 @@ __global__ void __launch_bounds__(kSmThreads, sm_min_blocks(FMT, NT)) k_smallm(c
         const int m = i / kSmRows, row = rb * kSmRows + (i - m * kSmRows);
         if (row < p.N) yout[(size_t)m * p.N + row] = sum;
     }
-    sm_cluster_sync();  // peers keep their shared memory until every rank has read it
+    sm_cluster_sync();
 }
 
 struct SmPlan {
     int nsteps, L, S, blocks, NT;
+    bool push;
     size_t smem;
     bool ok;
 };
@@ -727,10 +762,20 @@ static SmPlan sm_plan(int fmt, int M, int N, int K, int sms, int R = 1)
     P.blocks = (N + kSmRows - 1) / kSmRows * R;
     if (M < 2 || M > maxm || N < 1 || K % stepk != 0 || P.nsteps < 1 || R < 1 || R > kSmMaxR) return P;
     const size_t ring = (size_t)kSmWarps * kSmWStages * (fmt == 1 ? kSmStageBytes : kI4sStageBytes);
-    P.smem = 128 /*alignment*/ + sg_xring_bytes(fmt, kSmSlots, P.NT) + ring + (size_t)M * kSmRows * 4;
+    // the partial sums; with push, the peers' pushed partial sums after them
+    // (up to S - 1 entries more).  Pushing was measured faster up to M = 8
+    // (Q1_0_g128 5120x5120: 7.7 -> 7.2 us) and slower above (INT4_G64
+    // 11008x4096 M=32: 23.5 -> 26.6 us, about 4096 remote stores per CTA), so
+    // it is taken for M <= 8, where it also costs no residency
+    const size_t base = 128 /*alignment*/ + sg_xring_bytes(fmt, kSmSlots, P.NT) + ring + (size_t)M * kSmRows * 4;
+    const size_t with_recv = base + ((size_t)M * kSmRows + kSmMaxCluster) * 4;
     // CTAs resident per SM (shared memory, with 1 KB reserved per CTA, and registers)
-    const int resident =
-        (int)std::max<size_t>(1, std::min<size_t>(sm_min_blocks(fmt, P.NT), (228 * 1024) / (P.smem + 1024)));
+    auto resident_at = [&](size_t smem) {
+        return (int)std::max<size_t>(1, std::min<size_t>(sm_min_blocks(fmt, P.NT), (228 * 1024) / (smem + 1024)));
+    };
+    P.push = M <= 8 && with_recv <= (size_t)kSmMaxSmem && resident_at(with_recv) >= resident_at(base);
+    P.smem = P.push ? with_recv : base;
+    const int resident = resident_at(P.smem);
     // K slices: as many as keep every CTA resident in one wave
     P.S = (int)std::min<long long>(std::min(kSmMaxCluster, P.nsteps),
                                    std::max<long long>(1, (long long)resident * sms / P.blocks));
@@ -763,6 +808,7 @@ static lowbit_status sm_launch(int fmt, const uint8_t *const *bits, const uint16
     p.nsteps = P.nsteps;
     p.L = P.L;
     p.blocks = P.blocks / R;
+    p.push = P.push ? 1 : 0;
     void (*kern)(const CUtensorMap, const SmParams);
     if (fmt == 1)
         kern = P.NT == 1 ? k_smallm<1, 1> : k_smallm<1, 2>;

@@ -66,14 +66,14 @@ constexpr int kNormCThreads = 256;
 constexpr int kNormPer = 8;  // float4 of v per thread at most
 constexpr int kNormMaxD = 4 * kNormPer * kNormCThreads * kNormCluster;
 
-__device__ __forceinline__ float norm_ld_peer(const float *local, unsigned rank)
+// Store a float into rank `rank`'s shared memory, at the address `local`
+// has in this CTA.
+__device__ __forceinline__ void norm_st_peer(float *local, unsigned rank, float v)
 {
     unsigned ra;
-    float v;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"((unsigned)__cvta_generic_to_shared(local)),
                  "r"(rank));
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
-    return v;
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ void norm_cluster_sync()
@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kNormCThreads) k_rmsnorm_bf16_cl(const float *
                                                                    uint16_t *__restrict__ out)
 {
     __shared__ float red[kNormCThreads / 32];
-    __shared__ float part;
+    __shared__ float recv[kNormCluster];  // every CTA's partial sum of squares, pushed by its owner
     pdl_launch_dependents();
     pdl_wait_primary();
     const unsigned q = blockIdx.x;
@@ -123,12 +123,14 @@ __global__ void __launch_bounds__(kNormCThreads) k_rmsnorm_bf16_cl(const float *
     if (threadIdx.x < 32) {
         float t = threadIdx.x < kNormCThreads / 32 ? red[threadIdx.x] : 0.f;
         t = warp_sum(t);
-        if (threadIdx.x == 0) part = t;
+        // this CTA's partial sum (in every lane after the butterfly sum) goes
+        // into recv[q] of every CTA of the row, one lane per destination
+        if (threadIdx.x < kNormCluster) norm_st_peer(&recv[q], threadIdx.x, t);
     }
-    norm_cluster_sync();  // every CTA's partial sum is in its shared memory
+    norm_cluster_sync();  // every partial sum has arrived (release / acquire)
     float tot = 0.f;
 #pragma unroll
-    for (int r = 0; r < kNormCluster; ++r) tot += norm_ld_peer(&part, (unsigned)r);
+    for (int r = 0; r < kNormCluster; ++r) tot += recv[r];  // rank order
     const float inv = 1.0f / sqrtf(tot / (float)D + eps);
     uint2 *o = reinterpret_cast<uint2 *>(out + row * D);
 #pragma unroll
@@ -142,7 +144,7 @@ __global__ void __launch_bounds__(kNormCThreads) k_rmsnorm_bf16_cl(const float *
             o[i] = make_uint2(l, h);
         }
     }
-    norm_cluster_sync();  // peers keep their shared memory until every CTA has read it
+    // nothing reads another CTA's shared memory after the barrier: no second one
 }
 
 lowbit_status rmsnorm_launch(const float *a, const float *b, int M, int D, float eps, uint16_t *out,

@@ -59,6 +59,9 @@ constexpr int kI4MinExp = -96;
 constexpr int kI4MaxSmem = 226 * 1024;
 constexpr int kI4MaxCluster = 8;
 constexpr int kI4SplitRows = kI4SplitWarps * kI4StepRows;
+// dynamic shared memory of the split kernel at most: its static partial-sum
+// and receive buffers take the rest of the 227 KB
+constexpr int kI4SplitSmemCap = kI4MaxSmem - (kI4SplitRows + kI4MaxCluster) * 4;
 
 
 // ---------------------------------------------------------------------------
@@ -252,17 +255,14 @@ __device__ __forceinline__ void i4_cluster_sync()
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Read a float of rank `rank`'s shared memory.  volatile keeps the load after
-// the cluster barrier; the callers issue all ranks' loads before using any,
-// so they overlap.
-__device__ __forceinline__ float i4_ld_cluster(const float *local, unsigned rank)
+// Store a float into rank `rank`'s shared memory, at the address `local`
+// has in this CTA.
+__device__ __forceinline__ void i4_st_cluster(float *local, unsigned rank, float v)
 {
     const unsigned a = (unsigned)__cvta_generic_to_shared(local);
     unsigned ra;
-    float v;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra));
-    return v;
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
 // grid: x = K-slice (cluster rank), y = 128-row block.  With one slice the
@@ -271,6 +271,7 @@ __global__ void __launch_bounds__(kI4SplitWarps * 32) k_i4_m1_split(const I4Para
 {
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ float part[kI4SplitRows];
+    __shared__ float recv[kI4SplitRows + kI4MaxCluster];  // [slice][share]: the partial sums pushed to this rank
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int slice = blockIdx.x, nsl = gridDim.x, rb = blockIdx.y;
@@ -321,19 +322,24 @@ __global__ void __launch_bounds__(kI4SplitWarps * 32) k_i4_m1_split(const I4Para
             if (rb * kI4SplitRows + i < p.N) p.y[rb * kI4SplitRows + i] = part[i];
         return;
     }
-    i4_cluster_sync();  // every slice's partial sums are in its CTA's shared memory
-    // rank q adds up rows [q*per, (q+1)*per) over all ranks, in rank order
+    // rank q owns rows [q*per, (q+1)*per): every slice pushes its partial sums
+    // of those rows into rank q's recv[slice], and after one cluster barrier
+    // (release / acquire) rank q adds them up in rank order.  Nothing reads
+    // another CTA's shared memory after the barrier, so each CTA may then
+    // finish on its own.
     const int per = (kI4SplitRows + nsl - 1) / nsl;
-    for (int i = slice * per + threadIdx.x; i < min(kI4SplitRows, (slice + 1) * per); i += blockDim.x) {
-        float v[kI4MaxCluster];
-#pragma unroll
-        for (int q = 0; q < kI4MaxCluster; ++q) v[q] = q < nsl ? i4_ld_cluster(part + i, (unsigned)q) : 0.f;
-        float sum = 0.f;
-#pragma unroll
-        for (int q = 0; q < kI4MaxCluster; ++q) sum += v[q];
-        if (rb * kI4SplitRows + i < p.N) p.y[rb * kI4SplitRows + i] = sum;
+    __syncthreads();  // part[] is complete
+    for (int i = threadIdx.x; i < kI4SplitRows; i += blockDim.x) {
+        const int q = i / per;
+        i4_st_cluster(recv + slice * per + (i - q * per), (unsigned)q, part[i]);
     }
-    i4_cluster_sync();  // peers keep their shared memory until every rank has read it
+    i4_cluster_sync();
+    for (int j = threadIdx.x; j < per && slice * per + j < kI4SplitRows; j += blockDim.x) {
+        float sum = 0.f;
+        for (int q = 0; q < nsl; ++q) sum += recv[q * per + j];
+        const int row = rb * kI4SplitRows + slice * per + j;
+        if (row < p.N) p.y[row] = sum;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -500,10 +506,10 @@ static I4Plan i4_plan(int N, int K, int sms)
         P.nslices = (P.npairs + P.L - 1) / P.L;
         P.act_smem = ((size_t)P.L * per_pair + 15) & ~size_t(15);
         P.smem = P.act_smem + ring + kI4BuildScratch;
-        if (P.smem <= (size_t)kI4MaxSmem || S >= kI4MaxCluster) break;
+        if (P.smem <= (size_t)kI4SplitSmemCap || S >= kI4MaxCluster) break;
         S = std::min(kI4MaxCluster, S * 2);
     }
-    P.ok = P.smem <= (size_t)kI4MaxSmem && P.blocks < 65536 && (K / 64) % 2 == 0;
+    P.ok = P.smem <= (size_t)kI4SplitSmemCap && P.blocks < 65536 && (K / 64) % 2 == 0;
     return P;
 }
 
@@ -532,7 +538,7 @@ lowbit_status i4m1_launch(const uint8_t *q, const uint16_t *scales, const uint16
     p.npairs = P.npairs;
     p.L = P.L;
     p.act_smem = (int)P.act_smem;
-    if (cudaFuncSetAttribute(k_i4_m1_split, cudaFuncAttributeMaxDynamicSharedMemorySize, kI4MaxSmem) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_i4_m1_split, cudaFuncAttributeMaxDynamicSharedMemorySize, kI4SplitSmemCap) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(P.nslices, P.blocks);

@@ -889,17 +889,14 @@ __device__ __forceinline__ void cluster_sync()
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Read a float of rank `rank`'s shared memory.  volatile keeps the load after
-// the cluster barrier; the callers issue all ranks' loads before using any,
-// so they overlap.
-__device__ __forceinline__ float ld_cluster_f32(const float *local, unsigned rank)
+// Store a float into rank `rank`'s shared memory, at the address `local`
+// has in this CTA.
+__device__ __forceinline__ void st_cluster_f32(float *local, unsigned rank, float v)
 {
     const unsigned a = (unsigned)__cvta_generic_to_shared(local);
     unsigned ra;
-    float v;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra));
-    return v;
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
 #ifndef LOWBIT_Q1_SPLIT_STAGES
@@ -915,6 +912,9 @@ constexpr int kQ1SplitStages = LOWBIT_Q1_SPLIT_STAGES;  // steps of a split warp
 constexpr int kQ1SplitRing = kQ1SplitStages * kQ1StageBytes;
 
 constexpr int kQ1SplitRows = kQ1SplitWarps * kQ1StepRows;  // rows of one CTA
+// dynamic shared memory of the split kernel at most: its static partial-sum
+// and receive buffers take the rest of the 227 KB
+constexpr int kQ1SplitSmemCap = kQ1MaxSmem - (kQ1SplitRows + kQ1MaxCluster) * 4;
 
 // grid: x = slice (= cluster rank), y = r * blocks_per_matrix + row block
 __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid_constant__ Q1Group grp,
@@ -922,6 +922,7 @@ __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid
 {
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ float part[kQ1SplitRows];
+    __shared__ float recv[kQ1SplitRows + kQ1MaxCluster];  // [slice][share]: the partial sums pushed to this rank
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int slice = blockIdx.x, nsl = gridDim.x;
@@ -984,19 +985,24 @@ __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid
             if (rb * kQ1SplitRows + i < p.N) grp.y[r][rb * kQ1SplitRows + i] = part[i];
         return;
     }
-    cluster_sync();  // every slice's partial sums are in its CTA's shared memory
-    // rank q adds up rows [q*per, (q+1)*per) over all ranks, in rank order
+    // rank q owns rows [q*per, (q+1)*per): every slice pushes its partial sums
+    // of those rows into rank q's recv[slice], and after one cluster barrier
+    // (release / acquire) rank q adds them up in rank order.  Nothing reads
+    // another CTA's shared memory after the barrier, so each CTA may then
+    // finish on its own.
     const int per = (kQ1SplitRows + nsl - 1) / nsl;
-    for (int i = slice * per + threadIdx.x; i < min(kQ1SplitRows, (slice + 1) * per); i += blockDim.x) {
-        float v[kQ1MaxCluster];
-#pragma unroll
-        for (int q = 0; q < kQ1MaxCluster; ++q) v[q] = q < nsl ? ld_cluster_f32(part + i, (unsigned)q) : 0.f;
-        float sum = 0.f;
-#pragma unroll
-        for (int q = 0; q < kQ1MaxCluster; ++q) sum += v[q];
-        if (rb * kQ1SplitRows + i < p.N) grp.y[r][rb * kQ1SplitRows + i] = sum;
+    __syncthreads();  // part[] is complete
+    for (int i = threadIdx.x; i < kQ1SplitRows; i += blockDim.x) {
+        const int q = i / per;
+        st_cluster_f32(recv + slice * per + (i - q * per), (unsigned)q, part[i]);
     }
-    cluster_sync();  // peers keep their shared memory until every rank has read it
+    cluster_sync();
+    for (int j = threadIdx.x; j < per && slice * per + j < kQ1SplitRows; j += blockDim.x) {
+        float sum = 0.f;
+        for (int q = 0; q < nsl; ++q) sum += recv[q * per + j];
+        const int row = rb * kQ1SplitRows + slice * per + j;
+        if (row < p.N) grp.y[r][row] = sum;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1090,12 +1096,12 @@ static Q1Plan q1_plan(int R, int N, int K, int sms, bool aligned = false, int mv
         P.nslices = (P.nchunks + P.L - 1) / P.L;
         P.act_smem = (size_t)P.L * per_chunk + kQ1ZeroBytes;
         P.smem = P.act_smem + ring_split + kQ1BuildScratch;
-        if (P.smem <= (size_t)kQ1MaxSmem || S >= kQ1MaxCluster) break;
+        if (P.smem <= (size_t)kQ1SplitSmemCap || S >= kQ1MaxCluster) break;
         S = std::min(kQ1MaxCluster, S * 2);
     }
     P.grid_x = P.nslices;
     P.grid_y = (int)blocks;
-    P.ok = P.smem <= (size_t)kQ1MaxSmem && blocks < 65536;
+    P.ok = P.smem <= (size_t)kQ1SplitSmemCap && blocks < 65536;
     return P;
 }
 
