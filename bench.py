@@ -499,7 +499,9 @@ def run_q1_4096(args, world, rank, local):
     # call waits for the copy that last read its buffer set).  Several ranks:
     # one call at a time (the all-gather owns the output buffer).
     x_host = x.cpu().pin_memory()
-    e2e_calls = 200
+    # as many calls as the timed region above, so that both run for about as
+    # long (and at the clocks the power limit leaves)
+    e2e_calls = max(200, L * args.steps)
     if world == 1:
         x2 = torch.empty_like(x)
         y2 = torch.empty_like(y)
@@ -511,18 +513,33 @@ def run_q1_4096(args, world, rank, local):
         sets = [(graph, x, y), (graph2, x2, y2)]
         hosts = [torch.empty(out_host_shape, dtype=torch.float32).pin_memory() for _ in range(2)]
         y_host = hosts[0]
-        copy_stream = torch.cuda.Stream(device=dev)
+        copy_stream = torch.cuda.Stream(device=dev)  # outputs to the host
+        in_stream = torch.cuda.Stream(device=dev)    # inputs from the host
         done = [torch.cuda.Event() for _ in range(2)]
         copied = [torch.cuda.Event() for _ in range(2)]
+        loaded = [torch.cuda.Event() for _ in range(2)]
+
+        start = torch.cuda.Event()
 
         def e2e_run(n):
+            # the copy streams start after what `stream` has enqueued so far
+            # (the start of the timed region)
+            start.record(stream)
+            in_stream.wait_event(start)
+            copy_stream.wait_event(start)
             for i in range(n):
                 b = i % 2
                 g_b, x_b, y_b = sets[b]
-                with torch.cuda.stream(stream):
+                # x of call i comes in while call i-1 runs (x_b was last read by call i-2)
+                with torch.cuda.stream(in_stream):
                     if i >= 2:
-                        stream.wait_event(copied[b])
+                        in_stream.wait_event(done[b])
                     x_b.copy_(x_host, non_blocking=True)
+                    loaded[b].record(in_stream)
+                with torch.cuda.stream(stream):
+                    stream.wait_event(loaded[b])
+                    if i >= 2:
+                        stream.wait_event(copied[b])  # y_b of call i-2 has reached the host
                     g_b.replay()
                     done[b].record(stream)
                 with torch.cuda.stream(copy_stream):
@@ -532,8 +549,9 @@ def run_q1_4096(args, world, rank, local):
             stream.wait_event(copied[(n - 1) % 2])
             if n >= 2:
                 stream.wait_event(copied[(n - 2) % 2])
-        e2e_note = ("x in from pinned host, all outputs out, every call; two buffer sets: the outputs of "
-                    "one call copy out on a second stream during the next call")
+        e2e_note = ("x in from pinned host, all outputs out, every call; two buffer sets: the inputs of "
+                    "one call copy in and the outputs of the one before copy out on two more streams "
+                    "while a call runs")
     else:
         y_host = torch.empty(out_host_shape, dtype=torch.float32).pin_memory()
 
