@@ -98,12 +98,13 @@ struct SgFmt<3> {
 // filled by the tensor copy): the step's k plus 16 more.
 __host__ __device__ constexpr int sg_xrow(int fmt) { return fmt == 1 ? kSmStepK * 2 + 64 : (kI4sStepK + 16) * 2; }
 
-// Shared memory of both kernels starts with the raw ring (Q1_0_g128 only)
-// and the x ring, both written by tensor copies, which want 128-byte
-// aligned destinations: every slot size is a multiple of 128.
+// Shared memory of both kernels starts with the raw ring (the grouped
+// kernel: one step of the M rows of x per slot, natural order) and the x
+// ring, both written by tensor copies, which want 128-byte aligned
+// destinations: every slot size is a multiple of 128.
 __host__ __device__ constexpr size_t sg_raw_bytes(int fmt, int raw, int M)
 {
-    return fmt == 1 ? (size_t)raw * M * kSmStepK * 2 : 0;
+    return (size_t)raw * M * (fmt == 1 ? kSmStepK : kI4sStepK) * 2;
 }
 __host__ __device__ constexpr size_t sg_xring_bytes(int fmt, int slots, int NT)
 {
@@ -387,6 +388,62 @@ __device__ __forceinline__ void sg_consume_i4(const uint8_t *stage, const uint8_
     }
 }
 
+// The weight pair (k = j, j + 4) of a word of eight nibbles (k = 0..7, low
+// nibble first) as exact bf16: (word >> 4j) & 0x000F000F holds the two
+// nibbles in the low bits of each half; xor 8 and the exponent of 128 make
+// each half 136 + q, and one bf16x2 subtract leaves q.
+__device__ __forceinline__ uint32_t i4_pair4_bf16(uint32_t w, uint32_t sh)
+{
+    const uint32_t v = ((w >> sh) & 0x000F000Fu) ^ 0x43084308u;
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(0x43084308u));
+    return r;
+}
+
+// INT4_G64 step (two groups) from a weight stage and an x slot in pair order
+// (sg_rewrite_i4).  The MMA's k slots 2t, 2t+1 of a 16-k window carry k = t
+// and t + 4 of its first 8-k block, slots 2t+8, 2t+9 the same of the second,
+// in A and in B alike: a lane's A pair is one shift, one LOP3 and one bf16
+// subtract of a word of the row, its B registers one 8-byte word pair.
+template <int NT>
+__device__ __forceinline__ void sg_consume_i4p(const uint8_t *stage, const uint8_t *xs, int lane,
+                                               float (&yacc)[2][NT][4])
+{
+    constexpr int kXR = sg_xrow(3);
+    const int g = lane >> 2, t = lane & 3;
+    const uint8_t *xl = xs + g * kXR + 8 * t;
+    const uint32_t sh = 4u * (uint32_t)t;
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp) {
+        float acc[2][NT][4];
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const int ks = 4 * grp + s;  // 16-k window within the stage: bytes 8 ks .. 8 ks + 7 of a row
+            uint2 b[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) b[nt] = *reinterpret_cast<const uint2 *>(xl + 8 * nt * kXR + 32 * ks);
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                uint32_t a[2][2];  // [row g / g+8][block 0 / 1 of the window]
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const uint2 w = *reinterpret_cast<const uint2 *>(stage + (16 * tt + 8 * r + g) * kI4sRowStride + 8 * ks);
+                    a[r][0] = i4_pair4_bf16(w.x, sh);
+                    a[r][1] = i4_pair4_bf16(w.y, sh);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (s == 0)
+                        hmma0(acc[tt][nt], a[0][0], a[1][0], a[0][1], a[1][1], b[nt].x, b[nt].y);
+                    else
+                        hmma(acc[tt][nt], a[0][0], a[1][0], a[0][1], a[1][1], b[nt].x, b[nt].y);
+                }
+            }
+        }
+        sg_scale<3, NT>(stage, g, grp, acc, yacc);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // weight copies of one consumer warp
 // ---------------------------------------------------------------------------
@@ -451,11 +508,27 @@ __device__ __forceinline__ void sg_rewrite(const uint8_t *src, uint8_t *dst, int
         make_uint4(prmt(l0, h0, 0x5410u), prmt(l0, h0, 0x7632u), prmt(l1, h1, 0x5410u), prmt(l1, h1, 0x7632u));
 }
 
+// Producer task (INT4_G64): one 16-k window of one row, from its 32 raw
+// bytes at `src` (natural order) to `dst` in pair order: the eight bf16
+// pairs {x[8b + j], x[8b + j + 4]} (block b = 0, 1 of the window, j = 0..3)
+// as words in the order (b=0 j=0, b=1 j=0, b=0 j=1, b=1 j=1, ...), so that a
+// lane's two B registers of the window are one 8-byte word pair.
+__device__ __forceinline__ void sg_rewrite_i4(const uint8_t *src, uint8_t *dst)
+{
+    const uint4 A = *reinterpret_cast<const uint4 *>(src);       // x0x1 x2x3 x4x5 x6x7
+    const uint4 B = *reinterpret_cast<const uint4 *>(src + 16);  // x8x9 ... x14x15
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(prmt(A.x, A.z, 0x5410u), prmt(B.x, B.z, 0x5410u),
+                                                 prmt(A.x, A.z, 0x7632u), prmt(B.x, B.z, 0x7632u));
+    *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(prmt(A.y, A.w, 0x5410u), prmt(B.y, B.w, 0x5410u),
+                                                      prmt(A.y, A.w, 0x7632u), prmt(B.y, B.w, 0x7632u));
+}
+
 // Fill x-ring slot u % SLOTS with step s0 + u % ncycle of x, u = 0 .. total-1.
-// Direct (INT4_G64, or Q1_0_g128 with DIRECT): tensor copies straight into
-// the slot, boxes of all M rows and sg_xrow(3) / 2 k (one per INT4_G64 step,
-// one per 128-k half of a Q1_0_g128 step, the halves in two regions).
-// Otherwise (Q1_0_g128): raw slices of one step each, rewritten into P order.
+// DIRECT: tensor copies straight into the slot, boxes of all M rows and
+// sg_xrow(3) / 2 k (one per INT4_G64 step, one per 128-k half of a
+// Q1_0_g128 step, the halves in two regions), natural order.  Otherwise raw
+// slices of one step each, rewritten once into the consumers' order
+// (Q1_0_g128: {x[k], x[k+16]} pairs; INT4_G64: {x[k], x[k+4]} pairs).
 // Called by every lane of the producer warp; returns when done or when a
 // wait ran out.
 template <int FMT, int NT, int SLOTS, int RAW, bool DIRECT>
@@ -466,7 +539,7 @@ __device__ __forceinline__ void sg_produce(const CUtensorMap *xmap, uint8_t *raw
     constexpr int kXR = sg_xrow(FMT);
     constexpr int kXSlot = 8 * NT * kXR;
     pdl_wait_primary();  // x is produced by earlier kernels
-    if (FMT == 3 || DIRECT) {
+    if (DIRECT) {
         constexpr int kBoxes = FMT == 1 ? 2 : 1;
         constexpr int kRow = sg_xrow(3);  // bytes of a box row
         if (lane == 0) {
@@ -484,19 +557,21 @@ __device__ __forceinline__ void sg_produce(const CUtensorMap *xmap, uint8_t *raw
         return;
     }
     // raw slices by tensor copy, rewritten once into the x ring
-    const int rawslot = M * kSmStepK * 2;
+    constexpr int kStepK = SgFmt<FMT>::kStepK;
+    const int rawslot = M * kStepK * 2;
     auto copy_raw = [&](int v) {  // lane 0: step v of the sequence into raw slot v % RAW
         if (v >= total) return;
         uint64_t *bar = rawbar + v % RAW;
         mbar_arrive_expect_tx(bar, (unsigned)rawslot);
-        tma_load_2d(raw + (v % RAW) * rawslot, xmap, (s0 + v % ncycle) * kSmStepK, 0, bar);
+        tma_load_2d(raw + (v % RAW) * rawslot, xmap, (s0 + v % ncycle) * kStepK, 0, bar);
     };
     if (lane == 0)
         for (int v = 0; v < RAW; ++v) copy_raw(v);
-    // task T = (unit item T/4 = (row n, unit c), output chunk T%4); a quarter
-    // warp covers two adjacent units: 128 contiguous bytes each way
+    // Q1_0_g128: task T = (unit item T/4 = (row n, unit c), output chunk
+    // T%4); a quarter warp covers two adjacent units: 128 contiguous bytes
+    // each way.  INT4_G64: task T = (row T/8, 16-k window T%8).
     constexpr int kUnitsStep = kSmStepK / 32;
-    const int tasks = M * kUnitsStep * 4;
+    const int tasks = FMT == 1 ? M * kUnitsStep * 4 : M * (kI4sStepK / 16);
     constexpr int kUn = 4;
     for (int u = 0; u < total; ++u) {
         const int sl = u % SLOTS, rs = u % RAW;
@@ -510,8 +585,13 @@ __device__ __forceinline__ void sg_produce(const CUtensorMap *xmap, uint8_t *raw
             for (int i = 0; i < kUn; ++i) {
                 const int T = base + 32 * i + lane;
                 if (T < tasks) {
-                    const int item = T >> 2, n = item / kUnitsStep, c = item - n * kUnitsStep;
-                    sg_rewrite(rsrc + n * kSmStepK * 2 + 64 * c, xdst + n * kXR + 64 * c + 16 * (T & 3), T & 3);
+                    if (FMT == 1) {
+                        const int item = T >> 2, n = item / kUnitsStep, c = item - n * kUnitsStep;
+                        sg_rewrite(rsrc + n * kSmStepK * 2 + 64 * c, xdst + n * kXR + 64 * c + 16 * (T & 3), T & 3);
+                    } else {
+                        const int n = T >> 3, c = T & 7;
+                        sg_rewrite_i4(rsrc + n * kI4sStepK * 2 + 32 * c, xdst + n * kXR + 32 * c);
+                    }
                 }
             }
         }
@@ -547,7 +627,7 @@ __device__ __forceinline__ void sg_setup(uint8_t *xring, uint64_t *full, uint64_
     if (threadIdx.x < 16) multab[threadIdx.x >> 2][threadIdx.x & 3] = 1u << (15 - 4 * (threadIdx.x >> 2) - (threadIdx.x & 3));
     if (threadIdx.x == 0) {
         for (int s = 0; s < SLOTS; ++s) {
-            mbar_init(full + s, FMT == 1 && RAW > 0 ? 32 : 1);
+            mbar_init(full + s, RAW > 0 ? 32 : 1);
             mbar_init(empty + s, (unsigned)nc);
         }
         for (int s = 0; s < RAW; ++s) mbar_init(rawbar + s, 1);
@@ -557,15 +637,15 @@ __device__ __forceinline__ void sg_setup(uint8_t *xring, uint64_t *full, uint64_
 }
 
 // x [M][K] bf16 as a 2-D tensor whose box is the M rows of one step of k
-// (Q1_0_g128 into the raw ring) or of 128 k plus 16 (direct copies, the x
-// ring's row stride), rows dense in shared memory; k past K reads as zero.
+// (into the raw ring) or of 128 k plus 16 (direct copies, the x ring's row
+// stride), rows dense in shared memory; k past K reads as zero.
 static bool sg_xmap(CUtensorMap *map, int fmt, bool direct, const uint16_t *x, int M, int K)
 {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return false;
     const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)(fmt == 1 && !direct ? kSmStepK : sg_xrow(3) / 2), (cuuint32_t)M};
+    const cuuint32_t box[2] = {(cuuint32_t)(direct ? sg_xrow(3) / 2 : fmt == 1 ? kSmStepK : kI4sStepK), (cuuint32_t)M};
     const cuuint32_t estride[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), gdim, gstride, box, estride,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -909,7 +989,7 @@ __global__ void __launch_bounds__((sg_max_warps(FMT, NT) + 1) * 32, 1) k_smallm_
     const int total = q.rounds * q.nsteps;  // (round, step) sequence of every warp
     uint8_t *raw = smem;
     uint8_t *xring = raw + sg_raw_bytes(FMT, kSgRaw, q.M);
-    sg_setup<FMT, NT, kSgSlots, FMT == 1 ? kSgRaw : 0>(xring, full, empty, rawbar, multab, q.M, nw);
+    sg_setup<FMT, NT, kSgSlots, kSgRaw>(xring, full, empty, rawbar, multab, q.M, nw);
 
     if (warp == nw) {
         sg_produce<FMT, NT, kSgSlots, kSgRaw, false>(&xmap, raw, xring, full, empty, rawbar, q.M, total, 0, q.nsteps,
@@ -966,7 +1046,7 @@ __global__ void __launch_bounds__((sg_max_warps(FMT, NT) + 1) * 32, 1) k_smallm_
             if (FMT == 1)
                 sg_consume_q1<NT>(wring + stage * kSB, xring + sl * kXSlot, lane, mul, yacc);
             else
-                sg_consume_i4<NT>(wring + stage * kSB, xring + sl * kXSlot, lane, yacc);
+                sg_consume_i4p<NT>(wring + stage * kSB, xring + sl * kXSlot, lane, yacc);
         }
         __syncwarp();  // every lane has read the slot and the stage
         if (lane == 0) mbar_arrive(empty + sl);
