@@ -489,6 +489,71 @@ __device__ __forceinline__ void q1_build_chunk_warp(const uint16_t *__restrict__
     __syncwarp();  // the scratch is reused for the warp's next chunk
 }
 
+// Half h of q1_build_chunk_warp's work: group h (k = 256 ch + 128 h ..
+// +127) of the chunk, i.e. its constants info[2h], info[2h+1] and the eight
+// fragment entries whose k quarter t = e & 3 is 2h or 2h + 1 (each entry
+// reads only its group's limbs).  Two warps building the two halves of a
+// chunk write disjoint bytes, each with a limb scratch of its own; a warp's
+// chain of loads, reductions and stores is half as long.
+__device__ __forceinline__ void q1_build_half_warp(const uint16_t *__restrict__ x, int K, int ch, int h, uint8_t *frag,
+                                                   float2 *info, uint8_t *lw, int lane)
+{
+    float xv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int k = ch * kQ1ChunkK + 128 * h + 32 * j + lane;
+        xv[j] = k < K ? bf16_bits_to_float(x[k]) : 0.f;
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m = fmaxf(m, fabsf(xv[j]));
+    const float mh = warp_max_nonneg(m);
+    const int e8 = (int)((__float_as_uint(mh) >> 23) & 0xFFu);
+    const int E = max(e8 == 0 ? kQ1MinExp : e8 - 126, kQ1MinExp);  // smallest E with max|x| < 2^E
+    const int wpos = 4 * (lane & 7) + (lane >> 3);  // this lane's byte in each 32-k row of the scratch
+    int T = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int X = __float2int_rn(xv[j] * q1_pow2(23 - E));  // |X| <= 2^23
+        T += X;
+        const int B = X * (1 << (7 - (lane & 7)));              // k & 7 == lane & 7
+        const int l0 = (int)(int8_t)(B & 0xFF);
+        int r = (B - l0) >> 8;
+        const int l1 = (int)(int8_t)(r & 0xFF);
+        r = (r - l1) >> 8;
+        const int l2 = (int)(int8_t)(r & 0xFF);
+        const int row = 32 * (4 * h + j);  // the chunk's 32-k row of these k
+        lw[0 * kQ1LimbStride + row + wpos] = (uint8_t)l0;
+        lw[1 * kQ1LimbStride + row + wpos] = (uint8_t)l1;
+        lw[2 * kQ1LimbStride + row + wpos] = (uint8_t)l2;
+        lw[3 * kQ1LimbStride + row + wpos] = (uint8_t)((r - l2) >> 8);
+    }
+    const int Th = warp_sum_int(T);  // |T| <= 2^30
+    if (lane == 0) {
+        float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);
+        if ((2 * ch + h) * 128 < K) {
+            lo = make_float2(q1_pow2(E - 29), -((float)Th * q1_pow2(E - 23)));
+            hi = make_float2(q1_pow2(E - 13), 0.f);
+        }
+        info[2 * h] = lo;
+        info[2 * h + 1] = hi;
+    }
+    __syncwarp();
+    // lane l takes entry e = 4 (l' >> 1) + 2h + (l' & 1), l' = l & 7 (limb
+    // l' >> 1, k quarter t = 2h + (l' & 1)), of mmas 2 (l >> 3) and
+    // 2 (l >> 3) + 1
+    const int el = lane & 7, e = 4 * (el >> 1) + 2 * h + (el & 1), t = e & 3;
+    const uint8_t *lrow = lw + (e >> 2) * kQ1LimbStride;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int i = 2 * (lane >> 3) + q;
+        const uint32_t w0 = *reinterpret_cast<const uint32_t *>(lrow + 32 * (2 * t) + 4 * i);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(lrow + 32 * (2 * t + 1) + 4 * i);
+        *reinterpret_cast<uint2 *>(frag + e * kQ1FragLaneStride + q1_frag_plane(i)) = make_uint2(w0, w1);
+    }
+    __syncwarp();  // the scratch is reused for the warp's next task
+}
+
 __device__ __forceinline__ unsigned long long globaltimer_ns_q1()
 {
     unsigned long long t;
@@ -951,12 +1016,14 @@ __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid
     if (ch_hi > ch_lo) {
         const int n = ch_hi - ch_lo;
         if (p.x != nullptr) {
-            // fused: each warp turns its share of the slice's chunks of x into fragments
+            // fused: the warps turn the slice's chunks of x into fragments, one chunk half per task
             uint8_t *lw = smem + p.act_smem + kQ1SplitWarps * kQ1SplitRing + warp * kQ1LimbScratch;
             float2 *info = reinterpret_cast<float2 *>(smem + (size_t)n * kQ1FragBytesPerChunk);
-            for (int c = warp; c < n; c += kQ1SplitWarps)
-                q1_build_chunk_warp(p.x, p.K, ch_lo + c, smem + (size_t)c * kQ1FragBytesPerChunk, info + 4 * c, lw,
-                                    lane);
+            for (int c2 = warp; c2 < 2 * n; c2 += kQ1SplitWarps) {  // half c2 & 1 of chunk c2 >> 1
+                const int c = c2 >> 1;
+                q1_build_half_warp(p.x, p.K, ch_lo + c, c2 & 1, smem + (size_t)c * kQ1FragBytesPerChunk, info + 4 * c, lw,
+                                   lane);
+            }
         } else {
             stage_act(smem, p, ch_lo, n);
         }
@@ -1447,7 +1514,7 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
     uint8_t *zero = smem + kStSliceChunks * (kQ1FragBytesPerChunk + kQ1InfoBytesPerChunk);
     uint16_t *xs = reinterpret_cast<uint16_t *>(zero + kQ1ZeroBytes);
     uint8_t *lwall = reinterpret_cast<uint8_t *>(xs) + kStSliceK * 2;                         // limb scratch
-    float *xsf = reinterpret_cast<float *>(lwall + kStSliceChunks * kQ1LimbScratch);           // raw slice values
+    float *xsf = reinterpret_cast<float *>(lwall + 2 * kStSliceChunks * kQ1LimbScratch);       // raw slice values
     uint8_t *rings = reinterpret_cast<uint8_t *>(xsf) + kStSliceK * 4;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1562,10 +1629,10 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
             for (size_t i = (size_t)c * kStThreads + threadIdx.x; i < bufn; i += (size_t)G * kStThreads) z[i] = 0.f;
         }
         __syncthreads();
-        if (warp < kStSliceChunks)
-            q1_build_chunk_warp(xs - s * kStSliceK, q.K, s * kStSliceChunks + warp,
-                                frag + warp * kQ1FragBytesPerChunk, info + 4 * warp, lwall + warp * kQ1LimbScratch,
-                                lane);
+        if (warp < 2 * kStSliceChunks)  // half warp & 1 of chunk warp >> 1
+            q1_build_half_warp(xs - s * kStSliceK, q.K, s * kStSliceChunks + (warp >> 1), warp & 1,
+                               frag + (warp >> 1) * kQ1FragBytesPerChunk, info + 4 * (warp >> 1),
+                               lwall + warp * kQ1LimbScratch, lane);
         __syncthreads();
 
         // ---- this warp's units of the phase ----
@@ -1620,7 +1687,7 @@ lowbit_status q1stack_launch(const uint8_t *const *bits, const uint16_t *const *
     p.F = F;
     p.eps = eps;
     const size_t smem = kStSliceChunks * (kQ1FragBytesPerChunk + kQ1InfoBytesPerChunk) + kQ1ZeroBytes +
-                        kStSliceK * 2 + kStSliceChunks * kQ1LimbScratch + kStSliceK * 4 +
+                        kStSliceK * 2 + 2 * kStSliceChunks * kQ1LimbScratch + kStSliceK * 4 +
                         (size_t)kStWarps * kStStages * kQ1StageBytes;
     if (cudaFuncSetAttribute(k_q1_stack_m1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
