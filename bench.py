@@ -337,8 +337,11 @@ def _graph_time(step, stream, steps, warmup, min_ms=20.0):
     min_ms, so that the launch of the first replay is a small part of it."""
     import torch
     graph = _capture(step, stream)
-    for _ in range(warmup):
-        graph.replay()
+    # replay() launches on torch's current stream: the warm-up goes to
+    # `stream` too, so that it has finished before the first timed replay
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            graph.replay()
     stream.synchronize()
 
     def timed(n):
