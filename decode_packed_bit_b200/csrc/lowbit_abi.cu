@@ -328,7 +328,7 @@ lowbit_status lowbit_q1g128_stack_step(const uint8_t *const *w_bits, const uint1
 {
     LB_CHECK(w_bits && w_scales && x && workspace, LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(n_layers >= 1 && n_layers <= 73 && hidden >= 1 && ffn >= hidden && eps >= 0.f, LOWBIT_ERR_INVALID_ARG);
-    LB_CHECK(hidden % 1024 == 0 && ffn % 1024 == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
+    LB_CHECK(hidden % 512 == 0 && ffn % 512 == 0, LOWBIT_ERR_UNSUPPORTED_SHAPE);
     LB_CHECK(workspace_bytes >= lowbit_q1g128_stack_workspace_bytes(n_layers, hidden, ffn), LOWBIT_ERR_INVALID_ARG);
     LB_CHECK(aligned16(x) && aligned16(workspace), LOWBIT_ERR_MISALIGNED);
     LB_CHECK(record_inputs == nullptr || aligned16(record_inputs), LOWBIT_ERR_MISALIGNED);

@@ -14,15 +14,21 @@
 // touch once, so the inner loop must consume several weights per
 // instruction.  The kernels feed raw sign bits to the integer tensor cores:
 //
-//   A operand: for bit position i (0..7) one lop3 keeps bit i of each of the
+//   A operand: for bit position i (1..7) one lop3 keeps bit i of each of the
 //     four bytes of a 32-bit word of packed signs, giving four u8 values
-//     b*2^i -- four weights per instruction, no shifts, no table.
+//     b_i*2^i -- four weights per instruction, no shifts, no table.  Plane 0
+//     takes the packed bytes themselves, w = sum_i b_i 2^i, with no
+//     instruction: seven masks per eight bit planes.
 //   B operand: x rewritten exactly as integers.  Per 128-group, x is scaled
 //     to 24-bit fixed point X_k = round(x_k * 2^(23-E_g)) (E_g = the group's
-//     binary exponent ceiling), multiplied by 2^(7-i) to cancel the bit
-//     weight of its A slot, and split into four signed 8-bit limbs, one limb
-//     per B column.  Each D column then holds sum_k b_k * limb_l(X_k 2^(7-i))
-//     exactly, in int32.
+//     binary exponent ceiling).  For a byte whose bit i is weight k_i, plane
+//     0 carries Y_0 = 2^7 X_{k_0} and plane i >= 1 carries
+//     Y_i = 2^(7-i) X_{k_i} - 2^7 X_{k_0}, so that
+//         w Y_0 + sum_{i>=1} (b_i 2^i) Y_i = 2^7 sum_i b_i X_{k_i}
+//     (the bits of w in plane 0 are taken back out by the -2^7 X_{k_0} of
+//     the other planes).  |Y| < 2^30 + 2^29; each Y is split into four
+//     signed 8-bit limbs, one limb per B column, and each D column holds its
+//     limb's share exactly in int32 (|D| < 16 * 509 * 128 < 2^20).
 //   Two groups share one accumulator: B columns 0-3 carry the four limbs of
 //     the first group of a 256-k chunk, columns 4-7 those of the second.  A
 //     lane's B registers are zero whenever its column group differs from the
@@ -123,6 +129,14 @@ __device__ __forceinline__ uint2 q1_fragment(const int8_t (*lb)[256], int i, int
     return make_uint2(w[0], w[1]);
 }
 
+// The B value of weight k in bit plane i = k & 7, from its fixed-point x X
+// and X0, that of the byte's plane-0 weight k & ~7: 2^7 X0 for i = 0, else
+// 2^(7-i) X - 2^7 X0.  |X|, |X0| <= 2^23 give |result| <= 2^30 + 2^29.
+__device__ __forceinline__ int q1_plane_value(int X, int X0, int i)
+{
+    return i == 0 ? X * 128 : X * (1 << (7 - i)) - X0 * 128;
+}
+
 // One CTA of 256 threads per 256-k chunk.  Thread kk first turns x[k] into
 // four limbs; then thread t < 128 writes the 8-byte B fragment of live entry
 // t%16 for mma t/16.  A plain bf16 copy of x is kept after the fragments for
@@ -153,14 +167,15 @@ __global__ void __launch_bounds__(256) k_q1_prep_m1(const uint16_t *__restrict__
     // E = smallest integer with m < 2^E (m normal: exponent field - 126)
     const int e8 = (int)((__float_as_uint(m) >> 23) & 0xFFu);
     const int E = max(e8 == 0 ? kQ1MinExp : e8 - 126, kQ1MinExp);
-    const int X = __float2int_rn(ldexpf(xv, 23 - E));       // |X| < 2^23
-    const int B = X * (1 << (7 - (k & 7)));                 // cancels the A slot weight 2^i
+    const int X = __float2int_rn(ldexpf(xv, 23 - E));       // |X| <= 2^23
+    // k & 7 == lane & 7: the byte's plane-0 weight is in lane (lane & ~7)
+    const int B = q1_plane_value(X, __shfl_sync(0xffffffffu, X, lane & ~7), k & 7);
     int l0 = (int)(int8_t)(B & 0xFF);
     int r = (B - l0) >> 8;
     int l1 = (int)(int8_t)(r & 0xFF);
     r = (r - l1) >> 8;
     int l2 = (int)(int8_t)(r & 0xFF);
-    const int l3 = (r - l2) >> 8;                           // |B| < 2^30 keeps it in [-64, 64]
+    const int l3 = (r - l2) >> 8;                           // |B| <= 2^30 + 2^29 keeps it in [-97, 97]
     limb[0][kk] = (int8_t)l0;
     limb[1][kk] = (int8_t)l1;
     limb[2][kk] = (int8_t)l2;
@@ -315,6 +330,11 @@ __device__ __forceinline__ const uint8_t *bfrag_base(const uint8_t *frags, const
                    : zero + lc.e * kQ1FragLaneStride;
 }
 
+// A register of bit plane i from a word of packed signs: the word itself
+// for plane 0 (its B values take the other planes' bits back out), bit i of
+// each byte for the others.
+__device__ __forceinline__ uint32_t q1_plane(uint32_t w, int i) { return i == 0 ? w : w & (0x01010101u << i); }
+
 // D_lo + 256 D_hi of one limb pair, as a float (one rounding; |v| < 2^29).
 __device__ __forceinline__ float limb_pair(int lo, int hi) { return (float)(lo + (hi << 8)); }
 
@@ -337,34 +357,32 @@ __device__ __forceinline__ void consume_step(const uint8_t *st, const uint8_t *b
     if (nch == kQ1StepChunks) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const uint32_t m = 0x01010101u << i;
 #pragma unroll
             for (int c = 0; c < kQ1StepChunks; ++c) {
                 const uint2 b = *reinterpret_cast<const uint2 *>(bf + c * kQ1FragBytesPerChunk + q1_frag_plane(i));
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
+                    const uint32_t a0 = q1_plane(w[t][0][c].x, i), a1 = q1_plane(w[t][1][c].x, i);
+                    const uint32_t a2 = q1_plane(w[t][0][c].y, i), a3 = q1_plane(w[t][1][c].y, i);
                     if (i == 0)
-                        mma_u8s8_z(d[t][c], w[t][0][c].x & m, w[t][1][c].x & m, w[t][0][c].y & m, w[t][1][c].y & m,
-                                   b.x, b.y);
+                        mma_u8s8_z(d[t][c], a0, a1, a2, a3, b.x, b.y);
                     else
-                        mma_u8s8(d[t][c], w[t][0][c].x & m, w[t][1][c].x & m, w[t][0][c].y & m, w[t][1][c].y & m,
-                                 b.x, b.y);
+                        mma_u8s8(d[t][c], a0, a1, a2, a3, b.x, b.y);
                 }
             }
         }
     } else {  // one chunk left
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const uint32_t m = 0x01010101u << i;
             const uint2 b = *reinterpret_cast<const uint2 *>(bf + q1_frag_plane(i));
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
+                const uint32_t a0 = q1_plane(w[t][0][0].x, i), a1 = q1_plane(w[t][1][0].x, i);
+                const uint32_t a2 = q1_plane(w[t][0][0].y, i), a3 = q1_plane(w[t][1][0].y, i);
                 if (i == 0)
-                    mma_u8s8_z(d[t][0], w[t][0][0].x & m, w[t][1][0].x & m, w[t][0][0].y & m, w[t][1][0].y & m, b.x,
-                               b.y);
+                    mma_u8s8_z(d[t][0], a0, a1, a2, a3, b.x, b.y);
                 else
-                    mma_u8s8(d[t][0], w[t][0][0].x & m, w[t][1][0].x & m, w[t][0][0].y & m, w[t][1][0].y & m, b.x,
-                             b.y);
+                    mma_u8s8(d[t][0], a0, a1, a2, a3, b.x, b.y);
             }
         }
 #pragma unroll
@@ -448,7 +466,8 @@ __device__ __forceinline__ void q1_build_chunk_warp(const uint16_t *__restrict__
     for (int j = 0; j < 8; ++j) {
         const int X = __float2int_rn(xv[j] * q1_pow2(23 - E[j >> 2]));  // |X| <= 2^23
         T[j >> 2] += X;
-        const int B = X * (1 << (7 - (lane & 7)));                      // k & 7 == lane & 7
+        // k & 7 == lane & 7: the byte's plane-0 weight is in lane (lane & ~7)
+        const int B = q1_plane_value(X, __shfl_sync(0xffffffffu, X, lane & ~7), lane & 7);
         const int l0 = (int)(int8_t)(B & 0xFF);
         int r = (B - l0) >> 8;
         const int l1 = (int)(int8_t)(r & 0xFF);
@@ -516,7 +535,8 @@ __device__ __forceinline__ void q1_build_half_warp(const uint16_t *__restrict__ 
     for (int j = 0; j < 4; ++j) {
         const int X = __float2int_rn(xv[j] * q1_pow2(23 - E));  // |X| <= 2^23
         T += X;
-        const int B = X * (1 << (7 - (lane & 7)));              // k & 7 == lane & 7
+        // k & 7 == lane & 7: the byte's plane-0 weight is in lane (lane & ~7)
+        const int B = q1_plane_value(X, __shfl_sync(0xffffffffu, X, lane & ~7), lane & 7);
         const int l0 = (int)(int8_t)(B & 0xFF);
         int r = (B - l0) >> 8;
         const int l1 = (int)(int8_t)(r & 0xFF);
@@ -744,11 +764,11 @@ __device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *b
 #pragma unroll
                 for (int o = 0; o < 2; ++o) {
                     const int i = 2 * j + o;
-                    const uint32_t m = 0x01010101u << i;
-#pragma unroll
+        #pragma unroll
                     for (int t = 0; t < 2; ++t) {
                         const uint2 w0 = w[q][t][0], w1 = w[q][t][1];
-                        const uint32_t a0 = w0.x & m, a1 = w1.x & m, a2 = w0.y & m, a3 = w1.y & m;
+                        const uint32_t a0 = q1_plane(w0.x, i), a1 = q1_plane(w1.x, i);
+                        const uint32_t a2 = q1_plane(w0.y, i), a3 = q1_plane(w1.y, i);
 #pragma unroll
                         for (int v = 0; v < MV; ++v) {
                             if (i == 0)
@@ -1318,7 +1338,7 @@ lowbit_status q1m1_gemv_fused_launch(const uint8_t *bits, const uint16_t *scales
 
 constexpr int kStWarps = 16;
 constexpr int kStThreads = kStWarps * 32;
-constexpr int kStSliceK = 1024;                 // k per slice: four 256-k chunks
+constexpr int kStSliceK = 512;                  // k per slice: two 256-k chunks (one step)
 constexpr int kStSliceChunks = kStSliceK / kQ1ChunkK;
 constexpr int kStStages = 3;
 constexpr int kStMaxProj = 512;
@@ -1695,6 +1715,8 @@ lowbit_status q1stack_launch(const uint8_t *const *bits, const uint16_t *const *
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_q1_stack_m1, kStThreads, smem) != cudaSuccess ||
         per_sm < 1)
         return LOWBIT_ERR_CUDA;
+    // every K slice needs a CTA of its own (CTA c takes slice c % S)
+    if (F / kStSliceK > sms * per_sm || H / kStSliceK > sms * per_sm) return LOWBIT_ERR_UNSUPPORTED_SHAPE;
     // the barrier counter and phase 0's output start at zero
     if (cudaMemsetAsync(w8, 0, 256 + 2 * (size_t)F * 4, st) != cudaSuccess) return LOWBIT_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};

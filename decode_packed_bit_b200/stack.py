@@ -76,7 +76,11 @@ class Q1Stack:
         return per * len(self.layers)
 
     def fused_supported(self) -> bool:
-        return self.M == 1 and self.hidden % 1024 == 0 and self.ffn % 1024 == 0
+        if not (self.M == 1 and self.hidden % 512 == 0 and self.ffn % 512 == 0):
+            return False
+        # one CTA per SM, and every 512-k slice of the ffn-wide input needs one
+        dev = self.x.device
+        return dev.type != "cuda" or self.ffn // 512 <= torch.cuda.get_device_properties(dev).multi_processor_count
 
     def step_fused(self, stream=None, record: StackRecord | None = None):
         """The same step as step() at M = 1, as one launch of

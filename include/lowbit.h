@@ -272,8 +272,9 @@ lowbit_status lowbit_q1g128_gemv_noalloc(const uint8_t *w_bits, const uint16_t *
  *   record_inputs / record_outputs: NULL, or [7 * n_layers][ffn] bf16 /
  *     fp32 that receive every projection's input and fp32 output (row i
  *     uses the first K or N entries).
- * Needs hidden and ffn multiples of 1024, ffn >= hidden, 1 <= n_layers <=
- * 73.  The kernel is a cooperative launch (every CTA resident) whose phases
+ * Needs hidden and ffn multiples of 512, ffn >= hidden, 1 <= n_layers <=
+ * 73, and ffn / 512 at most the number of CTAs resident at once (one per SM;
+ * else LOWBIT_ERR_UNSUPPORTED_SHAPE).  The kernel is a cooperative launch (every CTA resident) whose phases
  * are separated by a grid barrier; a barrier wait bounded at 2 s that runs
  * out sets bit 2 of lowbit_fault_flags().  The projections' partial sums
  * are added with fp32 atomics, so results can differ in the last bits from

@@ -171,6 +171,23 @@ def test_group_validation(L):
     assert i(pp, pp, FAKE, pp, 2, 1, 16, 96, None) == 3        # K % 64
 
 
+def test_stack_step_validation(L):
+    """Every case fails before the pointer loop, so nothing reaches a launch."""
+    ptrs = (ctypes.c_void_p * 14)(*([0x10000] * 14))
+    pp = ctypes.cast(ptrs, ctypes.c_void_p)
+    s = L.lowbit_q1g128_stack_step
+    ws = L.lowbit_q1g128_stack_workspace_bytes(2, 1536, 2560)
+    assert ws >= 256 + 2 * 2560 * 4
+    assert s(pp, pp, 2, 1536, 2560, None, 1e-6, FAKE, ws, None, None, None) == 1      # null x
+    assert s(pp, pp, 0, 1536, 2560, FAKE, 1e-6, FAKE, ws, None, None, None) == 1      # no layers
+    assert s(pp, pp, 74, 1536, 2560, FAKE, 1e-6, FAKE, ws, None, None, None) == 1     # too many layers
+    assert s(pp, pp, 2, 2560, 1536, FAKE, 1e-6, FAKE, ws, None, None, None) == 1      # ffn < hidden
+    assert s(pp, pp, 2, 768, 2560, FAKE, 1e-6, FAKE, ws, None, None, None) == 3       # hidden % 512
+    assert s(pp, pp, 2, 1536, 2816, FAKE, 1e-6, FAKE, ws, None, None, None) == 3      # ffn % 512
+    assert s(pp, pp, 2, 1536, 2560, FAKE, 1e-6, FAKE, ws - 1, None, None, None) == 1  # workspace too small
+    assert s(pp, pp, 2, 1536, 2560, MIS, 1e-6, FAKE, ws, None, None, None) == 2       # misaligned x
+
+
 def test_z80_generate_validation(L):
     layers = (ctypes.c_void_p * 3)(0x10000, 0x10000, 0x10000)
     lp = ctypes.cast(layers, ctypes.c_void_p)

@@ -131,12 +131,13 @@ def test_stack_m1_one_launch_teacher_forced(stack_weights):
     assert (np.abs(got - r64) <= tol).all()
 
 
-@pytest.mark.parametrize("hidden,ffn,n_layers", [(1024, 8192, 2), (2048, 3072, 3)])
+@pytest.mark.parametrize("hidden,ffn,n_layers", [(1024, 8192, 2), (2048, 3072, 3), (1536, 2560, 2)])
 def test_stack_one_launch_other_widths(cuda_device, hidden, ffn, n_layers):
-    """The one-launch step at widths whose K-slice counts (1 and 8, 2 and
-    3 slices of 1024) differ from the 5120/17408 stack's, so every CTA's
-    slice, rank and share of the blocks take other values; checked
-    teacher-forced like the full stack, plus the step output."""
+    """The one-launch step at widths whose K-slice counts (2 and 16, 4 and
+    6, 3 and 5 slices of 512) differ from the 5120/17408 stack's (10 and
+    34), so every CTA's slice, rank and share of the blocks take other
+    values; checked teacher-forced like the full stack, plus the step
+    output."""
     from decode_packed_bit_b200 import build
     build.build()
     from decode_packed_bit_b200 import lowbit as lb
