@@ -622,7 +622,7 @@ def run_q1_4096(args, world, rank, local):
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes_per_launch": bytes_launch,
                      "us_per_launch": round(ms * 1e3 / launches, 3),
-                     "kernel": "k_q1_m1_lean<1>",
+                     "kernel": "k_q1_m1_lean<1, 4096>",
                      "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)"},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),

@@ -815,21 +815,25 @@ __device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *b
 // they run at most 12 warps (168 registers a thread).
 __host__ __device__ constexpr int q1l_max_warps(int mv) { return mv == 1 ? kQ1LMaxWarps : 12; }
 
-template <int MV>
+template <int MV, int KF>
 __global__ void __launch_bounds__(q1l_max_warps(MV) * 32, 1) k_q1_m1_lean(const __grid_constant__ Q1Group grp,
                                                                           const Q1Params p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ float part[2][q1l_max_warps(MV)][MV][kQ1StepRows];  // [head / tail][warp][vector][row] of cut cells
     pdl_launch_dependents();
+    // KF > 0: K known at compile time, so the copy addresses of a step are
+    // one register plus immediate offsets and the per-cell counts constants
+    const int K = KF > 0 ? KF : p.K;
+    const int nchunks = KF > 0 ? KF / kQ1ChunkK : p.nchunks;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int c0 = (int)((long long)blockIdx.x * p.cells / gridDim.x);
     const int c1 = (int)((long long)(blockIdx.x + 1) * p.cells / gridDim.x);
-    const int spc = p.nchunks / kQ1LChunks;  // steps per cell
+    const int spc = nchunks / kQ1LChunks;  // steps per cell
     const int T = (c1 - c0) * spc;
     const int s0 = (int)((long long)warp * T / nw), s1 = (int)((long long)(warp + 1) * T / nw);
-    const size_t rowbytes = (size_t)(p.K >> 3);
-    const int G = p.K >> 7;
+    const size_t rowbytes = (size_t)(K >> 3);
+    const int G = K >> 7;
     uint8_t *ring = smem + p.act_smem + warp * (kQ1LStages * kQ1LStageBytes);
     const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
 
@@ -880,18 +884,18 @@ __global__ void __launch_bounds__(q1l_max_warps(MV) * 32, 1) k_q1_m1_lean(const 
     for (int t = 0; t < kQ1LStages; ++t) issue_next();
 
     pdl_wait_primary();  // x or the activation, and the outputs, follow stream order from here
-    const int vfrag = p.nchunks * kQ1FragBytesPerChunk;  // bytes of one vector's fragments
+    const int vfrag = nchunks * kQ1FragBytesPerChunk;  // bytes of one vector's fragments
     uint8_t *zero = smem + p.act_smem - kQ1ZeroBytes;
     float2 *info = reinterpret_cast<float2 *>(smem + (size_t)MV * vfrag);
     if (p.x != nullptr) {
         // this warp's limb scratch, after every warp's ring
         uint8_t *lw = smem + p.act_smem + (size_t)nw * (kQ1LStages * kQ1LStageBytes) + (size_t)warp * kQ1LimbScratch;
-        for (int idx = warp; idx < MV * p.nchunks; idx += nw) {
-            const int v = idx / p.nchunks, ch = idx - v * p.nchunks;
+        for (int idx = warp; idx < MV * nchunks; idx += nw) {
+            const int v = idx / nchunks, ch = idx - v * nchunks;
             uint8_t *frag = smem + (size_t)v * vfrag + (size_t)ch * kQ1FragBytesPerChunk;
-            float2 *inf = info + 4 * (v * p.nchunks + ch);
+            float2 *inf = info + 4 * (v * nchunks + ch);
             if (v < p.M) {
-                q1_build_chunk_warp(p.x + (size_t)v * p.K, p.K, ch, frag, inf, lw, lane);
+                q1_build_chunk_warp(p.x + (size_t)v * K, K, ch, frag, inf, lw, lane);
             } else {
                 for (int i = lane; i < kQ1FragBytesPerChunk / 16; i += 32)
                     reinterpret_cast<uint4 *>(frag)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -899,7 +903,7 @@ __global__ void __launch_bounds__(q1l_max_warps(MV) * 32, 1) k_q1_m1_lean(const 
             }
         }
     } else if (c1 > c0) {
-        stage_act(smem, p, 0, p.nchunks);  // one vector
+        stage_act(smem, p, 0, nchunks);  // one vector
     }
     clear_zero_block(zero);
     __syncthreads();
@@ -932,7 +936,7 @@ __global__ void __launch_bounds__(q1l_max_warps(MV) * 32, 1) k_q1_m1_lean(const 
             __syncwarp();
             lean_consume<MV>(ring + slot * kQ1LStageBytes,
                              live ? bf_live + t * (kQ1LChunks * kQ1FragBytesPerChunk) : bf_dead, bstride,
-                             inf0 + 4 * kQ1LChunks * t, 4 * p.nchunks, woff, soff, yacc);
+                             inf0 + 4 * kQ1LChunks * t, 4 * nchunks, woff, soff, yacc);
             __syncwarp();  // every lane is done with this stage before it is refilled
             issue_next();  // refill the slot just consumed
             slot = slot + 1 == kQ1LStages ? 0 : slot + 1;
@@ -1236,7 +1240,12 @@ static lowbit_status q1m1_launch(const Q1Plan &P, const uint8_t *const *bits, co
     p.M = M;
     void (*kern)(const Q1Group, const Q1Params) = k_q1_m1_split;
     if (P.lean)
-        kern = P.mv == 1 ? k_q1_m1_lean<1> : P.mv == 2 ? k_q1_m1_lean<2> : k_q1_m1_lean<4>;
+        kern = P.mv == 2   ? k_q1_m1_lean<2, 0>
+               : P.mv == 4 ? k_q1_m1_lean<4, 0>
+               : K == 4096 ? k_q1_m1_lean<1, 4096>
+               : K == 5120 ? k_q1_m1_lean<1, 5120>
+               : K == 17408 ? k_q1_m1_lean<1, 17408>
+                             : k_q1_m1_lean<1, 0>;
     else if (P.stream)
         kern = k_q1_m1_stream;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) != cudaSuccess)
