@@ -1504,13 +1504,15 @@ __device__ __forceinline__ float st_block_sum(float v, float *red)
     return t;
 }
 
-// Grid barrier: every CTA adds 1 per phase; wait until all G have.
+// Grid barrier: every CTA adds 1 per phase; wait until all G have.  The
+// add is a release at GPU scope (it orders every write of the CTA that the
+// block barrier made visible to thread 0) and the poll an acquire, so no
+// separate fence is needed on either side.
 __device__ __forceinline__ void st_grid_sync(const StackP &p, unsigned target)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(p.bar, 1u);
+        asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p.bar), "r"(1u) : "memory");
         unsigned v = 0;
         const unsigned long long t0 = globaltimer_ns_q1();
         while (true) {
@@ -1523,7 +1525,6 @@ __device__ __forceinline__ void st_grid_sync(const StackP &p, unsigned target)
                 break;
             }
         }
-        __threadfence();
     }
     __syncthreads();
 }
