@@ -764,7 +764,7 @@ __device__ __forceinline__ void lean_consume(const uint8_t *st, const uint8_t *b
 #pragma unroll
                 for (int o = 0; o < 2; ++o) {
                     const int i = 2 * j + o;
-        #pragma unroll
+#pragma unroll
                     for (int t = 0; t < 2; ++t) {
                         const uint2 w0 = w[q][t][0], w1 = w[q][t][1];
                         const uint32_t a0 = q1_plane(w0.x, i), a1 = q1_plane(w1.x, i);
