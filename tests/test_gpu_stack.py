@@ -162,3 +162,30 @@ def test_stack_one_launch_other_widths(cuda_device, hidden, ffn, n_layers):
     got = synth.bf16_bits_to_f32(host(st.x.view(torch.int16)).view(np.uint16)).astype(np.float64)
     tol = 0.5 * _bf16_ulp(r64) + 1e-6 * np.abs(r64) + 1e-30
     assert (np.abs(got - r64) <= tol).all()
+
+
+def test_stack_refuses_more_slices_than_resident_ctas(cuda_device):
+    """Every 512-k slice of the ffn-wide input needs a CTA of its own (one
+    per SM).  With one slice more than that the launcher returns
+    LOWBIT_ERR_UNSUPPORTED_SHAPE before it clears the workspace or launches;
+    the buffers are real (small, never read)."""
+    from decode_packed_bit_b200 import build
+    build.build()
+    from decode_packed_bit_b200 import lowbit as lb
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    hidden, ffn = 512, 512 * (sms + 1)
+    ws_bytes = lb.lowbit_q1g128_stack_workspace_bytes(1, hidden, ffn)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=cuda_device)
+    bufs = [torch.zeros(16, dtype=torch.uint8, device=cuda_device) for _ in range(14)]
+    x = torch.zeros(hidden, dtype=torch.int16, device=cuda_device)
+    bits, keep_b = lb._ptr_array(bufs[:7])
+    scales, keep_s = lb._ptr_array(bufs[7:])
+    status = lb.lib().lowbit_q1g128_stack_step(bits, scales, 1, hidden, ffn, lb._ptr(x), 1e-6, lb._ptr(ws),
+                                               ws_bytes, None, None, lb._stream(None))
+    torch.cuda.synchronize()
+    assert status == 3
+    assert lb.lowbit_fault_flags() == 0
+    # one slice per SM is still taken by the one-launch step's planner
+    from decode_packed_bit_b200.stack import Q1Stack
+    assert not Q1Stack([], hidden, ffn, 1, cuda_device).fused_supported()
+    assert Q1Stack([], hidden, 512 * sms, 1, cuda_device).fused_supported()
