@@ -513,15 +513,17 @@ __device__ __forceinline__ void q1_build_chunk_warp(const uint16_t *__restrict__
 // fragment entries whose k quarter t = e & 3 is 2h or 2h + 1 (each entry
 // reads only its group's limbs).  Two warps building the two halves of a
 // chunk write disjoint bytes, each with a limb scratch of its own; a warp's
-// chain of loads, reductions and stores is half as long.
-__device__ __forceinline__ void q1_build_half_warp(const uint16_t *__restrict__ x, int K, int ch, int h, uint8_t *frag,
-                                                   float2 *info, uint8_t *lw, int lane)
+// chain of loads, reductions and stores is half as long.  xat(k): x[k], a
+// bf16 number, as a float (k < K).
+template <typename XAt>
+__device__ __forceinline__ void q1_build_half_warp(XAt xat, int K, int ch, int h, uint8_t *frag, float2 *info,
+                                                   uint8_t *lw, int lane)
 {
     float xv[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int k = ch * kQ1ChunkK + 128 * h + 32 * j + lane;
-        xv[j] = k < K ? bf16_bits_to_float(x[k]) : 0.f;
+        xv[j] = k < K ? xat(k) : 0.f;
     }
     float m = 0.f;
 #pragma unroll
@@ -1045,8 +1047,8 @@ __global__ void __launch_bounds__(kQ1SplitWarps * 32) k_q1_m1_split(const __grid
             float2 *info = reinterpret_cast<float2 *>(smem + (size_t)n * kQ1FragBytesPerChunk);
             for (int c2 = warp; c2 < 2 * n; c2 += kQ1SplitWarps) {  // half c2 & 1 of chunk c2 >> 1
                 const int c = c2 >> 1;
-                q1_build_half_warp(p.x, p.K, ch_lo + c, c2 & 1, smem + (size_t)c * kQ1FragBytesPerChunk, info + 4 * c, lw,
-                                   lane);
+                q1_build_half_warp([&](int k) { return bf16_bits_to_float(p.x[k]); }, p.K, ch_lo + c, c2 & 1,
+                                   smem + (size_t)c * kQ1FragBytesPerChunk, info + 4 * c, lw, lane);
             }
         } else {
             stage_act(smem, p, ch_lo, n);
@@ -1492,10 +1494,12 @@ __device__ __forceinline__ void st_prefetch_l2(const StackW &W, const StackP &p,
     }
 }
 
+// Sum over the CTA.  red needs no barrier before it is written: its
+// readers in the previous phase have passed the block barrier after that
+// phase's fragment build since.
 __device__ __forceinline__ float st_block_sum(float v, float *red)
 {
     v = warp_sum(v);
-    __syncthreads();  // red is free
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
     __syncthreads();
     float t = 0.f;
@@ -1542,8 +1546,7 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
     uint8_t *frag = smem;                                                  // 4 chunks of fragments
     float2 *info = reinterpret_cast<float2 *>(smem + kStSliceChunks * kQ1FragBytesPerChunk);
     uint8_t *zero = smem + kStSliceChunks * (kQ1FragBytesPerChunk + kQ1InfoBytesPerChunk);
-    uint16_t *xs = reinterpret_cast<uint16_t *>(zero + kQ1ZeroBytes);
-    uint8_t *lwall = reinterpret_cast<uint8_t *>(xs) + kStSliceK * 2;                         // limb scratch
+    uint8_t *lwall = zero + kQ1ZeroBytes;                                                     // limb scratch
     float *xsf = reinterpret_cast<float *>(lwall + 2 * kStSliceChunks * kQ1LimbScratch);       // raw slice values
     uint8_t *rings = reinterpret_cast<uint8_t *>(xsf) + kStSliceK * 4;
 
@@ -1642,27 +1645,29 @@ __global__ void __launch_bounds__(kStThreads, 1) k_q1_stack_m1(const __grid_cons
                 p.x[i] = __bfloat16_as_ushort(__float2bfloat16_rn(prev[i] * inv));
             break;
         }
-        for (int i = threadIdx.x; i < kStSliceK; i += kStThreads) {
-            const int k = s * kStSliceK + i;
-            uint16_t xb;
-            if (prev == nullptr)
-                xb = p.x[k];
-            else
-                xb = __bfloat16_as_ushort(__float2bfloat16_rn(xsf[i] * inv));  // stored before the block sum
-            xs[i] = xb;
-            if (p.rec_in != nullptr && c < S)  // the first CTA of each slice records it
+        // the projections' input: x_k = bf16(raw_k * inv) over this CTA's
+        // slice; the builders round it themselves from the raw values (kept
+        // in xsf before the block sum, whose barrier makes them visible)
+        if (p.rec_in != nullptr && c < S)  // the first CTA of each slice records it
+            for (int i = threadIdx.x; i < kStSliceK; i += kStThreads) {
+                const int k = s * kStSliceK + i;
+                const uint16_t xb = prev == nullptr ? p.x[k] : __bfloat16_as_ushort(__float2bfloat16_rn(xsf[i] * inv));
                 for (int m = 0; m < q.nmat; ++m) p.rec_in[(size_t)st_proj(q, m) * p.F + k] = xb;
+            }
+        if (prev == nullptr) {  // the step input, exact as a float (inv = 1)
+            for (int i = threadIdx.x; i < kStSliceK; i += kStThreads) xsf[i] = bf16_bits_to_float(p.x[s * kStSliceK + i]);
+            __syncthreads();
         }
         // zero the buffer two phases ahead (read last by the previous phase's prologue)
         {
             float *z = p.buf + (size_t)((ph_idx + 1) % 3) * bufn;
             for (size_t i = (size_t)c * kStThreads + threadIdx.x; i < bufn; i += (size_t)G * kStThreads) z[i] = 0.f;
         }
-        __syncthreads();
         if (warp < 2 * kStSliceChunks)  // half warp & 1 of chunk warp >> 1
-            q1_build_half_warp(xs - s * kStSliceK, q.K, s * kStSliceChunks + (warp >> 1), warp & 1,
-                               frag + (warp >> 1) * kQ1FragBytesPerChunk, info + 4 * (warp >> 1),
-                               lwall + warp * kQ1LimbScratch, lane);
+            q1_build_half_warp(
+                [&](int k) { return __bfloat162float(__float2bfloat16_rn(xsf[k - s * kStSliceK] * inv)); }, q.K,
+                s * kStSliceChunks + (warp >> 1), warp & 1, frag + (warp >> 1) * kQ1FragBytesPerChunk,
+                info + 4 * (warp >> 1), lwall + warp * kQ1LimbScratch, lane);
         __syncthreads();
 
         // ---- this warp's units of the phase ----
@@ -1717,7 +1722,7 @@ lowbit_status q1stack_launch(const uint8_t *const *bits, const uint16_t *const *
     p.F = F;
     p.eps = eps;
     const size_t smem = kStSliceChunks * (kQ1FragBytesPerChunk + kQ1InfoBytesPerChunk) + kQ1ZeroBytes +
-                        kStSliceK * 2 + 2 * kStSliceChunks * kQ1LimbScratch + kStSliceK * 4 +
+                        2 * kStSliceChunks * kQ1LimbScratch + kStSliceK * 4 +
                         (size_t)kStWarps * kStStages * kQ1StageBytes;
     if (cudaFuncSetAttribute(k_q1_stack_m1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
