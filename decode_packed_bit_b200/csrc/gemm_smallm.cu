@@ -452,9 +452,12 @@ __device__ __forceinline__ void sg_consume_i4p(const uint8_t *stage, const uint8
 // L%2 of rows L/2 and L/2 + 16; INT4_G64: the 16-byte column L%4 of rows
 // L/4 + {0, 8, 16, 24}; both: the scale pair of row L.  Rows past N copy
 // nothing (zero fill).
-template <int FMT>
+// KF > 0: K fixed at compile time, so the copies' row stride is an
+// immediate offset.
+template <int FMT, int KF = 0>
 struct SgCopy {
     static constexpr int kCopies = FMT == 1 ? 2 : 4;
+    static constexpr unsigned kStride = KF > 0 ? (unsigned)((FMT == 1 ? 16 : 8) * (FMT == 1 ? KF / 8 : KF / 2)) : 0u;
     static constexpr unsigned kDstStride = FMT == 1 ? 16 * kSmRowStride : 8 * kI4sRowStride;
     const uint8_t *src = nullptr;  // copy 0's bytes of step 0; copy c reads c * stride bytes further
     const uint16_t *scale = nullptr;
@@ -483,7 +486,8 @@ struct SgCopy {
 #pragma unroll
         for (int c = 0; c < kCopies; ++c) {
             const bool v = (ok >> c) & 1u;
-            sm_cp16(st + dst0 + kDstStride * c, v ? src + c * stride + s * SgFmt<FMT>::kStepBytes : dummy, v);
+            const unsigned cs = KF > 0 ? kStride * c : stride * c;
+            sm_cp16(st + dst0 + kDstStride * c, v ? src + cs + s * SgFmt<FMT>::kStepBytes : dummy, v);
         }
         const bool sv = (ok >> kCopies) & 1u;
         sm_cp4(st + SgFmt<FMT>::kStageW + lane * 4, sv ? scale + 2 * s : dummy, sv);
@@ -972,7 +976,7 @@ struct SmGParams {
     int M, N, K, nsteps, blocksN, nblocks, rounds;
 };
 
-template <int FMT, int NT>
+template <int FMT, int NT, int KF = 0>
 __global__ void __launch_bounds__((sg_max_warps(FMT, NT) + 1) * 32, 1) k_smallm_grp(const __grid_constant__ SmGroup grp,
                                                                  const __grid_constant__ CUtensorMap xmap,
                                                                  const SmGParams q)
@@ -1005,7 +1009,7 @@ __global__ void __launch_bounds__((sg_max_warps(FMT, NT) + 1) * 32, 1) k_smallm_
     for (int i = 0; i < 4; ++i) mul[i] = multab[lane & 3][i];
 
     // copy cursor: the (round, step) whose weights go out next
-    SgCopy<FMT> cp;
+    SgCopy<FMT, KF> cp;
     int cj = 0, cs = 0, cstage = 0;
     bool clive = false;
     auto set_round = [&](int j) {
@@ -1147,11 +1151,15 @@ lowbit_status smg_launch(int fmt, const uint8_t *const *bits, const uint16_t *co
     q.rounds = P.rounds;
     void (*kern)(const SmGroup, const CUtensorMap, const SmGParams);
     if (fmt == 1)
-        kern = P.NT == 1 ? k_smallm_grp<1, 1> : k_smallm_grp<1, 2>;
+        kern = P.NT == 1     ? k_smallm_grp<1, 1>
+               : K == 5120  ? k_smallm_grp<1, 2, 5120>
+               : K == 17408 ? k_smallm_grp<1, 2, 17408>
+                            : k_smallm_grp<1, 2>;
     else
         kern = P.NT == 1 ? k_smallm_grp<3, 1>
              : P.NT == 2 ? k_smallm_grp<3, 2>
              : P.NT == 3 ? k_smallm_grp<3, 3>
+             : K == 4096 ? k_smallm_grp<3, 4, 4096>
                          : k_smallm_grp<3, 4>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
